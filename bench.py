@@ -1,0 +1,420 @@
+#!/usr/bin/env python
+"""Benchmark of the KDA forward path on B200: chunkwise prefill (the step) and
+single-step decode, printed as one JSON line by rank 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Step: one kda_chunk_fwd over the long-context workload (B=1, H=32,
+T=1,048,576, dk=dv=128; bf16 q/k/v, fp32 g and beta, zero h0, out bf16 +
+final state fp32).  Inputs are synthetic (gated_delta_rule_100_b200.inputs),
+resident in HBM before the timed region, and 51.7 GB per step (far above the
+126 MB L2, so no flush is needed between steps).  Value: tokens (B*T) per
+second over all ranks; each rank runs its own copy of the workload (weak
+scaling, no collective on the data path).  Timing: CUDA events on the
+launching stream, barrier + synchronize on both sides, max over ranks.
+
+Also measured and reported in the same line:
+  decode   64 consecutive kda_decode_step calls on B=256, H=32, d=128 with a
+           512 MiB fp32 state (GB/s of algorithmic traffic);
+  e2e      the same prefill metric through the public API with pinned host
+           buffers: H2D of the inputs, the kernel, D2H of out and hT per step;
+  roofline achieved algorithmic GB/s of the prefill kernel vs measured HBM peak;
+  cpu_baseline  the fp64 oracle on a bounded sample of the workload (rank 0,
+           N = 1 only).
+
+--impl reference times the fp64 oracle (the only reference that exists for
+this method) on the host cores, on bounded samples of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = "long_context_B1_H32_T1M_d128"
+METRIC = "KDA prefill tokens/s & TFLOP/s; decode-step state GB/s vs B200 HBM peak"
+CHUNK = 64
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ------------------------------------------------------------------ helpers ----
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def prefill_bytes(B, T, H, dk, dv, with_h0, with_hT):
+    """Algorithmic HBM bytes of one prefill launch: q, k, v (bf16), g (fp32),
+    beta (fp32) read once, out (bf16) written once, h0/hT (fp32) once."""
+    per_token_head = 2 * dk * 2 + dv * 2 + 4 * dk + 4 + 2 * dv
+    state = 4 * dk * dv * B * H
+    return B * T * H * per_token_head + (state if with_h0 else 0) + (state if with_hT else 0)
+
+
+def prefill_flops(B, T, H, dk, dv, C=CHUNK):
+    """Algorithmic flops of the chunkwise form (triangles counted once): the three
+    state contractions, A, the triangular solve, the causal q k^T and P Vnew."""
+    per = (6 * dk * dv + (C - 1) * dk + (C - 1) * (dk + dv) + (C + 1) * (dk + dv))
+    return B * T * H * per
+
+
+def decode_bytes(B, H, dk, dv):
+    """State read + written (fp32) and q, k, v, g, beta, out per (b, h)."""
+    return B * H * (2 * 4 * dk * dv + 2 * dk * 2 + dv * 2 + 4 * dk + 4 + 2 * dv)
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "gated_delta_rule_100_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(kernel):
+    """Per-launch DRAM bytes from the committed ncu summary, if it was taken on
+    the current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        t = json.load(f)
+    e = t.get(kernel)
+    if not e or e.get("source_hash") != kernel_source_hash():
+        return None
+    return e.get("bytes_per_launch_full_workload")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 100 ms."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        time.sleep(0.2)
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out = ""
+        else:
+            self.out = ""
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[4:8]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup(args):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "gloo" if args.impl == "reference" else "nccl"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world, device):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------- cpu oracle ----
+def oracle_rate(d, scale, heads, tokens, threads):
+    """Run the fp64 oracle on `heads` x first `tokens` tokens; returns (seconds, token-heads)."""
+    import oracle
+    import torch
+
+    def cut(t):
+        return t[:, :tokens, :heads].to("cpu", torch.float64).numpy()
+
+    args = [cut(d[k]) for k in ("q", "k", "v", "g", "beta")]
+    t0 = time.perf_counter()
+    oracle.kda_fwd(*args, scale, None, threads=threads)
+    return time.perf_counter() - t0, heads * tokens * d["q"].shape[0]
+
+
+def cpu_baseline(d, cfg, budget_s):
+    """Oracle throughput on a bounded sample sized to about `budget_s` seconds."""
+    cores = os.cpu_count() or 1
+    heads = min(cfg.H, cores)
+    dt, n = oracle_rate(d, cfg.scale, heads, 512, heads)
+    rate = n / max(dt, 1e-9)
+    tokens = int(min(cfg.T, max(512, rate * budget_s / heads)))
+    tokens = max(512, (tokens // 512) * 512)
+    dt, n = oracle_rate(d, cfg.scale, heads, tokens, heads)
+    th_per_s = n / dt
+    return {"value": th_per_s / cfg.H, "unit": "tokens/s", "cores": heads, "kind": "oracle",
+            "sample": f"fp64 oracle on heads 0-{heads - 1} x first {tokens} tokens of the workload "
+                      f"({n} token-heads, {dt:.1f} s, {heads} threads); tokens/s = token-heads/s / {cfg.H}"}
+
+
+# -------------------------------------------------------------------- arms ----
+def run_reference(args):
+    """The fp64 oracle on the host cores (rank 0 only)."""
+    import torch
+    from gated_delta_rule_100_b200 import inputs
+
+    world, rank, _ = dist_setup(args)
+    if rank != 0:
+        return 0
+    cfg = inputs.CONFIGS[WORKLOAD]
+    cores = os.cpu_count() or 1
+    heads = min(cfg.H, cores)
+    tokens = 2048
+    d = inputs.make_prefill(cfg.B, tokens, heads, cfg.dk, cfg.dv, decay=cfg.decay, seed=cfg.seed)
+    times = []
+    for i in range(args.warmup + args.steps):
+        dt, n = oracle_rate(d, cfg.scale, heads, tokens, heads)
+        if i >= args.warmup:
+            times.append(dt)
+    step = statistics.mean(times)
+    value = heads * tokens / step / cfg.H
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": step * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "B": cfg.B, "H": cfg.H, "T": cfg.T, "dk": cfg.dk, "dv": cfg.dv},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": heads, "kind": "oracle",
+                         "sample": f"each step: fp64 oracle on {heads} heads x {tokens} tokens "
+                                   f"(synthetic, workload recipe); tokens/s = token-heads/s / {cfg.H}"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args):
+    import torch
+
+    from gated_delta_rule_100_b200 import inputs, kda
+
+    world, rank, local = dist_setup(args)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    kda.load()
+    cfg = inputs.CONFIGS[args.workload]
+    P, peak_src = peaks()
+    stream = torch.cuda.current_stream()
+
+    # ---------------- prefill (the step) ----------------
+    d = inputs.make_config(cfg, device=dev) if rank == 0 else inputs.make_prefill(
+        cfg.B, cfg.T, cfg.H, cfg.dk, cfg.dv, decay=cfg.decay, h0_std=cfg.h0_std, seed=cfg.seed + 1000 * rank,
+        device=dev)
+    out = torch.empty((cfg.B, cfg.T, cfg.H, cfg.dv), dtype=torch.bfloat16, device=dev)
+    hT = torch.empty((cfg.B, cfg.H, cfg.dk, cfg.dv), dtype=torch.float32, device=dev)
+
+    def step():
+        kda.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], cfg.scale, d["h0"], out=out, hT=hT,
+                      stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if kda.stream_status(stream) != kda.KDA_OK:
+        raise RuntimeError("device-side error during warm-up")
+
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    with ClockSampler(local) as clk:
+        barrier(world)
+        torch.cuda.synchronize()
+        ev[0].record(stream)
+        for i in range(args.steps):
+            step()
+            ev[i + 1].record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+    if kda.stream_status(stream) != kda.KDA_OK:
+        raise RuntimeError("device-side error in the timed region")
+    launch_ms = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
+    total_ms = ev[0].elapsed_time(ev[-1])
+    total_ms = max_over_ranks(total_ms, world, dev)
+    ms_per_step = total_ms / args.steps
+    tokens_per_step = cfg.B * cfg.T
+    value = tokens_per_step * world * args.steps / (total_ms / 1e3)
+
+    nbytes = prefill_bytes(cfg.B, cfg.T, cfg.H, cfg.dk, cfg.dv, cfg.h0_std > 0, True)
+    nflops = prefill_flops(cfg.B, cfg.T, cfg.H, cfg.dk, cfg.dv)
+    avg_launch_s = statistics.mean(launch_ms) / 1e3
+    achieved = nbytes / avg_launch_s / 1e9
+    roof = {"kernel": "chunk_fwd_kernel", "bound": "hbm", "achieved": achieved, "peak": P["hbm_gbs"],
+            "unit": "GB/s", "frac": achieved / P["hbm_gbs"], "peak_source": peak_src,
+            "traffic": measured_traffic("chunk_fwd_kernel"),
+            "algorithmic_bytes_per_launch": nbytes,
+            "tensor_view": {"achieved_tflops": nflops / avg_launch_s / 1e12,
+                            "peak_tflops": P["bf16_tflops_sustained"],
+                            "frac": nflops / avg_launch_s / 1e12 / P["bf16_tflops_sustained"]}}
+
+    # ---------------- decode ----------------
+    dec = None
+    if not args.no_decode:
+        dcfg = inputs.DECODE_CONFIG
+        dd = inputs.make_decode_config(dcfg, device=dev)
+        state = dd["state"]
+        dout = torch.empty((dcfg.B, dcfg.H, dcfg.dv), dtype=torch.bfloat16, device=dev)
+        for s in range(3):
+            kda.decode_step(dd["q"][s], dd["k"][s], dd["v"][s], dd["g"][s], dd["beta"][s], dcfg.scale, state,
+                            out=dout, stream=stream)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        e0.record(stream)
+        for s in range(dcfg.steps):
+            kda.decode_step(dd["q"][s], dd["k"][s], dd["v"][s], dd["g"][s], dd["beta"][s], dcfg.scale, state,
+                            out=dout, stream=stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        dms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+        db = decode_bytes(dcfg.B, dcfg.H, dcfg.dk, dcfg.dv)
+        gbs = db * dcfg.steps / (dms / 1e3) / 1e9
+        dec = {"metric": "decode-step state GB/s", "value": gbs * world, "unit": "GB/s",
+               "per_gpu_gbs": gbs, "us_per_step": dms * 1e3 / dcfg.steps, "steps": dcfg.steps,
+               "config": {"workload": dcfg.name, "B": dcfg.B, "H": dcfg.H, "dk": dcfg.dk, "dv": dcfg.dv},
+               "gpu_launches": dcfg.steps,
+               "roofline": {"kernel": "decode_step_kernel", "bound": "hbm", "achieved": gbs,
+                            "peak": P["hbm_gbs"], "unit": "GB/s", "frac": gbs / P["hbm_gbs"],
+                            "peak_source": peak_src, "traffic": measured_traffic("decode_step_kernel"),
+                            "algorithmic_bytes_per_launch": db}}
+        del dd, state
+
+    # ---------------- end to end from pinned host buffers ----------------
+    e2e = None
+    if not args.no_e2e:
+        host = {k: (torch.empty(v.shape, dtype=v.dtype, pin_memory=True).copy_(v) if v is not None else None)
+                for k, v in d.items()}
+        h_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        h_hT = torch.empty(hT.shape, dtype=hT.dtype, pin_memory=True)
+        bufs = kda.DeviceBuffers.__new__(kda.DeviceBuffers)
+        bufs.q, bufs.k, bufs.v, bufs.g, bufs.beta, bufs.h0 = d["q"], d["k"], d["v"], d["g"], d["beta"], d["h0"]
+        bufs.out, bufs.hT = out, hT
+        e2e_steps = max(1, min(args.steps, 3))
+        nin = nout = 0
+        kda.chunk_fwd_host(host["q"], host["k"], host["v"], host["g"], host["beta"], cfg.scale, host["h0"],
+                           out=h_out, hT=h_hT, bufs=bufs, stream=stream)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            nin, nout = kda.chunk_fwd_host(host["q"], host["k"], host["v"], host["g"], host["beta"], cfg.scale,
+                                           host["h0"], out=h_out, hT=h_hT, bufs=bufs, stream=stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        ems = max_over_ranks(e0.elapsed_time(e1), world, dev)
+        e2e = {"value": tokens_per_step * world * e2e_steps / (ems / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": nin, "d2h_bytes_per_step": nout, "steps": e2e_steps,
+               "ms_per_step": ems / e2e_steps}
+        del host, h_out, h_hT
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(d, cfg, args.cpu_seconds)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": args.workload, "B": cfg.B, "H": cfg.H, "T": cfg.T, "dk": cfg.dk,
+                       "dv": cfg.dv, "chunk": CHUNK, "seed": cfg.seed,
+                       "operands": "bf16 q/k/v, fp32 g/beta/state; tcgen05 bf16 + tf32 MMA, fp32 accumulate",
+                       "l2": "inputs larger than L2 (51.7 GB per step); no flush",
+                       "parallelism": f"weak: one workload copy per GPU x{world}"},
+            "tflops": nflops / (ms_per_step / 1e3) / 1e12 * world,
+            "roofline": roof, "decode": dec, "e2e": e2e, "cpu_baseline": cpu,
+            "clocks": clk.summary(), "gpu_launches": args.steps,
+            "launch_ms": {"mean": statistics.mean(launch_ms), "min": min(launch_ms), "max": max(launch_ms)},
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=WORKLOAD)
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)  # at least three untimed warm-up steps
+    return run_reference(args) if args.impl == "reference" else run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

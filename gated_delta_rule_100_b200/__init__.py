@@ -1,0 +1,9 @@
+"""B200-native Kimi Delta Attention (KDA) forward: chunkwise prefill and
+single-step decode, as CUDA kernels for sm_100a behind the C ABI in
+``include/kda.h``.  This package holds the ctypes binding (``kda``), the
+in-tree build (``build``) and the seeded synthetic inputs (``inputs``)."""
+from .kda import (KdaError, chunk_fwd, chunk_fwd_host, decode_step, inject_timeout,  # noqa: F401
+                  load, set_wait_limit, status_string, stream_status)
+
+__all__ = ["chunk_fwd", "chunk_fwd_host", "decode_step", "stream_status", "status_string",
+           "set_wait_limit", "inject_timeout", "load", "KdaError"]

@@ -1,0 +1,142 @@
+// decode.cu -- one recurrent KDA step per (b, h), state updated in place.
+//
+// For each column j of the fp32 state S (dk x dv):
+//   s'  = alpha .* S[:, j]                 (decay first)
+//   p_j = k . s'                           (what the memory returns for k)
+//   u_j = beta (v_j - p_j)                 (erase along k, then write v)
+//   S[:, j] = s' + k u_j
+//   o_j = scale (q . s' + (q . k) u_j)     (read after the write)
+// which is the combined update of "Kimi Linear's Hybrid Linear Attention
+// Architecture: A Technical Breakdown", section 3.3, for one token.
+//
+// The step is HBM-bound: the state (4 dk dv bytes per head) is read and
+// written once.  One CTA owns one (b, h): 256 threads tile the state as
+// (row groups) x (dv / 4 float4 column groups), so every warp-wide load or
+// store covers one contiguous 512-byte state row.  The two column reductions
+// (k.s' and q.s') go through shared memory across row groups.
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "kda_device.cuh"
+
+namespace kda {
+
+constexpr int DEC_THREADS = 256;
+
+template <int DK, int DV>
+__global__ void __launch_bounds__(DEC_THREADS)
+decode_step_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ k,
+                   const uint16_t *__restrict__ v, const float *__restrict__ g,
+                   const float *__restrict__ beta, float scale, float *__restrict__ state,
+                   uint16_t *__restrict__ out) {
+    constexpr int NCG = DV / 4;              // float4 column groups
+    constexpr int NRG = DEC_THREADS / NCG;   // row groups
+    constexpr int RPT = DK / NRG;            // state rows per thread
+    static_assert(DK % NRG == 0 && NCG <= 32, "tile shape");
+
+    __shared__ float s_k[DK], s_q[DK], s_a[DK];
+    __shared__ float s_red[2][NRG][DV];
+    __shared__ float s_qk;
+
+    const int bh = blockIdx.x;
+    const int tid = threadIdx.x;
+    const int cg = tid % NCG;   // column group
+    const int rg = tid / NCG;   // row group
+
+    const uint16_t *qh = q + (size_t)bh * DK;
+    const uint16_t *kh = k + (size_t)bh * DK;
+    const float *gh = g + (size_t)bh * DK;
+    float *S = state + (size_t)bh * DK * DV;
+
+    // Issue the state loads first: they are the long-latency part.
+    float4 s[RPT];
+#pragma unroll
+    for (int i = 0; i < RPT; ++i) {
+        const int r = rg * RPT + i;
+        s[i] = __ldcs(reinterpret_cast<const float4 *>(S + (size_t)r * DV) + cg);
+    }
+    for (int r = tid; r < DK; r += DEC_THREADS) {
+        s_k[r] = bf16_bits_to_f32(kh[r]);
+        s_q[r] = bf16_bits_to_f32(qh[r]);
+        s_a[r] = __expf(gh[r]);
+    }
+    __syncthreads();
+    if (tid < 32) {
+        float acc = 0.f;
+        for (int r = tid; r < DK; r += 32) acc += s_q[r] * s_k[r];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        if (tid == 0) s_qk = acc;
+    }
+
+    float4 pk = make_float4(0.f, 0.f, 0.f, 0.f), pq = pk;
+#pragma unroll
+    for (int i = 0; i < RPT; ++i) {
+        const int r = rg * RPT + i;
+        const float a = s_a[r], kr = s_k[r], qr = s_q[r];
+        s[i].x *= a; s[i].y *= a; s[i].z *= a; s[i].w *= a;
+        pk.x += kr * s[i].x; pk.y += kr * s[i].y; pk.z += kr * s[i].z; pk.w += kr * s[i].w;
+        pq.x += qr * s[i].x; pq.y += qr * s[i].y; pq.z += qr * s[i].z; pq.w += qr * s[i].w;
+    }
+    reinterpret_cast<float4 *>(&s_red[0][rg][0])[cg] = pk;
+    reinterpret_cast<float4 *>(&s_red[1][rg][0])[cg] = pq;
+    __syncthreads();
+
+    // Column totals: every thread needs u for its own 4 columns.
+    float4 p = make_float4(0.f, 0.f, 0.f, 0.f), y = p;
+#pragma unroll
+    for (int j = 0; j < NRG; ++j) {
+        const float4 a = reinterpret_cast<const float4 *>(&s_red[0][j][0])[cg];
+        const float4 b = reinterpret_cast<const float4 *>(&s_red[1][j][0])[cg];
+        p.x += a.x; p.y += a.y; p.z += a.z; p.w += a.w;
+        y.x += b.x; y.y += b.y; y.z += b.z; y.w += b.w;
+    }
+    const float bt = beta[bh];
+    const uint16_t *vh = v + (size_t)bh * DV + cg * 4;
+    float4 u;
+    u.x = bt * (bf16_bits_to_f32(vh[0]) - p.x);
+    u.y = bt * (bf16_bits_to_f32(vh[1]) - p.y);
+    u.z = bt * (bf16_bits_to_f32(vh[2]) - p.z);
+    u.w = bt * (bf16_bits_to_f32(vh[3]) - p.w);
+
+#pragma unroll
+    for (int i = 0; i < RPT; ++i) {
+        const int r = rg * RPT + i;
+        const float kr = s_k[r];
+        float4 o = s[i];
+        o.x += kr * u.x; o.y += kr * u.y; o.z += kr * u.z; o.w += kr * u.w;
+        __stcs(reinterpret_cast<float4 *>(S + (size_t)r * DV) + cg, o);
+    }
+
+    if (rg == 0) {
+        const float qk = s_qk;
+        uint2 pk2;
+        pk2.x = pack_bf16x2(scale * (y.x + qk * u.x), scale * (y.y + qk * u.y));
+        pk2.y = pack_bf16x2(scale * (y.z + qk * u.z), scale * (y.w + qk * u.w));
+        *reinterpret_cast<uint2 *>(out + (size_t)bh * DV + cg * 4) = pk2;
+    }
+}
+
+template <int DK, int DV>
+static cudaError_t launch_decode_t(const void *q, const void *k, const void *v, const float *g,
+                                   const float *beta, float scale, float *state, void *out,
+                                   int BH, cudaStream_t stream) {
+    decode_step_kernel<DK, DV><<<BH, DEC_THREADS, 0, stream>>>(
+        (const uint16_t *)q, (const uint16_t *)k, (const uint16_t *)v, g, beta, scale, state,
+        (uint16_t *)out);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_decode(const void *q, const void *k, const void *v, const float *g,
+                          const float *beta, float scale, float *state, void *out, int BH, int dk,
+                          int dv, cudaStream_t stream) {
+    if (dk == 128 && dv == 128)
+        return launch_decode_t<128, 128>(q, k, v, g, beta, scale, state, out, BH, stream);
+    if (dk == 128 && dv == 64)
+        return launch_decode_t<128, 64>(q, k, v, g, beta, scale, state, out, BH, stream);
+    if (dk == 64 && dv == 128)
+        return launch_decode_t<64, 128>(q, k, v, g, beta, scale, state, out, BH, stream);
+    return launch_decode_t<64, 64>(q, k, v, g, beta, scale, state, out, BH, stream);
+}
+
+}  // namespace kda

@@ -1,0 +1,189 @@
+// kda_api.cu -- the extern "C" boundary of libkda: argument validation,
+// TMA descriptor encoding, kernel launch, and the per-device status word.
+// Declarations and the contract of every entry point are in include/kda.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+#include <stdint.h>
+
+#include <atomic>
+#include <mutex>
+
+#include "../../include/kda.h"
+#include "kda_device.cuh"
+
+namespace kda {
+cudaError_t launch_decode(const void *q, const void *k, const void *v, const float *g,
+                          const float *beta, float scale, float *state, void *out, int BH, int dk,
+                          int dv, cudaStream_t stream);
+}
+
+#include "chunk_params.cuh"
+
+namespace kda {
+cudaError_t launch_chunk(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                         const float *g, const ChunkParams &prm, int dk, cudaStream_t stream);
+int chunk_value_slice();
+}
+
+// Device-side status word: kernels OR error bits into it (one per device,
+// part of this module's image, so nothing is allocated for it).
+__device__ uint32_t g_kda_status_word;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+uint32_t *g_status_ptr[kMaxDevices] = {};
+std::atomic<unsigned long long> g_wait_polls{0};
+std::atomic<unsigned long long> g_inject_polls{0};
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+int current_status_word(uint32_t **out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return KDA_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (g_status_ptr[dev] == nullptr) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_kda_status_word) != cudaSuccess) return KDA_ERR_CUDA;
+        g_status_ptr[dev] = static_cast<uint32_t *>(p);
+    }
+    *out = g_status_ptr[dev];
+    return KDA_OK;
+}
+
+int get_encoder(PFN_cuTensorMapEncodeTiled_v12000 *fn) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (g_encode == nullptr) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || p == nullptr)
+            return KDA_ERR_CUDA;
+        g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    *fn = g_encode;
+    return KDA_OK;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+// 4-D map over a [B][T][H][inner] tensor; box {box_inner, 1, 64, 1}.
+int make_map(CUtensorMap *map, PFN_cuTensorMapEncodeTiled_v12000 enc, const void *ptr,
+             CUtensorMapDataType dt, int esize, int inner, int H, int T, int B, int box_inner,
+             CUtensorMapSwizzle swz) {
+    cuuint64_t dims[4] = {(cuuint64_t)inner, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+    cuuint64_t strides[3] = {(cuuint64_t)inner * esize, (cuuint64_t)H * inner * esize,
+                             (cuuint64_t)T * H * inner * esize};
+    cuuint32_t box[4] = {(cuuint32_t)box_inner, 1u, 64u, 1u};
+    cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+    CUresult r = enc(map, dt, 4, const_cast<void *>(ptr), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? KDA_OK : KDA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int kda_abi_version(void) { return 100; }
+
+const char *kda_status_string(int status) {
+    switch (status) {
+        case KDA_OK: return "KDA_OK";
+        case KDA_ERR_INVALID_ARG: return "KDA_ERR_INVALID_ARG";
+        case KDA_ERR_UNSUPPORTED: return "KDA_ERR_UNSUPPORTED";
+        case KDA_ERR_ALIGNMENT: return "KDA_ERR_ALIGNMENT";
+        case KDA_ERR_CUDA: return "KDA_ERR_CUDA";
+        case KDA_ERR_TIMEOUT: return "KDA_ERR_TIMEOUT";
+        default: return "KDA_ERR_UNKNOWN";
+    }
+}
+
+void kda_chunk_fwd_debug_wait_limit(unsigned long long polls) { g_wait_polls.store(polls); }
+
+void kda_chunk_fwd_debug_inject_timeout(unsigned long long polls) { g_inject_polls.store(polls); }
+
+int kda_stream_status(void *stream) {
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return KDA_ERR_CUDA;
+    uint32_t *word = nullptr;
+    if (current_status_word(&word) != KDA_OK) return KDA_ERR_CUDA;
+    uint32_t v = 0;
+    if (cudaMemcpy(&v, word, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return KDA_ERR_CUDA;
+    if (v != 0) {
+        const uint32_t zero = 0;
+        if (cudaMemcpy(word, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return KDA_ERR_CUDA;
+    }
+    return (v & kda::DEV_TIMEOUT) ? KDA_ERR_TIMEOUT : KDA_OK;
+}
+
+int kda_chunk_fwd(const void *q, const void *k, const void *v, const float *g, const float *beta,
+                  float scale, const float *h0, void *out, float *hT, int B, int T, int H, int dk,
+                  int dv, void *stream) {
+    if (B < 1 || H < 1 || T < 0) return KDA_ERR_INVALID_ARG;
+    if (T > 0 && (!q || !k || !v || !g || !beta || !out)) return KDA_ERR_INVALID_ARG;
+    if ((dk != 64 && dk != 128) || (dv != 64 && dv != 128)) return KDA_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(g) || !aligned4(beta) ||
+        !aligned16(out) || !aligned16(h0) || !aligned16(hT))
+        return KDA_ERR_ALIGNMENT;
+    if ((long long)B * H * 4 > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+    if (T == 0) {  // nothing to scan: hT = h0 (or zero)
+        if (hT == nullptr) return KDA_OK;
+        const size_t bytes = (size_t)B * H * dk * dv * sizeof(float);
+        cudaError_t e = h0 ? (h0 == hT ? cudaSuccess : cudaMemcpyAsync(hT, h0, bytes, cudaMemcpyDeviceToDevice, s))
+                           : cudaMemsetAsync(hT, 0, bytes, s);
+        return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+    }
+
+    uint32_t *word = nullptr;
+    if (current_status_word(&word) != KDA_OK) return KDA_ERR_CUDA;
+    PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
+    if (get_encoder(&enc) != KDA_OK) return KDA_ERR_CUDA;
+
+    // Each CTA carries a 32-column slice of the value dimension.
+    const int vs = kda::chunk_value_slice();
+
+    CUtensorMap tq, tk, tv;
+    if (make_map(&tq, enc, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dk, H, T, B, 64,
+                 CU_TENSOR_MAP_SWIZZLE_128B) != KDA_OK ||
+        make_map(&tk, enc, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dk, H, T, B, 64,
+                 CU_TENSOR_MAP_SWIZZLE_128B) != KDA_OK ||
+        make_map(&tv, enc, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dv, H, T, B, vs,
+                 CU_TENSOR_MAP_SWIZZLE_NONE) != KDA_OK)
+        return KDA_ERR_CUDA;
+
+    kda::ChunkParams prm;
+    prm.beta = beta;
+    prm.h0 = h0;
+    prm.out = static_cast<uint16_t *>(out);
+    prm.hT = hT;
+    prm.scale = scale;
+    prm.B = B; prm.T = T; prm.H = H; prm.DV = dv;
+    prm.nslices = dv / vs;
+    prm.st.word = word;
+    const unsigned long long polls = g_wait_polls.load();
+    prm.st.wait_polls = polls ? polls : ~0ull;
+    prm.inject_wait_polls = g_inject_polls.load();
+    cudaError_t e = kda::launch_chunk(tq, tk, tv, g, prm, dk, s);
+    return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+int kda_decode_step(const void *q, const void *k, const void *v, const float *g, const float *beta,
+                    float scale, float *state, void *out, int B, int H, int dk, int dv, void *stream) {
+    if (!q || !k || !v || !g || !beta || !state || !out) return KDA_ERR_INVALID_ARG;
+    if (B < 1 || H < 1) return KDA_ERR_INVALID_ARG;
+    if ((dk != 64 && dk != 128) || (dv != 64 && dv != 128)) return KDA_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(g) || !aligned4(beta) ||
+        !aligned16(state) || !aligned16(out))
+        return KDA_ERR_ALIGNMENT;
+    if ((long long)B * H > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
+    cudaError_t e = kda::launch_decode(q, k, v, g, beta, scale, state, out, B * H, dk, dv,
+                                       static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+}  // extern "C"

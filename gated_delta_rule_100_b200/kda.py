@@ -1,0 +1,187 @@
+"""Python binding of libkda (ctypes).  Argument marshalling only: every step of
+the computation runs in the library's CUDA kernels.
+
+The entry points mirror ``include/kda.h``:
+
+* ``chunk_fwd``   -> ``kda_chunk_fwd``   (chunkwise prefill)
+* ``decode_step`` -> ``kda_decode_step`` (one recurrent step, state in place)
+* ``stream_status`` -> ``kda_stream_status``
+
+plus ``chunk_fwd_host``, the same prefill for host (pinned) tensors: it copies
+the inputs to the device, runs ``kda_chunk_fwd`` and copies the results back,
+all on one stream.
+
+If ``libkda.so`` is missing the calls raise; there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libkda.so")
+
+KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_ALIGNMENT, KDA_ERR_CUDA, KDA_ERR_TIMEOUT = range(6)
+EXPORTED = ("kda_chunk_fwd", "kda_decode_step", "kda_status_string", "kda_stream_status",
+            "kda_chunk_fwd_debug_wait_limit", "kda_chunk_fwd_debug_inject_timeout", "kda_abi_version")
+
+_lib = None
+
+
+class KdaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} ({status})")
+
+
+def load():
+    """Load libkda.so (built in-tree by ``gated_delta_rule_100_b200.build``)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                           "`python -m gated_delta_rule_100_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, fp, i, f = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    lib.kda_chunk_fwd.argtypes = [vp, vp, vp, fp, fp, f, fp, vp, fp, i, i, i, i, i, vp]
+    lib.kda_chunk_fwd.restype = i
+    lib.kda_decode_step.argtypes = [vp, vp, vp, fp, fp, f, fp, vp, i, i, i, i, vp]
+    lib.kda_decode_step.restype = i
+    lib.kda_status_string.argtypes = [i]
+    lib.kda_status_string.restype = ctypes.c_char_p
+    lib.kda_stream_status.argtypes = [vp]
+    lib.kda_stream_status.restype = i
+    lib.kda_chunk_fwd_debug_wait_limit.argtypes = [ctypes.c_ulonglong]
+    lib.kda_chunk_fwd_debug_wait_limit.restype = None
+    lib.kda_chunk_fwd_debug_inject_timeout.argtypes = [ctypes.c_ulonglong]
+    lib.kda_chunk_fwd_debug_inject_timeout.restype = None
+    lib.kda_abi_version.restype = i
+    _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    return load().kda_status_string(int(status)).decode()
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(t, name, dtype, shape):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def chunk_fwd(q, k, v, g, beta, scale, h0=None, *, out=None, hT=None, final_state=True, stream=None):
+    """Chunkwise prefill.  q, k [B,T,H,dk] bf16; v [B,T,H,dv] bf16; g [B,T,H,dk] fp32;
+    beta [B,T,H] fp32; h0 [B,H,dk,dv] fp32 or None.  Returns (out, hT); hT is None
+    when ``final_state`` is False and no ``hT`` buffer was given."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    _check(q, "q", torch.bfloat16, (B, T, H, dk))
+    _check(k, "k", torch.bfloat16, (B, T, H, dk))
+    _check(v, "v", torch.bfloat16, (B, T, H, dv))
+    _check(g, "g", torch.float32, (B, T, H, dk))
+    _check(beta, "beta", torch.float32, (B, T, H))
+    if h0 is not None:
+        _check(h0, "h0", torch.float32, (B, H, dk, dv))
+    if out is None:
+        out = torch.empty((B, T, H, dv), device=q.device, dtype=torch.bfloat16)
+    _check(out, "out", torch.bfloat16, (B, T, H, dv))
+    if hT is None and final_state:
+        hT = torch.empty((B, H, dk, dv), device=q.device, dtype=torch.float32)
+    if hT is not None:
+        _check(hT, "hT", torch.float32, (B, H, dk, dv))
+    rc = load().kda_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale),
+                              _ptr(h0), _ptr(out), _ptr(hT), B, T, H, dk, dv, _stream(stream))
+    if rc != KDA_OK:
+        raise KdaError(rc, "kda_chunk_fwd")
+    return out, hT
+
+
+def decode_step(q, k, v, g, beta, scale, state, *, out=None, stream=None):
+    """One recurrent step.  q, k [B,H,dk] bf16; v [B,H,dv] bf16; g [B,H,dk] fp32;
+    beta [B,H] fp32; state [B,H,dk,dv] fp32 (updated in place).  Returns out [B,H,dv] bf16."""
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    _check(q, "q", torch.bfloat16, (B, H, dk))
+    _check(k, "k", torch.bfloat16, (B, H, dk))
+    _check(v, "v", torch.bfloat16, (B, H, dv))
+    _check(g, "g", torch.float32, (B, H, dk))
+    _check(beta, "beta", torch.float32, (B, H))
+    _check(state, "state", torch.float32, (B, H, dk, dv))
+    if out is None:
+        out = torch.empty((B, H, dv), device=q.device, dtype=torch.bfloat16)
+    _check(out, "out", torch.bfloat16, (B, H, dv))
+    rc = load().kda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale),
+                                _ptr(state), _ptr(out), B, H, dk, dv, _stream(stream))
+    if rc != KDA_OK:
+        raise KdaError(rc, "kda_decode_step")
+    return out
+
+
+def stream_status(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device status word."""
+    return int(load().kda_stream_status(_stream(stream)))
+
+
+def set_wait_limit(polls: int) -> None:
+    """Test hook: polls a device-side wait makes before giving up (0 = default)."""
+    load().kda_chunk_fwd_debug_wait_limit(int(polls))
+
+
+def inject_timeout(polls: int) -> None:
+    """Test hook: nonzero makes each prefill CTA first wait on a barrier nothing
+    signals (at most ``polls`` polls) and take its timeout path; 0 = off."""
+    load().kda_chunk_fwd_debug_inject_timeout(int(polls))
+
+
+class DeviceBuffers:
+    """Device copies of one prefill problem, allocated once and reused."""
+
+    def __init__(self, B, T, H, dk, dv, device, with_h0):
+        z = dict(device=device)
+        self.q = torch.empty((B, T, H, dk), dtype=torch.bfloat16, **z)
+        self.k = torch.empty((B, T, H, dk), dtype=torch.bfloat16, **z)
+        self.v = torch.empty((B, T, H, dv), dtype=torch.bfloat16, **z)
+        self.g = torch.empty((B, T, H, dk), dtype=torch.float32, **z)
+        self.beta = torch.empty((B, T, H), dtype=torch.float32, **z)
+        self.h0 = torch.empty((B, H, dk, dv), dtype=torch.float32, **z) if with_h0 else None
+        self.out = torch.empty((B, T, H, dv), dtype=torch.bfloat16, **z)
+        self.hT = torch.empty((B, H, dk, dv), dtype=torch.float32, **z)
+
+
+def chunk_fwd_host(q, k, v, g, beta, scale, h0=None, *, out, hT, bufs: DeviceBuffers, stream=None):
+    """Prefill from host tensors (pinned for asynchronous copies): H2D of the inputs,
+    ``kda_chunk_fwd`` on the device copies, D2H of out and hT, all enqueued on
+    ``stream``.  Returns the (bytes_h2d, bytes_d2h) it moved."""
+    st = torch.cuda.current_stream() if stream is None else stream
+    with torch.cuda.stream(st):
+        nin = 0
+        for src, dst in ((q, bufs.q), (k, bufs.k), (v, bufs.v), (g, bufs.g), (beta, bufs.beta),
+                         (h0, bufs.h0)):
+            if src is not None:
+                dst.copy_(src, non_blocking=True)
+                nin += src.numel() * src.element_size()
+        chunk_fwd(bufs.q, bufs.k, bufs.v, bufs.g, bufs.beta, scale,
+                  bufs.h0 if h0 is not None else None, out=bufs.out, hT=bufs.hT, stream=st)
+        out.copy_(bufs.out, non_blocking=True)
+        hT.copy_(bufs.hT, non_blocking=True)
+    nout = out.numel() * out.element_size() + hT.numel() * hT.element_size()
+    return nin, nout

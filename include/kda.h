@@ -1,0 +1,148 @@
+/*
+ * kda.h -- C ABI of libkda, the B200 (sm_100a) Kimi Delta Attention forward.
+ *
+ * KDA is a per-head recurrence over a matrix state S in R^{dk x dv}:
+ *
+ *   S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T
+ *   o_t = scale * S_t^T q_t,              alpha_t = exp(g_t) per key channel
+ *
+ * The update is the "combined form" of section 3.3 of "Kimi Linear's Hybrid
+ * Linear Attention Architecture: A Technical Breakdown" (decay first, then the
+ * erase along k_t and the write), with the state oriented dk x dv as in the
+ * update printed in "Kimi Linear: How Moonshot AI Built a Hybrid Attention
+ * Architecture That Beats Full Attention" (beta_t k_t v_t^T).  The query reads
+ * the state after its own token's write ("Kimi Linear" explainer,
+ * math.kryvik.com, "Step 4: Query").  Prefill evaluates the recurrence in the
+ * chunkwise form of section 4 of the Baidu breakdown (state passing across
+ * chunks, causal intra-chunk output); decode is one step of the recurrence.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - All pointers are DEVICE pointers (cudaMalloc / torch CUDA tensors) on the
+ *   current device, row-major and contiguous, 16-byte aligned (beta: 4-byte).
+ * - bf16 tensors are passed as void* holding IEEE bfloat16 (uint16 bits).
+ * - The caller owns every buffer.  The library keeps no pointer after a call
+ *   returns and allocates no device memory for the data path.  The only
+ *   library-owned device memory is one 4-byte status word per device,
+ *   created on first use.
+ * - Work is enqueued on `stream` (a cudaStream_t, NULL = legacy default
+ *   stream) and the call returns without synchronising.  The return value
+ *   reports argument validation and launch errors only.  Device-side
+ *   conditions (a bounded wait that gave up) are reported by
+ *   kda_stream_status().
+ * - Supported sizes: dk, dv in {64, 128}; B, H >= 1; T >= 0.  Anything else
+ *   returns KDA_ERR_UNSUPPORTED (or KDA_ERR_INVALID_ARG for negative sizes
+ *   and NULL required pointers) without enqueueing work.
+ * - Value domain: g <= 0 and finite, beta in [0, 1].  Keys are used as given
+ *   (the caller L2-normalises them if the model does).  Results are exact up
+ *   to rounding when, for every key channel, the log-decay summed over any
+ *   16-token block aligned to a multiple of 16 within the sequence is >= -160;
+ *   beyond that the kernel stays finite but the within-block decay factors of
+ *   that channel are clamped.
+ */
+#ifndef KDA_H_
+#define KDA_H_
+
+#if defined(__GNUC__)
+#define KDA_API __attribute__((visibility("default")))
+#else
+#define KDA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    KDA_OK = 0,
+    KDA_ERR_INVALID_ARG = 1, /* NULL required pointer, negative size           */
+    KDA_ERR_UNSUPPORTED = 2, /* dk/dv outside {64,128}, other unsupported shape */
+    KDA_ERR_ALIGNMENT = 3,   /* a pointer below its required alignment        */
+    KDA_ERR_CUDA = 4,        /* a CUDA runtime/driver call or launch failed    */
+    KDA_ERR_TIMEOUT = 5      /* a device-side bounded wait gave up             */
+} kda_status;
+
+/*
+ * kda_chunk_fwd -- chunkwise prefill over whole sequences.
+ *
+ *   q, k  : bf16 [B, T, H, dk]
+ *   v     : bf16 [B, T, H, dv]
+ *   g     : fp32 [B, T, H, dk]   log-decay, g = log(alpha) <= 0
+ *   beta  : fp32 [B, T, H]       write/erase strength in [0, 1]
+ *   scale : readout scale (commonly dk^-0.5)
+ *   h0    : fp32 [B, H, dk, dv]  initial state, or NULL for a zero state
+ *   out   : bf16 [B, T, H, dv]   o_t for every token (written)
+ *   hT    : fp32 [B, H, dk, dv]  final state, or NULL to skip; may alias h0
+ *           (h0 is read in full before hT is written, per (b, h))
+ *   stream: cudaStream_t
+ *
+ * Internally each sequence is cut into chunks of 64 tokens; the last chunk of
+ * a sequence may be partial.  The state is carried in fp32 from chunk to
+ * chunk; the chunk contractions run on the tcgen05 tensor cores with fp32
+ * accumulation.  T == 0 copies h0 to hT (or zeroes hT) and writes no output;
+ * q, k, v, g, beta and out are then not read and may be NULL.
+ */
+KDA_API int kda_chunk_fwd(const void *q, const void *k, const void *v,
+                  const float *g, const float *beta, float scale,
+                  const float *h0, void *out, float *hT,
+                  int B, int T, int H, int dk, int dv, void *stream);
+
+/*
+ * kda_decode_step -- one recurrent step for every (b, h), state updated in place.
+ *
+ *   q, k  : bf16 [B, H, dk]
+ *   v     : bf16 [B, H, dv]
+ *   g     : fp32 [B, H, dk]
+ *   beta  : fp32 [B, H]
+ *   scale : readout scale
+ *   state : fp32 [B, H, dk, dv]  S_{t-1} on entry, S_t on return
+ *   out   : bf16 [B, H, dv]      o_t
+ *   stream: cudaStream_t
+ *
+ * The state layout is the one kda_chunk_fwd uses for h0/hT, so a decode can
+ * continue a prefill directly.  This is the recurrence itself, evaluated in
+ * fp32: decay each key row of S, project on k, erase-and-write, read with q.
+ */
+KDA_API int kda_decode_step(const void *q, const void *k, const void *v,
+                    const float *g, const float *beta, float scale,
+                    float *state, void *out,
+                    int B, int H, int dk, int dv, void *stream);
+
+/* Human-readable name of a kda_status value (static string, never NULL). */
+KDA_API const char *kda_status_string(int status);
+
+/*
+ * kda_stream_status -- synchronise `stream`, then read and clear the current
+ * device's status word.  Returns KDA_OK, KDA_ERR_TIMEOUT when a kernel's
+ * bounded wait gave up since the last call (that kernel's outputs are then
+ * unspecified), or KDA_ERR_CUDA when the synchronisation itself failed.
+ */
+KDA_API int kda_stream_status(void *stream);
+
+/*
+ * kda_chunk_fwd_debug_wait_limit -- test hook.  Sets the number of polls a
+ * device-side wait makes before it gives up (0 restores the default, about
+ * one second of polling).  A tiny limit lets a test exercise the timeout path
+ * on a healthy GPU: the kernel records KDA_ERR_TIMEOUT, releases what it
+ * holds and returns.  Applies to launches made after the call, process-wide.
+ */
+KDA_API void kda_chunk_fwd_debug_wait_limit(unsigned long long polls);
+
+/*
+ * kda_chunk_fwd_debug_inject_timeout -- test hook for the failure path.  When
+ * `polls` is nonzero, every prefill CTA launched afterwards first waits (at
+ * most `polls` polls, at most about one second) on a barrier that nothing
+ * signals, gives up, records KDA_ERR_TIMEOUT, waits for its own copies in
+ * flight, frees its tensor memory and returns without writing results.  The
+ * GPU context stays usable.  0 turns the hook off.  Process-wide.
+ */
+KDA_API void kda_chunk_fwd_debug_inject_timeout(unsigned long long polls);
+
+/* Version of this ABI (major * 100 + minor). */
+KDA_API int kda_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_H_ */

@@ -1,0 +1,99 @@
+"""The C ABI loads on a CPU-only host, exports what include/kda.h declares, and
+rejects bad arguments before touching a GPU (no compute calls here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from gated_delta_rule_100_b200 import build as kbuild
+from gated_delta_rule_100_b200 import kda
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "kda.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    kbuild.build()
+    return kda.load()
+
+
+def declared_symbols():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"KDA_API\s+[\w\s\*]*?\b(kda_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_symbols()
+    assert "kda_chunk_fwd" in names and "kda_decode_step" in names
+    assert set(names) == set(kda.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+    assert lib.kda_abi_version() == 100
+
+
+def test_status_strings(lib):
+    for code, name in enumerate(["KDA_OK", "KDA_ERR_INVALID_ARG", "KDA_ERR_UNSUPPORTED",
+                                 "KDA_ERR_ALIGNMENT", "KDA_ERR_CUDA", "KDA_ERR_TIMEOUT"]):
+        assert kda.status_string(code) == name
+    assert kda.status_string(99) == "KDA_ERR_UNKNOWN"
+
+
+A = ctypes.c_void_p(0x10000)     # stand-in device addresses: only validated, never dereferenced
+MIS = ctypes.c_void_p(0x10008)   # 8-byte aligned, not 16
+ODD = ctypes.c_void_p(0x10002)   # 2-byte aligned
+
+
+def chunk(lib, q=A, k=A, v=A, g=A, beta=A, h0=None, out=A, hT=None, B=1, T=64, H=1, dk=64, dv=64):
+    return lib.kda_chunk_fwd(q, k, v, g, beta, 1.0, h0, out, hT, B, T, H, dk, dv, None)
+
+
+def decode(lib, q=A, k=A, v=A, g=A, beta=A, state=A, out=A, B=1, H=1, dk=64, dv=64):
+    return lib.kda_decode_step(q, k, v, g, beta, 1.0, state, out, B, H, dk, dv, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), kda.KDA_ERR_INVALID_ARG),
+    (dict(beta=None), kda.KDA_ERR_INVALID_ARG),
+    (dict(out=None), kda.KDA_ERR_INVALID_ARG),
+    (dict(B=0), kda.KDA_ERR_INVALID_ARG),
+    (dict(H=0), kda.KDA_ERR_INVALID_ARG),
+    (dict(B=0, T=0), kda.KDA_ERR_INVALID_ARG),
+    (dict(T=-1), kda.KDA_ERR_INVALID_ARG),
+    (dict(dk=96), kda.KDA_ERR_UNSUPPORTED),
+    (dict(dv=256), kda.KDA_ERR_UNSUPPORTED),
+    (dict(k=MIS), kda.KDA_ERR_ALIGNMENT),
+    (dict(beta=ODD), kda.KDA_ERR_ALIGNMENT),
+    (dict(h0=MIS), kda.KDA_ERR_ALIGNMENT),
+    (dict(hT=MIS), kda.KDA_ERR_ALIGNMENT),
+])
+def test_chunk_fwd_rejects(lib, kw, code):
+    assert chunk(lib, **kw) == code
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(state=None), kda.KDA_ERR_INVALID_ARG),
+    (dict(out=None), kda.KDA_ERR_INVALID_ARG),
+    (dict(B=0), kda.KDA_ERR_INVALID_ARG),
+    (dict(dk=32), kda.KDA_ERR_UNSUPPORTED),
+    (dict(v=MIS), kda.KDA_ERR_ALIGNMENT),
+    (dict(beta=ODD), kda.KDA_ERR_ALIGNMENT),
+])
+def test_decode_step_rejects(lib, kw, code):
+    assert decode(lib, **kw) == code
+
+
+def test_zero_length_accepts_null_inputs(lib):
+    # T == 0 with no h0/hT: nothing to read or write, so nothing is enqueued
+    assert chunk(lib, q=None, k=None, v=None, g=None, beta=None, out=None, T=0) == kda.KDA_OK
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(kda, "_lib", None)
+    monkeypatch.setattr(kda, "LIB_PATH", str(tmp_path / "libkda.so"))
+    with pytest.raises(RuntimeError, match="missing"):
+        kda.load()

@@ -1,0 +1,184 @@
+"""kda_chunk_fwd (CUDA, through the C ABI) against the fp64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+from gated_delta_rule_100_b200 import inputs, kda
+from kda_testlib import assert_close, f64, oracle_prefill
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+
+@pytest.fixture(autouse=True)
+def _reset_hooks():
+    kda.inject_timeout(0)
+    kda.set_wait_limit(0)
+    yield
+    kda.inject_timeout(0)
+    kda.set_wait_limit(0)
+    assert kda.stream_status() == kda.KDA_OK
+
+
+def run(d, scale, **kw):
+    out, hT = kda.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], scale, d["h0"], **kw)
+    torch.cuda.synchronize()
+    return out, hT
+
+
+def check(d, scale, what, **kw):
+    out, hT = run(d, scale, **kw)
+    o_ref, s_ref = oracle_prefill(d, scale)
+    assert_close(f64(out), o_ref, f"{what} out")
+    assert_close(f64(hT), s_ref, f"{what} hT")
+    return out, hT
+
+
+@pytest.mark.parametrize("name", ["oracle_scale_B1_H1_T256_d64", "prefill_B1_H4_T2048_d128"])
+def test_config_full(name):
+    cfg = inputs.CONFIGS[name]
+    d = inputs.make_config(cfg, device=DEV)
+    check(d, cfg.scale, name)
+
+
+@pytest.mark.parametrize("T", [1, 15, 63, 64, 65, 129, 1000])
+def test_ragged_lengths(T):
+    d = inputs.make_prefill(2, T, 3, 128, 128, decay=0.05, h0_std=0.02, seed=100 + T, device=DEV)
+    check(d, 128 ** -0.5, f"T={T}")
+
+
+@pytest.mark.parametrize("dk,dv", [(64, 64), (64, 128), (128, 64), (128, 128)])
+def test_head_dims(dk, dv):
+    d = inputs.make_prefill(1, 300, 2, dk, dv, decay=0.1, h0_std=0.02, seed=7, device=DEV)
+    check(d, dk ** -0.5, f"dk={dk} dv={dv}")
+
+
+def test_value_slices_are_independent():
+    """Each CTA carries 32 value columns; the columns of the state evolve
+    independently, so the first 64 columns of a dv = 128 run must equal, bit
+    for bit, a dv = 64 run on those columns alone."""
+    d = inputs.make_prefill(2, 200, 2, 128, 128, decay=0.05, h0_std=0.02, seed=8, device=DEV)
+    out, hT = check(d, 0.1, "dv=128")
+    half = dict(d)
+    half["v"] = d["v"][..., :64].contiguous()
+    half["h0"] = d["h0"][..., :64].contiguous()
+    out2, hT2 = run(half, 0.1)
+    assert torch.equal(out2, out[..., :64])
+    assert torch.equal(hT2, hT[..., :64])
+
+
+def test_null_h0_and_null_hT():
+    d = inputs.make_prefill(1, 130, 2, 128, 128, decay=0.05, h0_std=0.0, seed=9, device=DEV)
+    out, hT = run(d, 0.2, final_state=False)
+    assert hT is None
+    o_ref, _ = oracle_prefill(d, 0.2)
+    assert_close(f64(out), o_ref, "hT=NULL out")
+
+
+def test_h0_aliases_hT():
+    d = inputs.make_prefill(2, 150, 2, 128, 128, decay=0.05, h0_std=0.02, seed=10, device=DEV)
+    o_ref, s_ref = oracle_prefill(d, 0.3)
+    state = d["h0"].clone()
+    out, hT = kda.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], 0.3, state, hT=state)
+    torch.cuda.synchronize()
+    assert hT.data_ptr() == state.data_ptr()
+    assert_close(f64(out), o_ref, "aliased out")
+    assert_close(f64(state), s_ref, "aliased state")
+
+
+def test_zero_length():
+    d = inputs.make_prefill(1, 0, 2, 64, 64, decay=0.05, h0_std=0.02, seed=11, device=DEV)
+    out, hT = run(d, 0.3)
+    assert out.shape[1] == 0
+    assert torch.equal(hT, d["h0"])
+
+
+def test_beta_zero_closed_form():
+    """beta = 0: the state only decays, S_t = Diag(e^{Gamma_t}) h0."""
+    d = inputs.make_prefill(1, 333, 2, 128, 128, decay=0.1, h0_std=0.5, seed=12, device=DEV)
+    d["beta"].zero_()
+    out, hT = run(d, 0.25)
+    g = f64(d["g"])
+    Gam = np.cumsum(g, axis=1)
+    h0 = f64(d["h0"])
+    want = 0.25 * np.einsum("bthc,bhcd->bthd", np.exp(Gam) * f64(d["q"]), h0)
+    assert_close(f64(out), want, "beta=0 out")
+    assert_close(f64(hT), np.exp(Gam[:, -1])[..., None] * h0, "beta=0 hT")
+
+
+def test_beta_one_write_then_read():
+    """beta = 1 and q = k: reading right after the write returns |k|^2-weighted v
+    (S_t^T k_t = (1-|k|^2)(D S)^T k + |k|^2 v); checked against the oracle."""
+    d = inputs.make_prefill(1, 200, 2, 128, 128, decay=0.05, h0_std=0.02, seed=13, device=DEV)
+    d["beta"].fill_(1.0)
+    d["q"] = d["k"].clone()
+    check(d, 1.0, "beta=1 q=k")
+
+
+@pytest.mark.parametrize("decay", [0.0, 5.0])
+def test_decay_extremes(decay):
+    """g = 0 (no decay) and g = -5 softplus(N(0,1)) (fast forgetting)."""
+    d = inputs.make_prefill(1, 500, 2, 128, 128, decay=decay, h0_std=0.02, seed=14, device=DEV)
+    check(d, 128 ** -0.5, f"decay={decay}")
+
+
+def test_continuation():
+    """chunk_fwd(T1) then chunk_fwd(T2) from its hT equals the oracle over T1 + T2
+    (the split is not on a chunk boundary)."""
+    d = inputs.make_prefill(1, 400, 2, 128, 128, decay=0.05, h0_std=0.02, seed=15, device=DEV)
+    cut = 136
+    a = {k: (v[:, :cut].contiguous() if k != "h0" else v) for k, v in d.items()}
+    o1, s1 = run(a, 0.2)
+    b = {k: (v[:, cut:].contiguous() if k != "h0" else s1) for k, v in d.items()}
+    o2, s2 = run(b, 0.2)
+    o_ref, s_ref = oracle_prefill(d, 0.2)
+    assert_close(f64(torch.cat([o1, o2], dim=1)), o_ref, "continuation out")
+    assert_close(f64(s2), s_ref, "continuation hT")
+
+
+def test_value_column_permutation():
+    d = inputs.make_prefill(1, 180, 2, 128, 128, decay=0.05, h0_std=0.02, seed=16, device=DEV)
+    out, hT = run(d, 0.2)
+    perm = torch.randperm(128, generator=torch.Generator().manual_seed(0)).to(DEV)
+    dp = dict(d)
+    dp["v"] = d["v"][..., perm].contiguous()
+    dp["h0"] = d["h0"][..., perm].contiguous()
+    out_p, hT_p = run(dp, 0.2)
+    o_ref, s_ref = oracle_prefill(dp, 0.2)
+    assert_close(f64(out_p), o_ref, "permuted out")
+    assert_close(f64(hT_p), s_ref, "permuted hT")
+    assert_close(f64(out_p), f64(out[..., perm]), "permuted vs unpermuted out")
+
+
+def test_timeout_path_reports_and_recovers():
+    """The fault-injection hook makes every CTA wait on a barrier nothing signals:
+    the bounded wait must give up, the kernel must record KDA_ERR_TIMEOUT,
+    release what it holds and return; the next call must be correct."""
+    d = inputs.make_prefill(1, 256, 2, 128, 128, decay=0.05, h0_std=0.02, seed=17, device=DEV)
+    kda.inject_timeout(1000)
+    run(d, 0.2)
+    assert kda.stream_status() == kda.KDA_ERR_TIMEOUT
+    kda.inject_timeout(0)
+    check(d, 0.2, "after timeout")
+
+
+def test_training_shape_full():
+    cfg = inputs.CONFIGS["training_B8_H32_T4096_d128"]
+    d = inputs.make_config(cfg, device=DEV)
+    out, hT = run(d, cfg.scale)
+    o_ref, s_ref = oracle_prefill(d, cfg.scale)
+    assert_close(f64(out), o_ref, "training out")
+    assert_close(f64(hT), s_ref, "training hT")
+
+
+def test_long_context_sampled():
+    """Full 1M-token launch; the oracle checks heads 0-1 over the first 65,536
+    tokens and head 0's final state over all tokens."""
+    cfg = inputs.CONFIGS["long_context_B1_H32_T1M_d128"]
+    d = inputs.make_config(cfg, device=DEV)
+    out, hT = run(d, cfg.scale)
+    o_ref, _ = oracle_prefill(d, cfg.scale, heads=slice(0, 2), tokens=65536)
+    assert_close(f64(out[:, :65536, 0:2]), o_ref, "long-context out (heads 0-1, 64k tokens)")
+    _, s_ref = oracle_prefill(d, cfg.scale, heads=slice(0, 1))
+    assert_close(f64(hT[:, 0:1]), s_ref, "long-context hT (head 0)")
