@@ -174,6 +174,11 @@ def barrier(world):
         dist.barrier()
 
 
+def weak_value(units_per_step, world, steps, total_ms):
+    """Whole-job throughput: every rank processes its own units each step."""
+    return units_per_step * world * steps / (total_ms / 1e3)
+
+
 def max_over_ranks(x, world, device):
     if world == 1:
         return x
@@ -297,7 +302,7 @@ def run_ours(args):
     total_ms = max_over_ranks(total_ms, world, dev)
     ms_per_step = total_ms / args.steps
     tokens_per_step = cfg.B * cfg.T
-    value = tokens_per_step * world * args.steps / (total_ms / 1e3)
+    value = weak_value(tokens_per_step, world, args.steps, total_ms)
 
     nbytes = prefill_bytes(cfg.B, cfg.T, cfg.H, cfg.dk, cfg.dv, cfg.h0_std > 0, True)
     nflops = prefill_flops(cfg.B, cfg.T, cfg.H, cfg.dk, cfg.dv)
