@@ -25,10 +25,11 @@
 // >= -160.  All factors come from running products of alpha = e^g (one exp
 // per input element) plus one reciprocal per factor above 1.
 //
-// One CTA (256 threads; threads c and c + 128 share key channel c) owns one
-// (b, h, 32-column value slice) and walks its chunks in order:
-//   E  alpha, running products; bf16 / tf32 operand tiles, written
-//      channel-major with 16-byte stores                       (CUDA cores)
+// One CTA (512 threads; thread (c, I) = key channel c, 16-token block I)
+// owns one (b, h, 32-column value slice) and walks its chunks in order:
+//   E  alpha, running products as a two-level scan (within the 16-token block,
+//      then across the four block totals); bf16 / tf32 operand tiles,
+//      written channel-major with 16-byte stores               (CUDA cores)
 //   F  X * Y^(I) for the four row blocks -> A, P                (UMMA bf16)
 //   AP A -> fp32 scratch, P -> tf32 tile                        (TMEM -> smem)
 //   T  (I + A)^{-1}: 16x16 diagonal blocks by substitution, off-diagonal
@@ -54,8 +55,8 @@ constexpr int CH = 64;          // chunk length
 constexpr int SUB = 16;         // sub-block of the decay references
 constexpr int NSUB = CH / SUB;  // 4
 constexpr int VSL = 32;         // value columns per CTA
-constexpr int CHUNK_THREADS = 256;  // two threads per key channel
-constexpr int VSH = VSL / 2;        // value columns per thread in the state update
+constexpr int CHUNK_THREADS = 512;  // four threads per key channel
+constexpr int VSQ = VSL / 4;        // value columns per thread in the state update
 constexpr int A_LD = 68;        // fp32 row stride of the A / T scratch
 constexpr float EXP_CLAMP_HI = 5.5406223843935098e34f;  // e^80
 constexpr float EXP_CLAMP_LO = 1.8048513878454153e-35f; // e^-80
@@ -120,8 +121,13 @@ __device__ __forceinline__ uint4 pack8_bf16(const float (&v)[8]) {
                       pack_bf16x2(v[6], v[7]));
 }
 
+// tf32 operands are stored as fp32 bit patterns: the tensor core reads the
+// sign, exponent and top 10 mantissa bits (the conversion instruction runs at
+// a sixteenth of the FMA rate, so it is skipped).
+__device__ __forceinline__ uint32_t tf32_bits(float x) { return __float_as_uint(x); }
+
 __device__ __forceinline__ uint4 pack4_tf32(float a, float b, float c, float d) {
-    return make_uint4(to_tf32(a), to_tf32(b), to_tf32(c), to_tf32(d));
+    return make_uint4(tf32_bits(a), tf32_bits(b), tf32_bits(c), tf32_bits(d));
 }
 
 template <int DK>
@@ -136,6 +142,7 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 
     float *s_beta = reinterpret_cast<float *>(sm + L::OFF_MISC);        // [64]
     float *s_dec = reinterpret_cast<float *>(sm + L::OFF_MISC + 256);   // [128]: e^{Gamma_C} per key channel
+    float *s_xch = reinterpret_cast<float *>(sm + L::OFF_KH);            // [2][4][128] block products, phase E
     uint64_t *s_bars = reinterpret_cast<uint64_t *>(sm + L::OFF_MISC + 768);
     uint32_t *s_tmem = reinterpret_cast<uint32_t *>(sm + L::OFF_MISC + 800);
     int *s_abort = reinterpret_cast<int *>(sm + L::OFF_MISC + 808);
@@ -146,7 +153,7 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
     const int ch = tid & 127;        // key channel / TMEM lane of this thread
-    const int half = tid >> 7;       // which of the channel's two threads
+    const int qb = tid >> 7;         // 16-token block (phase E) / column quarter (elsewhere)
     const int unit = blockIdx.x;
     const int slice = unit % prm.nslices;
     const int bh = unit / prm.nslices;
@@ -173,29 +180,19 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const uint32_t tmem = *s_tmem;
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;  // this warp's TMEM lanes
 
-    // ---- state: thread (ch, half) holds S[ch][16 half .. 16 half + 15] in fp32 ----
-    float S[VSH];
+    // ---- state: thread (ch, qb) holds S[ch][8 qb .. 8 qb + 7] in fp32 ----
+    float S[VSQ];
 #pragma unroll
-    for (int n = 0; n < VSH; ++n) S[n] = 0.f;
-    const int scol = col0 + half * VSH;
+    for (int n = 0; n < VSQ; ++n) S[n] = 0.f;
+    const int scol = col0 + qb * VSQ;
     if (ch < DK && prm.h0 != nullptr) {
         const float *src = prm.h0 + (((size_t)b * H + h) * DK + ch) * DV + scol;
-#pragma unroll
-        for (int n = 0; n < VSH; n += 4) {
-            const float4 x = *reinterpret_cast<const float4 *>(src + n);
-            S[n] = x.x; S[n + 1] = x.y; S[n + 2] = x.z; S[n + 3] = x.w;
-        }
+        const float4 x0 = *reinterpret_cast<const float4 *>(src), x1 = *reinterpret_cast<const float4 *>(src + 4);
+        S[0] = x0.x; S[1] = x0.y; S[2] = x0.z; S[3] = x0.w; S[4] = x1.x; S[5] = x1.y; S[6] = x1.z; S[7] = x1.w;
     }
     auto store_state_bf16 = [&]() {
-        if (ch < DK) {
-#pragma unroll
-            for (int n = 0; n < VSH; n += 8) {
-                float v8[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) v8[e] = S[n + e];
-                *reinterpret_cast<uint4 *>(sm + L::OFF_S + mnmaj<64, 2>(ch, half * VSH + n, DK)) = pack8_bf16(v8);
-            }
-        }
+        if (ch < DK)
+            *reinterpret_cast<uint4 *>(sm + L::OFF_S + mnmaj<64, 2>(ch, qb * VSQ, DK)) = pack8_bf16(S);
     };
     store_state_bf16();
 
@@ -211,14 +208,13 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         }
         tma_load_4d(sbase + L::OFF_V, &tm_v, bar_in, col0, h, t0, b);
     };
-    // g (fp32) of one chunk for channel tid, straight from global into registers
-    float al[CH];
+    // g (fp32) of this thread's 16 tokens for channel ch, straight into registers
+    float al[SUB];
     auto load_g = [&](int n) {
-        const int t0 = n * CH;
-        const int Lc = min(CH, T - t0);
+        const int t0 = n * CH + qb * SUB;
         const float *gp = gptr + (((size_t)b * T + t0) * H + h) * DK + ch;
 #pragma unroll
-        for (int t = 0; t < CH; ++t) al[t] = (t < Lc && ch < DK) ? __ldg(gp + (size_t)t * H * DK) : 0.f;
+        for (int u = 0; u < SUB; ++u) al[u] = (t0 + u < T && ch < DK) ? __ldg(gp + (size_t)u * H * DK) : 0.f;
     };
     auto load_beta = [&](int n) -> float {
         const int t0 = n * CH;
@@ -270,201 +266,208 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         if (!wait_all(bar_in, ph_in, tma_pending)) { aborted = true; break; }
 
         // ---------------- E: decay factors and operand tiles ----------------
-        // half 0: e^{Gamma} (Q e^G, (beta K e^G)^T), e^{Gamma_C - Gamma} (K-hat^T), X rows
-        // half 1: Y^(I) columns, (beta V)^T
-        if (ch < DK) {
-            const int c = ch;
+        // Thread (c, I = qb) covers key channel c, tokens 16 I .. 16 I + 15.
+        // Local running products inside the block, then the four block totals
+        // and mid-block products are exchanged through shared memory.  The
+        // formation operands (X, Y) are written first so the formation UMMA
+        // runs while the remaining tiles are built.
+        {
+            const int c = ch, I = qb, tb = SUB * I;
+            const bool active = c < DK;
             const uint8_t *qs = sm + L::OFF_Q, *ks = sm + L::OFF_K;
-            auto kval = [&](int i) { return bf16_bits_to_f32(*reinterpret_cast<const uint16_t *>(ks + kmaj<128, 2>(i, c, CH))); };
-            auto qval = [&](int i) { return bf16_bits_to_f32(*reinterpret_cast<const uint16_t *>(qs + kmaj<128, 2>(i, c, CH))); };
+            auto kval = [&](int t) { return bf16_bits_to_f32(*reinterpret_cast<const uint16_t *>(ks + kmaj<128, 2>(t, c, CH))); };
+            auto qval = [&](int t) { return bf16_bits_to_f32(*reinterpret_cast<const uint16_t *>(qs + kmaj<128, 2>(t, c, CH))); };
+            float lp[SUB];  // lp[u] = prod_{s=tb..tb+u} alpha_s
+            float p = 1.f;
 #pragma unroll
-            for (int t = 0; t < CH; ++t) al[t] = __expf(al[t]);
-
-            if (half == 0) {
-                float pre = 1.f;
+            for (int u = 0; u < SUB; ++u) { al[u] = __expf(al[u]); p *= al[u]; lp[u] = p; }
+            if (active) { s_xch[I * 128 + c] = lp[SUB - 1]; s_xch[512 + I * 128 + c] = lp[SUB / 2]; }
+            __syncthreads();
+            float bt[NSUB], l8[NSUB];
 #pragma unroll
-                for (int g8 = 0; g8 < CH / 8; ++g8) {
-                    float qv[8], bk[8];
+            for (int J = 0; J < NSUB; ++J) { bt[J] = s_xch[J * 128 + c]; l8[J] = s_xch[512 + J * 128 + c]; }
+            __syncthreads();  // s_xch aliases the K-hat tile written below
+            float ls[SUB];  // ls[u] = prod_{s=tb+u+1..tb+15} alpha_s
+            ls[SUB - 1] = 1.f;
 #pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        const int t = g8 * 8 + u;
-                        pre *= al[t];
-                        qv[u] = qval(t) * pre;
-                        bk[u] = s_beta[t] * kval(t) * pre;
+            for (int u = SUB - 2; u >= 0; --u) ls[u] = ls[u + 1] * al[u + 1];
+            float kv[SUB], qv[SUB];
+#pragma unroll
+            for (int u = 0; u < SUB; ++u) { kv[u] = kval(tb + u); qv[u] = qval(tb + u); }
+            if (active) {
+                // Own block, reference m = tb + 8:
+                //   u >= 8: f_u = prod_{s=9..u} alpha     X = k f,   Y^(I) = k / f
+                //   u <  8: y_u = prod_{s=u+1..8} alpha   X = k / y, Y^(I) = k y
+                float xk[SUB], xq[SUB], yo[SUB];
+                {
+                    float f = 1.f;
+#pragma unroll
+                    for (int u = SUB / 2; u < SUB; ++u) {
+                        if (u > SUB / 2) f *= al[u];
+                        xk[u] = kv[u] * f;
+                        xq[u] = qv[u] * f;
+                        yo[u] = u == SUB / 2 ? kv[u] : kv[u] * rcp_clamped(f);
                     }
-                    *reinterpret_cast<uint4 *>(sm + L::OFF_WQ + mnmaj<128, 2>(c, 64 + g8 * 8, DK)) = pack8_bf16(qv);
-                    *reinterpret_cast<uint4 *>(sm + L::OFF_BK + kmaj<128, 4>(c, g8 * 8, 128)) = pack4_tf32(bk[0], bk[1], bk[2], bk[3]);
-                    *reinterpret_cast<uint4 *>(sm + L::OFF_BK + kmaj<128, 4>(c, g8 * 8 + 4, 128)) = pack4_tf32(bk[4], bk[5], bk[6], bk[7]);
-                }
-                s_dec[c] = pre;
-                float suf = 1.f;
-#pragma unroll
-                for (int g4 = CH / 4 - 1; g4 >= 0; --g4) {
-                    float kh[4];
-#pragma unroll
-                    for (int u = 3; u >= 0; --u) {
-                        const int t = g4 * 4 + u;
-                        kh[u] = kval(t) * suf;
-                        suf *= al[t];
-                    }
-                    *reinterpret_cast<uint4 *>(sm + L::OFF_KH + kmaj<128, 4>(c, g4 * 4, 128)) = pack4_tf32(kh[0], kh[1], kh[2], kh[3]);
-                }
-                // X rows of block I (reference m = 16 I + 8): F_t = e^{Gamma_t - Gamma_m}
-#pragma unroll
-                for (int I = 0; I < NSUB; ++I) {
-                    const int m = SUB * I + SUB / 2;
-                    float xk[8], xq[8];
-                    float p = 1.f;
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) {  // tokens m .. m+7
-                        const int t = m + u;
-                        if (u > 0) p *= al[t];
-                        xk[u] = kval(t) * p;
-                        xq[u] = qval(t) * p;
-                    }
-                    *reinterpret_cast<uint4 *>(sm + L::OFF_X + mnmaj<128, 2>(c, m, DK)) = pack8_bf16(xk);
-                    *reinterpret_cast<uint4 *>(sm + L::OFF_X + mnmaj<128, 2>(c, 64 + m, DK)) = pack8_bf16(xq);
                     float y = 1.f;
 #pragma unroll
-                    for (int u = 7; u >= 0; --u) {  // tokens m-1 down to 16 I
-                        const int t = SUB * I + u;
-                        y *= al[t + 1];
+                    for (int u = SUB / 2 - 1; u >= 0; --u) {
+                        y *= al[u + 1];
                         const float r = rcp_clamped(y);
-                        xk[u] = kval(t) * r;
-                        xq[u] = qval(t) * r;
+                        xk[u] = kv[u] * r;
+                        xq[u] = qv[u] * r;
+                        yo[u] = kv[u] * y;
                     }
-                    *reinterpret_cast<uint4 *>(sm + L::OFF_X + mnmaj<128, 2>(c, SUB * I, DK)) = pack8_bf16(xk);
-                    *reinterpret_cast<uint4 *>(sm + L::OFF_X + mnmaj<128, 2>(c, 64 + SUB * I, DK)) = pack8_bf16(xq);
                 }
-            } else {
-                // Y^(I) columns j <= 16 I + 15: e^{Gamma_m - Gamma_j}
+                auto yput = [&](int Iy, int j0, const float *v) {
+                    float v8[8];
 #pragma unroll
-                for (int I = 0; I < NSUB; ++I) {
-                    const int m = SUB * I + SUB / 2;
-                    const int yofs = I == 0 ? L::OFF_Y0 : I == 1 ? L::OFF_Y1 : I == 2 ? L::OFF_Y2 : L::OFF_Y3;
-                    auto yput = [&](int j0, const float (&v)[8]) {
-                        uint8_t *dst = sm + yofs;
-                        if (I == 0)      *reinterpret_cast<uint4 *>(dst + mnmaj<32, 2>(c, j0, DK)) = pack8_bf16(v);
-                        else if (I == 1) *reinterpret_cast<uint4 *>(dst + mnmaj<64, 2>(c, j0, DK)) = pack8_bf16(v);
-                        else             *reinterpret_cast<uint4 *>(dst + mnmaj<128, 2>(c, j0, DK)) = pack8_bf16(v);
-                    };
-                    {
-                        float yv[8];
-                        float p = 1.f;
+                    for (int e = 0; e < 8; ++e) v8[e] = v[e];
+                    if (Iy == 0)      *reinterpret_cast<uint4 *>(sm + L::OFF_Y0 + mnmaj<32, 2>(c, j0, DK)) = pack8_bf16(v8);
+                    else if (Iy == 1) *reinterpret_cast<uint4 *>(sm + L::OFF_Y1 + mnmaj<64, 2>(c, j0, DK)) = pack8_bf16(v8);
+                    else if (Iy == 2) *reinterpret_cast<uint4 *>(sm + L::OFF_Y2 + mnmaj<128, 2>(c, j0, DK)) = pack8_bf16(v8);
+                    else              *reinterpret_cast<uint4 *>(sm + L::OFF_Y3 + mnmaj<128, 2>(c, j0, DK)) = pack8_bf16(v8);
+                };
 #pragma unroll
-                        for (int u = 0; u < 8; ++u) {  // tokens m .. m+7: 1 / prod_{s=m+1..t} alpha_s
-                            const int t = m + u;
-                            if (u > 0) p *= al[t];
-                            yv[u] = u == 0 ? kval(t) : kval(t) * rcp_clamped(p);
-                        }
-                        yput(m, yv);
-                    }
-                    float y = 1.f;
+                for (int h8 = 0; h8 < 2; ++h8) {
+                    float a8[8], b8[8];
 #pragma unroll
-                    for (int g8 = m / 8 - 1; g8 >= 0; --g8) {  // tokens below m: prod_{s=t+1..m} alpha_s
-                        float yv[8];
+                    for (int e = 0; e < 8; ++e) { a8[e] = xk[h8 * 8 + e]; b8[e] = xq[h8 * 8 + e]; }
+                    *reinterpret_cast<uint4 *>(sm + L::OFF_X + mnmaj<128, 2>(c, tb + h8 * 8, DK)) = pack8_bf16(a8);
+                    *reinterpret_cast<uint4 *>(sm + L::OFF_X + mnmaj<128, 2>(c, 64 + tb + h8 * 8, DK)) = pack8_bf16(b8);
+                    yput(I, tb + h8 * 8, yo + h8 * 8);
+                }
+                // Later blocks I' > I see this block through e^{Gamma_{m'} - Gamma_j}
+                //   = ls_u * prod_{J = I+1 .. I'-1} bt_J * l8_{I'}   (all factors <= 1)
+                float mid = 1.f;
 #pragma unroll
-                        for (int u = 7; u >= 0; --u) {
-                            const int t = g8 * 8 + u;
-                            y *= al[t + 1];
-                            yv[u] = kval(t) * y;
-                        }
-                        yput(g8 * 8, yv);
+                for (int Ip = 1; Ip < NSUB; ++Ip) {
+                    if (Ip > I) {
+                        const float sc = mid * l8[Ip];
+                        float yv[SUB];
+#pragma unroll
+                        for (int u = 0; u < SUB; ++u) yv[u] = kv[u] * (ls[u] * sc);
+                        yput(Ip, tb, yv);
+                        yput(Ip, tb + 8, yv + 8);
+                        mid *= bt[Ip];
                     }
                 }
             }
-        }
-        if (half == 1 && ch >= DK - VSL && ch < DK) {  // (beta V)^T: row n = value column
-            const int nn = ch - (DK - VSL);
-            const uint16_t *vs = reinterpret_cast<const uint16_t *>(sm + L::OFF_V);
-#pragma unroll
-            for (int g4 = 0; g4 < CH / 4; ++g4) {
-                float w[4];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int t = g4 * 4 + u;
-                    w[u] = s_beta[t] * bf16_bits_to_f32(vs[t * VSL + nn]);
-                }
-                *reinterpret_cast<uint4 *>(sm + L::OFF_BV + kmaj<128, 4>(nn, g4 * 4, VSL)) = pack4_tf32(w[0], w[1], w[2], w[3]);
-            }
-        }
-        sync_for_mma();
+            sync_for_mma();
 
-        // ---------------- F: formation products (bf16) ----------------
-        if (tid == 0) {
-            if (n + 1 < nchunks) issue_loads(n + 1);  // R_in is consumed: prefetch
+            // ---------------- F: formation products (bf16), overlapped with the rest of E ----------------
+            if (tid == 0) {
 #pragma unroll
-            for (int I = 0; I < NSUB; ++I) {
-                const uint32_t idesc = make_idesc(1, true, true, 128, SUB * (I + 1));
+                for (int If = 0; If < NSUB; ++If) {
+                    const uint32_t idesc = make_idesc(1, true, true, 128, SUB * (If + 1));
 #pragma unroll
-                for (int kk = 0; kk < DK / 16; ++kk) {
-                    const uint64_t da = desc_mnmaj<128>(sbase + L::OFF_X, DK, kk * 16);
-                    uint64_t db;
-                    if (I == 0)      db = desc_mnmaj<32>(sbase + L::OFF_Y0, DK, kk * 16);
-                    else if (I == 1) db = desc_mnmaj<64>(sbase + L::OFF_Y1, DK, kk * 16);
-                    else if (I == 2) db = desc_mnmaj<128>(sbase + L::OFF_Y2, DK, kk * 16);
-                    else             db = desc_mnmaj<128>(sbase + L::OFF_Y3, DK, kk * 16);
-                    umma<0>(tmem + L::TM_AP + yoff(I), da, db, idesc, kk > 0);
+                    for (int kk = 0; kk < DK / 16; ++kk) {
+                        const uint64_t da = desc_mnmaj<128>(sbase + L::OFF_X, DK, kk * 16);
+                        uint64_t db;
+                        if (If == 0)      db = desc_mnmaj<32>(sbase + L::OFF_Y0, DK, kk * 16);
+                        else if (If == 1) db = desc_mnmaj<64>(sbase + L::OFF_Y1, DK, kk * 16);
+                        else if (If == 2) db = desc_mnmaj<128>(sbase + L::OFF_Y2, DK, kk * 16);
+                        else              db = desc_mnmaj<128>(sbase + L::OFF_Y3, DK, kk * 16);
+                        umma<0>(tmem + L::TM_AP + yoff(If), da, db, idesc, kk > 0);
+                    }
+                }
+                umma_commit(bar_mma);
+            }
+            mma_pending = true;
+
+            if (active) {
+                float preB = 1.f, postB = 1.f;
+#pragma unroll
+                for (int J = 0; J < NSUB; ++J) { if (J < I) preB *= bt[J]; if (J > I) postB *= bt[J]; }
+                if (I == 0) s_dec[c] = bt[0] * bt[1] * bt[2] * bt[3];
+                // e^{Gamma_t}: Q e^G (rows 64.. of [W; Q e^G]) and (beta K e^G)^T;  e^{Gamma_C - Gamma_t}: K-hat^T
+#pragma unroll
+                for (int h8 = 0; h8 < 2; ++h8) {
+                    const float4 b0 = *reinterpret_cast<const float4 *>(s_beta + tb + h8 * 8);
+                    const float4 b1 = *reinterpret_cast<const float4 *>(s_beta + tb + h8 * 8 + 4);
+                    const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+                    float qe[8], bk[8], kh[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int u = h8 * 8 + e;
+                        const float pre = preB * lp[u];
+                        qe[e] = qv[u] * pre;
+                        bk[e] = bb[e] * kv[u] * pre;
+                        kh[e] = kv[u] * (ls[u] * postB);
+                    }
+                    const int t8 = tb + h8 * 8;
+                    *reinterpret_cast<uint4 *>(sm + L::OFF_WQ + mnmaj<128, 2>(c, 64 + t8, DK)) = pack8_bf16(qe);
+                    *reinterpret_cast<uint4 *>(sm + L::OFF_BK + kmaj<128, 4>(c, t8, 128)) = pack4_tf32(bk[0], bk[1], bk[2], bk[3]);
+                    *reinterpret_cast<uint4 *>(sm + L::OFF_BK + kmaj<128, 4>(c, t8 + 4, 128)) = pack4_tf32(bk[4], bk[5], bk[6], bk[7]);
+                    *reinterpret_cast<uint4 *>(sm + L::OFF_KH + kmaj<128, 4>(c, t8, 128)) = pack4_tf32(kh[0], kh[1], kh[2], kh[3]);
+                    *reinterpret_cast<uint4 *>(sm + L::OFF_KH + kmaj<128, 4>(c, t8 + 4, 128)) = pack4_tf32(kh[4], kh[5], kh[6], kh[7]);
                 }
             }
-            umma_commit(bar_mma);
+            if (c < VSL) {  // (beta V)^T: row c = value column, tokens of block I
+                const uint16_t *vs = reinterpret_cast<const uint16_t *>(sm + L::OFF_V);
+#pragma unroll
+                for (int g4 = 0; g4 < SUB / 4; ++g4) {
+                    const float4 b4 = *reinterpret_cast<const float4 *>(s_beta + tb + g4 * 4);
+                    const float bb[4] = {b4.x, b4.y, b4.z, b4.w};
+                    float w[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) w[e] = bb[e] * bf16_bits_to_f32(vs[(tb + g4 * 4 + e) * VSL + c]);
+                    *reinterpret_cast<uint4 *>(sm + L::OFF_BV + kmaj<128, 4>(c, tb + g4 * 4, VSL)) = pack4_tf32(w[0], w[1], w[2], w[3]);
+                }
+            }
         }
+        __syncthreads();  // R_in consumed
+        if (tid == 0 && n + 1 < nchunks) issue_loads(n + 1);
         tma_pending = n + 1 < nchunks;
-        mma_pending = true;
         beta_next = n + 1 < nchunks ? load_beta(n + 1) : 0.f;
         if (!wait_all(bar_mma, ph_mma, mma_pending)) { aborted = true; break; }
 
         // ---------------- AP: A -> fp32 scratch, P -> tf32 tile ----------------
-        // TMEM lane = row of [k; q]; the two warps of a lane quarter split the
-        // four 16-column chunks of each row (half 0: chunks 0-1, half 1: 2-3).
+        // TMEM lane = row of [k; q]; the four warps of a lane quarter take one
+        // 16-column chunk each (chunk = qb).
         {
             float *sA = reinterpret_cast<float *>(sm + L::OFF_A);
-            const int row = ch;
-            const int i = row & 63;
+            const int i = ch & 63;
             const int myI = i / SUB;
-            const bool is_q = row >= 64;
+            const bool is_q = ch >= 64;
             const float bi = s_beta[i];
-            const int I0 = (((warp & 3) & 1) * 32) / SUB;  // the lane quarter covers blocks I0, I0 + 1
+            const int I0 = ((warp & 1) * 32) / SUB;  // the lane quarter covers blocks I0, I0 + 1
+            const int cc = qb;
+            float v16[16];
 #pragma unroll
-            for (int c2 = 0; c2 < 2; ++c2) {
-                const int cc = half * 2 + c2;
-                float v16[16];
+            for (int e = 0; e < 16; ++e) v16[e] = 0.f;
 #pragma unroll
-                for (int e = 0; e < 16; ++e) v16[e] = 0.f;
+            for (int dI = 0; dI < 2; ++dI) {
+                const int I = I0 + dI;
+                if (cc <= I) {
+                    float t[16];
+                    tmem_ld16(tmem + lane_base + L::TM_AP + yoff(I) + cc * 16, t);
+                    tmem_wait_ld();
+                    if (myI == I) {
 #pragma unroll
-                for (int dI = 0; dI < 2; ++dI) {
-                    const int I = I0 + dI;
-                    if (cc <= I) {
-                        float t[16];
-                        tmem_ld16(tmem + lane_base + L::TM_AP + yoff(I) + cc * 16, t);
-                        tmem_wait_ld();
-                        if (myI == I) {
-#pragma unroll
-                            for (int e = 0; e < 16; ++e) v16[e] = t[e];
-                        }
+                        for (int e = 0; e < 16; ++e) v16[e] = t[e];
                     }
                 }
-                const int j0 = cc * 16;
-                if (!is_q) {
+            }
+            const int j0 = cc * 16;
+            if (!is_q) {
 #pragma unroll
-                    for (int e = 0; e < 16; e += 4) {
-                        float4 w;
-                        w.x = (j0 + e + 0 < i) ? bi * v16[e + 0] : 0.f;
-                        w.y = (j0 + e + 1 < i) ? bi * v16[e + 1] : 0.f;
-                        w.z = (j0 + e + 2 < i) ? bi * v16[e + 2] : 0.f;
-                        w.w = (j0 + e + 3 < i) ? bi * v16[e + 3] : 0.f;
-                        *reinterpret_cast<float4 *>(sA + i * A_LD + j0 + e) = w;
-                    }
-                } else {
+                for (int e = 0; e < 16; e += 4) {
+                    float4 w;
+                    w.x = (j0 + e + 0 < i) ? bi * v16[e + 0] : 0.f;
+                    w.y = (j0 + e + 1 < i) ? bi * v16[e + 1] : 0.f;
+                    w.z = (j0 + e + 2 < i) ? bi * v16[e + 2] : 0.f;
+                    w.w = (j0 + e + 3 < i) ? bi * v16[e + 3] : 0.f;
+                    *reinterpret_cast<float4 *>(sA + i * A_LD + j0 + e) = w;
+                }
+            } else {
 #pragma unroll
-                    for (int e = 0; e < 16; e += 4) {
-                        uint4 w;
-                        w.x = (j0 + e + 0 <= i) ? to_tf32(v16[e + 0]) : 0u;
-                        w.y = (j0 + e + 1 <= i) ? to_tf32(v16[e + 1]) : 0u;
-                        w.z = (j0 + e + 2 <= i) ? to_tf32(v16[e + 2]) : 0u;
-                        w.w = (j0 + e + 3 <= i) ? to_tf32(v16[e + 3]) : 0u;
-                        *reinterpret_cast<uint4 *>(sm + L::OFF_PB + kmaj_s<128, 4>(64 + i, j0 + e, 8192)) = w;
-                    }
+                for (int e = 0; e < 16; e += 4) {
+                    uint4 w;
+                    w.x = (j0 + e + 0 <= i) ? tf32_bits(v16[e + 0]) : 0u;
+                    w.y = (j0 + e + 1 <= i) ? tf32_bits(v16[e + 1]) : 0u;
+                    w.z = (j0 + e + 2 <= i) ? tf32_bits(v16[e + 2]) : 0u;
+                    w.w = (j0 + e + 3 <= i) ? tf32_bits(v16[e + 3]) : 0u;
+                    *reinterpret_cast<uint4 *>(sm + L::OFF_PB + kmaj_s<128, 4>(64 + i, j0 + e, 8192)) = w;
                 }
             }
         }
@@ -491,36 +494,72 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 for (int ii = 0; ii < SUB; ++ii) sTf[(base + ii) * A_LD + base + jj] = x[ii];
             }
             __syncthreads();
-            // off-diagonal blocks by distance d: T_{I,J} = -T_II sum_{K=J}^{I-1} A_IK T_KJ, J = I - d
-#pragma unroll
-            for (int d = 1; d < NSUB; ++d) {
-                const int nt = NSUB - d;
-                for (int e = tid; e < nt * 256; e += CHUNK_THREADS) {
-                    const int blk = e >> 8, I = d + blk, J = blk, r = (e >> 4) & 15, cc = e & 15;
-                    float acc = 0.f;
-                    for (int K = J; K < I; ++K) {
-                        const float *arow = sA + (SUB * I + r) * A_LD + SUB * K;
-#pragma unroll
-                        for (int m4 = 0; m4 < SUB; m4 += 4) {
-                            const float4 a4 = *reinterpret_cast<const float4 *>(arow + m4);
-                            const float *tc = sTf + (SUB * K + m4) * A_LD + SUB * J + cc;
-                            acc += a4.x * tc[0] + a4.y * tc[A_LD] + a4.z * tc[2 * A_LD] + a4.w * tc[3 * A_LD];
-                        }
-                    }
-                    sZ[blk * 256 + r * 16 + cc] = acc;
-                }
-                __syncthreads();
-                for (int e = tid; e < nt * 256; e += CHUNK_THREADS) {
-                    const int blk = e >> 8, I = d + blk, J = blk, r = (e >> 4) & 15, cc = e & 15;
-                    const float *trow = sTf + (SUB * I + r) * A_LD + SUB * I;
-                    float acc = 0.f;
+            // Off-diagonal blocks.  With D = diag(T_II) and N = D A_offdiag (strictly block
+            // lower, N^4 = 0):  T = (I - N + N^2 - N^3) D, i.e. T_IJ = M_IJ T_JJ with
+            //   M_{I,I-1} = -N_{I,I-1},  M_20 = -N_20 + N_21 N_10,  M_31 = -N_31 + N_32 N_21,
+            //   M_30 = -N_30 + N_31 N_10 - N_32 M_20.
+            // Scratch slots (16x16, row stride 16): 0 N10, 1 N20, 2 N21, 3 N30, 4 N31, 5 N32, 6 M31.
+            // One warp per 16x16 product; lane (r = lane / 2, c0 = 8 (lane % 2)) owns 8 outputs.
+            {
+                const int r = lane >> 1, c0 = (lane & 1) * 8;
+                // 16x16 * 16x16 row-times-block: out[0..7] += sum_m a[r][m] * B[m][c0..c0+7]
+                auto rowblk = [&](const float *arow, const float *bblk, int bld, float (&o)[8]) {
 #pragma unroll
                     for (int m4 = 0; m4 < SUB; m4 += 4) {
-                        const float4 t4 = *reinterpret_cast<const float4 *>(trow + m4);  // zero above the diagonal
-                        const float *z = sZ + blk * 256 + m4 * 16 + cc;
-                        acc += t4.x * z[0] + t4.y * z[16] + t4.z * z[32] + t4.w * z[48];
+                        const float4 a4 = *reinterpret_cast<const float4 *>(arow + m4);
+                        const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+                        for (int mm = 0; mm < 4; ++mm) {
+                            const float *brow = bblk + (m4 + mm) * bld + c0;
+                            const float4 b0 = *reinterpret_cast<const float4 *>(brow);
+                            const float4 b1 = *reinterpret_cast<const float4 *>(brow + 4);
+                            o[0] += av[mm] * b0.x; o[1] += av[mm] * b0.y; o[2] += av[mm] * b0.z; o[3] += av[mm] * b0.w;
+                            o[4] += av[mm] * b1.x; o[5] += av[mm] * b1.y; o[6] += av[mm] * b1.z; o[7] += av[mm] * b1.w;
+                        }
                     }
-                    sTf[(SUB * I + r) * A_LD + SUB * J + cc] = -acc;
+                };
+                auto store8 = [&](float *dst, const float (&o)[8], float sgn) {
+                    *reinterpret_cast<float4 *>(dst) = make_float4(sgn * o[0], sgn * o[1], sgn * o[2], sgn * o[3]);
+                    *reinterpret_cast<float4 *>(dst + 4) = make_float4(sgn * o[4], sgn * o[5], sgn * o[6], sgn * o[7]);
+                };
+                const int BI = warp == 0 ? 1 : (warp < 3 ? 2 : 3);            // block pair of warp < 6:
+                const int BJ = warp == 0 ? 0 : (warp < 3 ? warp - 1 : warp - 3);  // (1,0) (2,0) (2,1) (3,0) (3,1) (3,2)
+                if (warp < 6) {  // N_IJ = T_II A_IJ
+                    const int I = BI, J = BJ;
+                    float o[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                    rowblk(sTf + (SUB * I + r) * A_LD + SUB * I, sA + (SUB * I) * A_LD + SUB * J, A_LD, o);
+                    store8(sZ + warp * 256 + r * 16 + c0, o, 1.f);
+                }
+                __syncthreads();
+                if (warp < 2) {  // M20 = -N20 + N21 N10 (slot 1);  M31 = -N31 + N32 N21 (slot 6)
+                    const int so = warp == 0 ? 1 : 4, sa = warp == 0 ? 2 : 5, sb = warp == 0 ? 0 : 2;
+                    float o[8];
+                    const float *own = sZ + so * 256 + r * 16 + c0;
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) o[e] = -own[e];
+                    rowblk(sZ + sa * 256 + r * 16, sZ + sb * 256, 16, o);
+                    store8(sZ + (warp == 0 ? 1 : 6) * 256 + r * 16 + c0, o, 1.f);
+                }
+                __syncthreads();
+                if (warp == 0) {  // M30 = -N30 + N31 N10 - N32 M20 (slot 3)
+                    float o[8], o2[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                    const float *own = sZ + 3 * 256 + r * 16 + c0;
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) o[e] = -own[e];
+                    rowblk(sZ + 4 * 256 + r * 16, sZ + 0 * 256, 16, o);
+                    rowblk(sZ + 5 * 256 + r * 16, sZ + 1 * 256, 16, o2);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) o[e] -= o2[e];
+                    store8(sZ + 3 * 256 + r * 16 + c0, o, 1.f);
+                }
+                __syncthreads();
+                if (warp < 6) {  // T_IJ = M_IJ T_JJ; adjacent blocks carry M = -N
+                    const int I = BI, J = BJ;
+                    const int msl = warp == 4 ? 6 : warp;
+                    const float sgn = (warp == 0 || warp == 2 || warp == 5) ? -1.f : 1.f;
+                    float o[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                    rowblk(sZ + msl * 256 + r * 16, sTf + (SUB * J) * A_LD + SUB * J, A_LD, o);
+                    store8(sTf + (SUB * I + r) * A_LD + SUB * J + c0, o, sgn);
                 }
                 __syncthreads();
             }
@@ -551,18 +590,16 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         mma_pending = true;
         if (!wait_all(bar_mma, ph_mma, mma_pending)) { aborted = true; break; }
         if (n + 1 < nchunks) load_g(n + 1);  // consumed at the next chunk's phase E
-        if (ch < DK) {  // W^T row ch -> W columns of [W; Q e^G]; half h takes tokens 32 h .. 32 h + 31
+        if ((warp & 3) < DK / 32) {  // W^T row ch -> W columns of [W; Q e^G]; thread takes tokens 16 qb ..
+            const int i0 = qb * 16;
+            float t[16];
+            tmem_ld16(tmem + lane_base + L::TM_W + i0, t);
+            tmem_wait_ld();
+            float a8[8], b8[8];
 #pragma unroll
-            for (int i0 = half * 32; i0 < half * 32 + 32; i0 += 16) {
-                float t[16];
-                tmem_ld16(tmem + lane_base + L::TM_W + i0, t);
-                tmem_wait_ld();
-                float a8[8], b8[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) { a8[e] = t[e]; b8[e] = t[8 + e]; }
-                *reinterpret_cast<uint4 *>(sm + L::OFF_WQ + mnmaj<128, 2>(ch, i0, DK)) = pack8_bf16(a8);
-                *reinterpret_cast<uint4 *>(sm + L::OFF_WQ + mnmaj<128, 2>(ch, i0 + 8, DK)) = pack8_bf16(b8);
-            }
+            for (int e = 0; e < 8; ++e) { a8[e] = t[e]; b8[e] = t[8 + e]; }
+            *reinterpret_cast<uint4 *>(sm + L::OFF_WQ + mnmaj<128, 2>(ch, i0, DK)) = pack8_bf16(a8);
+            *reinterpret_cast<uint4 *>(sm + L::OFF_WQ + mnmaj<128, 2>(ch, i0 + 8, DK)) = pack8_bf16(b8);
         }
         sync_for_mma();
 
@@ -579,16 +616,16 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         if (!wait_all(bar_mma, ph_mma, mma_pending)) { aborted = true; break; }
 
         // ---------------- 2: Vnew = U - W S0 -> Vnew^T tile (tf32) ----------------
-        if ((warp & 3) < 2) {  // lanes 0..63 = tokens; half picks 16 of the 32 columns
+        if ((warp & 3) < 2) {  // lanes 0..63 = tokens; qb picks 8 of the 32 columns
             const int i = ch;
-            const int n0 = half * VSH;
-            float u[16], ws[16];
-            tmem_ld16(tmem + lane_base + L::TM_U + n0, u);
-            tmem_ld16(tmem + lane_base + L::TM_D1 + n0, ws);
+            const int n0 = qb * VSQ;
+            float u[8], ws[8];
+            tmem_ld8(tmem + lane_base + L::TM_U + n0, u);
+            tmem_ld8(tmem + lane_base + L::TM_D1 + n0, ws);
             tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 16; ++e)
-                *reinterpret_cast<uint32_t *>(sm + L::OFF_VN + kmaj_s<128, 4>(n0 + e, i, VSL * 128)) = to_tf32(u[e] - ws[e]);
+            for (int e = 0; e < 8; ++e)
+                *reinterpret_cast<uint32_t *>(sm + L::OFF_VN + kmaj_s<128, 4>(n0 + e, i, VSL * 128)) = tf32_bits(u[e] - ws[e]);
         }
         sync_for_mma();
 
@@ -607,28 +644,26 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         if (!wait_all(bar_mma, ph_mma, mma_pending)) { aborted = true; break; }
 
         // ---------------- 4: output and state update ----------------
-        if ((warp & 3) >= 2) {  // lanes 64..127 = output rows
+        if ((warp & 3) >= 2) {  // lanes 64..127 = output rows; qb picks 8 of the 32 columns
             const int i = ch - 64;
-            const int n0 = half * VSH;
-            float t[16];
-            tmem_ld16(tmem + lane_base + L::TM_D1 + n0, t);
+            const int n0 = qb * VSQ;
+            float t[8];
+            tmem_ld8(tmem + lane_base + L::TM_D1 + n0, t);
             tmem_wait_ld();
             if (i < Lc) {
-                uint16_t *dst = prm.out + (((size_t)b * T + t0 + i) * H + h) * DV + col0 + n0;
-                float a8[8], b8[8];
+                float a8[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) { a8[e] = prm.scale * t[e]; b8[e] = prm.scale * t[8 + e]; }
-                reinterpret_cast<uint4 *>(dst)[0] = pack8_bf16(a8);
-                reinterpret_cast<uint4 *>(dst)[1] = pack8_bf16(b8);
+                for (int e = 0; e < 8; ++e) a8[e] = prm.scale * t[e];
+                *reinterpret_cast<uint4 *>(prm.out + (((size_t)b * T + t0 + i) * H + h) * DV + col0 + n0) = pack8_bf16(a8);
             }
         }
         if ((warp & 3) < DK / 32) {
-            float t[16];
-            tmem_ld16(tmem + lane_base + L::TM_D3 + half * VSH, t);
+            float t[8];
+            tmem_ld8(tmem + lane_base + L::TM_D3 + qb * VSQ, t);
             tmem_wait_ld();
             const float dc = s_dec[ch];
 #pragma unroll
-            for (int e = 0; e < VSH; ++e) S[e] = dc * S[e] + t[e];
+            for (int e = 0; e < VSQ; ++e) S[e] = dc * S[e] + t[e];
         }
         store_state_bf16();
         tc_fence_before();
@@ -645,9 +680,8 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         __syncthreads();
     } else if (prm.hT != nullptr && ch < DK) {
         float *dst = prm.hT + (((size_t)b * H + h) * DK + ch) * DV + scol;
-#pragma unroll
-        for (int n = 0; n < VSH; n += 4)
-            *reinterpret_cast<float4 *>(dst + n) = make_float4(S[n], S[n + 1], S[n + 2], S[n + 3]);
+        *reinterpret_cast<float4 *>(dst) = make_float4(S[0], S[1], S[2], S[3]);
+        *reinterpret_cast<float4 *>(dst + 4) = make_float4(S[4], S[5], S[6], S[7]);
     }
     tc_fence_after();
     if (warp == 0) tmem_dealloc(tmem, L::TM_COLS);

@@ -1,5 +1,5 @@
-// chunk_params.cuh -- launch parameters of the chunkwise prefill kernel,
-// shared by the kernel (chunk_fwd.cu) and the C ABI (kda_api.cu).
+// chunk_params.cuh -- launch parameters of the two prefill kernels, shared by
+// the kernels (prep_fwd.cu, chain_fwd.cu) and the C ABI (kda_api.cu).
 #pragma once
 #include <stdint.h>
 
@@ -7,6 +7,7 @@
 
 namespace kda {
 
+// Fused single-kernel prefill: one CTA per (b, h, value slice).
 struct ChunkParams {
     const float *beta;   // [B, T, H]
     const float *h0;     // [B, H, dk, dv] or NULL
@@ -14,6 +15,28 @@ struct ChunkParams {
     float *hT;           // [B, H, dk, dv] or NULL
     float scale;
     int B, T, H, DV, nslices;
+    DeviceStatus st;
+    uint64_t inject_wait_polls;  // test hook: nonzero = first wait on a barrier nothing signals
+};
+
+// One CTA per (b, h, chunk) of chunks [n_begin, n_begin + nseg).
+struct PrepParams {
+    const float *g;      // [B, T, H, dk]
+    const float *beta;   // [B, T, H]
+    uint8_t *ws;         // records [B*H][nseg][REC_BYTES]
+    int B, T, H, n_begin, nseg;
+    DeviceStatus st;
+};
+
+// One CTA per (b, h); walks chunks [n_begin, n_begin + nseg) in order.
+struct ChainParams {
+    const float *beta;   // [B, T, H]
+    const float *h0;     // [B, H, dk, dv] or NULL (state at chunk n_begin)
+    uint16_t *out;       // bf16 [B, T, H, dv]
+    float *hT;           // [B, H, dk, dv] or NULL (state after the last chunk of the segment)
+    const uint8_t *ws;   // records written by the prep kernel
+    float scale;
+    int B, T, H, DV, n_begin, nseg;
     DeviceStatus st;
     uint64_t inject_wait_polls;  // test hook: nonzero = first wait on a barrier nothing signals
 };
