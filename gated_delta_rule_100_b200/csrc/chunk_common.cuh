@@ -1,0 +1,63 @@
+// chunk_common.cuh -- constants, the per-chunk record layout and small helpers
+// shared by the two prefill kernels (prep_fwd.cu, chain_fwd.cu).
+//
+// The chunkwise prefill is split in two:
+//   prep  (one CTA per (b, h, chunk), no dependence between chunks): builds the
+//         decay-scaled operands, the intra-chunk blocks A and P, T = (I + A)^-1
+//         and W = T Diag(beta) (K * e^Gamma), and writes one record per chunk;
+//   chain (one CTA per (b, h), chunks in order): U = T Diag(beta) V, then the
+//         state pass Vnew = U - W S, S <- e^{Gamma_C} S + K-hat^T Vnew and the
+//         outputs (Q e^Gamma) S + P Vnew.
+// A record holds, in the exact shared-memory layouts the chain's UMMAs read
+// (offsets relative to a 1024-byte aligned base, so the swizzle carries over):
+//   WQ   bf16 MN-major [dk][128]: columns 0..63 = W^T, 64..127 = (Q e^Gamma)^T
+//   P    tf32 K-major  [64][64], K-block stride 8 KB (causal q-k block, incl. diagonal)
+//   KH   tf32 K-major  [128][64] (K-hat^T: row = key channel, K = token)
+//   T'   tf32 K-major  [64][64], K-block stride 8 KB: T' = T Diag(beta)
+//   DEC  fp32 [128]    e^{Gamma_C} per key channel
+#pragma once
+#include <stdint.h>
+
+#include "kda_device.cuh"
+
+namespace kda {
+
+constexpr int CH = 64;          // chunk length
+constexpr int SUB = 16;         // sub-block of the decay references
+constexpr int NSUB = CH / SUB;  // 4
+constexpr int A_LD = 68;        // fp32 row stride of the A / T scratch
+constexpr float EXP_CLAMP_HI = 5.5406223843935098e34f;  // e^80
+constexpr float EXP_CLAMP_LO = 1.8048513878454153e-35f; // e^-80
+
+constexpr int REC_WQ = 0;
+constexpr int REC_P = 32768;
+constexpr int REC_KH = 49152;
+constexpr int REC_T = 81920;
+constexpr int REC_DEC = 98304;
+constexpr int REC_BYTES = 99328;
+
+__host__ __device__ constexpr int align1k(int x) { return (x + 1023) & ~1023; }
+__host__ __device__ constexpr int cmax(int a, int b) { return a > b ? a : b; }
+
+// First TMEM column / Y row of block I's formation product: 16 * I (I + 1) / 2.
+__device__ __forceinline__ constexpr int yoff(int I) { return SUB * (I * (I + 1) / 2); }
+
+__device__ __forceinline__ float rcp_clamped(float p) {
+    return p < EXP_CLAMP_LO ? EXP_CLAMP_HI : __fdividef(1.0f, p);
+}
+
+__device__ __forceinline__ uint4 pack8_bf16(const float (&v)[8]) {
+    return make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                      pack_bf16x2(v[6], v[7]));
+}
+
+// tf32 operands are stored as fp32 bit patterns: the tensor core reads the
+// sign, exponent and top 10 mantissa bits (the conversion instruction runs at
+// a sixteenth of the FMA rate, so it is skipped).
+__device__ __forceinline__ uint32_t tf32_bits(float x) { return __float_as_uint(x); }
+
+__device__ __forceinline__ uint4 pack4_tf32(float a, float b, float c, float d) {
+    return make_uint4(tf32_bits(a), tf32_bits(b), tf32_bits(c), tf32_bits(d));
+}
+
+}  // namespace kda

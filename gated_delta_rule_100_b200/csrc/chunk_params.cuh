@@ -7,18 +7,6 @@
 
 namespace kda {
 
-// Fused single-kernel prefill: one CTA per (b, h, value slice).
-struct ChunkParams {
-    const float *beta;   // [B, T, H]
-    const float *h0;     // [B, H, dk, dv] or NULL
-    uint16_t *out;       // bf16 [B, T, H, dv]
-    float *hT;           // [B, H, dk, dv] or NULL
-    float scale;
-    int B, T, H, DV, nslices;
-    DeviceStatus st;
-    uint64_t inject_wait_polls;  // test hook: nonzero = first wait on a barrier nothing signals
-};
-
 // One CTA per (b, h, chunk) of chunks [n_begin, n_begin + nseg).
 struct PrepParams {
     const float *g;      // [B, T, H, dk]
@@ -28,15 +16,15 @@ struct PrepParams {
     DeviceStatus st;
 };
 
-// One CTA per (b, h); walks chunks [n_begin, n_begin + nseg) in order.
+// One CTA per (b, h, value slice); walks chunks [n_begin, n_begin + nseg) in order.
 struct ChainParams {
-    const float *beta;   // [B, T, H]
+    const uint16_t *v;   // bf16 [B, T, H, dv]
     const float *h0;     // [B, H, dk, dv] or NULL (state at chunk n_begin)
     uint16_t *out;       // bf16 [B, T, H, dv]
     float *hT;           // [B, H, dk, dv] or NULL (state after the last chunk of the segment)
     const uint8_t *ws;   // records written by the prep kernel
     float scale;
-    int B, T, H, DV, n_begin, nseg;
+    int B, T, H, DV, n_begin, nseg, nslices;
     DeviceStatus st;
     uint64_t inject_wait_polls;  // test hook: nonzero = first wait on a barrier nothing signals
 };

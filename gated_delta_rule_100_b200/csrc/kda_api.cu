@@ -18,12 +18,13 @@ cudaError_t launch_decode(const void *q, const void *k, const void *v, const flo
                           int dv, cudaStream_t stream);
 }
 
+#include "chunk_common.cuh"
 #include "chunk_params.cuh"
 
 namespace kda {
-cudaError_t launch_chunk(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
-                         const float *g, const ChunkParams &prm, int dk, cudaStream_t stream);
-int chunk_value_slice();
+cudaError_t launch_prep(const CUtensorMap &tq, const CUtensorMap &tk, const PrepParams &prm, int dk,
+                        cudaStream_t stream);
+cudaError_t launch_chain(const ChainParams &prm, int dk, cudaStream_t stream);
 }
 
 // Device-side status word: kernels OR error bits into it (one per device,
@@ -63,6 +64,54 @@ int get_encoder(PFN_cuTensorMapEncodeTiled_v12000 *fn) {
         g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
     }
     *fn = g_encode;
+    return KDA_OK;
+}
+
+// Per-device workspace of the prefill: the per-chunk records written by the
+// prep kernel and read by the chain kernel, plus a state buffer carried
+// between segments.  Grown on demand (cudaFree synchronises the device, so no
+// kernel still reads the old buffer) and kept for later calls.  Calls on
+// different streams are ordered on it by `done`, recorded after each call's
+// last kernel and waited on by the next call's stream.
+constexpr size_t kWorkspaceCap = size_t(2) << 30;  // records of one segment, bytes
+struct Workspace {
+    uint8_t *rec = nullptr;
+    size_t rec_bytes = 0;
+    float *state = nullptr;
+    size_t state_bytes = 0;
+    cudaEvent_t done = nullptr;
+};
+Workspace g_ws[kMaxDevices];
+
+size_t rec_row_bytes(int B, int H) { return (size_t)B * H * kda::REC_BYTES; }
+
+// Chunks per segment: as many as fit the cap, at least one.
+int segment_chunks(int B, int T, int H) {
+    const int nchunks = (T + kda::CH - 1) / kda::CH;
+    const size_t fit = kWorkspaceCap / rec_row_bytes(B, H);
+    return (int)(fit < 1 ? 1 : (fit < (size_t)nchunks ? fit : (size_t)nchunks));
+}
+
+// Called with g_mu held.
+int reserve_workspace(int dev, size_t rec_bytes, size_t state_bytes, Workspace **out) {
+    Workspace &w = g_ws[dev];
+    if (w.rec_bytes < rec_bytes) {
+        if (w.rec != nullptr && cudaFree(w.rec) != cudaSuccess) return KDA_ERR_CUDA;
+        w.rec = nullptr;
+        w.rec_bytes = 0;
+        if (cudaMalloc(&w.rec, rec_bytes) != cudaSuccess) return KDA_ERR_CUDA;
+        w.rec_bytes = rec_bytes;
+    }
+    if (w.state_bytes < state_bytes) {
+        if (w.state != nullptr && cudaFree(w.state) != cudaSuccess) return KDA_ERR_CUDA;
+        w.state = nullptr;
+        w.state_bytes = 0;
+        if (cudaMalloc(&w.state, state_bytes) != cudaSuccess) return KDA_ERR_CUDA;
+        w.state_bytes = state_bytes;
+    }
+    if (w.done == nullptr && cudaEventCreateWithFlags(&w.done, cudaEventDisableTiming) != cudaSuccess)
+        return KDA_ERR_CUDA;
+    *out = &w;
     return KDA_OK;
 }
 
@@ -143,33 +192,88 @@ int kda_chunk_fwd(const void *q, const void *k, const void *v, const float *g, c
     if (current_status_word(&word) != KDA_OK) return KDA_ERR_CUDA;
     PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
     if (get_encoder(&enc) != KDA_OK) return KDA_ERR_CUDA;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return KDA_ERR_CUDA;
 
-    // Each CTA carries a 32-column slice of the value dimension.
-    const int vs = kda::chunk_value_slice();
-
-    CUtensorMap tq, tk, tv;
+    CUtensorMap tq, tk;
     if (make_map(&tq, enc, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dk, H, T, B, 64,
                  CU_TENSOR_MAP_SWIZZLE_128B) != KDA_OK ||
         make_map(&tk, enc, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dk, H, T, B, 64,
-                 CU_TENSOR_MAP_SWIZZLE_128B) != KDA_OK ||
-        make_map(&tv, enc, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dv, H, T, B, vs,
-                 CU_TENSOR_MAP_SWIZZLE_NONE) != KDA_OK)
+                 CU_TENSOR_MAP_SWIZZLE_128B) != KDA_OK)
         return KDA_ERR_CUDA;
 
-    kda::ChunkParams prm;
-    prm.beta = beta;
-    prm.h0 = h0;
-    prm.out = static_cast<uint16_t *>(out);
-    prm.hT = hT;
-    prm.scale = scale;
-    prm.B = B; prm.T = T; prm.H = H; prm.DV = dv;
-    prm.nslices = dv / vs;
-    prm.st.word = word;
+    const int nchunks = (T + kda::CH - 1) / kda::CH;
+    const int seg = segment_chunks(B, T, H);
+    const bool multi = seg < nchunks;
+    const size_t state_bytes = (multi && hT == nullptr) ? (size_t)B * H * dk * dv * sizeof(float) : 0;
+
+    std::lock_guard<std::mutex> lk(g_mu);
+    Workspace *w = nullptr;
+    if (int st = reserve_workspace(dev, (size_t)seg * rec_row_bytes(B, H), state_bytes, &w); st != KDA_OK)
+        return st;
+    if (cudaStreamWaitEvent(s, w->done, 0) != cudaSuccess) return KDA_ERR_CUDA;
+
     const unsigned long long polls = g_wait_polls.load();
-    prm.st.wait_polls = polls ? polls : ~0ull;
-    prm.inject_wait_polls = g_inject_polls.load();
-    cudaError_t e = kda::launch_chunk(tq, tk, tv, g, prm, dk, s);
-    return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+    kda::DeviceStatus dst;
+    dst.word = word;
+    dst.wait_polls = polls ? polls : ~0ull;
+    // State carried between segments: the caller's hT when given, else the workspace's.
+    float *carry = hT != nullptr ? hT : w->state;
+
+    for (int n0 = 0; n0 < nchunks; n0 += seg) {
+        const int cnt = nchunks - n0 < seg ? nchunks - n0 : seg;
+        const bool last = n0 + cnt == nchunks;
+        kda::PrepParams pp;
+        pp.g = g;
+        pp.beta = beta;
+        pp.ws = w->rec;
+        pp.B = B; pp.T = T; pp.H = H;
+        pp.n_begin = n0;
+        pp.nseg = cnt;
+        pp.st = dst;
+        cudaError_t e = kda::launch_prep(tq, tk, pp, dk, s);
+        if (e != cudaSuccess) return KDA_ERR_CUDA;
+
+        kda::ChainParams cp;
+        cp.v = static_cast<const uint16_t *>(v);
+        cp.h0 = n0 == 0 ? h0 : carry;
+        cp.out = static_cast<uint16_t *>(out);
+        cp.hT = last ? hT : carry;
+        cp.ws = w->rec;
+        cp.scale = scale;
+        cp.B = B; cp.T = T; cp.H = H; cp.DV = dv;
+        cp.n_begin = n0;
+        cp.nseg = cnt;
+        cp.nslices = 1;
+        cp.st = dst;
+        cp.inject_wait_polls = g_inject_polls.load();
+        e = kda::launch_chain(cp, dk, s);
+        if (e != cudaSuccess) return KDA_ERR_CUDA;
+    }
+    if (cudaEventRecord(w->done, s) != cudaSuccess) return KDA_ERR_CUDA;
+    return KDA_OK;
+}
+
+size_t kda_chunk_fwd_workspace_bytes(int B, int T, int H, int dk, int dv) {
+    if (B < 1 || H < 1 || T < 0 || (dk != 64 && dk != 128) || (dv != 64 && dv != 128)) return 0;
+    if (T == 0) return 0;
+    const int nchunks = (T + kda::CH - 1) / kda::CH;
+    const int seg = segment_chunks(B, T, H);
+    const size_t state = seg < nchunks ? (size_t)B * H * dk * dv * sizeof(float) : 0;
+    return (size_t)seg * rec_row_bytes(B, H) + state;
+}
+
+int kda_release_workspace(void) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return KDA_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_mu);
+    Workspace &w = g_ws[dev];
+    int st = KDA_OK;
+    if (w.rec != nullptr && cudaFree(w.rec) != cudaSuccess) st = KDA_ERR_CUDA;
+    if (w.state != nullptr && cudaFree(w.state) != cudaSuccess) st = KDA_ERR_CUDA;
+    w.rec = nullptr; w.rec_bytes = 0;
+    w.state = nullptr; w.state_bytes = 0;
+    return st;
 }
 
 int kda_decode_step(const void *q, const void *k, const void *v, const float *g, const float *beta,

@@ -1,0 +1,505 @@
+// prep_fwd.cu -- the intra-chunk half of the chunkwise KDA prefill (sm_100a).
+//
+// Per chunk of C = 64 tokens of one head (Gamma = inclusive running sum of g
+// inside the chunk, every exp factor per key channel):
+//   A_ij = beta_i sum_c k_ic k_jc e^{Gamma_ic - Gamma_jc}   (i > j, else 0)
+//   P_ij =        sum_c q_ic k_jc e^{Gamma_ic - Gamma_jc}   (i >= j, else 0)
+//   T    = (I + A)^{-1}                                   (unit lower)
+//   T'   = T Diag(beta),   W = T' (K * e^Gamma)
+//   plus Q * e^Gamma, K-hat = K * e^{Gamma_C - Gamma} and e^{Gamma_C}.
+// These are the intra-chunk pieces of the chunkwise rewrite of the KDA
+// recurrence (section 4 of "Kimi Linear's Hybrid Linear Attention
+// Architecture: A Technical Breakdown"), with the chunk's rank-1 updates
+// packed in the WY form (W, and U = T' V in the chain kernel).
+// None of them depends on the state, so every chunk is an independent CTA;
+// the result goes to a per-chunk record (layout in chunk_common.cuh).
+//
+// Decay factors.  e^{Gamma_i - Gamma_j} is split into two factors, one per
+// side of the contraction over key channels.  Rows of 16-token block I use
+// the reference m = 16 I + 8: row factor e^{Gamma_i - Gamma_m}, column factor
+// e^{Gamma_m - Gamma_j}.  For j in an earlier block both factors are <= 1; in
+// the block itself a factor can exceed 1 and is clamped at e^80, so results
+// are exact when a channel's log-decay over one aligned 16-token block is
+// >= -160.  All factors come from running products of alpha = e^g (one exp
+// per input element) plus one reciprocal per factor above 1.
+//
+// CTA: 512 threads; in the elementwise phase thread (c, I) owns key channel c
+// and tokens 16 I .. 16 I + 15 (a two-level scan: products inside the block,
+// then the four block totals through shared memory).  Phases:
+//   E  alpha, running products, operand tiles X, Y^(I) (bf16, smem) for the
+//      formation; Q e^G, K-hat (global record); (K e^G)^T (tf32, smem)
+//   F  X Y^(I)^T -> A, P                    (UMMA bf16, overlapped with E's tail)
+//   AP A -> fp32 scratch, P -> record
+//   T  (I + A)^{-1}: 16x16 diagonal blocks by substitution, off-diagonal blocks
+//      from N = D A_off as T = (I - N + N^2 - N^3) D, fp32 on CUDA cores
+//   W  T' = T Diag(beta) -> record;  W^T = (K e^G)^T T'^T  (UMMA tf32) -> record
+// Shared memory is 110 KB and TMEM 256 columns, so two CTAs share an SM.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "chunk_common.cuh"
+#include "chunk_params.cuh"
+#include "kda_device.cuh"
+
+namespace kda {
+
+constexpr int PREP_THREADS = 512;
+
+template <int DK>
+struct PrepLayout {
+    static_assert(DK == 64 || DK == 128, "dk");
+    // R_form: formation operands (E..F), then A, T scratch, T, the N/M scratch
+    static constexpr int OFF_F = 0;
+    static constexpr int OFF_XCH = OFF_F;                    // block products exchange (E only)
+    static constexpr int OFF_X = OFF_F;                      // MN-major bf16 [DK][128]
+    static constexpr int OFF_Y0 = OFF_X + DK * 256;          // SW32  [DK][16]
+    static constexpr int OFF_Y1 = OFF_Y0 + DK * 32;          // SW64  [DK][32]
+    static constexpr int OFF_Y2 = OFF_Y1 + DK * 64;          // SW128 [DK][64] (48 used)
+    static constexpr int OFF_Y3 = OFF_Y2 + DK * 128;         // SW128 [DK][64]
+    static constexpr int FORM_B = DK * (256 + 32 + 64 + 128 + 128);
+    static constexpr int OFF_A = OFF_F;                      // fp32 [64][A_LD]
+    static constexpr int OFF_TF = OFF_A + 64 * A_LD * 4;     // fp32 [64][A_LD]
+    static constexpr int OFF_T = OFF_F + align1k(2 * 64 * A_LD * 4);  // tf32 K-major [64][64], 8 KB K-blocks (+8 KB read overhang)
+    static constexpr int OFF_ZS = OFF_T + 24576;             // N / M scratch, 7 x 1 KB
+    static constexpr int POST_B = OFF_ZS + 7 * 1024 - OFF_F;
+    static constexpr int RF_B = align1k(cmax(FORM_B, POST_B));
+    // (K e^G)^T: tf32 K-major [128][64]; holds the q, k TMA tiles during E
+    static constexpr int OFF_BK = OFF_F + RF_B;
+    static constexpr int OFF_QIN = OFF_BK;                   // bf16 [64][DK], 128B swizzle
+    static constexpr int OFF_KIN = OFF_BK + CH * DK * 2;
+    static constexpr int OFF_MISC = OFF_BK + 128 * 64 * 4;   // beta, e^{Gamma_C}, barriers, TMEM address
+    static constexpr int TOTAL = OFF_MISC + 1024;
+    static constexpr int SMEM_BYTES = TOTAL + 1024;          // slack for the 1 KB base alignment
+    static_assert(SMEM_BYTES <= 113 * 1024, "two CTAs per SM");
+    static_assert(POST_B <= RF_B && FORM_B <= RF_B, "R_form");
+
+    static constexpr uint32_t TM_AP = 0;    // 160: formation products D^(I)
+    static constexpr uint32_t TM_W = 160;   // 64: W^T (lane = key channel, column = token)
+    static constexpr uint32_t TM_COLS = 256;
+};
+
+template <int DK>
+__global__ void __launch_bounds__(PREP_THREADS, 2)
+prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+            const PrepParams prm) {
+    using L = PrepLayout<DK>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    const uint32_t sbase = smem_u32(sm);
+
+    float *s_beta = reinterpret_cast<float *>(sm + L::OFF_MISC);        // [64]
+    float *s_xch = reinterpret_cast<float *>(sm + L::OFF_XCH);          // [2][4][128]
+    uint64_t *s_bars = reinterpret_cast<uint64_t *>(sm + L::OFF_MISC + 768);
+    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(sm + L::OFF_MISC + 800);
+    const uint32_t bar_in = smem_u32(&s_bars[0]);
+    const uint32_t bar_mma = smem_u32(&s_bars[1]);
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5, lane = tid & 31;
+    const int ch = tid & 127;        // key channel / TMEM lane of this thread
+    const int qb = tid >> 7;         // 16-token block (phase E) / 16-column quarter (elsewhere)
+    const int item = blockIdx.x;     // (b, h) major, chunk minor
+    const int ni = item % prm.nseg;
+    const int bh = item / prm.nseg;
+    const int h = bh % prm.H, b = bh / prm.H;
+    const int T = prm.T, H = prm.H;
+    const int n = prm.n_begin + ni;
+    const int t0 = n * CH;
+    uint8_t *rec = prm.ws + (size_t)item * REC_BYTES;
+    const uint64_t polls = prm.st.wait_polls;
+
+    if (tid == 0) {
+        mbar_init(bar_in, 1);
+        mbar_init(bar_mma, 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(smem_u32(s_tmem), L::TM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *s_tmem;
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+
+    bool tma_pending = false, mma_pending = false, aborted = false;
+    uint32_t ph_mma = 0;  // phase of bar_mma that the MMAs in flight complete
+    auto wait_all = [&](uint32_t bar, uint32_t ph, bool &pending) -> bool {
+        const bool ok = mbar_wait(bar, ph, polls, prm.st);
+        if (__syncthreads_or(!ok)) return false;
+        pending = false;
+        tc_fence_after();
+        return true;
+    };
+    auto sync_for_mma = [&]() {
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+    };
+
+    // ---------------- inputs: q, k by TMA; g (this thread's 16 tokens) and beta by plain loads
+    if (tid == 0) {
+        mbar_expect_tx(bar_in, (uint32_t)(2 * CH * DK * 2));
+#pragma unroll
+        for (int kb = 0; kb < DK / 64; ++kb) {
+            tma_load_4d(sbase + L::OFF_QIN + kb * CH * 128, &tm_q, bar_in, kb * 64, h, t0, b);
+            tma_load_4d(sbase + L::OFF_KIN + kb * CH * 128, &tm_k, bar_in, kb * 64, h, t0, b);
+        }
+    }
+    tma_pending = true;
+    const int c = ch, I = qb, tb = SUB * I;
+    const bool active = c < DK;
+    float al[SUB];
+    {
+        const float *gp = prm.g + (((size_t)b * T + t0 + tb) * H + h) * DK + c;
+#pragma unroll
+        for (int u = 0; u < SUB; ++u) al[u] = (t0 + tb + u < T && active) ? __ldg(gp + (size_t)u * H * DK) : 0.f;
+    }
+    if (tid < CH) s_beta[tid] = (t0 + tid < T) ? prm.beta[((size_t)b * T + t0 + tid) * H + h] : 0.f;
+    if (!wait_all(bar_in, 0, tma_pending)) aborted = true;
+
+    if (!aborted) {
+        // ---------------- E: decay factors and operand tiles ----------------
+        float kv[SUB], qv[SUB];
+        {
+            const uint8_t *qs = sm + L::OFF_QIN, *ks = sm + L::OFF_KIN;
+#pragma unroll
+            for (int u = 0; u < SUB; ++u) {
+                kv[u] = bf16_bits_to_f32(*reinterpret_cast<const uint16_t *>(ks + kmaj<128, 2>(tb + u, c, CH)));
+                qv[u] = bf16_bits_to_f32(*reinterpret_cast<const uint16_t *>(qs + kmaj<128, 2>(tb + u, c, CH)));
+            }
+        }
+        float lp[SUB];  // lp[u] = prod_{s=tb..tb+u} alpha_s
+        {
+            float p = 1.f;
+#pragma unroll
+            for (int u = 0; u < SUB; ++u) { al[u] = __expf(al[u]); p *= al[u]; lp[u] = p; }
+        }
+        if (active) { s_xch[I * 128 + c] = lp[SUB - 1]; s_xch[512 + I * 128 + c] = lp[SUB / 2]; }
+        __syncthreads();
+        float bt[NSUB], l8[NSUB];
+#pragma unroll
+        for (int J = 0; J < NSUB; ++J) { bt[J] = s_xch[J * 128 + c]; l8[J] = s_xch[512 + J * 128 + c]; }
+        __syncthreads();  // the exchange area becomes X; the q, k tiles are consumed
+        float ls[SUB];    // ls[u] = prod_{s=tb+u+1..tb+15} alpha_s
+        ls[SUB - 1] = 1.f;
+#pragma unroll
+        for (int u = SUB - 2; u >= 0; --u) ls[u] = ls[u + 1] * al[u + 1];
+        if (active) {
+            // Own block, reference m = tb + 8:
+            //   u >= 8: f_u = prod_{s=9..u} alpha     X = k f,   Y^(I) = k / f
+            //   u <  8: y_u = prod_{s=u+1..8} alpha   X = k / y, Y^(I) = k y
+            float xk[SUB], xq[SUB], yo[SUB];
+            {
+                float f = 1.f;
+#pragma unroll
+                for (int u = SUB / 2; u < SUB; ++u) {
+                    if (u > SUB / 2) f *= al[u];
+                    xk[u] = kv[u] * f;
+                    xq[u] = qv[u] * f;
+                    yo[u] = u == SUB / 2 ? kv[u] : kv[u] * rcp_clamped(f);
+                }
+                float y = 1.f;
+#pragma unroll
+                for (int u = SUB / 2 - 1; u >= 0; --u) {
+                    y *= al[u + 1];
+                    const float r = rcp_clamped(y);
+                    xk[u] = kv[u] * r;
+                    xq[u] = qv[u] * r;
+                    yo[u] = kv[u] * y;
+                }
+            }
+            auto yput = [&](int Iy, int j0, const float *v) {
+                float v8[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) v8[e] = v[e];
+                if (Iy == 0)      *reinterpret_cast<uint4 *>(sm + L::OFF_Y0 + mnmaj<32, 2>(c, j0, DK)) = pack8_bf16(v8);
+                else if (Iy == 1) *reinterpret_cast<uint4 *>(sm + L::OFF_Y1 + mnmaj<64, 2>(c, j0, DK)) = pack8_bf16(v8);
+                else if (Iy == 2) *reinterpret_cast<uint4 *>(sm + L::OFF_Y2 + mnmaj<128, 2>(c, j0, DK)) = pack8_bf16(v8);
+                else              *reinterpret_cast<uint4 *>(sm + L::OFF_Y3 + mnmaj<128, 2>(c, j0, DK)) = pack8_bf16(v8);
+            };
+#pragma unroll
+            for (int h8 = 0; h8 < 2; ++h8) {
+                float a8[8], b8[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) { a8[e] = xk[h8 * 8 + e]; b8[e] = xq[h8 * 8 + e]; }
+                *reinterpret_cast<uint4 *>(sm + L::OFF_X + mnmaj<128, 2>(c, tb + h8 * 8, DK)) = pack8_bf16(a8);
+                *reinterpret_cast<uint4 *>(sm + L::OFF_X + mnmaj<128, 2>(c, 64 + tb + h8 * 8, DK)) = pack8_bf16(b8);
+                yput(I, tb + h8 * 8, yo + h8 * 8);
+            }
+            // Later blocks I' > I see this block through e^{Gamma_{m'} - Gamma_j}
+            //   = ls_u * prod_{J = I+1 .. I'-1} bt_J * l8_{I'}   (all factors <= 1)
+            float mid = 1.f;
+#pragma unroll
+            for (int Ip = 1; Ip < NSUB; ++Ip) {
+                if (Ip > I) {
+                    const float sc = mid * l8[Ip];
+                    float yv[SUB];
+#pragma unroll
+                    for (int u = 0; u < SUB; ++u) yv[u] = kv[u] * (ls[u] * sc);
+                    yput(Ip, tb, yv);
+                    yput(Ip, tb + 8, yv + 8);
+                    mid *= bt[Ip];
+                }
+            }
+        }
+        sync_for_mma();
+
+        // ---------------- F: formation products (bf16), overlapped with the rest of E ----------------
+        if (tid == 0) {
+#pragma unroll
+            for (int If = 0; If < NSUB; ++If) {
+                const uint32_t idesc = make_idesc(1, true, true, 128, SUB * (If + 1));
+#pragma unroll
+                for (int kk = 0; kk < DK / 16; ++kk) {
+                    const uint64_t da = desc_mnmaj<128>(sbase + L::OFF_X, DK, kk * 16);
+                    uint64_t db;
+                    if (If == 0)      db = desc_mnmaj<32>(sbase + L::OFF_Y0, DK, kk * 16);
+                    else if (If == 1) db = desc_mnmaj<64>(sbase + L::OFF_Y1, DK, kk * 16);
+                    else if (If == 2) db = desc_mnmaj<128>(sbase + L::OFF_Y2, DK, kk * 16);
+                    else              db = desc_mnmaj<128>(sbase + L::OFF_Y3, DK, kk * 16);
+                    umma<0>(tmem + L::TM_AP + yoff(If), da, db, idesc, kk > 0);
+                }
+            }
+            umma_commit(bar_mma);
+        }
+        mma_pending = true;
+
+        if (active) {
+            float preB = 1.f, postB = 1.f;
+#pragma unroll
+            for (int J = 0; J < NSUB; ++J) { if (J < I) preB *= bt[J]; if (J > I) postB *= bt[J]; }
+            if (I == 0) reinterpret_cast<float *>(rec + REC_DEC)[c] = bt[0] * bt[1] * bt[2] * bt[3];
+            // e^{Gamma_t}: Q e^G (record, WQ columns 64..) and (K e^G)^T (smem);
+            // e^{Gamma_C - Gamma_t}: K-hat^T (record)
+#pragma unroll
+            for (int h8 = 0; h8 < 2; ++h8) {
+                float qe[8], bk[8], kh[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int u = h8 * 8 + e;
+                    const float pre = preB * lp[u];
+                    qe[e] = qv[u] * pre;
+                    bk[e] = kv[u] * pre;
+                    kh[e] = kv[u] * (ls[u] * postB);
+                }
+                const int t8 = tb + h8 * 8;
+                *reinterpret_cast<uint4 *>(rec + REC_WQ + mnmaj<128, 2>(c, 64 + t8, DK)) = pack8_bf16(qe);
+                *reinterpret_cast<uint4 *>(sm + L::OFF_BK + kmaj<128, 4>(c, t8, 128)) = pack4_tf32(bk[0], bk[1], bk[2], bk[3]);
+                *reinterpret_cast<uint4 *>(sm + L::OFF_BK + kmaj<128, 4>(c, t8 + 4, 128)) = pack4_tf32(bk[4], bk[5], bk[6], bk[7]);
+                *reinterpret_cast<uint4 *>(rec + REC_KH + kmaj<128, 4>(c, t8, 128)) = pack4_tf32(kh[0], kh[1], kh[2], kh[3]);
+                *reinterpret_cast<uint4 *>(rec + REC_KH + kmaj<128, 4>(c, t8 + 4, 128)) = pack4_tf32(kh[4], kh[5], kh[6], kh[7]);
+            }
+        }
+        if (!wait_all(bar_mma, 0, mma_pending)) aborted = true;
+        else ph_mma = 1;
+    }
+
+    if (!aborted) {
+        // ---------------- AP: A -> fp32 scratch, P -> record ----------------
+        // TMEM lane = row of [k; q]; the four warps of a lane quarter take one
+        // 16-column chunk each (chunk = qb).
+        {
+            float *sA = reinterpret_cast<float *>(sm + L::OFF_A);
+            const int i = ch & 63;
+            const int myI = i / SUB;
+            const bool is_q = ch >= 64;
+            const float bi = s_beta[i];
+            const int I0 = ((warp & 1) * 32) / SUB;  // the lane quarter covers blocks I0, I0 + 1
+            const int cc = qb;
+            float v16[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) v16[e] = 0.f;
+#pragma unroll
+            for (int dI = 0; dI < 2; ++dI) {
+                const int Ib = I0 + dI;
+                if (cc <= Ib) {
+                    float t[16];
+                    tmem_ld16(tmem + lane_base + L::TM_AP + yoff(Ib) + cc * 16, t);
+                    tmem_wait_ld();
+                    if (myI == Ib) {
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) v16[e] = t[e];
+                    }
+                }
+            }
+            const int j0 = cc * 16;
+            if (!is_q) {
+#pragma unroll
+                for (int e = 0; e < 16; e += 4) {
+                    float4 w;
+                    w.x = (j0 + e + 0 < i) ? bi * v16[e + 0] : 0.f;
+                    w.y = (j0 + e + 1 < i) ? bi * v16[e + 1] : 0.f;
+                    w.z = (j0 + e + 2 < i) ? bi * v16[e + 2] : 0.f;
+                    w.w = (j0 + e + 3 < i) ? bi * v16[e + 3] : 0.f;
+                    *reinterpret_cast<float4 *>(sA + i * A_LD + j0 + e) = w;
+                }
+            } else {
+#pragma unroll
+                for (int e = 0; e < 16; e += 4) {
+                    const uint4 w = pack4_tf32((j0 + e + 0 <= i) ? v16[e + 0] : 0.f, (j0 + e + 1 <= i) ? v16[e + 1] : 0.f,
+                                               (j0 + e + 2 <= i) ? v16[e + 2] : 0.f, (j0 + e + 3 <= i) ? v16[e + 3] : 0.f);
+                    *reinterpret_cast<uint4 *>(rec + REC_P + kmaj_s<128, 4>(i, j0 + e, 8192)) = w;
+                }
+            }
+        }
+        tc_fence_before();
+        __syncthreads();
+
+        // ---------------- T: (I + A)^{-1}, fp32 ----------------
+        {
+            const float *sA = reinterpret_cast<const float *>(sm + L::OFF_A);
+            float *sTf = reinterpret_cast<float *>(sm + L::OFF_TF);
+            float *sZ = reinterpret_cast<float *>(sm + L::OFF_ZS);
+            // diagonal 16x16 blocks: thread (I, jj) solves column jj of (I + A_II) x = e_jj
+            if (tid < 64) {
+                const int Ib = tid >> 4, jj = tid & 15, base = SUB * Ib;
+                float x[SUB];
+#pragma unroll
+                for (int ii = 0; ii < SUB; ++ii) {
+                    float acc = (ii == jj) ? 1.f : 0.f;
+#pragma unroll
+                    for (int mm = 0; mm < ii; ++mm) acc -= sA[(base + ii) * A_LD + base + mm] * x[mm];
+                    x[ii] = (ii < jj) ? 0.f : acc;
+                }
+#pragma unroll
+                for (int ii = 0; ii < SUB; ++ii) sTf[(base + ii) * A_LD + base + jj] = x[ii];
+            }
+            __syncthreads();
+            // Off-diagonal blocks.  With D = diag(T_II) and N = D A_offdiag (strictly block
+            // lower, N^4 = 0):  T = (I - N + N^2 - N^3) D, i.e. T_IJ = M_IJ T_JJ with
+            //   M_{I,I-1} = -N_{I,I-1},  M_20 = -N_20 + N_21 N_10,  M_31 = -N_31 + N_32 N_21,
+            //   M_30 = -N_30 + N_31 N_10 - N_32 M_20.
+            // Scratch slots (16x16, row stride 16): 0 N10, 1 N20, 2 N21, 3 N30, 4 N31, 5 N32, 6 M31.
+            // One warp per 16x16 product; lane (r = lane / 2, c0 = 8 (lane % 2)) owns 8 outputs.
+            {
+                const int r = lane >> 1, c0 = (lane & 1) * 8;
+                auto rowblk = [&](const float *arow, const float *bblk, int bld, float (&o)[8]) {
+#pragma unroll
+                    for (int m4 = 0; m4 < SUB; m4 += 4) {
+                        const float4 a4 = *reinterpret_cast<const float4 *>(arow + m4);
+                        const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+                        for (int mm = 0; mm < 4; ++mm) {
+                            const float *brow = bblk + (m4 + mm) * bld + c0;
+                            const float4 b0 = *reinterpret_cast<const float4 *>(brow);
+                            const float4 b1 = *reinterpret_cast<const float4 *>(brow + 4);
+                            o[0] += av[mm] * b0.x; o[1] += av[mm] * b0.y; o[2] += av[mm] * b0.z; o[3] += av[mm] * b0.w;
+                            o[4] += av[mm] * b1.x; o[5] += av[mm] * b1.y; o[6] += av[mm] * b1.z; o[7] += av[mm] * b1.w;
+                        }
+                    }
+                };
+                auto store8 = [&](float *dst, const float (&o)[8], float sgn) {
+                    *reinterpret_cast<float4 *>(dst) = make_float4(sgn * o[0], sgn * o[1], sgn * o[2], sgn * o[3]);
+                    *reinterpret_cast<float4 *>(dst + 4) = make_float4(sgn * o[4], sgn * o[5], sgn * o[6], sgn * o[7]);
+                };
+                const int BI = warp == 0 ? 1 : (warp < 3 ? 2 : 3);            // block pair of warp < 6:
+                const int BJ = warp == 0 ? 0 : (warp < 3 ? warp - 1 : warp - 3);  // (1,0) (2,0) (2,1) (3,0) (3,1) (3,2)
+                if (warp < 6) {  // N_IJ = T_II A_IJ
+                    float o[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                    rowblk(sTf + (SUB * BI + r) * A_LD + SUB * BI, sA + (SUB * BI) * A_LD + SUB * BJ, A_LD, o);
+                    store8(sZ + warp * 256 + r * 16 + c0, o, 1.f);
+                }
+                __syncthreads();
+                if (warp < 2) {  // M20 = -N20 + N21 N10 (slot 1);  M31 = -N31 + N32 N21 (slot 6)
+                    const int so = warp == 0 ? 1 : 4, sa = warp == 0 ? 2 : 5, sb = warp == 0 ? 0 : 2;
+                    float o[8];
+                    const float *own = sZ + so * 256 + r * 16 + c0;
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) o[e] = -own[e];
+                    rowblk(sZ + sa * 256 + r * 16, sZ + sb * 256, 16, o);
+                    store8(sZ + (warp == 0 ? 1 : 6) * 256 + r * 16 + c0, o, 1.f);
+                }
+                __syncthreads();
+                if (warp == 0) {  // M30 = -N30 + N31 N10 - N32 M20 (slot 3)
+                    float o[8], o2[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                    const float *own = sZ + 3 * 256 + r * 16 + c0;
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) o[e] = -own[e];
+                    rowblk(sZ + 4 * 256 + r * 16, sZ + 0 * 256, 16, o);
+                    rowblk(sZ + 5 * 256 + r * 16, sZ + 1 * 256, 16, o2);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) o[e] -= o2[e];
+                    store8(sZ + 3 * 256 + r * 16 + c0, o, 1.f);
+                }
+                __syncthreads();
+                if (warp < 6) {  // T_IJ = M_IJ T_JJ; adjacent blocks carry M = -N
+                    const int msl = warp == 4 ? 6 : warp;
+                    const float sgn = (warp == 0 || warp == 2 || warp == 5) ? -1.f : 1.f;
+                    float o[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                    rowblk(sZ + msl * 256 + r * 16, sTf + (SUB * BJ) * A_LD + SUB * BJ, A_LD, o);
+                    store8(sTf + (SUB * BI + r) * A_LD + SUB * BJ + c0, o, sgn);
+                }
+                __syncthreads();
+            }
+            // T' = T Diag(beta) -> tf32 K-major tile (smem operand of W, and the record),
+            // zeros above the diagonal
+            for (int e = tid; e < 64 * 16; e += PREP_THREADS) {
+                const int i = e >> 4, j = (e & 15) * 4;
+                const float *src = sTf + i * A_LD + j;
+                const float4 bj = *reinterpret_cast<const float4 *>(s_beta + j);
+                const uint4 w = pack4_tf32(j + 0 <= i ? src[0] * bj.x : 0.f, j + 1 <= i ? src[1] * bj.y : 0.f,
+                                           j + 2 <= i ? src[2] * bj.z : 0.f, j + 3 <= i ? src[3] * bj.w : 0.f);
+                const uint32_t off = kmaj_s<128, 4>(i, j, 8192);
+                *reinterpret_cast<uint4 *>(sm + L::OFF_T + off) = w;
+                *reinterpret_cast<uint4 *>(rec + REC_T + off) = w;
+            }
+        }
+        sync_for_mma();
+
+        // ---------------- W: W^T = (K e^G)^T T'^T  (tf32) ----------------
+        if (tid == 0) {
+            const uint32_t id_w = make_idesc(2, false, false, 128, 64);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+                umma<1>(tmem + L::TM_W, desc_kmaj_s<128, 4>(sbase + L::OFF_BK, 128 * 128, kk * 8),
+                        desc_kmaj_s<128, 4>(sbase + L::OFF_T, 8192, kk * 8), id_w, kk > 0);
+            umma_commit(bar_mma);
+        }
+        mma_pending = true;
+        if (!wait_all(bar_mma, 1, mma_pending)) aborted = true;
+    }
+    if (!aborted && (warp & 3) < DK / 32) {  // W^T row ch -> W columns (tokens 16 qb ..) of the record's WQ
+        const int i0 = qb * 16;
+        float t[16];
+        tmem_ld16(tmem + lane_base + L::TM_W + i0, t);
+        tmem_wait_ld();
+        float a8[8], b8[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) { a8[e] = t[e]; b8[e] = t[8 + e]; }
+        *reinterpret_cast<uint4 *>(rec + REC_WQ + mnmaj<128, 2>(ch, i0, DK)) = pack8_bf16(a8);
+        *reinterpret_cast<uint4 *>(rec + REC_WQ + mnmaj<128, 2>(ch, i0 + 8, DK)) = pack8_bf16(b8);
+    }
+
+    if (aborted && tid == 0) {
+        // Leave nothing in flight that targets this CTA's smem or TMEM.
+        if (tma_pending) mbar_wait(bar_in, 0, ~0ull, prm.st);
+        if (mma_pending) mbar_wait(bar_mma, ph_mma, ~0ull, prm.st);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tmem, L::TM_COLS);
+}
+
+template <int DK>
+static cudaError_t launch_prep_t(const CUtensorMap &tq, const CUtensorMap &tk, const PrepParams &prm,
+                                 cudaStream_t stream) {
+    using L = PrepLayout<DK>;
+    cudaError_t e = cudaFuncSetAttribute(prep_kernel<DK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         L::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    prep_kernel<DK><<<prm.B * prm.H * prm.nseg, PREP_THREADS, L::SMEM_BYTES, stream>>>(tq, tk, prm);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_prep(const CUtensorMap &tq, const CUtensorMap &tk, const PrepParams &prm, int dk,
+                        cudaStream_t stream) {
+    if (dk == 128) return launch_prep_t<128>(tq, tk, prm, stream);
+    return launch_prep_t<64>(tq, tk, prm, stream);
+}
+
+}  // namespace kda

@@ -6,6 +6,8 @@ The entry points mirror ``include/kda.h``:
 * ``chunk_fwd``   -> ``kda_chunk_fwd``   (chunkwise prefill)
 * ``decode_step`` -> ``kda_decode_step`` (one recurrent step, state in place)
 * ``stream_status`` -> ``kda_stream_status``
+* ``workspace_bytes`` / ``release_workspace`` -> ``kda_chunk_fwd_workspace_bytes`` /
+  ``kda_release_workspace``
 
 plus ``chunk_fwd_host``, the same prefill for host (pinned) tensors: it copies
 the inputs to the device, runs ``kda_chunk_fwd`` and copies the results back,
@@ -24,8 +26,9 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libkda.so")
 
 KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_ALIGNMENT, KDA_ERR_CUDA, KDA_ERR_TIMEOUT = range(6)
-EXPORTED = ("kda_chunk_fwd", "kda_decode_step", "kda_status_string", "kda_stream_status",
-            "kda_chunk_fwd_debug_wait_limit", "kda_chunk_fwd_debug_inject_timeout", "kda_abi_version")
+EXPORTED = ("kda_chunk_fwd", "kda_decode_step", "kda_chunk_fwd_workspace_bytes", "kda_release_workspace",
+            "kda_status_string", "kda_stream_status", "kda_chunk_fwd_debug_wait_limit",
+            "kda_chunk_fwd_debug_inject_timeout", "kda_abi_version")
 
 _lib = None
 
@@ -50,6 +53,10 @@ def load():
     lib.kda_chunk_fwd.restype = i
     lib.kda_decode_step.argtypes = [vp, vp, vp, fp, fp, f, fp, vp, i, i, i, i, vp]
     lib.kda_decode_step.restype = i
+    lib.kda_chunk_fwd_workspace_bytes.argtypes = [i, i, i, i, i]
+    lib.kda_chunk_fwd_workspace_bytes.restype = ctypes.c_size_t
+    lib.kda_release_workspace.argtypes = []
+    lib.kda_release_workspace.restype = i
     lib.kda_status_string.argtypes = [i]
     lib.kda_status_string.restype = ctypes.c_char_p
     lib.kda_stream_status.argtypes = [vp]
@@ -134,6 +141,18 @@ def decode_step(q, k, v, g, beta, scale, state, *, out=None, stream=None):
     if rc != KDA_OK:
         raise KdaError(rc, "kda_decode_step")
     return out
+
+
+def workspace_bytes(B: int, T: int, H: int, dk: int, dv: int) -> int:
+    """Device memory ``chunk_fwd`` holds for these sizes (0 when unsupported)."""
+    return int(load().kda_chunk_fwd_workspace_bytes(int(B), int(T), int(H), int(dk), int(dv)))
+
+
+def release_workspace() -> None:
+    """Free the current device's prefill workspace (synchronises the device)."""
+    rc = load().kda_release_workspace()
+    if rc != KDA_OK:
+        raise KdaError(rc, "kda_release_workspace")
 
 
 def stream_status(stream=None) -> int:

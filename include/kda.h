@@ -21,10 +21,10 @@
  * - All pointers are DEVICE pointers (cudaMalloc / torch CUDA tensors) on the
  *   current device, row-major and contiguous, 16-byte aligned (beta: 4-byte).
  * - bf16 tensors are passed as void* holding IEEE bfloat16 (uint16 bits).
- * - The caller owns every buffer.  The library keeps no pointer after a call
- *   returns and allocates no device memory for the data path.  The only
- *   library-owned device memory is one 4-byte status word per device,
- *   created on first use.
+ * - The caller owns every buffer it passes.  The library keeps no pointer to
+ *   them after a call returns.  Library-owned device memory: one 4-byte status
+ *   word per device (part of the module image), and the prefill workspace
+ *   described at kda_chunk_fwd_workspace_bytes().
  * - Work is enqueued on `stream` (a cudaStream_t, NULL = legacy default
  *   stream) and the call returns without synchronising.  The return value
  *   reports argument validation and launch errors only.  Device-side
@@ -42,6 +42,8 @@
  */
 #ifndef KDA_H_
 #define KDA_H_
+
+#include <stddef.h>
 
 #if defined(__GNUC__)
 #define KDA_API __attribute__((visibility("default")))
@@ -77,10 +79,20 @@ typedef enum {
  *   stream: cudaStream_t
  *
  * Internally each sequence is cut into chunks of 64 tokens; the last chunk of
- * a sequence may be partial.  The state is carried in fp32 from chunk to
- * chunk; the chunk contractions run on the tcgen05 tensor cores with fp32
- * accumulation.  T == 0 copies h0 to hT (or zeroes hT) and writes no output;
- * q, k, v, g, beta and out are then not read and may be NULL.
+ * a sequence may be partial.  Two kernels run per segment of chunks: one
+ * builds every chunk's state-independent pieces in parallel (decay-scaled
+ * operands, the intra-chunk blocks, the inverse of the unit-lower system and
+ * the WY factors) into the workspace; the other walks the chunks of each
+ * (b, h) in order, carrying the state in fp32.  The chunk contractions run on
+ * the tcgen05 tensor cores with fp32 accumulation.  T == 0 copies h0 to hT
+ * (or zeroes hT) and writes no output; q, k, v, g, beta and out are then not
+ * read and may be NULL.
+ *
+ * Workspace: the first call on a device, and any call that needs more than
+ * the workspace held so far, allocates it with cudaMalloc (freeing the old
+ * one first, which synchronises the device), so make such a call before any
+ * stream capture.  Calls on different streams are ordered on the workspace by
+ * an event.  Allocation failure returns KDA_ERR_CUDA.
  */
 KDA_API int kda_chunk_fwd(const void *q, const void *k, const void *v,
                   const float *g, const float *beta, float scale,
@@ -107,6 +119,22 @@ KDA_API int kda_decode_step(const void *q, const void *k, const void *v,
                     const float *g, const float *beta, float scale,
                     float *state, void *out,
                     int B, int H, int dk, int dv, void *stream);
+
+/*
+ * kda_chunk_fwd_workspace_bytes -- device memory kda_chunk_fwd holds for these
+ * sizes: the per-chunk records of one segment (about 97 KB per 64-token chunk
+ * and (b, h); a segment spans as many chunks as fit in 2 GiB, at least one)
+ * plus, when the sequence takes more than one segment, an fp32 state buffer
+ * [B, H, dk, dv].  0 for unsupported sizes or T == 0.
+ */
+KDA_API size_t kda_chunk_fwd_workspace_bytes(int B, int T, int H, int dk, int dv);
+
+/*
+ * kda_release_workspace -- free the current device's prefill workspace (the
+ * next kda_chunk_fwd allocates it again).  cudaFree synchronises the device,
+ * so no launched work still uses it.  KDA_OK, or KDA_ERR_CUDA.
+ */
+KDA_API int kda_release_workspace(void);
 
 /* Human-readable name of a kda_status value (static string, never NULL). */
 KDA_API const char *kda_status_string(int status);
