@@ -18,7 +18,8 @@ Also measured and reported in the same line:
            512 MiB fp32 state (GB/s of algorithmic traffic);
   e2e      the same prefill metric through the public API with pinned host
            buffers: H2D of the inputs, the kernel, D2H of out and hT per step;
-  roofline achieved algorithmic GB/s of the prefill kernel vs measured HBM peak;
+  roofline achieved algorithmic GB/s of the prefill call (its two kernels, timed
+           per launch with CUDA events on the stream) vs measured HBM peak;
   cpu_baseline  the fp64 oracle on a bounded sample of the workload (rank 0,
            N = 1 only).
 
@@ -285,6 +286,8 @@ def run_ours(args):
     if kda.stream_status(stream) != kda.KDA_OK:
         raise RuntimeError("device-side error during warm-up")
 
+    kda.kernel_times()  # forget launches timed before this point (none: the hook is off)
+    kda.kernel_timing(True)
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
     with ClockSampler(local) as clk:
         barrier(world)
@@ -295,8 +298,10 @@ def run_ours(args):
             ev[i + 1].record(stream)
         torch.cuda.synchronize()
         barrier(world)
+    kda.kernel_timing(False)
     if kda.stream_status(stream) != kda.KDA_OK:
         raise RuntimeError("device-side error in the timed region")
+    ktimes = kda.kernel_times()
     launch_ms = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
     total_ms = ev[0].elapsed_time(ev[-1])
     total_ms = max_over_ranks(total_ms, world, dev)
@@ -308,10 +313,15 @@ def run_ours(args):
     nflops = prefill_flops(cfg.B, cfg.T, cfg.H, cfg.dk, cfg.dv)
     avg_launch_s = statistics.mean(launch_ms) / 1e3
     achieved = nbytes / avg_launch_s / 1e9
-    roof = {"kernel": "chunk_fwd_kernel", "bound": "hbm", "achieved": achieved, "peak": P["hbm_gbs"],
-            "unit": "GB/s", "frac": achieved / P["hbm_gbs"], "peak_source": peak_src,
-            "traffic": measured_traffic("chunk_fwd_kernel"),
-            "algorithmic_bytes_per_launch": nbytes,
+    kernel_ms = sum(t for t, _ in ktimes.values())
+    kernels = {k: {"ms_per_step": t / args.steps, "launches_per_step": n / args.steps,
+                   "share": t / kernel_ms if kernel_ms > 0 else None}
+               for k, (t, n) in ktimes.items()}
+    gpu_launches = sum(n for _, n in ktimes.values())
+    roof = {"kernel": "kda_chunk_fwd (prep_kernel + chain_kernel)", "bound": "hbm", "achieved": achieved,
+            "peak": P["hbm_gbs"], "unit": "GB/s", "frac": achieved / P["hbm_gbs"], "peak_source": peak_src,
+            "traffic": measured_traffic("kda_chunk_fwd"),
+            "algorithmic_bytes_per_launch": nbytes, "kernels": kernels,
             "tensor_view": {"achieved_tflops": nflops / avg_launch_s / 1e12,
                             "peak_tflops": P["bf16_tflops_sustained"],
                             "frac": nflops / avg_launch_s / 1e12 / P["bf16_tflops_sustained"]}}
@@ -395,7 +405,7 @@ def run_ours(args):
                        "parallelism": f"weak: one workload copy per GPU x{world}"},
             "tflops": nflops / (ms_per_step / 1e3) / 1e12 * world,
             "roofline": roof, "decode": dec, "e2e": e2e, "cpu_baseline": cpu,
-            "clocks": clk.summary(), "gpu_launches": args.steps,
+            "clocks": clk.summary(), "gpu_launches": gpu_launches,
             "launch_ms": {"mean": statistics.mean(launch_ms), "min": min(launch_ms), "max": max(launch_ms)},
         }
         print(json.dumps(line), flush=True)

@@ -8,6 +8,8 @@
 
 #include <atomic>
 #include <mutex>
+#include <utility>
+#include <vector>
 
 #include "../../include/kda.h"
 #include "kda_device.cuh"
@@ -113,6 +115,43 @@ int reserve_workspace(int dev, size_t rec_bytes, size_t state_bytes, Workspace *
         return KDA_ERR_CUDA;
     *out = &w;
     return KDA_OK;
+}
+
+// Per-kernel timing hook (measurement only): CUDA events recorded on the
+// launching stream around every prefill kernel while enabled.
+constexpr int kKernelKinds = 2;  // 0 = prep, 1 = chain
+struct TimedLaunch {
+    int dev, kind;
+    cudaEvent_t start, stop;
+};
+std::atomic<int> g_timing{0};
+std::vector<TimedLaunch> g_timed;            // recorded, not yet read
+std::vector<std::pair<int, cudaEvent_t>> g_event_pool;  // (device, event)
+
+cudaEvent_t pooled_event(int dev) {  // called with g_mu held
+    for (size_t i = 0; i < g_event_pool.size(); ++i) {
+        if (g_event_pool[i].first == dev) {
+            cudaEvent_t e = g_event_pool[i].second;
+            g_event_pool.erase(g_event_pool.begin() + i);
+            return e;
+        }
+    }
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    return e;
+}
+
+// Launch `fn` on `s`, bracketed by timing events when the hook is on.
+template <class F>
+cudaError_t timed_launch(int dev, int kind, cudaStream_t s, F &&fn) {
+    if (!g_timing.load()) return fn();
+    cudaEvent_t a = pooled_event(dev), b = pooled_event(dev);
+    if (a == nullptr || b == nullptr) return cudaErrorMemoryAllocation;
+    cudaError_t e = cudaEventRecord(a, s);
+    if (e == cudaSuccess) e = fn();
+    if (e == cudaSuccess) e = cudaEventRecord(b, s);
+    g_timed.push_back({dev, kind, a, b});
+    return e;
 }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -231,7 +270,7 @@ int kda_chunk_fwd(const void *q, const void *k, const void *v, const float *g, c
         pp.n_begin = n0;
         pp.nseg = cnt;
         pp.st = dst;
-        cudaError_t e = kda::launch_prep(tq, tk, pp, dk, s);
+        cudaError_t e = timed_launch(dev, 0, s, [&] { return kda::launch_prep(tq, tk, pp, dk, s); });
         if (e != cudaSuccess) return KDA_ERR_CUDA;
 
         kda::ChainParams cp;
@@ -247,7 +286,7 @@ int kda_chunk_fwd(const void *q, const void *k, const void *v, const float *g, c
         cp.nslices = 1;
         cp.st = dst;
         cp.inject_wait_polls = g_inject_polls.load();
-        e = kda::launch_chain(cp, dk, s);
+        e = timed_launch(dev, 1, s, [&] { return kda::launch_chain(cp, dk, s); });
         if (e != cudaSuccess) return KDA_ERR_CUDA;
     }
     if (cudaEventRecord(w->done, s) != cudaSuccess) return KDA_ERR_CUDA;
@@ -261,6 +300,25 @@ size_t kda_chunk_fwd_workspace_bytes(int B, int T, int H, int dk, int dv) {
     const int seg = segment_chunks(B, T, H);
     const size_t state = seg < nchunks ? (size_t)B * H * dk * dv * sizeof(float) : 0;
     return (size_t)seg * rec_row_bytes(B, H) + state;
+}
+
+void kda_debug_kernel_timing(int enable) { g_timing.store(enable != 0); }
+
+int kda_debug_kernel_times(double *ms, long long *launches, int nkinds) {
+    if (ms == nullptr || launches == nullptr || nkinds < 0) return KDA_ERR_INVALID_ARG;
+    for (int i = 0; i < nkinds; ++i) { ms[i] = 0.0; launches[i] = 0; }
+    std::lock_guard<std::mutex> lk(g_mu);
+    int st = KDA_OK;
+    for (const TimedLaunch &t : g_timed) {
+        float e_ms = 0.f;
+        if (cudaEventSynchronize(t.stop) != cudaSuccess || cudaEventElapsedTime(&e_ms, t.start, t.stop) != cudaSuccess)
+            st = KDA_ERR_CUDA;
+        if (t.kind < nkinds) { ms[t.kind] += e_ms; launches[t.kind] += 1; }
+        g_event_pool.push_back({t.dev, t.start});
+        g_event_pool.push_back({t.dev, t.stop});
+    }
+    g_timed.clear();
+    return st;
 }
 
 int kda_release_workspace(void) {

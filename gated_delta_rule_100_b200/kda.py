@@ -28,7 +28,8 @@ LIB_PATH = os.path.join(_HERE, "libkda.so")
 KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_ALIGNMENT, KDA_ERR_CUDA, KDA_ERR_TIMEOUT = range(6)
 EXPORTED = ("kda_chunk_fwd", "kda_decode_step", "kda_chunk_fwd_workspace_bytes", "kda_release_workspace",
             "kda_status_string", "kda_stream_status", "kda_chunk_fwd_debug_wait_limit",
-            "kda_chunk_fwd_debug_inject_timeout", "kda_abi_version")
+            "kda_chunk_fwd_debug_inject_timeout", "kda_debug_kernel_timing", "kda_debug_kernel_times",
+            "kda_abi_version")
 
 _lib = None
 
@@ -65,6 +66,10 @@ def load():
     lib.kda_chunk_fwd_debug_wait_limit.restype = None
     lib.kda_chunk_fwd_debug_inject_timeout.argtypes = [ctypes.c_ulonglong]
     lib.kda_chunk_fwd_debug_inject_timeout.restype = None
+    lib.kda_debug_kernel_timing.argtypes = [i]
+    lib.kda_debug_kernel_timing.restype = None
+    lib.kda_debug_kernel_times.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_longlong), i]
+    lib.kda_debug_kernel_times.restype = i
     lib.kda_abi_version.restype = i
     _lib = lib
     return lib
@@ -169,6 +174,25 @@ def inject_timeout(polls: int) -> None:
     """Test hook: nonzero makes each prefill CTA first wait on a barrier nothing
     signals (at most ``polls`` polls) and take its timeout path; 0 = off."""
     load().kda_chunk_fwd_debug_inject_timeout(int(polls))
+
+
+KERNEL_KINDS = ("prep", "chain")
+
+
+def kernel_timing(enable: bool) -> None:
+    """Measurement hook: time every prefill kernel launch with CUDA events."""
+    load().kda_debug_kernel_timing(1 if enable else 0)
+
+
+def kernel_times() -> dict:
+    """{kind: (ms summed, launches)} of the launches timed since the last call."""
+    n = len(KERNEL_KINDS)
+    ms = (ctypes.c_double * n)()
+    cnt = (ctypes.c_longlong * n)()
+    rc = load().kda_debug_kernel_times(ms, cnt, n)
+    if rc != KDA_OK:
+        raise KdaError(rc, "kda_debug_kernel_times")
+    return {k: (ms[i], int(cnt[i])) for i, k in enumerate(KERNEL_KINDS)}
 
 
 class DeviceBuffers:

@@ -166,6 +166,20 @@ KDA_API void kda_chunk_fwd_debug_wait_limit(unsigned long long polls);
  */
 KDA_API void kda_chunk_fwd_debug_inject_timeout(unsigned long long polls);
 
+/*
+ * kda_debug_kernel_timing -- measurement hook.  While enabled (enable != 0),
+ * every kda_chunk_fwd records a pair of CUDA events on its stream around each
+ * kernel it launches (kind 0 = the per-chunk prep kernel, kind 1 = the state
+ * chain kernel).  Process-wide; off by default.
+ *
+ * kda_debug_kernel_times -- waits for the events recorded so far, writes per
+ * kind the summed device time in ms (ms[kind]) and the number of launches
+ * (launches[kind]) for kinds < nkinds, and forgets them.  The host arrays are
+ * the caller's.  KDA_OK, KDA_ERR_INVALID_ARG for NULL arrays, or KDA_ERR_CUDA.
+ */
+KDA_API void kda_debug_kernel_timing(int enable);
+KDA_API int kda_debug_kernel_times(double *ms, long long *launches, int nkinds);
+
 /* Version of this ABI (major * 100 + minor). */
 KDA_API int kda_abi_version(void);
 
