@@ -186,6 +186,7 @@ const char *kda_status_string(int status) {
         case KDA_ERR_ALIGNMENT: return "KDA_ERR_ALIGNMENT";
         case KDA_ERR_CUDA: return "KDA_ERR_CUDA";
         case KDA_ERR_TIMEOUT: return "KDA_ERR_TIMEOUT";
+        case KDA_ERR_SCRATCH_LIMIT: return "KDA_ERR_SCRATCH_LIMIT";
         default: return "KDA_ERR_UNKNOWN";
     }
 }
@@ -346,6 +347,129 @@ int kda_decode_step(const void *q, const void *k, const void *v, const float *g,
     cudaError_t e = kda::launch_decode(q, k, v, g, beta, scale, state, out, B * H, dk, dv,
                                        static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Fixed-scratch prefill (kda_chunk_fwd_noalloc).
+//
+// Some callers cannot allocate device memory when they call the prefill: a
+// process whose device memory is handed out up front to another allocator (a
+// serving stack that reserves nearly all of HBM for its own caching allocator
+// leaves cudaMalloc nothing to give), or code that must not pay the
+// device-wide synchronisation that freeing a grown workspace costs.  This
+// variant runs the same two kernels over chunk records kept in a fixed array
+// that is part of the module image, in as many segments as the array holds.
+// Nothing in it needs to start at zero: the prep kernel writes every record
+// byte the chain kernel's results depend on before the chain kernel reads it
+// (rows it leaves unwritten feed accumulator lanes that are discarded), and
+// the carried state is written before it is read.
+namespace {
+
+constexpr size_t kScratchBytes = size_t(64) << 20;  // 64 MiB per device
+static __device__ __align__(256) uint8_t g_kda_scratch[kScratchBytes];
+
+uint8_t *g_scratch_ptr[kMaxDevices] = {};
+
+// Once per device, with that device current: the device address of the array.
+int scratch_base(int dev, uint8_t **out) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (g_scratch_ptr[dev] == nullptr) {
+        uint8_t *p = nullptr;
+        if (cudaGetSymbolAddress((void **)&p, g_kda_scratch) != cudaSuccess || p == nullptr) return KDA_ERR_CUDA;
+        g_scratch_ptr[dev] = p;
+    }
+    *out = g_scratch_ptr[dev];
+    return KDA_OK;
+}
+
+size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
+
+}  // namespace
+
+extern "C" {
+
+int kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const float *g, const float *beta,
+                          float scale, const float *h0, void *out, float *hT, int B, int T, int H, int dk,
+                          int dv, void *stream) {
+    if (B < 1 || H < 1 || T < 0) return KDA_ERR_INVALID_ARG;
+    if (T > 0 && (!q || !k || !v || !g || !beta || !out)) return KDA_ERR_INVALID_ARG;
+    if ((dk != 64 && dk != 128) || (dv != 64 && dv != 128)) return KDA_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(g) || !aligned4(beta) ||
+        !aligned16(out) || !aligned16(h0) || !aligned16(hT))
+        return KDA_ERR_ALIGNMENT;
+    if ((long long)B * H * 4 > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+    if (T == 0) {  // nothing to scan: hT = h0 (or zero)
+        if (hT == nullptr) return KDA_OK;
+        const size_t bytes = (size_t)B * H * dk * dv * sizeof(float);
+        cudaError_t e = h0 ? (h0 == hT ? cudaSuccess : cudaMemcpyAsync(hT, h0, bytes, cudaMemcpyDeviceToDevice, s))
+                           : cudaMemsetAsync(hT, 0, bytes, s);
+        return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+    }
+
+    // Scratch layout: [carried state, when hT is NULL][records of one segment].
+    const int nchunks = (T + kda::CH - 1) / kda::CH;
+    const size_t row = rec_row_bytes(B, H);
+    const size_t state_bytes = hT == nullptr ? round256((size_t)B * H * dk * dv * sizeof(float)) : 0;
+    if (state_bytes + row > kScratchBytes) return KDA_ERR_SCRATCH_LIMIT;
+    const size_t fit = (kScratchBytes - state_bytes) / row;
+    const int seg = fit < (size_t)nchunks ? (int)fit : nchunks;
+
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return KDA_ERR_CUDA;
+    uint8_t *scratch = nullptr;
+    if (scratch_base(dev, &scratch) != KDA_OK) return KDA_ERR_CUDA;
+    uint32_t *word = nullptr;
+    if (current_status_word(&word) != KDA_OK) return KDA_ERR_CUDA;
+    PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
+    if (get_encoder(&enc) != KDA_OK) return KDA_ERR_CUDA;
+
+    CUtensorMap tq, tk;
+    if (make_map(&tq, enc, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dk, H, T, B, 64,
+                 CU_TENSOR_MAP_SWIZZLE_128B) != KDA_OK ||
+        make_map(&tk, enc, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dk, H, T, B, 64,
+                 CU_TENSOR_MAP_SWIZZLE_128B) != KDA_OK)
+        return KDA_ERR_CUDA;
+
+    const unsigned long long polls = g_wait_polls.load();
+    kda::DeviceStatus dst;
+    dst.word = word;
+    dst.wait_polls = polls ? polls : ~0ull;
+    float *carry = hT != nullptr ? hT : reinterpret_cast<float *>(scratch);
+    uint8_t *recs = scratch + state_bytes;
+
+    for (int n0 = 0; n0 < nchunks; n0 += seg) {
+        const int cnt = nchunks - n0 < seg ? nchunks - n0 : seg;
+        const bool last = n0 + cnt == nchunks;
+        kda::PrepParams pp;
+        pp.g = g;
+        pp.beta = beta;
+        pp.ws = recs;
+        pp.B = B; pp.T = T; pp.H = H;
+        pp.n_begin = n0;
+        pp.nseg = cnt;
+        pp.st = dst;
+        if (kda::launch_prep(tq, tk, pp, dk, s) != cudaSuccess) return KDA_ERR_CUDA;
+
+        kda::ChainParams cp;
+        cp.v = static_cast<const uint16_t *>(v);
+        cp.h0 = n0 == 0 ? h0 : carry;
+        cp.out = static_cast<uint16_t *>(out);
+        cp.hT = last ? hT : carry;
+        cp.ws = recs;
+        cp.scale = scale;
+        cp.B = B; cp.T = T; cp.H = H; cp.DV = dv;
+        cp.n_begin = n0;
+        cp.nseg = cnt;
+        cp.nslices = 1;
+        cp.st = dst;
+        cp.inject_wait_polls = g_inject_polls.load();
+        if (kda::launch_chain(cp, dk, s) != cudaSuccess) return KDA_ERR_CUDA;
+    }
+    return KDA_OK;
 }
 
 }  // extern "C"

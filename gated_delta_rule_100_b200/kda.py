@@ -4,6 +4,8 @@ the computation runs in the library's CUDA kernels.
 The entry points mirror ``include/kda.h``:
 
 * ``chunk_fwd``   -> ``kda_chunk_fwd``   (chunkwise prefill)
+* ``chunk_fwd_noalloc`` -> ``kda_chunk_fwd_noalloc`` (the same prefill over a fixed
+  scratch array: no device allocation)
 * ``decode_step`` -> ``kda_decode_step`` (one recurrent step, state in place)
 * ``stream_status`` -> ``kda_stream_status``
 * ``workspace_bytes`` / ``release_workspace`` -> ``kda_chunk_fwd_workspace_bytes`` /
@@ -25,8 +27,9 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libkda.so")
 
-KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_ALIGNMENT, KDA_ERR_CUDA, KDA_ERR_TIMEOUT = range(6)
-EXPORTED = ("kda_chunk_fwd", "kda_decode_step", "kda_chunk_fwd_workspace_bytes", "kda_release_workspace",
+(KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_ALIGNMENT, KDA_ERR_CUDA, KDA_ERR_TIMEOUT,
+ KDA_ERR_SCRATCH_LIMIT) = range(7)
+EXPORTED = ("kda_chunk_fwd", "kda_chunk_fwd_noalloc", "kda_decode_step", "kda_chunk_fwd_workspace_bytes", "kda_release_workspace",
             "kda_status_string", "kda_stream_status", "kda_chunk_fwd_debug_wait_limit",
             "kda_chunk_fwd_debug_inject_timeout", "kda_debug_kernel_timing", "kda_debug_kernel_times",
             "kda_abi_version")
@@ -52,6 +55,8 @@ def load():
     vp, fp, i, f = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_float
     lib.kda_chunk_fwd.argtypes = [vp, vp, vp, fp, fp, f, fp, vp, fp, i, i, i, i, i, vp]
     lib.kda_chunk_fwd.restype = i
+    lib.kda_chunk_fwd_noalloc.argtypes = [vp, vp, vp, fp, fp, f, fp, vp, fp, i, i, i, i, i, vp]
+    lib.kda_chunk_fwd_noalloc.restype = i
     lib.kda_decode_step.argtypes = [vp, vp, vp, fp, fp, f, fp, vp, i, i, i, i, vp]
     lib.kda_decode_step.restype = i
     lib.kda_chunk_fwd_workspace_bytes.argtypes = [i, i, i, i, i]
@@ -124,6 +129,29 @@ def chunk_fwd(q, k, v, g, beta, scale, h0=None, *, out=None, hT=None, final_stat
                               _ptr(h0), _ptr(out), _ptr(hT), B, T, H, dk, dv, _stream(stream))
     if rc != KDA_OK:
         raise KdaError(rc, "kda_chunk_fwd")
+    return out, hT
+
+
+def chunk_fwd_noalloc(q, k, v, g, beta, scale, h0=None, *, out, hT=None, stream=None):
+    """``chunk_fwd`` through ``kda_chunk_fwd_noalloc``: the caller passes ``out``
+    (and ``hT`` unless the final state is not wanted); the library allocates
+    nothing.  Returns (out, hT)."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    _check(q, "q", torch.bfloat16, (B, T, H, dk))
+    _check(k, "k", torch.bfloat16, (B, T, H, dk))
+    _check(v, "v", torch.bfloat16, (B, T, H, dv))
+    _check(g, "g", torch.float32, (B, T, H, dk))
+    _check(beta, "beta", torch.float32, (B, T, H))
+    if h0 is not None:
+        _check(h0, "h0", torch.float32, (B, H, dk, dv))
+    _check(out, "out", torch.bfloat16, (B, T, H, dv))
+    if hT is not None:
+        _check(hT, "hT", torch.float32, (B, H, dk, dv))
+    rc = load().kda_chunk_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale),
+                                      _ptr(h0), _ptr(out), _ptr(hT), B, T, H, dk, dv, _stream(stream))
+    if rc != KDA_OK:
+        raise KdaError(rc, "kda_chunk_fwd_noalloc")
     return out, hT
 
 

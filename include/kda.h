@@ -61,7 +61,8 @@ typedef enum {
     KDA_ERR_UNSUPPORTED = 2, /* dk/dv outside {64,128}, other unsupported shape */
     KDA_ERR_ALIGNMENT = 3,   /* a pointer below its required alignment        */
     KDA_ERR_CUDA = 4,        /* a CUDA runtime/driver call or launch failed    */
-    KDA_ERR_TIMEOUT = 5      /* a device-side bounded wait gave up             */
+    KDA_ERR_TIMEOUT = 5,     /* a device-side bounded wait gave up             */
+    KDA_ERR_SCRATCH_LIMIT = 6 /* kda_chunk_fwd_noalloc: problem exceeds its fixed scratch */
 } kda_status;
 
 /*
@@ -119,6 +120,34 @@ KDA_API int kda_decode_step(const void *q, const void *k, const void *v,
                     const float *g, const float *beta, float scale,
                     float *state, void *out,
                     int B, int H, int dk, int dv, void *stream);
+
+/*
+ * kda_chunk_fwd_noalloc -- kda_chunk_fwd without any device allocation.  The
+ * method itself has no counterpart: this is a deployment variant for callers
+ * that cannot allocate device memory at call time (a process whose device
+ * memory is reserved up front by another allocator, or code that must not pay
+ * the device-wide synchronisation of freeing a grown workspace).
+ *
+ * Same arguments, layouts, results and error codes as kda_chunk_fwd; the
+ * outputs are bit-identical to it.  The chunk records live in a fixed 64 MiB
+ * array per device that is part of the library's module image, so a long
+ * sequence runs in several segments of two kernel launches each.  Limit: the
+ * records of one 64-token chunk of every (b, h) (B * H * 99,328 bytes), plus,
+ * when hT is NULL, the fp32 state [B, H, dk, dv] carried between segments,
+ * must fit in 64 MiB (B * H <= 675 with hT given); a larger problem returns
+ * KDA_ERR_SCRATCH_LIMIT without enqueueing work.  Nothing in the scratch
+ * needs to start at zero.
+ *
+ * The first call on a device looks up the array's device address (with that
+ * device current) and caches it: make that first call before any stream
+ * capture.  The scratch is shared by every call on the device, so calls that
+ * overlap on the GPU (different streams, no ordering between them) race on
+ * it and give wrong results; the caller orders them.
+ */
+KDA_API int kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v,
+                  const float *g, const float *beta, float scale,
+                  const float *h0, void *out, float *hT,
+                  int B, int T, int H, int dk, int dv, void *stream);
 
 /*
  * kda_chunk_fwd_workspace_bytes -- device memory kda_chunk_fwd holds for these

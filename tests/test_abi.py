@@ -112,3 +112,21 @@ def test_workspace_bytes(lib):
     assert kda.workspace_bytes(1, 0, 1, 128, 128) == 0
     assert kda.workspace_bytes(1, 64, 1, 96, 128) == 0
     assert kda.workspace_bytes(0, 64, 1, 128, 128) == 0
+
+
+def test_noalloc_rejects_beyond_its_scratch(lib):
+    def call(B, H, hT, dk=128, dv=128):
+        return lib.kda_chunk_fwd_noalloc(A, A, A, A, A, 1.0, None, A, hT, B, 64, H, dk, dv, None)
+    # one chunk record of every (b, h) must fit in the 64 MiB array: B * H <= 675 with hT given
+    assert call(1, 676, A) == kda.KDA_ERR_SCRATCH_LIMIT
+    assert call(2, 338, A) == kda.KDA_ERR_SCRATCH_LIMIT
+    # without hT the carried fp32 state shares the array
+    assert call(1, 600, None) == kda.KDA_ERR_SCRATCH_LIMIT
+    assert kda.status_string(kda.KDA_ERR_SCRATCH_LIMIT) == "KDA_ERR_SCRATCH_LIMIT"
+    # the usual argument checks come first
+    assert lib.kda_chunk_fwd_noalloc(None, A, A, A, A, 1.0, None, A, None, 1, 64, 1, 64, 64, None) == \
+        kda.KDA_ERR_INVALID_ARG
+    assert lib.kda_chunk_fwd_noalloc(A, A, A, A, A, 1.0, None, A, None, 1, 64, 1, 96, 64, None) == \
+        kda.KDA_ERR_UNSUPPORTED
+    assert lib.kda_chunk_fwd_noalloc(MIS, A, A, A, A, 1.0, None, A, None, 1, 64, 1, 64, 64, None) == \
+        kda.KDA_ERR_ALIGNMENT
