@@ -33,6 +33,7 @@
 namespace kda {
 
 constexpr int CHAIN_THREADS = 512;
+constexpr int CHAIN_PREFETCH = 4;  // chunks between the L2 prefetch of a record and its use
 
 template <int DK, int VS>
 struct ChainLayout {
@@ -57,7 +58,10 @@ struct ChainLayout {
 };
 
 template <int DK, int VS>
-__global__ void __launch_bounds__(CHAIN_THREADS, 1) chain_kernel(const ChainParams prm) {
+__global__ void __launch_bounds__(CHAIN_THREADS, 1)
+chain_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ CUtensorMap tm_p,
+             const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUtensorMap tm_t,
+             const ChainParams prm) {
     using L = ChainLayout<DK, VS>;
     constexpr int CPT = VS / 4;            // value columns per thread (state, Vnew, output)
     constexpr int NP = VS / 2;             // value column pairs (V loads)
@@ -91,11 +95,13 @@ __global__ void __launch_bounds__(CHAIN_THREADS, 1) chain_kernel(const ChainPara
     const int col0 = slice * VS;
     const int nseg = prm.nseg;
     const uint8_t *recs = prm.ws + (size_t)bh * nseg * REC_BYTES;
+    const int rec0 = bh * nseg;  // index of this (b, h)'s first record in the tensor maps
     const uint64_t polls = prm.st.wait_polls;
 
     if (tid == 0) {
         for (int i = 0; i < 6; ++i) mbar_init(smem_u32(&s_bars[i]), 1);
         fence_mbar_init();
+        prefetch_tmap(&tm_wq); prefetch_tmap(&tm_p); prefetch_tmap(&tm_kh); prefetch_tmap(&tm_t);
     }
     if (warp == 0) {
         tmem_alloc(smem_u32(s_tmem), L::TM_COLS);
@@ -107,18 +113,24 @@ __global__ void __launch_bounds__(CHAIN_THREADS, 1) chain_kernel(const ChainPara
     const uint32_t tmem = *s_tmem;
     const uint32_t lane_base = (uint32_t)(lq * 32) << 16;
 
+    // Record parts are plain row-major in global memory; the tensor loads
+    // write them in the swizzled operand layouts.
     auto issue_a = [&](int n) {
         const uint8_t *r = recs + (size_t)n * REC_BYTES;
         mbar_expect_tx(bar_a, TX_A);
-        bulk_load(sbase + REC_WQ, r + REC_WQ, DK * 256, bar_a);
-        bulk_load(sbase + REC_T, r + REC_T, 16384, bar_a);
+#pragma unroll
+        for (int nb = 0; nb < 2; ++nb) tma_load_3d(sbase + REC_WQ + nb * DK * 128, &tm_wq, bar_a, nb * 64, 0, rec0 + n);
+#pragma unroll
+        for (int kb = 0; kb < 2; ++kb) tma_load_3d(sbase + REC_T + kb * 8192, &tm_t, bar_a, kb * 32, 0, rec0 + n);
         bulk_load(sbase + L::OFF_DEC + (n & 1) * 512, r + REC_DEC, 512, bar_a);
     };
     auto issue_b = [&](int n) {
-        const uint8_t *r = recs + (size_t)n * REC_BYTES;
         mbar_expect_tx(bar_b, TX_B);
-        bulk_load(sbase + REC_P, r + REC_P, 16384, bar_b);
-        bulk_load(sbase + REC_KH, r + REC_KH, 32768, bar_b);
+#pragma unroll
+        for (int kb = 0; kb < 2; ++kb) {
+            tma_load_3d(sbase + REC_P + kb * 8192, &tm_p, bar_b, kb * 32, 0, rec0 + n);
+            tma_load_3d(sbase + REC_KH + kb * 16384, &tm_kh, bar_b, kb * 32, 0, rec0 + n);
+        }
     };
 
     // ---- state: thread (ch, cg) holds S[ch][cg CPT .. cg CPT + CPT - 1] in fp32 ----
@@ -196,6 +208,9 @@ __global__ void __launch_bounds__(CHAIN_THREADS, 1) chain_kernel(const ChainPara
     };
 
     store_state_bf16();
+    if (tid == 32) {
+        for (int n = 1; n < CHAIN_PREFETCH && n < nseg; ++n) prefetch_l2(recs + (size_t)n * REC_BYTES, REC_BYTES);
+    }
     if (nseg > 0) {
         if (tid == 0) { issue_a(0); issue_b(0); }
         pend_a = pend_b = true;
@@ -223,6 +238,8 @@ __global__ void __launch_bounds__(CHAIN_THREADS, 1) chain_kernel(const ChainPara
         const int t0 = (prm.n_begin + n) * CH;
 
         // ---- 1: D1 = [W; Q e^G] S0 (U of this chunk is already queued ahead of it) ----
+        if (tid == 32 && n + CHAIN_PREFETCH < nseg)  // records a few chunks ahead -> L2
+            prefetch_l2(recs + (size_t)(n + CHAIN_PREFETCH) * REC_BYTES, REC_BYTES);
         if (tid == 0) {
 #pragma unroll
             for (int kk = 0; kk < DK / 16; ++kk)
@@ -338,19 +355,22 @@ __global__ void __launch_bounds__(CHAIN_THREADS, 1) chain_kernel(const ChainPara
 }
 
 template <int DK, int VS>
-static cudaError_t launch_chain_t(const ChainParams &prm, cudaStream_t stream) {
+static cudaError_t launch_chain_t(const CUtensorMap *maps, const ChainParams &prm, cudaStream_t stream) {
     using L = ChainLayout<DK, VS>;
     cudaError_t e = cudaFuncSetAttribute(chain_kernel<DK, VS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          L::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    chain_kernel<DK, VS><<<prm.B * prm.H * prm.nslices, CHAIN_THREADS, L::SMEM_BYTES, stream>>>(prm);
+    chain_kernel<DK, VS><<<prm.B * prm.H * prm.nslices, CHAIN_THREADS, L::SMEM_BYTES, stream>>>(
+        maps[0], maps[1], maps[2], maps[3], prm);
     return cudaGetLastError();
 }
 
-cudaError_t launch_chain(const ChainParams &prm, int dk, cudaStream_t stream) {
+// maps: the record parts WQ, P, K-hat, T' (see chunk_common.cuh)
+cudaError_t launch_chain(const CUtensorMap *maps, const ChainParams &prm, int dk, cudaStream_t stream) {
     const int vs = prm.DV / prm.nslices;
-    if (dk == 128) return vs == 128 ? launch_chain_t<128, 128>(prm, stream) : launch_chain_t<128, 64>(prm, stream);
-    return vs == 128 ? launch_chain_t<64, 128>(prm, stream) : launch_chain_t<64, 64>(prm, stream);
+    if (dk == 128)
+        return vs == 128 ? launch_chain_t<128, 128>(maps, prm, stream) : launch_chain_t<128, 64>(maps, prm, stream);
+    return vs == 128 ? launch_chain_t<64, 128>(maps, prm, stream) : launch_chain_t<64, 64>(maps, prm, stream);
 }
 
 }  // namespace kda

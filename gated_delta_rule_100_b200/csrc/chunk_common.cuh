@@ -8,13 +8,14 @@
 //   chain (one CTA per (b, h), chunks in order): U = T Diag(beta) V, then the
 //         state pass Vnew = U - W S, S <- e^{Gamma_C} S + K-hat^T Vnew and the
 //         outputs (Q e^Gamma) S + P Vnew.
-// A record holds, in the exact shared-memory layouts the chain's UMMAs read
-// (offsets relative to a 1024-byte aligned base, so the swizzle carries over):
-//   WQ   bf16 MN-major [dk][128]: columns 0..63 = W^T, 64..127 = (Q e^Gamma)^T
-//   P    tf32 K-major  [64][64], K-block stride 8 KB (causal q-k block, incl. diagonal)
-//   KH   tf32 K-major  [128][64] (K-hat^T: row = key channel, K = token)
-//   T'   tf32 K-major  [64][64], K-block stride 8 KB: T' = T Diag(beta)
-//   DEC  fp32 [128]    e^{Gamma_C} per key channel
+// A record holds plain row-major arrays (the chain kernel's tensor loads put
+// them in the swizzled UMMA operand layouts):
+//   WQ   bf16 [dk][128]  row = key channel; columns 0..63 = W^T, 64..127 = (Q e^Gamma)^T
+//   P    fp32 [64][64]   causal q-k block (incl. diagonal), rows = queries
+//   KH   fp32 [128][64]  K-hat^T: row = key channel, column = token
+//   T'   fp32 [64][64]   T' = T Diag(beta), unit-lower times beta
+//   DEC  fp32 [128]      e^{Gamma_C} per key channel
+// at the offsets below (each a multiple of 1 KB; 97 KB per record).
 #pragma once
 #include <stdint.h>
 

@@ -25,8 +25,8 @@ cudaError_t launch_decode(const void *q, const void *k, const void *v, const flo
 
 namespace kda {
 cudaError_t launch_prep(const CUtensorMap &tq, const CUtensorMap &tk, const PrepParams &prm, int dk,
-                        cudaStream_t stream);
-cudaError_t launch_chain(const ChainParams &prm, int dk, cudaStream_t stream);
+                        int num_sms, cudaStream_t stream);
+cudaError_t launch_chain(const CUtensorMap *maps, const ChainParams &prm, int dk, cudaStream_t stream);
 }
 
 // Device-side status word: kernels OR error bits into it (one per device,
@@ -119,7 +119,6 @@ int reserve_workspace(int dev, size_t rec_bytes, size_t state_bytes, Workspace *
 
 // Per-kernel timing hook (measurement only): CUDA events recorded on the
 // launching stream around every prefill kernel while enabled.
-constexpr int kKernelKinds = 2;  // 0 = prep, 1 = chain
 struct TimedLaunch {
     int dev, kind;
     cudaEvent_t start, stop;
@@ -171,6 +170,48 @@ int make_map(CUtensorMap *map, PFN_cuTensorMapEncodeTiled_v12000 enc, const void
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? KDA_OK : KDA_ERR_CUDA;
 }
+
+// Streaming multiprocessors of a device (cached; its own lock, so callers may hold g_mu).
+std::mutex g_sms_mu;
+int g_num_sms[kMaxDevices] = {};
+int num_sms(int dev) {
+    std::lock_guard<std::mutex> lk(g_sms_mu);
+    if (g_num_sms[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1) n = 148;
+        g_num_sms[dev] = n;
+    }
+    return g_num_sms[dev];
+}
+
+// Tensor maps over the record parts of `nrec` consecutive records at `rec`
+// (plain row-major arrays, see chunk_common.cuh), with the boxes and the
+// 128-byte swizzle of the chain kernel's operand tiles.
+int make_rec_maps(PFN_cuTensorMapEncodeTiled_v12000 enc, const uint8_t *rec, long long nrec, int dk,
+                  CUtensorMap *maps) {
+    struct Part { size_t off; CUtensorMapDataType dt; int esize, cols, rows, box_cols; };
+    const Part parts[4] = {{(size_t)kda::REC_WQ, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 128, dk, 64},
+                           {(size_t)kda::REC_P, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, 64, 64, 32},
+                           {(size_t)kda::REC_KH, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, 64, 128, 32},
+                           {(size_t)kda::REC_T, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, 64, 64, 32}};
+    for (int i = 0; i < 4; ++i) {
+        const Part &p = parts[i];
+        cuuint64_t dims[3] = {(cuuint64_t)p.cols, (cuuint64_t)p.rows, (cuuint64_t)nrec};
+        cuuint64_t strides[2] = {(cuuint64_t)p.cols * p.esize, (cuuint64_t)kda::REC_BYTES};
+        cuuint32_t box[3] = {(cuuint32_t)p.box_cols, (cuuint32_t)p.rows, 1u};
+        cuuint32_t estr[3] = {1u, 1u, 1u};
+        CUresult r = enc(&maps[i], p.dt, 3, const_cast<uint8_t *>(rec + p.off), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return KDA_ERR_CUDA;
+    }
+    return KDA_OK;
+}
+
+// Value-column slices per (b, h) in the chain kernel: two 64-column CTAs when
+// that still fits one CTA per SM (the chain is latency-bound, and half the
+// columns halve every state product), else one.
+int chain_slices(int B, int H, int dv, int sms) { return (dv == 128 && 2LL * B * H <= sms) ? 2 : 1; }
 
 }  // namespace
 
@@ -259,6 +300,9 @@ int kda_chunk_fwd(const void *q, const void *k, const void *v, const float *g, c
     dst.wait_polls = polls ? polls : ~0ull;
     // State carried between segments: the caller's hT when given, else the workspace's.
     float *carry = hT != nullptr ? hT : w->state;
+    const int sms = num_sms(dev);
+    CUtensorMap rmaps[4];
+    if (make_rec_maps(enc, w->rec, (long long)B * H * seg, dk, rmaps) != KDA_OK) return KDA_ERR_CUDA;
 
     for (int n0 = 0; n0 < nchunks; n0 += seg) {
         const int cnt = nchunks - n0 < seg ? nchunks - n0 : seg;
@@ -271,7 +315,7 @@ int kda_chunk_fwd(const void *q, const void *k, const void *v, const float *g, c
         pp.n_begin = n0;
         pp.nseg = cnt;
         pp.st = dst;
-        cudaError_t e = timed_launch(dev, 0, s, [&] { return kda::launch_prep(tq, tk, pp, dk, s); });
+        cudaError_t e = timed_launch(dev, 0, s, [&] { return kda::launch_prep(tq, tk, pp, dk, sms, s); });
         if (e != cudaSuccess) return KDA_ERR_CUDA;
 
         kda::ChainParams cp;
@@ -284,10 +328,10 @@ int kda_chunk_fwd(const void *q, const void *k, const void *v, const float *g, c
         cp.B = B; cp.T = T; cp.H = H; cp.DV = dv;
         cp.n_begin = n0;
         cp.nseg = cnt;
-        cp.nslices = 1;
+        cp.nslices = chain_slices(B, H, dv, sms);
         cp.st = dst;
         cp.inject_wait_polls = g_inject_polls.load();
-        e = timed_launch(dev, 1, s, [&] { return kda::launch_chain(cp, dk, s); });
+        e = timed_launch(dev, 1, s, [&] { return kda::launch_chain(rmaps, cp, dk, s); });
         if (e != cudaSuccess) return KDA_ERR_CUDA;
     }
     if (cudaEventRecord(w->done, s) != cudaSuccess) return KDA_ERR_CUDA;
@@ -440,6 +484,9 @@ int kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const flo
     dst.wait_polls = polls ? polls : ~0ull;
     float *carry = hT != nullptr ? hT : reinterpret_cast<float *>(scratch);
     uint8_t *recs = scratch + state_bytes;
+    const int sms = num_sms(dev);
+    CUtensorMap rmaps[4];
+    if (make_rec_maps(enc, recs, (long long)B * H * seg, dk, rmaps) != KDA_OK) return KDA_ERR_CUDA;
 
     for (int n0 = 0; n0 < nchunks; n0 += seg) {
         const int cnt = nchunks - n0 < seg ? nchunks - n0 : seg;
@@ -452,7 +499,7 @@ int kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const flo
         pp.n_begin = n0;
         pp.nseg = cnt;
         pp.st = dst;
-        if (kda::launch_prep(tq, tk, pp, dk, s) != cudaSuccess) return KDA_ERR_CUDA;
+        if (kda::launch_prep(tq, tk, pp, dk, sms, s) != cudaSuccess) return KDA_ERR_CUDA;
 
         kda::ChainParams cp;
         cp.v = static_cast<const uint16_t *>(v);
@@ -464,10 +511,10 @@ int kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const flo
         cp.B = B; cp.T = T; cp.H = H; cp.DV = dv;
         cp.n_begin = n0;
         cp.nseg = cnt;
-        cp.nslices = 1;
+        cp.nslices = chain_slices(B, H, dv, sms);
         cp.st = dst;
         cp.inject_wait_polls = g_inject_polls.load();
-        if (kda::launch_chain(cp, dk, s) != cudaSuccess) return KDA_ERR_CUDA;
+        if (kda::launch_chain(rmaps, cp, dk, s) != cudaSuccess) return KDA_ERR_CUDA;
     }
     return KDA_OK;
 }

@@ -11,8 +11,8 @@
 // recurrence (section 4 of "Kimi Linear's Hybrid Linear Attention
 // Architecture: A Technical Breakdown"), with the chunk's rank-1 updates
 // packed in the WY form (W, and U = T' V in the chain kernel).
-// None of them depends on the state, so every chunk is an independent CTA;
-// the result goes to a per-chunk record (layout in chunk_common.cuh).
+// None of them depends on the state, so chunks are independent work items;
+// each result goes to a per-chunk record (layout in chunk_common.cuh).
 //
 // Decay factors.  e^{Gamma_i - Gamma_j} is split into two factors, one per
 // side of the contraction over key channels.  Rows of 16-token block I use
@@ -23,17 +23,21 @@
 // >= -160.  All factors come from running products of alpha = e^g (one exp
 // per input element) plus one reciprocal per factor above 1.
 //
-// CTA: 512 threads; in the elementwise phase thread (c, I) owns key channel c
-// and tokens 16 I .. 16 I + 15 (a two-level scan: products inside the block,
-// then the four block totals through shared memory).  Phases:
-//   E  alpha, running products, operand tiles X, Y^(I) (bf16, smem) for the
-//      formation; Q e^G, K-hat (global record); (K e^G)^T (tf32, smem)
+// Persistent CTAs (two per SM, 512 threads) loop over the items; while one
+// item is processed the next one's q, k and g are prefetched into L2.  In the
+// elementwise phase thread (c, I) owns key channel c and tokens 16 I .. 16 I +
+// 15 (a two-level scan: products inside the block, then the four block
+// totals through shared memory); its key and query values are held as bf16
+// pairs, so the phase fits in 64 registers.  Phases per item:
+//   E  alpha, running products; operand tiles X, Y^(I) (bf16, smem) for the
+//      formation; Q e^G, K-hat (record); (K e^G)^T (tf32, smem)
 //   F  X Y^(I)^T -> A, P                    (UMMA bf16, overlapped with E's tail)
 //   AP A -> fp32 scratch, P -> record
 //   T  (I + A)^{-1}: 16x16 diagonal blocks by substitution, off-diagonal blocks
 //      from N = D A_off as T = (I - N + N^2 - N^3) D, fp32 on CUDA cores
 //   W  T' = T Diag(beta) -> record;  W^T = (K e^G)^T T'^T  (UMMA tf32) -> record
-// Shared memory is 110 KB and TMEM 256 columns, so two CTAs share an SM.
+// Record parts are plain row-major arrays written with contiguous 16-byte
+// stores; the chain kernel's tensor loads apply the operand swizzle.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <stdint.h>
@@ -60,15 +64,15 @@ struct PrepLayout {
     static constexpr int FORM_B = DK * (256 + 32 + 64 + 128 + 128);
     static constexpr int OFF_A = OFF_F;                      // fp32 [64][A_LD]
     static constexpr int OFF_TF = OFF_A + 64 * A_LD * 4;     // fp32 [64][A_LD]
-    static constexpr int OFF_T = OFF_F + align1k(2 * 64 * A_LD * 4);  // tf32 K-major [64][64], 8 KB K-blocks (+8 KB read overhang)
-    static constexpr int OFF_ZS = OFF_T + 24576;             // N / M scratch, 7 x 1 KB
+    static constexpr int OFF_T = OFF_F + align1k(2 * 64 * A_LD * 4);  // tf32 K-major [64][64], 8 KB K-blocks
+    static constexpr int OFF_ZS = OFF_T + 16384;             // N / M scratch, 7 x 1 KB
     static constexpr int POST_B = OFF_ZS + 7 * 1024 - OFF_F;
     static constexpr int RF_B = align1k(cmax(FORM_B, POST_B));
     // (K e^G)^T: tf32 K-major [128][64]; holds the q, k TMA tiles during E
     static constexpr int OFF_BK = OFF_F + RF_B;
     static constexpr int OFF_QIN = OFF_BK;                   // bf16 [64][DK], 128B swizzle
     static constexpr int OFF_KIN = OFF_BK + CH * DK * 2;
-    static constexpr int OFF_MISC = OFF_BK + 128 * 64 * 4;   // beta, e^{Gamma_C}, barriers, TMEM address
+    static constexpr int OFF_MISC = OFF_BK + 128 * 64 * 4;   // beta, barriers, TMEM address
     static constexpr int TOTAL = OFF_MISC + 1024;
     static constexpr int SMEM_BYTES = TOTAL + 1024;          // slack for the 1 KB base alignment
     static_assert(SMEM_BYTES <= 113 * 1024, "two CTAs per SM");
@@ -78,6 +82,13 @@ struct PrepLayout {
     static constexpr uint32_t TM_W = 160;   // 64: W^T (lane = key channel, column = token)
     static constexpr uint32_t TM_COLS = 256;
 };
+
+__device__ __forceinline__ void prefetch_tensor_4d(const CUtensorMap *map, int c0, int c1, int c2, int c3) {
+    asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+                 : "memory");
+}
 
 template <int DK>
 __global__ void __launch_bounds__(PREP_THREADS, 2)
@@ -99,20 +110,16 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     const int warp = tid >> 5, lane = tid & 31;
     const int ch = tid & 127;        // key channel / TMEM lane of this thread
     const int qb = tid >> 7;         // 16-token block (phase E) / 16-column quarter (elsewhere)
-    const int item = blockIdx.x;     // (b, h) major, chunk minor
-    const int ni = item % prm.nseg;
-    const int bh = item / prm.nseg;
-    const int h = bh % prm.H, b = bh / prm.H;
     const int T = prm.T, H = prm.H;
-    const int n = prm.n_begin + ni;
-    const int t0 = n * CH;
-    uint8_t *rec = prm.ws + (size_t)item * REC_BYTES;
+    const int nitems = prm.B * prm.H * prm.nseg;  // (b, h) major, chunk minor
     const uint64_t polls = prm.st.wait_polls;
 
     if (tid == 0) {
         mbar_init(bar_in, 1);
         mbar_init(bar_mma, 1);
         fence_mbar_init();
+        prefetch_tmap(&tm_q);
+        prefetch_tmap(&tm_k);
     }
     if (warp == 0) {
         tmem_alloc(smem_u32(s_tmem), L::TM_COLS);
@@ -125,7 +132,8 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
 
     bool tma_pending = false, mma_pending = false, aborted = false;
-    uint32_t ph_mma = 0;  // phase of bar_mma that the MMAs in flight complete
+    uint32_t ph_in = 0;   // phase of bar_in the TMA in flight completes
+    uint32_t ph_mma = 0;  // phase of bar_mma the MMAs in flight complete
     auto wait_all = [&](uint32_t bar, uint32_t ph, bool &pending) -> bool {
         const bool ok = mbar_wait(bar, ph, polls, prm.st);
         if (__syncthreads_or(!ok)) return false;
@@ -139,110 +147,172 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         __syncthreads();
         tc_fence_after();
     };
+    // first token, batch and head of an item
+    auto item_coords = [&](int it, int &b, int &h, int &t0) {
+        const int ni = it % prm.nseg, bh = it / prm.nseg;
+        h = bh % H;
+        b = bh / H;
+        t0 = (prm.n_begin + ni) * CH;
+    };
 
-    // ---------------- inputs: q, k by TMA; g (this thread's 16 tokens) and beta by plain loads
-    if (tid == 0) {
-        mbar_expect_tx(bar_in, (uint32_t)(2 * CH * DK * 2));
-#pragma unroll
-        for (int kb = 0; kb < DK / 64; ++kb) {
-            tma_load_4d(sbase + L::OFF_QIN + kb * CH * 128, &tm_q, bar_in, kb * 64, h, t0, b);
-            tma_load_4d(sbase + L::OFF_KIN + kb * CH * 128, &tm_k, bar_in, kb * 64, h, t0, b);
-        }
-    }
-    tma_pending = true;
     const int c = ch, I = qb, tb = SUB * I;
     const bool active = c < DK;
-    float al[SUB];
-    {
-        const float *gp = prm.g + (((size_t)b * T + t0 + tb) * H + h) * DK + c;
-#pragma unroll
-        for (int u = 0; u < SUB; ++u) al[u] = (t0 + tb + u < T && active) ? __ldg(gp + (size_t)u * H * DK) : 0.f;
-    }
-    if (tid < CH) s_beta[tid] = (t0 + tid < T) ? prm.beta[((size_t)b * T + t0 + tid) * H + h] : 0.f;
-    if (!wait_all(bar_in, 0, tma_pending)) aborted = true;
 
-    if (!aborted) {
+    for (int item = blockIdx.x; item < nitems && !aborted; item += gridDim.x) {
+        int b, h, t0;
+        item_coords(item, b, h, t0);
+        uint8_t *rec = prm.ws + (size_t)item * REC_BYTES;
+
+        // ---------------- inputs: q, k by TMA; g (this thread's 16 tokens) and beta by plain loads
+        if (tid == 0) {
+            mbar_expect_tx(bar_in, (uint32_t)(2 * CH * DK * 2));
+#pragma unroll
+            for (int kb = 0; kb < DK / 64; ++kb) {
+                tma_load_4d(sbase + L::OFF_QIN + kb * CH * 128, &tm_q, bar_in, kb * 64, h, t0, b);
+                tma_load_4d(sbase + L::OFF_KIN + kb * CH * 128, &tm_k, bar_in, kb * 64, h, t0, b);
+            }
+        }
+        tma_pending = true;
+        float al[SUB];
+        {
+            const float *gp = prm.g + (((size_t)b * T + t0 + tb) * H + h) * DK + c;
+#pragma unroll
+            for (int u = 0; u < SUB; ++u) al[u] = (t0 + tb + u < T && active) ? __ldg(gp + (size_t)u * H * DK) : 0.f;
+        }
+        if (tid < CH) s_beta[tid] = (t0 + tid < T) ? prm.beta[((size_t)b * T + t0 + tid) * H + h] : 0.f;
+        // the next item's q, k and g into L2 while this one is processed
+        if (item + (int)gridDim.x < nitems) {
+            int nb, nh, nt0;
+            item_coords(item + gridDim.x, nb, nh, nt0);
+            if (tid == 0) {
+#pragma unroll
+                for (int kb = 0; kb < DK / 64; ++kb) {
+                    prefetch_tensor_4d(&tm_q, kb * 64, nh, nt0, nb);
+                    prefetch_tensor_4d(&tm_k, kb * 64, nh, nt0, nb);
+                }
+            } else if (tid >= 64 && tid < 64 + CH && nt0 + tid - 64 < T) {
+                prefetch_l2(prm.g + (((size_t)nb * T + nt0 + tid - 64) * H + nh) * DK, DK * 4);
+            }
+        }
+        if (!wait_all(bar_in, ph_in, tma_pending)) { aborted = true; break; }
+        ph_in ^= 1u;
+
         // ---------------- E: decay factors and operand tiles ----------------
-        float kv[SUB], qv[SUB];
+        // This thread's 16 key and query values, kept as bf16 pairs (tokens 2e, 2e + 1).
+        uint32_t kp[SUB / 2], qp[SUB / 2];
         {
             const uint8_t *qs = sm + L::OFF_QIN, *ks = sm + L::OFF_KIN;
 #pragma unroll
-            for (int u = 0; u < SUB; ++u) {
-                kv[u] = bf16_bits_to_f32(*reinterpret_cast<const uint16_t *>(ks + kmaj<128, 2>(tb + u, c, CH)));
-                qv[u] = bf16_bits_to_f32(*reinterpret_cast<const uint16_t *>(qs + kmaj<128, 2>(tb + u, c, CH)));
+            for (int e = 0; e < SUB / 2; ++e) {
+                const uint32_t k0 = *reinterpret_cast<const uint16_t *>(ks + kmaj<128, 2>(tb + 2 * e, c, CH));
+                const uint32_t k1 = *reinterpret_cast<const uint16_t *>(ks + kmaj<128, 2>(tb + 2 * e + 1, c, CH));
+                const uint32_t q0 = *reinterpret_cast<const uint16_t *>(qs + kmaj<128, 2>(tb + 2 * e, c, CH));
+                const uint32_t q1 = *reinterpret_cast<const uint16_t *>(qs + kmaj<128, 2>(tb + 2 * e + 1, c, CH));
+                kp[e] = k0 | (k1 << 16);
+                qp[e] = q0 | (q1 << 16);
             }
         }
-        float lp[SUB];  // lp[u] = prod_{s=tb..tb+u} alpha_s
+        auto unpack = [](const uint32_t (&pr)[SUB / 2], int u) {
+            return __uint_as_float((u & 1) ? (pr[u >> 1] & 0xFFFF0000u) : (pr[u >> 1] << 16));
+        };
+        auto kval = [&](int u) { return unpack(kp, u); };
+        auto qval = [&](int u) { return unpack(qp, u); };
+#pragma unroll
+        for (int u = 0; u < SUB; ++u) al[u] = __expf(al[u]);
         {
-            float p = 1.f;
+            float p = 1.f, p8 = 1.f;
 #pragma unroll
-            for (int u = 0; u < SUB; ++u) { al[u] = __expf(al[u]); p *= al[u]; lp[u] = p; }
+            for (int u = 0; u < SUB; ++u) { p *= al[u]; if (u == SUB / 2) p8 = p; }
+            if (active) { s_xch[I * 128 + c] = p; s_xch[512 + I * 128 + c] = p8; }
         }
-        if (active) { s_xch[I * 128 + c] = lp[SUB - 1]; s_xch[512 + I * 128 + c] = lp[SUB / 2]; }
-        __syncthreads();
-        float bt[NSUB], l8[NSUB];
+        __syncthreads();  // also: every thread holds its q, k values, so their tiles' space is free
+        // From the block totals bt_J and the products l8_J through each block's
+        // reference token: preB = prod_{J<I} bt_J, postB = prod_{J>I} bt_J, and
+        // sc[I'] = prod_{J=I+1..I'-1} bt_J * l8_{I'} for the later blocks I' > I.
+        float preB = 1.f, postB = 1.f, dec = 1.f, sc[NSUB];
+        {
+            float mid = 1.f;
 #pragma unroll
-        for (int J = 0; J < NSUB; ++J) { bt[J] = s_xch[J * 128 + c]; l8[J] = s_xch[512 + J * 128 + c]; }
-        __syncthreads();  // the exchange area becomes X; the q, k tiles are consumed
-        float ls[SUB];    // ls[u] = prod_{s=tb+u+1..tb+15} alpha_s
-        ls[SUB - 1] = 1.f;
-#pragma unroll
-        for (int u = SUB - 2; u >= 0; --u) ls[u] = ls[u + 1] * al[u + 1];
+            for (int J = 0; J < NSUB; ++J) {
+                const float btJ = s_xch[J * 128 + c], l8J = s_xch[512 + J * 128 + c];
+                sc[J] = mid * l8J;
+                if (J > I) mid *= btJ;
+                if (J < I) preB *= btJ;
+                if (J > I) postB *= btJ;
+                dec *= btJ;
+            }
+        }
+        __syncthreads();  // the exchange area becomes X
+
+        auto yput = [&](int Iy, int j0, const float (&v8)[8]) {
+            if (Iy == 0)      *reinterpret_cast<uint4 *>(sm + L::OFF_Y0 + mnmaj<32, 2>(c, j0, DK)) = pack8_bf16(v8);
+            else if (Iy == 1) *reinterpret_cast<uint4 *>(sm + L::OFF_Y1 + mnmaj<64, 2>(c, j0, DK)) = pack8_bf16(v8);
+            else if (Iy == 2) *reinterpret_cast<uint4 *>(sm + L::OFF_Y2 + mnmaj<128, 2>(c, j0, DK)) = pack8_bf16(v8);
+            else              *reinterpret_cast<uint4 *>(sm + L::OFF_Y3 + mnmaj<128, 2>(c, j0, DK)) = pack8_bf16(v8);
+        };
+        auto xput = [&](int col, const float (&v8)[8]) {
+            *reinterpret_cast<uint4 *>(sm + L::OFF_X + mnmaj<128, 2>(c, col, DK)) = pack8_bf16(v8);
+        };
         if (active) {
             // Own block, reference m = tb + 8:
             //   u >= 8: f_u = prod_{s=9..u} alpha     X = k f,   Y^(I) = k / f
             //   u <  8: y_u = prod_{s=u+1..8} alpha   X = k / y, Y^(I) = k y
-            float xk[SUB], xq[SUB], yo[SUB];
             {
-                float f = 1.f;
+                float f[8], v8[8];
+                float ff = 1.f;
 #pragma unroll
-                for (int u = SUB / 2; u < SUB; ++u) {
-                    if (u > SUB / 2) f *= al[u];
-                    xk[u] = kv[u] * f;
-                    xq[u] = qv[u] * f;
-                    yo[u] = u == SUB / 2 ? kv[u] : kv[u] * rcp_clamped(f);
-                }
-                float y = 1.f;
+                for (int e = 0; e < 8; ++e) { if (e > 0) ff *= al[8 + e]; f[e] = ff; }
 #pragma unroll
-                for (int u = SUB / 2 - 1; u >= 0; --u) {
-                    y *= al[u + 1];
-                    const float r = rcp_clamped(y);
-                    xk[u] = kv[u] * r;
-                    xq[u] = qv[u] * r;
-                    yo[u] = kv[u] * y;
-                }
+                for (int e = 0; e < 8; ++e) v8[e] = kval(8 + e) * f[e];
+                xput(tb + 8, v8);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) v8[e] = qval(8 + e) * f[e];
+                xput(64 + tb + 8, v8);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) v8[e] = e == 0 ? kval(8) : kval(8 + e) * rcp_clamped(f[e]);
+                yput(I, tb + 8, v8);
             }
-            auto yput = [&](int Iy, int j0, const float *v) {
-                float v8[8];
+            {
+                float y[8], v8[8];
+                float yy = 1.f;
 #pragma unroll
-                for (int e = 0; e < 8; ++e) v8[e] = v[e];
-                if (Iy == 0)      *reinterpret_cast<uint4 *>(sm + L::OFF_Y0 + mnmaj<32, 2>(c, j0, DK)) = pack8_bf16(v8);
-                else if (Iy == 1) *reinterpret_cast<uint4 *>(sm + L::OFF_Y1 + mnmaj<64, 2>(c, j0, DK)) = pack8_bf16(v8);
-                else if (Iy == 2) *reinterpret_cast<uint4 *>(sm + L::OFF_Y2 + mnmaj<128, 2>(c, j0, DK)) = pack8_bf16(v8);
-                else              *reinterpret_cast<uint4 *>(sm + L::OFF_Y3 + mnmaj<128, 2>(c, j0, DK)) = pack8_bf16(v8);
-            };
+                for (int e = 7; e >= 0; --e) { yy *= al[e + 1]; y[e] = yy; }
 #pragma unroll
-            for (int h8 = 0; h8 < 2; ++h8) {
-                float a8[8], b8[8];
+                for (int e = 0; e < 8; ++e) v8[e] = kval(e) * y[e];
+                yput(I, tb, v8);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) { a8[e] = xk[h8 * 8 + e]; b8[e] = xq[h8 * 8 + e]; }
-                *reinterpret_cast<uint4 *>(sm + L::OFF_X + mnmaj<128, 2>(c, tb + h8 * 8, DK)) = pack8_bf16(a8);
-                *reinterpret_cast<uint4 *>(sm + L::OFF_X + mnmaj<128, 2>(c, 64 + tb + h8 * 8, DK)) = pack8_bf16(b8);
-                yput(I, tb + h8 * 8, yo + h8 * 8);
+                for (int e = 0; e < 8; ++e) y[e] = rcp_clamped(y[e]);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) v8[e] = kval(e) * y[e];
+                xput(tb, v8);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) v8[e] = qval(e) * y[e];
+                xput(64 + tb, v8);
             }
             // Later blocks I' > I see this block through e^{Gamma_{m'} - Gamma_j}
-            //   = ls_u * prod_{J = I+1 .. I'-1} bt_J * l8_{I'}   (all factors <= 1)
-            float mid = 1.f;
+            //   = ls_u * prod_{J = I+1 .. I'-1} bt_J * l8_{I'},  ls_u = prod_{s=u+1..15} alpha_s
+            // (all factors <= 1).  Half by half, from the top token down.
 #pragma unroll
-            for (int Ip = 1; Ip < NSUB; ++Ip) {
-                if (Ip > I) {
-                    const float sc = mid * l8[Ip];
-                    float yv[SUB];
+            for (int hh = 1; hh >= 0; --hh) {
+                float ls[8];
+                float r = 1.f;
+                if (hh == 0) {
 #pragma unroll
-                    for (int u = 0; u < SUB; ++u) yv[u] = kv[u] * (ls[u] * sc);
-                    yput(Ip, tb, yv);
-                    yput(Ip, tb + 8, yv + 8);
-                    mid *= bt[Ip];
+                    for (int s = 8; s < SUB; ++s) r *= al[s];
+                }
+#pragma unroll
+                for (int e = 7; e >= 0; --e) { ls[e] = r; r *= al[hh * 8 + e]; }
+                float kk[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) kk[e] = kval(hh * 8 + e) * ls[e];
+#pragma unroll
+                for (int Ip = 1; Ip < NSUB; ++Ip) {
+                    if (Ip > I) {
+                        float v8[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) v8[e] = kk[e] * sc[Ip];
+                        yput(Ip, tb + hh * 8, v8);
+                    }
                 }
             }
         }
@@ -268,37 +338,42 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         }
         mma_pending = true;
 
-        if (active) {
-            float preB = 1.f, postB = 1.f;
+        // e^{Gamma_C - Gamma_t}: K-hat^T (record);  e^{Gamma_t}: Q e^G (record) and (K e^G)^T (smem)
+        {
+            if (active) {
+                if (I == 0) reinterpret_cast<float *>(rec + REC_DEC)[c] = dec;
+                float *khr = reinterpret_cast<float *>(rec + REC_KH) + c * CH + tb;
+                float r = postB;
 #pragma unroll
-            for (int J = 0; J < NSUB; ++J) { if (J < I) preB *= bt[J]; if (J > I) postB *= bt[J]; }
-            if (I == 0) reinterpret_cast<float *>(rec + REC_DEC)[c] = bt[0] * bt[1] * bt[2] * bt[3];
-            // e^{Gamma_t}: Q e^G (record, WQ columns 64..) and (K e^G)^T (smem);
-            // e^{Gamma_C - Gamma_t}: K-hat^T (record)
+                for (int hh = 1; hh >= 0; --hh) {
+                    float kh[8];
 #pragma unroll
-            for (int h8 = 0; h8 < 2; ++h8) {
-                float qe[8], bk[8], kh[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const int u = h8 * 8 + e;
-                    const float pre = preB * lp[u];
-                    qe[e] = qv[u] * pre;
-                    bk[e] = kv[u] * pre;
-                    kh[e] = kv[u] * (ls[u] * postB);
+                    for (int e = 7; e >= 0; --e) { kh[e] = kval(hh * 8 + e) * r; r *= al[hh * 8 + e]; }
+                    *reinterpret_cast<float4 *>(khr + hh * 8) = make_float4(kh[0], kh[1], kh[2], kh[3]);
+                    *reinterpret_cast<float4 *>(khr + hh * 8 + 4) = make_float4(kh[4], kh[5], kh[6], kh[7]);
                 }
-                const int t8 = tb + h8 * 8;
-                *reinterpret_cast<uint4 *>(rec + REC_WQ + mnmaj<128, 2>(c, 64 + t8, DK)) = pack8_bf16(qe);
-                *reinterpret_cast<uint4 *>(sm + L::OFF_BK + kmaj<128, 4>(c, t8, 128)) = pack4_tf32(bk[0], bk[1], bk[2], bk[3]);
-                *reinterpret_cast<uint4 *>(sm + L::OFF_BK + kmaj<128, 4>(c, t8 + 4, 128)) = pack4_tf32(bk[4], bk[5], bk[6], bk[7]);
-                *reinterpret_cast<uint4 *>(rec + REC_KH + kmaj<128, 4>(c, t8, 128)) = pack4_tf32(kh[0], kh[1], kh[2], kh[3]);
-                *reinterpret_cast<uint4 *>(rec + REC_KH + kmaj<128, 4>(c, t8 + 4, 128)) = pack4_tf32(kh[4], kh[5], kh[6], kh[7]);
+                uint16_t *qer = reinterpret_cast<uint16_t *>(rec + REC_WQ) + c * 128 + 64 + tb;
+                float p = preB;
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    float qe[8], bk[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        p *= al[hh * 8 + e];
+                        qe[e] = qval(hh * 8 + e) * p;
+                        bk[e] = kval(hh * 8 + e) * p;
+                    }
+                    *reinterpret_cast<uint4 *>(qer + hh * 8) = pack8_bf16(qe);
+                    *reinterpret_cast<uint4 *>(sm + L::OFF_BK + kmaj<128, 4>(c, tb + hh * 8, 128)) =
+                        pack4_tf32(bk[0], bk[1], bk[2], bk[3]);
+                    *reinterpret_cast<uint4 *>(sm + L::OFF_BK + kmaj<128, 4>(c, tb + hh * 8 + 4, 128)) =
+                        pack4_tf32(bk[4], bk[5], bk[6], bk[7]);
+                }
             }
         }
-        if (!wait_all(bar_mma, 0, mma_pending)) aborted = true;
-        else ph_mma = 1;
-    }
+        if (!wait_all(bar_mma, ph_mma, mma_pending)) { aborted = true; break; }
+        ph_mma ^= 1u;
 
-    if (!aborted) {
         // ---------------- AP: A -> fp32 scratch, P -> record ----------------
         // TMEM lane = row of [k; q]; the four warps of a lane quarter take one
         // 16-column chunk each (chunk = qb).
@@ -316,7 +391,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 #pragma unroll
             for (int dI = 0; dI < 2; ++dI) {
                 const int Ib = I0 + dI;
-                if (cc <= Ib) {
+                if (cc <= Ib) {  // warp-uniform
                     float t[16];
                     tmem_ld16(tmem + lane_base + L::TM_AP + yoff(Ib) + cc * 16, t);
                     tmem_wait_ld();
@@ -338,12 +413,12 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     *reinterpret_cast<float4 *>(sA + i * A_LD + j0 + e) = w;
                 }
             } else {
+                float *pr = reinterpret_cast<float *>(rec + REC_P) + i * CH + j0;
 #pragma unroll
-                for (int e = 0; e < 16; e += 4) {
-                    const uint4 w = pack4_tf32((j0 + e + 0 <= i) ? v16[e + 0] : 0.f, (j0 + e + 1 <= i) ? v16[e + 1] : 0.f,
-                                               (j0 + e + 2 <= i) ? v16[e + 2] : 0.f, (j0 + e + 3 <= i) ? v16[e + 3] : 0.f);
-                    *reinterpret_cast<uint4 *>(rec + REC_P + kmaj_s<128, 4>(i, j0 + e, 8192)) = w;
-                }
+                for (int e = 0; e < 16; e += 4)
+                    *reinterpret_cast<float4 *>(pr + e) =
+                        make_float4((j0 + e + 0 <= i) ? v16[e + 0] : 0.f, (j0 + e + 1 <= i) ? v16[e + 1] : 0.f,
+                                    (j0 + e + 2 <= i) ? v16[e + 2] : 0.f, (j0 + e + 3 <= i) ? v16[e + 3] : 0.f);
             }
         }
         tc_fence_before();
@@ -435,17 +510,16 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 }
                 __syncthreads();
             }
-            // T' = T Diag(beta) -> tf32 K-major tile (smem operand of W, and the record),
+            // T' = T Diag(beta) -> tf32 K-major tile (smem operand of W) and the record,
             // zeros above the diagonal
             for (int e = tid; e < 64 * 16; e += PREP_THREADS) {
                 const int i = e >> 4, j = (e & 15) * 4;
                 const float *src = sTf + i * A_LD + j;
                 const float4 bj = *reinterpret_cast<const float4 *>(s_beta + j);
-                const uint4 w = pack4_tf32(j + 0 <= i ? src[0] * bj.x : 0.f, j + 1 <= i ? src[1] * bj.y : 0.f,
-                                           j + 2 <= i ? src[2] * bj.z : 0.f, j + 3 <= i ? src[3] * bj.w : 0.f);
-                const uint32_t off = kmaj_s<128, 4>(i, j, 8192);
-                *reinterpret_cast<uint4 *>(sm + L::OFF_T + off) = w;
-                *reinterpret_cast<uint4 *>(rec + REC_T + off) = w;
+                const float4 w = make_float4(j + 0 <= i ? src[0] * bj.x : 0.f, j + 1 <= i ? src[1] * bj.y : 0.f,
+                                             j + 2 <= i ? src[2] * bj.z : 0.f, j + 3 <= i ? src[3] * bj.w : 0.f);
+                *reinterpret_cast<uint4 *>(sm + L::OFF_T + kmaj_s<128, 4>(i, j, 8192)) = pack4_tf32(w.x, w.y, w.z, w.w);
+                *reinterpret_cast<float4 *>(rec + REC_T + (i * CH + j) * 4) = w;
             }
         }
         sync_for_mma();
@@ -460,23 +534,28 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             umma_commit(bar_mma);
         }
         mma_pending = true;
-        if (!wait_all(bar_mma, 1, mma_pending)) aborted = true;
-    }
-    if (!aborted && (warp & 3) < DK / 32) {  // W^T row ch -> W columns (tokens 16 qb ..) of the record's WQ
-        const int i0 = qb * 16;
-        float t[16];
-        tmem_ld16(tmem + lane_base + L::TM_W + i0, t);
-        tmem_wait_ld();
-        float a8[8], b8[8];
+        if (!wait_all(bar_mma, ph_mma, mma_pending)) { aborted = true; break; }
+        ph_mma ^= 1u;
+        if ((warp & 3) < DK / 32) {  // W^T row ch -> W columns (tokens 16 qb ..) of the record's WQ
+            const int i0 = qb * 16;
+            float t[16];
+            tmem_ld16(tmem + lane_base + L::TM_W + i0, t);
+            tmem_wait_ld();
+            float a8[8], b8[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) { a8[e] = t[e]; b8[e] = t[8 + e]; }
-        *reinterpret_cast<uint4 *>(rec + REC_WQ + mnmaj<128, 2>(ch, i0, DK)) = pack8_bf16(a8);
-        *reinterpret_cast<uint4 *>(rec + REC_WQ + mnmaj<128, 2>(ch, i0 + 8, DK)) = pack8_bf16(b8);
+            for (int e = 0; e < 8; ++e) { a8[e] = t[e]; b8[e] = t[8 + e]; }
+            uint16_t *wr = reinterpret_cast<uint16_t *>(rec + REC_WQ) + ch * 128 + i0;
+            *reinterpret_cast<uint4 *>(wr) = pack8_bf16(a8);
+            *reinterpret_cast<uint4 *>(wr + 8) = pack8_bf16(b8);
+        }
+        tc_fence_before();
+        __syncthreads();  // this item's shared memory and TMEM are free for the next one
+        tc_fence_after();
     }
 
     if (aborted && tid == 0) {
         // Leave nothing in flight that targets this CTA's smem or TMEM.
-        if (tma_pending) mbar_wait(bar_in, 0, ~0ull, prm.st);
+        if (tma_pending) mbar_wait(bar_in, ph_in, ~0ull, prm.st);
         if (mma_pending) mbar_wait(bar_mma, ph_mma, ~0ull, prm.st);
     }
     tc_fence_before();
@@ -487,19 +566,21 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 
 template <int DK>
 static cudaError_t launch_prep_t(const CUtensorMap &tq, const CUtensorMap &tk, const PrepParams &prm,
-                                 cudaStream_t stream) {
+                                 int num_sms, cudaStream_t stream) {
     using L = PrepLayout<DK>;
     cudaError_t e = cudaFuncSetAttribute(prep_kernel<DK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          L::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    prep_kernel<DK><<<prm.B * prm.H * prm.nseg, PREP_THREADS, L::SMEM_BYTES, stream>>>(tq, tk, prm);
+    const long long items = (long long)prm.B * prm.H * prm.nseg;
+    const int grid = (int)(items < 2LL * num_sms ? items : 2LL * num_sms);
+    prep_kernel<DK><<<grid, PREP_THREADS, L::SMEM_BYTES, stream>>>(tq, tk, prm);
     return cudaGetLastError();
 }
 
 cudaError_t launch_prep(const CUtensorMap &tq, const CUtensorMap &tk, const PrepParams &prm, int dk,
-                        cudaStream_t stream) {
-    if (dk == 128) return launch_prep_t<128>(tq, tk, prm, stream);
-    return launch_prep_t<64>(tq, tk, prm, stream);
+                        int num_sms, cudaStream_t stream) {
+    if (dk == 128) return launch_prep_t<128>(tq, tk, prm, num_sms, stream);
+    return launch_prep_t<64>(tq, tk, prm, num_sms, stream);
 }
 
 }  // namespace kda
