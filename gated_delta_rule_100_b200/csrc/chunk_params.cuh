@@ -7,11 +7,12 @@
 
 namespace kda {
 
-// One CTA per (b, h, chunk) of chunks [n_begin, n_begin + nseg).
+// Items (b, h, chunk) of chunks [n_begin, n_begin + nseg), claimed by persistent CTAs.
 struct PrepParams {
     const float *g;      // [B, T, H, dk]
     const float *beta;   // [B, T, H]
     uint8_t *ws;         // records [B*H][nseg][REC_BYTES]
+    int *ticket;         // item counter, zero at launch: CTAs claim items from it
     int B, T, H, n_begin, nseg;
     DeviceStatus st;
 };

@@ -27,6 +27,7 @@ namespace kda {
 cudaError_t launch_prep(const CUtensorMap &tq, const CUtensorMap &tk, const PrepParams &prm, int dk,
                         int num_sms, cudaStream_t stream);
 cudaError_t launch_chain(const CUtensorMap *maps, const ChainParams &prm, int dk, cudaStream_t stream);
+int chain_value_slice();
 }
 
 // Device-side status word: kernels OR error bits into it (one per device,
@@ -69,40 +70,61 @@ int get_encoder(PFN_cuTensorMapEncodeTiled_v12000 *fn) {
     return KDA_OK;
 }
 
-// Per-device workspace of the prefill: the per-chunk records written by the
-// prep kernel and read by the chain kernel, plus a state buffer carried
-// between segments.  Grown on demand (cudaFree synchronises the device, so no
-// kernel still reads the old buffer) and kept for later calls.  Calls on
-// different streams are ordered on it by `done`, recorded after each call's
-// last kernel and waited on by the next call's stream.
-constexpr size_t kWorkspaceCap = size_t(2) << 30;  // records of one segment, bytes
+// Per-device workspace of the prefill: the per-chunk records passed from the
+// prep kernel to the chain kernel, the prep kernel's item counters, and a
+// state buffer carried between segments.  Grown on demand (cudaFree
+// synchronises the device, so no kernel still reads the old buffer) and kept
+// for later calls.  Calls on different streams are ordered on it by `done`,
+// recorded after each call's last kernel and waited on by the next call's
+// stream.
+//
+// A sequence whose records fit the cap runs as one segment (prep, then chain,
+// on the caller's stream).  A longer one runs in segments over two record
+// buffers so that the prep kernel of segment i + 1 overlaps the chain kernel
+// of segment i: prep on a low-priority internal stream, chain on a
+// high-priority one (its few CTAs are placed first, prep fills the other SMs).
+constexpr size_t kWorkspaceCap = size_t(2) << 30;  // bytes of records
+constexpr size_t kTicketBytes = 256;               // two item counters at the front of the records
 struct Workspace {
-    uint8_t *rec = nullptr;
-    size_t rec_bytes = 0;
+    uint8_t *base = nullptr;  // [tickets][records]
+    size_t base_bytes = 0;
     float *state = nullptr;
     size_t state_bytes = 0;
     cudaEvent_t done = nullptr;
+    cudaStream_t lo = nullptr, hi = nullptr;  // prep and chain streams of the segmented path
+    cudaEvent_t fork = nullptr, prep_done[2] = {nullptr, nullptr}, chain_done[2] = {nullptr, nullptr};
 };
 Workspace g_ws[kMaxDevices];
 
 size_t rec_row_bytes(int B, int H) { return (size_t)B * H * kda::REC_BYTES; }
 
-// Chunks per segment: as many as fit the cap, at least one.
-int segment_chunks(int B, int T, int H) {
-    const int nchunks = (T + kda::CH - 1) / kda::CH;
-    const size_t fit = kWorkspaceCap / rec_row_bytes(B, H);
-    return (int)(fit < 1 ? 1 : (fit < (size_t)nchunks ? fit : (size_t)nchunks));
+struct SegPlan {
+    int nchunks, seg, nbuf;  // chunks, chunks per segment, record buffers
+};
+SegPlan plan_segments(int B, int T, int H) {
+    SegPlan p;
+    p.nchunks = (T + kda::CH - 1) / kda::CH;
+    const size_t row = rec_row_bytes(B, H);
+    if ((size_t)p.nchunks * row <= kWorkspaceCap) {
+        p.seg = p.nchunks;
+        p.nbuf = 1;
+    } else {
+        const size_t fit = kWorkspaceCap / (2 * row);
+        p.seg = (int)(fit < 1 ? 1 : fit);
+        p.nbuf = 2;
+    }
+    return p;
 }
 
 // Called with g_mu held.
-int reserve_workspace(int dev, size_t rec_bytes, size_t state_bytes, Workspace **out) {
+int reserve_workspace(int dev, size_t base_bytes, size_t state_bytes, bool streams, Workspace **out) {
     Workspace &w = g_ws[dev];
-    if (w.rec_bytes < rec_bytes) {
-        if (w.rec != nullptr && cudaFree(w.rec) != cudaSuccess) return KDA_ERR_CUDA;
-        w.rec = nullptr;
-        w.rec_bytes = 0;
-        if (cudaMalloc(&w.rec, rec_bytes) != cudaSuccess) return KDA_ERR_CUDA;
-        w.rec_bytes = rec_bytes;
+    if (w.base_bytes < base_bytes) {
+        if (w.base != nullptr && cudaFree(w.base) != cudaSuccess) return KDA_ERR_CUDA;
+        w.base = nullptr;
+        w.base_bytes = 0;
+        if (cudaMalloc(&w.base, base_bytes) != cudaSuccess) return KDA_ERR_CUDA;
+        w.base_bytes = base_bytes;
     }
     if (w.state_bytes < state_bytes) {
         if (w.state != nullptr && cudaFree(w.state) != cudaSuccess) return KDA_ERR_CUDA;
@@ -113,6 +135,16 @@ int reserve_workspace(int dev, size_t rec_bytes, size_t state_bytes, Workspace *
     }
     if (w.done == nullptr && cudaEventCreateWithFlags(&w.done, cudaEventDisableTiming) != cudaSuccess)
         return KDA_ERR_CUDA;
+    if (streams && w.lo == nullptr) {
+        int least = 0, greatest = 0;
+        if (cudaDeviceGetStreamPriorityRange(&least, &greatest) != cudaSuccess ||
+            cudaStreamCreateWithPriority(&w.lo, cudaStreamNonBlocking, least) != cudaSuccess ||
+            cudaStreamCreateWithPriority(&w.hi, cudaStreamNonBlocking, greatest) != cudaSuccess)
+            return KDA_ERR_CUDA;
+        cudaEvent_t *evs[5] = {&w.fork, &w.prep_done[0], &w.prep_done[1], &w.chain_done[0], &w.chain_done[1]};
+        for (cudaEvent_t *e : evs)
+            if (cudaEventCreateWithFlags(e, cudaEventDisableTiming) != cudaSuccess) return KDA_ERR_CUDA;
+    }
     *out = &w;
     return KDA_OK;
 }
@@ -208,10 +240,8 @@ int make_rec_maps(PFN_cuTensorMapEncodeTiled_v12000 enc, const uint8_t *rec, lon
     return KDA_OK;
 }
 
-// Value-column slices per (b, h) in the chain kernel: two 64-column CTAs when
-// that still fits one CTA per SM (the chain is latency-bound, and half the
-// columns halve every state product), else one.
-int chain_slices(int B, int H, int dv, int sms) { return (dv == 128 && 2LL * B * H <= sms) ? 2 : 1; }
+// Value-column slices per (b, h) in the chain kernel: one CTA per 64 columns.
+int chain_slices(int dv) { return dv / kda::chain_value_slice(); }
 
 }  // namespace
 
@@ -283,14 +313,16 @@ int kda_chunk_fwd(const void *q, const void *k, const void *v, const float *g, c
                  CU_TENSOR_MAP_SWIZZLE_128B) != KDA_OK)
         return KDA_ERR_CUDA;
 
-    const int nchunks = (T + kda::CH - 1) / kda::CH;
-    const int seg = segment_chunks(B, T, H);
-    const bool multi = seg < nchunks;
+    const SegPlan pl = plan_segments(B, T, H);
+    const int nchunks = pl.nchunks, seg = pl.seg;
+    const bool multi = pl.nbuf == 2;
+    const size_t row = rec_row_bytes(B, H);
     const size_t state_bytes = (multi && hT == nullptr) ? (size_t)B * H * dk * dv * sizeof(float) : 0;
+    const int sms = num_sms(dev);
 
     std::lock_guard<std::mutex> lk(g_mu);
     Workspace *w = nullptr;
-    if (int st = reserve_workspace(dev, (size_t)seg * rec_row_bytes(B, H), state_bytes, &w); st != KDA_OK)
+    if (int st = reserve_workspace(dev, kTicketBytes + pl.nbuf * seg * row, state_bytes, multi, &w); st != KDA_OK)
         return st;
     if (cudaStreamWaitEvent(s, w->done, 0) != cudaSuccess) return KDA_ERR_CUDA;
 
@@ -300,40 +332,62 @@ int kda_chunk_fwd(const void *q, const void *k, const void *v, const float *g, c
     dst.wait_polls = polls ? polls : ~0ull;
     // State carried between segments: the caller's hT when given, else the workspace's.
     float *carry = hT != nullptr ? hT : w->state;
-    const int sms = num_sms(dev);
-    CUtensorMap rmaps[4];
-    if (make_rec_maps(enc, w->rec, (long long)B * H * seg, dk, rmaps) != KDA_OK) return KDA_ERR_CUDA;
+    int *tickets = reinterpret_cast<int *>(w->base);
+    uint8_t *recs[2] = {w->base + kTicketBytes, w->base + kTicketBytes + (size_t)seg * row};
+    CUtensorMap rmaps[2][4];
+    for (int i = 0; i < pl.nbuf; ++i)
+        if (make_rec_maps(enc, recs[i], (long long)B * H * seg, dk, rmaps[i]) != KDA_OK) return KDA_ERR_CUDA;
 
-    for (int n0 = 0; n0 < nchunks; n0 += seg) {
+    cudaStream_t sp = s, sc = s;  // prep and chain streams
+    if (multi) {
+        sp = w->lo;
+        sc = w->hi;
+        if (cudaEventRecord(w->fork, s) != cudaSuccess || cudaStreamWaitEvent(sp, w->fork, 0) != cudaSuccess ||
+            cudaStreamWaitEvent(sc, w->fork, 0) != cudaSuccess)
+            return KDA_ERR_CUDA;
+    }
+    int i = 0;
+    for (int n0 = 0; n0 < nchunks; n0 += seg, ++i) {
         const int cnt = nchunks - n0 < seg ? nchunks - n0 : seg;
         const bool last = n0 + cnt == nchunks;
+        const int buf = multi ? (i & 1) : 0;
+        // buffer reuse: the chain kernel two segments back has read it
+        if (multi && i >= 2 && cudaStreamWaitEvent(sp, w->chain_done[buf], 0) != cudaSuccess) return KDA_ERR_CUDA;
+        if (cudaMemsetAsync(tickets + buf, 0, sizeof(int), sp) != cudaSuccess) return KDA_ERR_CUDA;
         kda::PrepParams pp;
         pp.g = g;
         pp.beta = beta;
-        pp.ws = w->rec;
+        pp.ws = recs[buf];
+        pp.ticket = tickets + buf;
         pp.B = B; pp.T = T; pp.H = H;
         pp.n_begin = n0;
         pp.nseg = cnt;
         pp.st = dst;
-        cudaError_t e = timed_launch(dev, 0, s, [&] { return kda::launch_prep(tq, tk, pp, dk, sms, s); });
+        cudaError_t e = timed_launch(dev, 0, sp, [&] { return kda::launch_prep(tq, tk, pp, dk, sms, sp); });
         if (e != cudaSuccess) return KDA_ERR_CUDA;
+        if (multi && (cudaEventRecord(w->prep_done[buf], sp) != cudaSuccess ||
+                      cudaStreamWaitEvent(sc, w->prep_done[buf], 0) != cudaSuccess))
+            return KDA_ERR_CUDA;
 
         kda::ChainParams cp;
         cp.v = static_cast<const uint16_t *>(v);
         cp.h0 = n0 == 0 ? h0 : carry;
         cp.out = static_cast<uint16_t *>(out);
         cp.hT = last ? hT : carry;
-        cp.ws = w->rec;
+        cp.ws = recs[buf];
         cp.scale = scale;
         cp.B = B; cp.T = T; cp.H = H; cp.DV = dv;
         cp.n_begin = n0;
         cp.nseg = cnt;
-        cp.nslices = chain_slices(B, H, dv, sms);
+        cp.nslices = chain_slices(dv);
         cp.st = dst;
         cp.inject_wait_polls = g_inject_polls.load();
-        e = timed_launch(dev, 1, s, [&] { return kda::launch_chain(rmaps, cp, dk, s); });
+        e = timed_launch(dev, 1, sc, [&] { return kda::launch_chain(rmaps[buf], cp, dk, sc); });
         if (e != cudaSuccess) return KDA_ERR_CUDA;
+        if (multi && cudaEventRecord(w->chain_done[buf], sc) != cudaSuccess) return KDA_ERR_CUDA;
     }
+    // join: the last chain kernel follows every prep kernel
+    if (multi && cudaStreamWaitEvent(s, w->chain_done[(i - 1) & 1], 0) != cudaSuccess) return KDA_ERR_CUDA;
     if (cudaEventRecord(w->done, s) != cudaSuccess) return KDA_ERR_CUDA;
     return KDA_OK;
 }
@@ -341,10 +395,9 @@ int kda_chunk_fwd(const void *q, const void *k, const void *v, const float *g, c
 size_t kda_chunk_fwd_workspace_bytes(int B, int T, int H, int dk, int dv) {
     if (B < 1 || H < 1 || T < 0 || (dk != 64 && dk != 128) || (dv != 64 && dv != 128)) return 0;
     if (T == 0) return 0;
-    const int nchunks = (T + kda::CH - 1) / kda::CH;
-    const int seg = segment_chunks(B, T, H);
-    const size_t state = seg < nchunks ? (size_t)B * H * dk * dv * sizeof(float) : 0;
-    return (size_t)seg * rec_row_bytes(B, H) + state;
+    const SegPlan pl = plan_segments(B, T, H);
+    const size_t state = pl.nbuf == 2 ? (size_t)B * H * dk * dv * sizeof(float) : 0;
+    return kTicketBytes + (size_t)pl.nbuf * pl.seg * rec_row_bytes(B, H) + state;
 }
 
 void kda_debug_kernel_timing(int enable) { g_timing.store(enable != 0); }
@@ -372,9 +425,9 @@ int kda_release_workspace(void) {
     std::lock_guard<std::mutex> lk(g_mu);
     Workspace &w = g_ws[dev];
     int st = KDA_OK;
-    if (w.rec != nullptr && cudaFree(w.rec) != cudaSuccess) st = KDA_ERR_CUDA;
+    if (w.base != nullptr && cudaFree(w.base) != cudaSuccess) st = KDA_ERR_CUDA;
     if (w.state != nullptr && cudaFree(w.state) != cudaSuccess) st = KDA_ERR_CUDA;
-    w.rec = nullptr; w.rec_bytes = 0;
+    w.base = nullptr; w.base_bytes = 0;
     w.state = nullptr; w.state_bytes = 0;
     return st;
 }
@@ -405,7 +458,8 @@ int kda_decode_step(const void *q, const void *k, const void *v, const float *g,
 // device-wide synchronisation that freeing a grown workspace costs.  This
 // variant runs the same two kernels over chunk records kept in a fixed array
 // that is part of the module image, in as many segments as the array holds.
-// Nothing in it needs to start at zero: the prep kernel writes every record
+// Of the scratch, only the prep kernel's item counter must start at zero, and
+// each call clears it before each launch; the prep kernel writes every record
 // byte the chain kernel's results depend on before the chain kernel reads it
 // (rows it leaves unwritten feed accumulator lanes that are discarded), and
 // the carried state is written before it is read.
@@ -458,8 +512,8 @@ int kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const flo
     const int nchunks = (T + kda::CH - 1) / kda::CH;
     const size_t row = rec_row_bytes(B, H);
     const size_t state_bytes = hT == nullptr ? round256((size_t)B * H * dk * dv * sizeof(float)) : 0;
-    if (state_bytes + row > kScratchBytes) return KDA_ERR_SCRATCH_LIMIT;
-    const size_t fit = (kScratchBytes - state_bytes) / row;
+    if (kTicketBytes + state_bytes + row > kScratchBytes) return KDA_ERR_SCRATCH_LIMIT;
+    const size_t fit = (kScratchBytes - kTicketBytes - state_bytes) / row;
     const int seg = fit < (size_t)nchunks ? (int)fit : nchunks;
 
     int dev = 0;
@@ -482,8 +536,10 @@ int kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const flo
     kda::DeviceStatus dst;
     dst.word = word;
     dst.wait_polls = polls ? polls : ~0ull;
-    float *carry = hT != nullptr ? hT : reinterpret_cast<float *>(scratch);
-    uint8_t *recs = scratch + state_bytes;
+    // [the prep kernel's item counter][carried state, when hT is NULL][records]
+    int *ticket = reinterpret_cast<int *>(scratch);
+    float *carry = hT != nullptr ? hT : reinterpret_cast<float *>(scratch + kTicketBytes);
+    uint8_t *recs = scratch + kTicketBytes + state_bytes;
     const int sms = num_sms(dev);
     CUtensorMap rmaps[4];
     if (make_rec_maps(enc, recs, (long long)B * H * seg, dk, rmaps) != KDA_OK) return KDA_ERR_CUDA;
@@ -495,11 +551,14 @@ int kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const flo
         pp.g = g;
         pp.beta = beta;
         pp.ws = recs;
+        pp.ticket = ticket;
         pp.B = B; pp.T = T; pp.H = H;
         pp.n_begin = n0;
         pp.nseg = cnt;
         pp.st = dst;
-        if (kda::launch_prep(tq, tk, pp, dk, sms, s) != cudaSuccess) return KDA_ERR_CUDA;
+        if (cudaMemsetAsync(ticket, 0, sizeof(int), s) != cudaSuccess ||  // the counter starts at zero
+            kda::launch_prep(tq, tk, pp, dk, sms, s) != cudaSuccess)
+            return KDA_ERR_CUDA;
 
         kda::ChainParams cp;
         cp.v = static_cast<const uint16_t *>(v);
@@ -511,7 +570,7 @@ int kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const flo
         cp.B = B; cp.T = T; cp.H = H; cp.DV = dv;
         cp.n_begin = n0;
         cp.nseg = cnt;
-        cp.nslices = chain_slices(B, H, dv, sms);
+        cp.nslices = chain_slices(dv);
         cp.st = dst;
         cp.inject_wait_polls = g_inject_polls.load();
         if (kda::launch_chain(rmaps, cp, dk, s) != cudaSuccess) return KDA_ERR_CUDA;

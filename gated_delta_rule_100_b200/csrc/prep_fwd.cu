@@ -23,8 +23,8 @@
 // >= -160.  All factors come from running products of alpha = e^g (one exp
 // per input element) plus one reciprocal per factor above 1.
 //
-// Persistent CTAs (two per SM, 512 threads) loop over the items; while one
-// item is processed the next one's q, k and g are prefetched into L2.  In the
+// Persistent CTAs (two per SM, 512 threads) claim items from a counter; while
+// one item is processed the next one's q, k and g are prefetched into L2.  In the
 // elementwise phase thread (c, I) owns key channel c and tokens 16 I .. 16 I +
 // 15 (a two-level scan: products inside the block, then the four block
 // totals through shared memory); its key and query values are held as bf16
@@ -57,11 +57,10 @@ struct PrepLayout {
     static constexpr int OFF_F = 0;
     static constexpr int OFF_XCH = OFF_F;                    // block products exchange (E only)
     static constexpr int OFF_X = OFF_F;                      // MN-major bf16 [DK][128]
-    static constexpr int OFF_Y0 = OFF_X + DK * 256;          // SW32  [DK][16]
-    static constexpr int OFF_Y1 = OFF_Y0 + DK * 32;          // SW64  [DK][32]
-    static constexpr int OFF_Y2 = OFF_Y1 + DK * 64;          // SW128 [DK][64] (48 used)
-    static constexpr int OFF_Y3 = OFF_Y2 + DK * 128;         // SW128 [DK][64]
-    static constexpr int FORM_B = DK * (256 + 32 + 64 + 128 + 128);
+    // [Y^(0) | Y^(1) | Y^(2) | Y^(3)]: MN-major bf16 [DK][160], 64B swizzle (32-column
+    // blocks); Y^(I) starts at column yoff(I), so one 160-wide product forms all four
+    static constexpr int OFF_Y = OFF_X + DK * 256;
+    static constexpr int FORM_B = DK * (256 + 320);
     static constexpr int OFF_A = OFF_F;                      // fp32 [64][A_LD]
     static constexpr int OFF_TF = OFF_A + 64 * A_LD * 4;     // fp32 [64][A_LD]
     static constexpr int OFF_T = OFF_F + align1k(2 * 64 * A_LD * 4);  // tf32 K-major [64][64], 8 KB K-blocks
@@ -103,6 +102,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     float *s_xch = reinterpret_cast<float *>(sm + L::OFF_XCH);          // [2][4][128]
     uint64_t *s_bars = reinterpret_cast<uint64_t *>(sm + L::OFF_MISC + 768);
     uint32_t *s_tmem = reinterpret_cast<uint32_t *>(sm + L::OFF_MISC + 800);
+    int *s_next = reinterpret_cast<int *>(sm + L::OFF_MISC + 808);  // the item claimed next
     const uint32_t bar_in = smem_u32(&s_bars[0]);
     const uint32_t bar_mma = smem_u32(&s_bars[1]);
 
@@ -158,7 +158,13 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     const int c = ch, I = qb, tb = SUB * I;
     const bool active = c < DK;
 
-    for (int item = blockIdx.x; item < nitems && !aborted; item += gridDim.x) {
+    if (tid == 0) *s_next = atomicAdd(prm.ticket, 1);
+    __syncthreads();
+    for (int item = *s_next; item < nitems && !aborted;) {
+        __syncthreads();  // every thread has read s_next
+        if (tid == 0) *s_next = atomicAdd(prm.ticket, 1);  // claimed now, so its inputs can be prefetched
+        __syncthreads();
+        const int next = *s_next;
         int b, h, t0;
         item_coords(item, b, h, t0);
         uint8_t *rec = prm.ws + (size_t)item * REC_BYTES;
@@ -181,9 +187,9 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         }
         if (tid < CH) s_beta[tid] = (t0 + tid < T) ? prm.beta[((size_t)b * T + t0 + tid) * H + h] : 0.f;
         // the next item's q, k and g into L2 while this one is processed
-        if (item + (int)gridDim.x < nitems) {
+        if (next < nitems) {
             int nb, nh, nt0;
-            item_coords(item + gridDim.x, nb, nh, nt0);
+            item_coords(next, nb, nh, nt0);
             if (tid == 0) {
 #pragma unroll
                 for (int kb = 0; kb < DK / 64; ++kb) {
@@ -245,10 +251,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         __syncthreads();  // the exchange area becomes X
 
         auto yput = [&](int Iy, int j0, const float (&v8)[8]) {
-            if (Iy == 0)      *reinterpret_cast<uint4 *>(sm + L::OFF_Y0 + mnmaj<32, 2>(c, j0, DK)) = pack8_bf16(v8);
-            else if (Iy == 1) *reinterpret_cast<uint4 *>(sm + L::OFF_Y1 + mnmaj<64, 2>(c, j0, DK)) = pack8_bf16(v8);
-            else if (Iy == 2) *reinterpret_cast<uint4 *>(sm + L::OFF_Y2 + mnmaj<128, 2>(c, j0, DK)) = pack8_bf16(v8);
-            else              *reinterpret_cast<uint4 *>(sm + L::OFF_Y3 + mnmaj<128, 2>(c, j0, DK)) = pack8_bf16(v8);
+            *reinterpret_cast<uint4 *>(sm + L::OFF_Y + mnmaj<64, 2>(c, yoff(Iy) + j0, DK)) = pack8_bf16(v8);
         };
         auto xput = [&](int col, const float (&v8)[8]) {
             *reinterpret_cast<uint4 *>(sm + L::OFF_X + mnmaj<128, 2>(c, col, DK)) = pack8_bf16(v8);
@@ -319,21 +322,12 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         sync_for_mma();
 
         // ---------------- F: formation products (bf16), overlapped with the rest of E ----------------
-        if (tid == 0) {
+        if (tid == 0) {  // X [Y^(0) | .. | Y^(3)]^T: 128 x 160, column block I' = D^(I')
+            const uint32_t idesc = make_idesc(1, true, true, 128, yoff(NSUB));
 #pragma unroll
-            for (int If = 0; If < NSUB; ++If) {
-                const uint32_t idesc = make_idesc(1, true, true, 128, SUB * (If + 1));
-#pragma unroll
-                for (int kk = 0; kk < DK / 16; ++kk) {
-                    const uint64_t da = desc_mnmaj<128>(sbase + L::OFF_X, DK, kk * 16);
-                    uint64_t db;
-                    if (If == 0)      db = desc_mnmaj<32>(sbase + L::OFF_Y0, DK, kk * 16);
-                    else if (If == 1) db = desc_mnmaj<64>(sbase + L::OFF_Y1, DK, kk * 16);
-                    else if (If == 2) db = desc_mnmaj<128>(sbase + L::OFF_Y2, DK, kk * 16);
-                    else              db = desc_mnmaj<128>(sbase + L::OFF_Y3, DK, kk * 16);
-                    umma<0>(tmem + L::TM_AP + yoff(If), da, db, idesc, kk > 0);
-                }
-            }
+            for (int kk = 0; kk < DK / 16; ++kk)
+                umma<0>(tmem + L::TM_AP, desc_mnmaj<128>(sbase + L::OFF_X, DK, kk * 16),
+                        desc_mnmaj<64>(sbase + L::OFF_Y, DK, kk * 16), idesc, kk > 0);
             umma_commit(bar_mma);
         }
         mma_pending = true;
@@ -551,6 +545,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         tc_fence_before();
         __syncthreads();  // this item's shared memory and TMEM are free for the next one
         tc_fence_after();
+        item = next;
     }
 
     if (aborted && tid == 0) {

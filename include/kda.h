@@ -135,8 +135,8 @@ KDA_API int kda_decode_step(const void *q, const void *k, const void *v,
  * records of one 64-token chunk of every (b, h) (B * H * 99,328 bytes), plus,
  * when hT is NULL, the fp32 state [B, H, dk, dv] carried between segments,
  * must fit in 64 MiB (B * H <= 675 with hT given); a larger problem returns
- * KDA_ERR_SCRATCH_LIMIT without enqueueing work.  Nothing in the scratch
- * needs to start at zero.
+ * KDA_ERR_SCRATCH_LIMIT without enqueueing work.  The only part of the
+ * scratch that must start at zero, an item counter, is cleared by each call.
  *
  * The first call on a device looks up the array's device address (with that
  * device current) and caches it: make that first call before any stream
@@ -151,10 +151,12 @@ KDA_API int kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v,
 
 /*
  * kda_chunk_fwd_workspace_bytes -- device memory kda_chunk_fwd holds for these
- * sizes: the per-chunk records of one segment (about 97 KB per 64-token chunk
- * and (b, h); a segment spans as many chunks as fit in 2 GiB, at least one)
- * plus, when the sequence takes more than one segment, an fp32 state buffer
- * [B, H, dk, dv].  0 for unsupported sizes or T == 0.
+ * sizes: the per-chunk records (about 97 KB per 64-token chunk and (b, h)) of
+ * the whole sequence when they fit in 2 GiB, else of two segments of as many
+ * chunks as fit in 1 GiB each (at least one; the prep kernel of one segment
+ * overlaps the state chain of the previous one on two internal streams),
+ * plus then an fp32 state buffer [B, H, dk, dv], plus 256 bytes of counters.
+ * 0 for unsupported sizes or T == 0.
  */
 KDA_API size_t kda_chunk_fwd_workspace_bytes(int B, int T, int H, int dk, int dv);
 

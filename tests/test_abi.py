@@ -101,13 +101,14 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
 
 def test_workspace_bytes(lib):
     rec = 99328  # bytes of one chunk record of one (b, h)
-    # one segment: 4 chunks of one head, no state buffer
-    assert kda.workspace_bytes(1, 256, 1, 128, 128) == 4 * rec
-    assert kda.workspace_bytes(2, 65, 3, 64, 64) == 2 * 6 * rec
-    # long sequence: segments of as many chunks as fit in 2 GiB, plus the carried state
+    tick = 256   # the prep kernel's item counters
+    # one segment: all chunks' records, no state buffer
+    assert kda.workspace_bytes(1, 256, 1, 128, 128) == tick + 4 * rec
+    assert kda.workspace_bytes(2, 65, 3, 64, 64) == tick + 2 * 6 * rec
+    # long sequence: two buffers of as many chunks as fit in 1 GiB each, plus the carried state
     row = 32 * rec
-    seg = (2 << 30) // row
-    assert kda.workspace_bytes(1, 1 << 20, 32, 128, 128) == seg * row + 32 * 128 * 128 * 4
+    seg = (1 << 30) // row
+    assert kda.workspace_bytes(1, 1 << 20, 32, 128, 128) == tick + 2 * seg * row + 32 * 128 * 128 * 4
     # unsupported or empty
     assert kda.workspace_bytes(1, 0, 1, 128, 128) == 0
     assert kda.workspace_bytes(1, 64, 1, 96, 128) == 0
