@@ -15,8 +15,10 @@
 // accumulators:
 //   1   D1 = [W; Q e^G] S0            bf16, A = record WQ (MN-major)
 //   U   U  = T' V                      tf32, A = record T' (rows 64..127 unused)
-//   3a  D3 = K-hat^T Vnew              tf32
-//   3b  D1 += [.; P] Vnew              tf32, rows 64..127 = the output block
+//   3a  D3 = K-hat^T Vnew              fp16
+//   3b  D1 += [.; P] Vnew              fp16, rows 64..127 = the output block
+// (fp16 keeps tf32's 10-bit mantissa; K-hat, P and Vnew are bounded in
+// magnitude, T' is kept in tf32 for its range).
 //
 // Warp roles.  One issuer warp (its lane 0) issues every tensor load and every
 // product; sixteen compute warps move data between TMEM, registers and shared
@@ -27,8 +29,8 @@
 // order, is fed as soon as each operand is ready.  Per chunk n it runs
 // 1(n), 3b(n-1), 3a(n), U(n+1): only 1 and 3a lie on the state's critical
 // path, the other two fill the pipe while the compute warps form Vnew(n) and
-// update the state.  Buffers: two output accumulators, two Vnew tiles, two
-// K-hat and two T' buffers; one each of WQ, P, V^T and S0.
+// update the state.  Buffers: two output accumulators and two each of the
+// Vnew tiles, WQ, P, K-hat and T'; one V^T and one S0.
 //
 // The state lives in fp32 registers (compute thread (c, g) holds row c, 16
 // columns); a bf16 copy in shared memory feeds the tensor core.  The values V
@@ -52,21 +54,21 @@ template <int DK>
 struct ChainLayout {
     static_assert(DK == 64 || DK == 128, "dk");
     static constexpr int VS = CHAIN_VS;
-    static constexpr int OFF_WQ = 0;          // bf16 MN-major [DK][128]: [W; Q e^G]
-    static constexpr int OFF_P = 32768;       // tf32 K-major [64][64] (8 KB K-blocks)
-    static constexpr int OFF_KH = 49152;      // two tf32 K-major [128][64] (16 KB K-blocks)
+    static constexpr int OFF_WQ = 0;          // two bf16 MN-major [DK][128]: [W; Q e^G] (32 KB slots)
+    static constexpr int OFF_P = 65536;       // two fp16 K-major [64][64] (8 KB)
+    static constexpr int OFF_KH = 81920;      // two fp16 K-major [128][64] (16 KB)
     static constexpr int OFF_T = 114688;      // two tf32 K-major [64][64] (8 KB K-blocks)
     static constexpr int OFF_DEC = 147456;    // two 512-byte slots of e^{Gamma_C} (with K-hat)
     static constexpr int OFF_S0 = 148480;     // bf16 MN-major S0 [DK][64], 128B swizzle
     static constexpr int OFF_VT = OFF_S0 + DK * VS * 2;   // tf32 K-major V^T [64][64]
-    static constexpr int OFF_VN = OFF_VT + VS * 256;      // two tf32 K-major Vnew^T [64][64]
-    static constexpr int OFF_MISC = OFF_VN + 2 * VS * 256;  // barriers, TMEM address, abort flag
+    static constexpr int OFF_VN = OFF_VT + VS * 256;      // two fp16 K-major Vnew^T [64][64]
+    static constexpr int OFF_MISC = OFF_VN + 2 * VS * 128;  // barriers, TMEM address, abort flag
     static constexpr int TOTAL = OFF_MISC + 1024;
     static constexpr int SMEM_BYTES = TOTAL + 1024;  // slack for the 1 KB base alignment
     static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
     static_assert(OFF_S0 % 1024 == 0 && OFF_VT % 1024 == 0 && OFF_VN % 1024 == 0, "1 KB aligned tiles");
-    // The 128-row views read 8 KB before P (rows 0..63, discarded) and 8 KB
-    // past T's second buffer (rows 64..127, discarded).
+    // The 128-row views read 8 KB before each P buffer (rows 0..63, discarded)
+    // and 8 KB past T's second buffer (rows 64..127, discarded).
     static_assert(OFF_P >= 8192 && OFF_T + 2 * 16384 + 8192 <= TOTAL, "operand views stay in bounds");
 
     static constexpr uint32_t TM_U = 0;          // U (lane = token)
@@ -87,7 +89,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
     constexpr int TG = CHAIN_WORKERS / NP;  // token groups (V loads)
     constexpr int TPT = CH / TG;            // tokens per compute thread (V loads)
     static_assert(TPT % 4 == 0 && CPT == 16, "thread mapping");
-    constexpr uint32_t TX_T = 16384, TX_W = DK * 256, TX_P = 16384, TX_K = 32768 + 512;
+    constexpr uint32_t TX_T = 16384, TX_W = DK * 256, TX_P = 8192, TX_K = 16384 + 512;
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -98,7 +100,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
 
     // mbarriers (each tracks one phase at a time; the protocol never arms a
     // barrier again before its previous phase was waited for)
-    enum { B_W, B_P, B_K0, B_K1, B_T0, B_T1, B_M1, B_MB, B_M3,  // issuer loads and commits (count 1)
+    enum { B_W0, B_W1, B_P0, B_P1, B_K0, B_K1, B_T0, B_T1, B_M1, B_MB, B_M3,  // issuer loads, commits (count 1)
            B_S0, B_VT, B_VN0, B_VN1, B_OUT0, B_OUT1,            // compute-warp arrivals
            B_NEVER, NBARS };
     auto bar = [&](int i) { return smem_u32(&s_bars[i]); };
@@ -158,29 +160,30 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
         // ================================ issuer warp ================================
         const uint32_t id_tf = make_idesc(2, false, false, 128, VS);
         const uint32_t id_bf = make_idesc(1, true, true, 128, VS);
+        const uint32_t id_h = make_idesc(0, false, false, 128, VS);
         int issued[B_M3 + 1] = {0};  // completions issued per barrier
-        auto load_w = [&](int n) {
+        auto load_w = [&](int n) {  // WQ(n) -> slot n & 1
+            const int s = n & 1, bi = B_W0 + s;
             if (lane == 0) {
-                mbar_expect_tx(bar(B_W), TX_W);
+                mbar_expect_tx(bar(bi), TX_W);
                 for (int nb = 0; nb < 2; ++nb)
-                    tma_load_3d(sbase + L::OFF_WQ + nb * DK * 128, &tm_wq, bar(B_W), nb * 64, 0, rec0 + n);
+                    tma_load_3d(sbase + L::OFF_WQ + s * 32768 + nb * DK * 128, &tm_wq, bar(bi), nb * 64, 0, rec0 + n);
             }
-            ++issued[B_W];
+            ++issued[bi];
         };
-        auto load_p = [&](int n) {
+        auto load_p = [&](int n) {  // P(n) -> slot n & 1
+            const int s = n & 1, bi = B_P0 + s;
             if (lane == 0) {
-                mbar_expect_tx(bar(B_P), TX_P);
-                for (int kb = 0; kb < 2; ++kb)
-                    tma_load_3d(sbase + L::OFF_P + kb * 8192, &tm_p, bar(B_P), kb * 32, 0, rec0 + n);
+                mbar_expect_tx(bar(bi), TX_P);
+                tma_load_3d(sbase + L::OFF_P + s * 8192, &tm_p, bar(bi), 0, 0, rec0 + n);
             }
-            ++issued[B_P];
+            ++issued[bi];
         };
         auto load_k = [&](int n) {  // K-hat(n) and e^{Gamma_C}(n) -> slot n & 1
             const int s = n & 1, bi = B_K0 + s;
             if (lane == 0) {
                 mbar_expect_tx(bar(bi), TX_K);
-                for (int kb = 0; kb < 2; ++kb)
-                    tma_load_3d(sbase + L::OFF_KH + s * 32768 + kb * 16384, &tm_kh, bar(bi), kb * 32, 0, rec0 + n);
+                tma_load_3d(sbase + L::OFF_KH + s * 16384, &tm_kh, bar(bi), 0, 0, rec0 + n);
                 bulk_load(sbase + L::OFF_DEC + s * 512, recs + (size_t)n * REC_BYTES + REC_DEC, 512, bar(bi));
             }
             ++issued[bi];
@@ -210,25 +213,25 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
             if (lane == 0) {
                 tc_fence_after();
                 for (int kk = 0; kk < DK / 16; ++kk)
-                    umma<0>(tmem + L::TM_D1 + (n & 1) * VS, desc_mnmaj<128>(sbase + L::OFF_WQ, DK, kk * 16),
+                    umma<0>(tmem + L::TM_D1 + (n & 1) * VS, desc_mnmaj<128>(sbase + L::OFF_WQ + (n & 1) * 32768, DK, kk * 16),
                             desc_mnmaj<128>(sbase + L::OFF_S0, DK, kk * 16), id_bf, kk > 0);
             }
         };
         auto mma_3a = [&](int n) {  // D3 = K-hat(n)^T Vnew(n)
             if (lane == 0) {
                 tc_fence_after();
-                for (int kk = 0; kk < 8; ++kk)
-                    umma<1>(tmem + L::TM_D3, desc_kmaj_s<128, 4>(sbase + L::OFF_KH + (n & 1) * 32768, 128 * 128, kk * 8),
-                            desc_kmaj_s<128, 4>(sbase + L::OFF_VN + (n & 1) * VS * 256, VS * 128, kk * 8), id_tf,
-                            kk > 0);
+                for (int kk = 0; kk < 4; ++kk)
+                    umma<0>(tmem + L::TM_D3, desc_kmaj<128, 2>(sbase + L::OFF_KH + (n & 1) * 16384, 128, kk * 16),
+                            desc_kmaj<128, 2>(sbase + L::OFF_VN + (n & 1) * VS * 128, VS, kk * 16), id_h, kk > 0);
             }
         };
         auto mma_3b = [&](int n) {  // D1[n & 1] rows 64..127 += P(n) Vnew(n)
             if (lane == 0) {
                 tc_fence_after();
-                for (int kk = 0; kk < 8; ++kk)
-                    umma<1>(tmem + L::TM_D1 + (n & 1) * VS, desc_kmaj_s<128, 4>(sbase + L::OFF_P - 8192, 8192, kk * 8),
-                            desc_kmaj_s<128, 4>(sbase + L::OFF_VN + (n & 1) * VS * 256, VS * 128, kk * 8), id_tf, 1u);
+                for (int kk = 0; kk < 4; ++kk)
+                    umma<0>(tmem + L::TM_D1 + (n & 1) * VS,
+                            desc_kmaj<128, 2>(sbase + L::OFF_P + (n & 1) * 8192 - 8192, 128, kk * 16),
+                            desc_kmaj<128, 2>(sbase + L::OFF_VN + (n & 1) * VS * 128, VS, kk * 16), id_h, 1u);
             }
         };
 
@@ -240,7 +243,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
                     prefetch_l2(recs + (size_t)n * REC_BYTES, REC_BYTES);
             }
             load_w(0); load_p(0); load_k(0); load_t(0);
-            if (nseg > 1) { load_k(1); load_t(1); }
+            if (nseg > 1) { load_w(1); load_p(1); load_k(1); load_t(1); }
             ok = wait_warp(B_VT, 0u) && wait_warp(B_T0, 0u);
             if (ok) mma_u(0);
         }
@@ -250,24 +253,26 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
                 prefetch_l2(recs + (size_t)(n + CHAIN_PREFETCH) * REC_BYTES, REC_BYTES);
             if (!(ok = wait_warp(B_S0, (uint32_t)(n & 1)))) break;      // S0(n); D3, e^{Gamma_C}(n-1) consumed
             if (n >= 1 && more) load_k(n + 1);                            // its slot held K-hat(n-1)
-            if (!(ok = wait_warp(B_W, (uint32_t)(n & 1)))) break;       // WQ(n)
+            if (!(ok = wait_warp(B_W0 + (n & 1), (uint32_t)((n >> 1) & 1)))) break;  // WQ(n)
             if (n >= 2 && !(ok = wait_warp(B_OUT0 + (n & 1), (uint32_t)(((n - 2) >> 1) & 1)))) break;  // D1[n&1] free
             mma_1(n);
             commit(B_M1);
             if (n >= 1) {
-                if (!(ok = wait_warp(B_P, (uint32_t)((n - 1) & 1)))) break;  // P(n-1)
+                if (!(ok = wait_warp(B_P0 + ((n - 1) & 1), (uint32_t)(((n - 1) >> 1) & 1)))) break;  // P(n-1)
                 mma_3b(n - 1);
                 commit(B_MB);
             }
             if (!(ok = wait_warp(B_VN0 + (n & 1), (uint32_t)((n >> 1) & 1)))) break;  // Vnew(n); U(n), WQ(n) consumed
-            if (more) load_w(n + 1);
-            if (n + 2 < nseg) load_t(n + 2);                              // T'(n)'s slot: U(n) is done
+            if (n + 2 < nseg) {  // the slots of WQ(n) and T'(n): product 1(n) and U(n) are done
+                load_w(n + 2);
+                load_t(n + 2);
+            }
             if (!(ok = wait_warp(B_K0 + (n & 1), (uint32_t)((n >> 1) & 1)))) break;  // K-hat(n)
             mma_3a(n);
             commit(B_M3);
             if (n >= 1) {
                 if (!(ok = wait_warp(B_MB, (uint32_t)((n - 1) & 1)))) break;  // 3b(n-1) has read P(n-1)
-                load_p(n);
+                if (more) load_p(n + 1);                                     // into P(n-1)'s slot
             }
             if (more) {
                 if (!(ok = wait_warp(B_VT, (uint32_t)((n + 1) & 1)))) break;                 // V^T(n+1)
@@ -277,7 +282,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
         }
         if (ok) {  // the last chunk's output block, once output(N-2) has been read
             if (nseg >= 2) ok = wait_warp(B_OUT0 + (nseg & 1), (uint32_t)(((nseg - 2) >> 1) & 1));
-            if (ok) ok = wait_warp(B_P, (uint32_t)((nseg - 1) & 1));
+            if (ok) ok = wait_warp(B_P0 + ((nseg - 1) & 1), (uint32_t)(((nseg - 1) >> 1) & 1));
             if (ok) { mma_3b(nseg - 1); commit(B_MB); }
         }
         if (*s_abort && lane == 0) {
@@ -376,10 +381,10 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
                 tmem_ld16(tmem + lane_base + L::TM_U + cg * CPT, u);
                 tmem_ld16(tmem + lane_base + L::TM_D1 + (n & 1) * VS + cg * CPT, w);
                 tmem_wait_ld();
-                uint8_t *vn = sm + L::OFF_VN + (n & 1) * VS * 256;
+                uint8_t *vn = sm + L::OFF_VN + (n & 1) * VS * 128;
 #pragma unroll
                 for (int e = 0; e < 16; ++e)
-                    *reinterpret_cast<uint32_t *>(vn + kmaj_s<128, 4>(cg * CPT + e, ch, VS * 128)) = tf32_bits(u[e] - w[e]);
+                    *reinterpret_cast<uint16_t *>(vn + kmaj<128, 2>(cg * CPT + e, ch, VS)) = f16_bits(u[e] - w[e]);
                 fence_async_smem();
                 tc_fence_before();
                 arrive(B_VN0 + (n & 1));

@@ -11,12 +11,13 @@
 // A record holds plain row-major arrays (the chain kernel's tensor loads put
 // them in the swizzled UMMA operand layouts):
 //   WQ   bf16 [dk][128]  row = key channel; columns 0..63 = W^T, 64..127 = (Q e^Gamma)^T
-//   P    fp32 [64][64]   causal q-k block (incl. diagonal), rows = queries
-//   KH   fp32 [128][64]  K-hat^T: row = key channel, column = token
+//   P    fp16 [64][64]   causal q-k block (incl. diagonal), rows = queries
+//   KH   fp16 [128][64]  K-hat^T: row = key channel, column = token
 //   T'   fp32 [64][64]   T' = T Diag(beta), unit-lower times beta
 //   DEC  fp32 [128]      e^{Gamma_C} per key channel
 // at the offsets below (each a multiple of 1 KB; 97 KB per record).
 #pragma once
+#include <cuda_fp16.h>
 #include <stdint.h>
 
 #include "kda_device.cuh"
@@ -45,6 +46,24 @@ __device__ __forceinline__ constexpr int yoff(int I) { return SUB * (I * (I + 1)
 
 __device__ __forceinline__ float rcp_clamped(float p) {
     return p < EXP_CLAMP_LO ? EXP_CLAMP_HI : __fdividef(1.0f, p);
+}
+
+// fp16 keeps tf32's 10-bit mantissa (rounded to nearest) in half the bytes;
+// the values stored as fp16 are bounded by |q| |k| and |k| (P, K-hat) or by
+// the values' and the state's magnitudes (Vnew).
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+    const __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t *>(&h);
+}
+
+__device__ __forceinline__ uint4 pack8_f16(const float (&v)[8]) {
+    return make_uint4(pack_f16x2(v[0], v[1]), pack_f16x2(v[2], v[3]), pack_f16x2(v[4], v[5]),
+                      pack_f16x2(v[6], v[7]));
+}
+
+__device__ __forceinline__ uint16_t f16_bits(float x) {
+    const __half h = __float2half_rn(x);
+    return *reinterpret_cast<const uint16_t *>(&h);
 }
 
 __device__ __forceinline__ uint4 pack8_bf16(const float (&v)[8]) {

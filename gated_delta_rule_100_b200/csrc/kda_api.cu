@@ -223,8 +223,8 @@ int make_rec_maps(PFN_cuTensorMapEncodeTiled_v12000 enc, const uint8_t *rec, lon
                   CUtensorMap *maps) {
     struct Part { size_t off; CUtensorMapDataType dt; int esize, cols, rows, box_cols; };
     const Part parts[4] = {{(size_t)kda::REC_WQ, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 128, dk, 64},
-                           {(size_t)kda::REC_P, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, 64, 64, 32},
-                           {(size_t)kda::REC_KH, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, 64, 128, 32},
+                           {(size_t)kda::REC_P, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, 64, 64, 64},
+                           {(size_t)kda::REC_KH, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, 64, 128, 64},
                            {(size_t)kda::REC_T, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, 64, 64, 32}};
     for (int i = 0; i < 4; ++i) {
         const Part &p = parts[i];

@@ -32,7 +32,7 @@
 //   E  alpha, running products; operand tiles X, Y^(I) (bf16, smem) for the
 //      formation; Q e^G, K-hat (record); (K e^G)^T (tf32, smem)
 //   F  X Y^(I)^T -> A, P                    (UMMA bf16, overlapped with E's tail)
-//   AP A -> fp32 scratch, P -> record
+//   AP A -> fp32 scratch, P -> record (fp16)
 //   T  (I + A)^{-1}: 16x16 diagonal blocks by substitution, off-diagonal blocks
 //      from N = D A_off as T = (I - N + N^2 - N^3) D, fp32 on CUDA cores
 //   W  T' = T Diag(beta) -> record;  W^T = (K e^G)^T T'^T  (UMMA tf32) -> record
@@ -336,15 +336,14 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         {
             if (active) {
                 if (I == 0) reinterpret_cast<float *>(rec + REC_DEC)[c] = dec;
-                float *khr = reinterpret_cast<float *>(rec + REC_KH) + c * CH + tb;
+                uint16_t *khr = reinterpret_cast<uint16_t *>(rec + REC_KH) + c * CH + tb;
                 float r = postB;
 #pragma unroll
                 for (int hh = 1; hh >= 0; --hh) {
                     float kh[8];
 #pragma unroll
                     for (int e = 7; e >= 0; --e) { kh[e] = kval(hh * 8 + e) * r; r *= al[hh * 8 + e]; }
-                    *reinterpret_cast<float4 *>(khr + hh * 8) = make_float4(kh[0], kh[1], kh[2], kh[3]);
-                    *reinterpret_cast<float4 *>(khr + hh * 8 + 4) = make_float4(kh[4], kh[5], kh[6], kh[7]);
+                    *reinterpret_cast<uint4 *>(khr + hh * 8) = pack8_f16(kh);
                 }
                 uint16_t *qer = reinterpret_cast<uint16_t *>(rec + REC_WQ) + c * 128 + 64 + tb;
                 float p = preB;
@@ -407,12 +406,14 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     *reinterpret_cast<float4 *>(sA + i * A_LD + j0 + e) = w;
                 }
             } else {
-                float *pr = reinterpret_cast<float *>(rec + REC_P) + i * CH + j0;
+                uint16_t *pr = reinterpret_cast<uint16_t *>(rec + REC_P) + i * CH + j0;
 #pragma unroll
-                for (int e = 0; e < 16; e += 4)
-                    *reinterpret_cast<float4 *>(pr + e) =
-                        make_float4((j0 + e + 0 <= i) ? v16[e + 0] : 0.f, (j0 + e + 1 <= i) ? v16[e + 1] : 0.f,
-                                    (j0 + e + 2 <= i) ? v16[e + 2] : 0.f, (j0 + e + 3 <= i) ? v16[e + 3] : 0.f);
+                for (int e8 = 0; e8 < 16; e8 += 8) {
+                    float p8[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) p8[e] = (j0 + e8 + e <= i) ? v16[e8 + e] : 0.f;
+                    *reinterpret_cast<uint4 *>(pr + e8) = pack8_f16(p8);
+                }
             }
         }
         tc_fence_before();
