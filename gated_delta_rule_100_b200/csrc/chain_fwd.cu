@@ -47,21 +47,25 @@ namespace kda {
 
 constexpr int CHAIN_WORKERS = 512;                   // sixteen compute warps
 constexpr int CHAIN_THREADS = CHAIN_WORKERS + 32;    // plus the issuer warp
-constexpr int CHAIN_VS = 64;                         // value columns per CTA
 constexpr int CHAIN_PREFETCH = 4;  // chunks between the L2 prefetch of a record and its use
 
-template <int DK>
+// VS value columns per CTA (64 or 128).  Every CTA of a (b, h) reads that
+// (b, h)'s whole records, so fewer, wider slices read fewer record bytes; the
+// 128-column layout has room for one WQ buffer, the 64-column one for two.
+template <int DK, int VS_>
 struct ChainLayout {
     static_assert(DK == 64 || DK == 128, "dk");
-    static constexpr int VS = CHAIN_VS;
-    static constexpr int OFF_WQ = 0;          // two bf16 MN-major [DK][128]: [W; Q e^G] (32 KB slots)
-    static constexpr int OFF_P = 65536;       // two fp16 K-major [64][64] (8 KB)
-    static constexpr int OFF_KH = 81920;      // two fp16 K-major [128][64] (16 KB)
-    static constexpr int OFF_T = 114688;      // two tf32 K-major [64][64] (8 KB K-blocks)
-    static constexpr int OFF_DEC = 147456;    // two 512-byte slots of e^{Gamma_C} (with K-hat)
-    static constexpr int OFF_S0 = 148480;     // bf16 MN-major S0 [DK][64], 128B swizzle
-    static constexpr int OFF_VT = OFF_S0 + DK * VS * 2;   // tf32 K-major V^T [64][64]
-    static constexpr int OFF_VN = OFF_VT + VS * 256;      // two fp16 K-major Vnew^T [64][64]
+    static_assert(VS_ == 64 || VS_ == 128, "value slice");
+    static constexpr int VS = VS_;
+    static constexpr int WS = VS == 64 ? 2 : 1;          // WQ buffers
+    static constexpr int OFF_WQ = 0;                     // bf16 MN-major [DK][128]: [W; Q e^G] (32 KB slots)
+    static constexpr int OFF_P = WS * 32768;             // two fp16 K-major [64][64] (8 KB)
+    static constexpr int OFF_KH = OFF_P + 16384;         // two fp16 K-major [128][64] (16 KB)
+    static constexpr int OFF_T = OFF_KH + 32768;         // two tf32 K-major [64][64] (8 KB K-blocks)
+    static constexpr int OFF_DEC = OFF_T + 32768;        // two 512-byte slots of e^{Gamma_C} (with K-hat)
+    static constexpr int OFF_S0 = OFF_DEC + 1024;        // bf16 MN-major S0 [DK][VS], 128B swizzle
+    static constexpr int OFF_VT = OFF_S0 + DK * VS * 2;  // tf32 K-major V^T [VS][64]
+    static constexpr int OFF_VN = OFF_VT + VS * 256;     // two fp16 K-major Vnew^T [VS][64]
     static constexpr int OFF_MISC = OFF_VN + 2 * VS * 128;  // barriers, TMEM address, abort flag
     static constexpr int TOTAL = OFF_MISC + 1024;
     static constexpr int SMEM_BYTES = TOTAL + 1024;  // slack for the 1 KB base alignment
@@ -74,21 +78,21 @@ struct ChainLayout {
     static constexpr uint32_t TM_U = 0;          // U (lane = token)
     static constexpr uint32_t TM_D1 = VS;        // two: [W; Q e^G] S0, then += P Vnew on lanes 64..127
     static constexpr uint32_t TM_D3 = 3 * VS;    // K-hat^T Vnew (lane = key channel)
-    static constexpr uint32_t TM_COLS = 256;
+    static constexpr uint32_t TM_COLS = 4 * VS;
 };
 
-template <int DK>
+template <int DK, int VS_>
 __global__ void __launch_bounds__(CHAIN_THREADS, 1)
 chain_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ CUtensorMap tm_p,
              const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUtensorMap tm_t,
              const ChainParams prm) {
-    using L = ChainLayout<DK>;
-    constexpr int VS = L::VS;
+    using L = ChainLayout<DK, VS_>;
+    constexpr int VS = L::VS, WS = L::WS;
     constexpr int CPT = VS / 4;             // value columns per compute thread
     constexpr int NP = VS / 2;              // value column pairs (V loads)
     constexpr int TG = CHAIN_WORKERS / NP;  // token groups (V loads)
     constexpr int TPT = CH / TG;            // tokens per compute thread (V loads)
-    static_assert(TPT % 4 == 0 && CPT == 16, "thread mapping");
+    static_assert(TPT % 4 == 0 && CPT % 16 == 0, "thread mapping");
     constexpr uint32_t TX_T = 16384, TX_W = DK * 256, TX_P = 8192, TX_K = 16384 + 512;
 
     extern __shared__ uint8_t smem_raw[];
@@ -162,8 +166,8 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
         const uint32_t id_bf = make_idesc(1, true, true, 128, VS);
         const uint32_t id_h = make_idesc(0, false, false, 128, VS);
         int issued[B_M3 + 1] = {0};  // completions issued per barrier
-        auto load_w = [&](int n) {  // WQ(n) -> slot n & 1
-            const int s = n & 1, bi = B_W0 + s;
+        auto load_w = [&](int n) {  // WQ(n) -> slot n % WS
+            const int s = n % WS, bi = B_W0 + s;
             if (lane == 0) {
                 mbar_expect_tx(bar(bi), TX_W);
                 for (int nb = 0; nb < 2; ++nb)
@@ -213,7 +217,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
             if (lane == 0) {
                 tc_fence_after();
                 for (int kk = 0; kk < DK / 16; ++kk)
-                    umma<0>(tmem + L::TM_D1 + (n & 1) * VS, desc_mnmaj<128>(sbase + L::OFF_WQ + (n & 1) * 32768, DK, kk * 16),
+                    umma<0>(tmem + L::TM_D1 + (n & 1) * VS, desc_mnmaj<128>(sbase + L::OFF_WQ + (n % WS) * 32768, DK, kk * 16),
                             desc_mnmaj<128>(sbase + L::OFF_S0, DK, kk * 16), id_bf, kk > 0);
             }
         };
@@ -243,7 +247,10 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
                     prefetch_l2(recs + (size_t)n * REC_BYTES, REC_BYTES);
             }
             load_w(0); load_p(0); load_k(0); load_t(0);
-            if (nseg > 1) { load_w(1); load_p(1); load_k(1); load_t(1); }
+            if (nseg > 1) {
+                if (WS == 2) load_w(1);
+                load_p(1); load_k(1); load_t(1);
+            }
             ok = wait_warp(B_VT, 0u) && wait_warp(B_T0, 0u);
             if (ok) mma_u(0);
         }
@@ -253,7 +260,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
                 prefetch_l2(recs + (size_t)(n + CHAIN_PREFETCH) * REC_BYTES, REC_BYTES);
             if (!(ok = wait_warp(B_S0, (uint32_t)(n & 1)))) break;      // S0(n); D3, e^{Gamma_C}(n-1) consumed
             if (n >= 1 && more) load_k(n + 1);                            // its slot held K-hat(n-1)
-            if (!(ok = wait_warp(B_W0 + (n & 1), (uint32_t)((n >> 1) & 1)))) break;  // WQ(n)
+            if (!(ok = wait_warp(B_W0 + (n % WS), (uint32_t)((n / WS) & 1)))) break;  // WQ(n)
             if (n >= 2 && !(ok = wait_warp(B_OUT0 + (n & 1), (uint32_t)(((n - 2) >> 1) & 1)))) break;  // D1[n&1] free
             mma_1(n);
             commit(B_M1);
@@ -263,10 +270,9 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
                 commit(B_MB);
             }
             if (!(ok = wait_warp(B_VN0 + (n & 1), (uint32_t)((n >> 1) & 1)))) break;  // Vnew(n); U(n), WQ(n) consumed
-            if (n + 2 < nseg) {  // the slots of WQ(n) and T'(n): product 1(n) and U(n) are done
-                load_w(n + 2);
-                load_t(n + 2);
-            }
+            // the slots of WQ(n) and T'(n): product 1(n) and U(n) are done
+            if (n + WS < nseg) load_w(n + WS);
+            if (n + 2 < nseg) load_t(n + 2);
             if (!(ok = wait_warp(B_K0 + (n & 1), (uint32_t)((n >> 1) & 1)))) break;  // K-hat(n)
             mma_3a(n);
             commit(B_M3);
@@ -349,16 +355,19 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
         auto write_output = [&](int n) {
             const int i = ch - 64;
             const int t = (prm.n_begin + n) * CH + i;
-            float o[16];
-            tmem_ld16(tmem + lane_base + L::TM_D1 + (n & 1) * VS + cg * CPT, o);
-            tmem_wait_ld();
-            if (t < T) {
-                uint16_t *dst = prm.out + (((size_t)b * T + t) * H + h) * DV + scol;
-                float a8[8], b8[8];
+            uint16_t *dst = prm.out + (((size_t)b * T + (t < T ? t : 0)) * H + h) * DV + scol;
 #pragma unroll
-                for (int e = 0; e < 8; ++e) { a8[e] = prm.scale * o[e]; b8[e] = prm.scale * o[8 + e]; }
-                *reinterpret_cast<uint4 *>(dst) = pack8_bf16(a8);
-                *reinterpret_cast<uint4 *>(dst + 8) = pack8_bf16(b8);
+            for (int c16 = 0; c16 < CPT; c16 += 16) {
+                float o[16];
+                tmem_ld16(tmem + lane_base + L::TM_D1 + (n & 1) * VS + cg * CPT + c16, o);
+                tmem_wait_ld();
+                if (t < T) {
+                    float a8[8], b8[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) { a8[e] = prm.scale * o[e]; b8[e] = prm.scale * o[8 + e]; }
+                    *reinterpret_cast<uint4 *>(dst + c16) = pack8_bf16(a8);
+                    *reinterpret_cast<uint4 *>(dst + c16 + 8) = pack8_bf16(b8);
+                }
             }
             tc_fence_before();
         };
@@ -377,14 +386,17 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
             if (!(ok = wait_warp(B_M1, (uint32_t)(n & 1)))) break;  // U(n), D1[n&1] rows 0..63
             tc_fence_after();
             if (lq < 2) {  // Vnew(n) = U - W S0 -> Vnew^T tile n & 1
-                float u[16], w[16];
-                tmem_ld16(tmem + lane_base + L::TM_U + cg * CPT, u);
-                tmem_ld16(tmem + lane_base + L::TM_D1 + (n & 1) * VS + cg * CPT, w);
-                tmem_wait_ld();
                 uint8_t *vn = sm + L::OFF_VN + (n & 1) * VS * 128;
 #pragma unroll
-                for (int e = 0; e < 16; ++e)
-                    *reinterpret_cast<uint16_t *>(vn + kmaj<128, 2>(cg * CPT + e, ch, VS)) = f16_bits(u[e] - w[e]);
+                for (int c16 = 0; c16 < CPT; c16 += 16) {
+                    float u[16], w[16];
+                    tmem_ld16(tmem + lane_base + L::TM_U + cg * CPT + c16, u);
+                    tmem_ld16(tmem + lane_base + L::TM_D1 + (n & 1) * VS + cg * CPT + c16, w);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        *reinterpret_cast<uint16_t *>(vn + kmaj<128, 2>(cg * CPT + c16 + e, ch, VS)) = f16_bits(u[e] - w[e]);
+                }
                 fence_async_smem();
                 tc_fence_before();
                 arrive(B_VN0 + (n & 1));
@@ -405,11 +417,14 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
             tc_fence_after();
             if (ch < DK) {  // warp-uniform
                 const float dc = reinterpret_cast<const float *>(sm + L::OFF_DEC + (n & 1) * 512)[ch];
-                float t[16];
-                tmem_ld16(tmem + lane_base + L::TM_D3 + cg * CPT, t);
-                tmem_wait_ld();
 #pragma unroll
-                for (int e = 0; e < 16; ++e) S[e] = dc * S[e] + t[e];
+                for (int c16 = 0; c16 < CPT; c16 += 16) {
+                    float t[16];
+                    tmem_ld16(tmem + lane_base + L::TM_D3 + cg * CPT + c16, t);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) S[c16 + e] = dc * S[c16 + e] + t[e];
+                }
             }
             store_state_bf16();  // S0 is free: product 1(n) completed
             tc_fence_before();
@@ -433,23 +448,23 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
     if (warp == 0) tmem_dealloc(tmem, L::TM_COLS);
 }
 
-template <int DK>
+template <int DK, int VS>
 static cudaError_t launch_chain_t(const CUtensorMap *maps, const ChainParams &prm, cudaStream_t stream) {
-    using L = ChainLayout<DK>;
-    cudaError_t e = cudaFuncSetAttribute(chain_kernel<DK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    using L = ChainLayout<DK, VS>;
+    cudaError_t e = cudaFuncSetAttribute(chain_kernel<DK, VS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          L::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    chain_kernel<DK><<<prm.B * prm.H * prm.nslices, CHAIN_THREADS, L::SMEM_BYTES, stream>>>(
+    chain_kernel<DK, VS><<<prm.B * prm.H * prm.nslices, CHAIN_THREADS, L::SMEM_BYTES, stream>>>(
         maps[0], maps[1], maps[2], maps[3], prm);
     return cudaGetLastError();
 }
 
-int chain_value_slice() { return CHAIN_VS; }
-
-// maps: the record parts WQ, P, K-hat, T' (see chunk_common.cuh)
+// maps: the record parts WQ, P, K-hat, T' (see chunk_common.cuh); the value
+// slice of a CTA is DV / nslices columns (64 or 128).
 cudaError_t launch_chain(const CUtensorMap *maps, const ChainParams &prm, int dk, cudaStream_t stream) {
-    if (dk == 128) return launch_chain_t<128>(maps, prm, stream);
-    return launch_chain_t<64>(maps, prm, stream);
+    const int vs = prm.DV / prm.nslices;
+    if (dk == 128) return vs == 128 ? launch_chain_t<128, 128>(maps, prm, stream) : launch_chain_t<128, 64>(maps, prm, stream);
+    return vs == 128 ? launch_chain_t<64, 128>(maps, prm, stream) : launch_chain_t<64, 64>(maps, prm, stream);
 }
 
 }  // namespace kda

@@ -25,9 +25,8 @@ cudaError_t launch_decode(const void *q, const void *k, const void *v, const flo
 
 namespace kda {
 cudaError_t launch_prep(const CUtensorMap &tq, const CUtensorMap &tk, const PrepParams &prm, int dk,
-                        int num_sms, cudaStream_t stream);
+                        int max_ctas, cudaStream_t stream);
 cudaError_t launch_chain(const CUtensorMap *maps, const ChainParams &prm, int dk, cudaStream_t stream);
-int chain_value_slice();
 }
 
 // Device-side status word: kernels OR error bits into it (one per device,
@@ -84,6 +83,7 @@ int get_encoder(PFN_cuTensorMapEncodeTiled_v12000 *fn) {
 // of segment i: prep on a low-priority internal stream, chain on a
 // high-priority one (its few CTAs are placed first, prep fills the other SMs).
 constexpr size_t kWorkspaceCap = size_t(2) << 30;  // bytes of records
+constexpr double kPrepCtasPerFreeSm = 2.0;         // prep density beside a chain kernel
 constexpr size_t kTicketBytes = 256;               // two item counters at the front of the records
 struct Workspace {
     uint8_t *base = nullptr;  // [tickets][records]
@@ -240,8 +240,12 @@ int make_rec_maps(PFN_cuTensorMapEncodeTiled_v12000 enc, const uint8_t *rec, lon
     return KDA_OK;
 }
 
-// Value-column slices per (b, h) in the chain kernel: one CTA per 64 columns.
-int chain_slices(int dv) { return dv / kda::chain_value_slice(); }
+// Value-column slices per (b, h) in the chain kernel.  Every CTA of a (b, h)
+// reads all of that (b, h)'s records, so one 128-column CTA reads them once;
+// two 64-column CTAs halve the per-chunk work on the sequential path.  Use the
+// narrow slices when they still fit one CTA per SM (few (b, h): latency
+// matters), the wide one otherwise (many (b, h): record traffic matters).
+int chain_slices(int B, int H, int dv, int sms) { return (dv == 128 && 2LL * B * H <= sms) ? 2 : 1; }
 
 }  // namespace
 
@@ -338,6 +342,13 @@ int kda_chunk_fwd(const void *q, const void *k, const void *v, const float *g, c
     for (int i = 0; i < pl.nbuf; ++i)
         if (make_rec_maps(enc, recs[i], (long long)B * H * seg, dk, rmaps[i]) != KDA_OK) return KDA_ERR_CUDA;
 
+    // Prep CTAs: two per SM when prep runs alone; beside a chain kernel, two
+    // per SM the chain leaves free (lower densities slowed the whole call on
+    // the long-context workload: the chain speeds up less than prep slows).
+    // Its CTAs claim items from a counter, so any that start late only share
+    // the remaining work.
+    const int chain_ctas = B * H * chain_slices(B, H, dv, sms);
+    const int prep_ctas = (multi && chain_ctas < sms) ? (int)(kPrepCtasPerFreeSm * (sms - chain_ctas) + 0.5) : 2 * sms;
     cudaStream_t sp = s, sc = s;  // prep and chain streams
     if (multi) {
         sp = w->lo;
@@ -363,7 +374,7 @@ int kda_chunk_fwd(const void *q, const void *k, const void *v, const float *g, c
         pp.n_begin = n0;
         pp.nseg = cnt;
         pp.st = dst;
-        cudaError_t e = timed_launch(dev, 0, sp, [&] { return kda::launch_prep(tq, tk, pp, dk, sms, sp); });
+        cudaError_t e = timed_launch(dev, 0, sp, [&] { return kda::launch_prep(tq, tk, pp, dk, prep_ctas > 0 ? prep_ctas : 1, sp); });
         if (e != cudaSuccess) return KDA_ERR_CUDA;
         if (multi && (cudaEventRecord(w->prep_done[buf], sp) != cudaSuccess ||
                       cudaStreamWaitEvent(sc, w->prep_done[buf], 0) != cudaSuccess))
@@ -379,7 +390,7 @@ int kda_chunk_fwd(const void *q, const void *k, const void *v, const float *g, c
         cp.B = B; cp.T = T; cp.H = H; cp.DV = dv;
         cp.n_begin = n0;
         cp.nseg = cnt;
-        cp.nslices = chain_slices(dv);
+        cp.nslices = chain_slices(B, H, dv, sms);
         cp.st = dst;
         cp.inject_wait_polls = g_inject_polls.load();
         e = timed_launch(dev, 1, sc, [&] { return kda::launch_chain(rmaps[buf], cp, dk, sc); });
@@ -557,7 +568,7 @@ int kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const flo
         pp.nseg = cnt;
         pp.st = dst;
         if (cudaMemsetAsync(ticket, 0, sizeof(int), s) != cudaSuccess ||  // the counter starts at zero
-            kda::launch_prep(tq, tk, pp, dk, sms, s) != cudaSuccess)
+            kda::launch_prep(tq, tk, pp, dk, 2 * sms, s) != cudaSuccess)
             return KDA_ERR_CUDA;
 
         kda::ChainParams cp;
@@ -570,7 +581,7 @@ int kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const flo
         cp.B = B; cp.T = T; cp.H = H; cp.DV = dv;
         cp.n_begin = n0;
         cp.nseg = cnt;
-        cp.nslices = chain_slices(dv);
+        cp.nslices = chain_slices(B, H, dv, sms);
         cp.st = dst;
         cp.inject_wait_polls = g_inject_polls.load();
         if (kda::launch_chain(rmaps, cp, dk, s) != cudaSuccess) return KDA_ERR_CUDA;

@@ -562,21 +562,22 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 
 template <int DK>
 static cudaError_t launch_prep_t(const CUtensorMap &tq, const CUtensorMap &tk, const PrepParams &prm,
-                                 int num_sms, cudaStream_t stream) {
+                                 int max_ctas, cudaStream_t stream) {
     using L = PrepLayout<DK>;
     cudaError_t e = cudaFuncSetAttribute(prep_kernel<DK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          L::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     const long long items = (long long)prm.B * prm.H * prm.nseg;
-    const int grid = (int)(items < 2LL * num_sms ? items : 2LL * num_sms);
+    const int grid = (int)(items < max_ctas ? items : max_ctas);
     prep_kernel<DK><<<grid, PREP_THREADS, L::SMEM_BYTES, stream>>>(tq, tk, prm);
     return cudaGetLastError();
 }
 
+// At most max_ctas persistent CTAs (two fit on an SM), at most one per item.
 cudaError_t launch_prep(const CUtensorMap &tq, const CUtensorMap &tk, const PrepParams &prm, int dk,
-                        int num_sms, cudaStream_t stream) {
-    if (dk == 128) return launch_prep_t<128>(tq, tk, prm, num_sms, stream);
-    return launch_prep_t<64>(tq, tk, prm, num_sms, stream);
+                        int max_ctas, cudaStream_t stream) {
+    if (dk == 128) return launch_prep_t<128>(tq, tk, prm, max_ctas, stream);
+    return launch_prep_t<64>(tq, tk, prm, max_ctas, stream);
 }
 
 }  // namespace kda
