@@ -15,7 +15,7 @@
 //   KH   fp16 [128][64]  K-hat^T: row = key channel, column = token
 //   T'   fp32 [64][64]   T' = T Diag(beta), unit-lower times beta
 //   DEC  fp32 [128]      e^{Gamma_C} per key channel
-// at the offsets below (each a multiple of 1 KB; 97 KB per record).
+// at the offsets below (each 16-byte aligned; 72.5 KB per record).
 #pragma once
 #include <cuda_fp16.h>
 #include <stdint.h>
@@ -31,12 +31,12 @@ constexpr int A_LD = 68;        // fp32 row stride of the A / T scratch
 constexpr float EXP_CLAMP_HI = 5.5406223843935098e34f;  // e^80
 constexpr float EXP_CLAMP_LO = 1.8048513878454153e-35f; // e^-80
 
-constexpr int REC_WQ = 0;
-constexpr int REC_P = 32768;
-constexpr int REC_KH = 49152;
-constexpr int REC_T = 81920;
-constexpr int REC_DEC = 98304;
-constexpr int REC_BYTES = 99328;
+constexpr int REC_WQ = 0;         // 32 KB (dk = 64 uses the first 16 KB)
+constexpr int REC_P = 32768;      // 8 KB
+constexpr int REC_KH = 40960;     // 16 KB
+constexpr int REC_T = 57344;      // 16 KB
+constexpr int REC_DEC = 73728;    // 512 B
+constexpr int REC_BYTES = 74240;
 
 __host__ __device__ constexpr int align1k(int x) { return (x + 1023) & ~1023; }
 __host__ __device__ constexpr int cmax(int a, int b) { return a > b ? a : b; }

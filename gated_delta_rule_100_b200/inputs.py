@@ -70,6 +70,9 @@ CONFIGS = {
     "prefill_B1_H4_T2048_d128": PrefillConfig("prefill_B1_H4_T2048_d128", 1, 4, 2048, 128, 128, 0.05, 0.02, 1),
     "training_B8_H32_T4096_d128": PrefillConfig("training_B8_H32_T4096_d128", 8, 32, 4096, 128, 128, 0.05, 0.0, 2),
     "long_context_B1_H32_T1M_d128": PrefillConfig("long_context_B1_H32_T1M_d128", 1, 32, 1 << 20, 128, 128, 0.01, 0.0, 3),
+    # the training shape at a quarter of the batch: inputs (0.34 GB) above L2, small enough for
+    # multi-pass counter captures
+    "profile_B2_H32_T4096_d128": PrefillConfig("profile_B2_H32_T4096_d128", 2, 32, 4096, 128, 128, 0.05, 0.0, 4),
 }
 DECODE_CONFIG = DecodeConfig("decode_B256_H32_d128_64steps", 256, 32, 128, 128, 0.05, 0.02, 64, 4)
 

@@ -132,9 +132,9 @@ KDA_API int kda_decode_step(const void *q, const void *k, const void *v,
  * outputs are bit-identical to it.  The chunk records live in a fixed 64 MiB
  * array per device that is part of the library's module image, so a long
  * sequence runs in several segments of two kernel launches each.  Limit: the
- * records of one 64-token chunk of every (b, h) (B * H * 99,328 bytes), plus,
+ * records of one 64-token chunk of every (b, h) (B * H * 74,240 bytes), plus,
  * when hT is NULL, the fp32 state [B, H, dk, dv] carried between segments,
- * must fit in 64 MiB (B * H <= 675 with hT given); a larger problem returns
+ * must fit in 64 MiB (B * H <= 903 with hT given); a larger problem returns
  * KDA_ERR_SCRATCH_LIMIT without enqueueing work.  The only part of the
  * scratch that must start at zero, an item counter, is cleared by each call.
  *
@@ -151,7 +151,7 @@ KDA_API int kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v,
 
 /*
  * kda_chunk_fwd_workspace_bytes -- device memory kda_chunk_fwd holds for these
- * sizes: the per-chunk records (about 97 KB per 64-token chunk and (b, h)) of
+ * sizes: the per-chunk records (72.5 KB per 64-token chunk and (b, h)) of
  * the whole sequence when they fit in 2 GiB, else of two segments of as many
  * chunks as fit in 1 GiB each (at least one; the prep kernel of one segment
  * overlaps the state chain of the previous one on two internal streams),

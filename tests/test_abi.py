@@ -100,7 +100,7 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
 
 
 def test_workspace_bytes(lib):
-    rec = 99328  # bytes of one chunk record of one (b, h)
+    rec = 74240  # bytes of one chunk record of one (b, h)
     tick = 256   # the prep kernel's item counters
     # one segment: all chunks' records, no state buffer
     assert kda.workspace_bytes(1, 256, 1, 128, 128) == tick + 4 * rec
@@ -118,9 +118,9 @@ def test_workspace_bytes(lib):
 def test_noalloc_rejects_beyond_its_scratch(lib):
     def call(B, H, hT, dk=128, dv=128):
         return lib.kda_chunk_fwd_noalloc(A, A, A, A, A, 1.0, None, A, hT, B, 64, H, dk, dv, None)
-    # one chunk record of every (b, h) must fit in the 64 MiB array: B * H <= 675 with hT given
-    assert call(1, 676, A) == kda.KDA_ERR_SCRATCH_LIMIT
-    assert call(2, 338, A) == kda.KDA_ERR_SCRATCH_LIMIT
+    # one chunk record of every (b, h) must fit in the 64 MiB array: B * H <= 903 with hT given
+    assert call(1, 904, A) == kda.KDA_ERR_SCRATCH_LIMIT
+    assert call(2, 452, A) == kda.KDA_ERR_SCRATCH_LIMIT
     # without hT the carried fp32 state shares the array
     assert call(1, 600, None) == kda.KDA_ERR_SCRATCH_LIMIT
     assert kda.status_string(kda.KDA_ERR_SCRATCH_LIMIT) == "KDA_ERR_SCRATCH_LIMIT"

@@ -65,8 +65,8 @@ def test_noalloc_zero_length_and_limit():
     assert rc == kda.KDA_OK
     torch.cuda.synchronize()
     assert torch.equal(hT, h0)
-    # one chunk record of each of 676 (b, h) exceeds the 64 MiB array: rejected, nothing enqueued
-    big = inputs.make_prefill(1, 64, 676, 128, 128, decay=0.05, h0_std=0.0, seed=13, device=dev)
-    out = torch.empty((1, 64, 676, 128), dtype=torch.bfloat16, device=dev)
-    hT2 = torch.empty((1, 676, 128, 128), dtype=torch.float32, device=dev)
+    # one chunk record of each of 904 (b, h) exceeds the 64 MiB array: rejected, nothing enqueued
+    big = inputs.make_prefill(1, 64, 904, 128, 128, decay=0.05, h0_std=0.0, seed=13, device=dev)
+    out = torch.empty((1, 64, 904, 128), dtype=torch.bfloat16, device=dev)
+    hT2 = torch.empty((1, 904, 128, 128), dtype=torch.float32, device=dev)
     assert _noalloc(lib, big, 0.1, out, hT2) == kda.KDA_ERR_SCRATCH_LIMIT
