@@ -160,11 +160,9 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 
     if (tid == 0) *s_next = atomicAdd(prm.ticket, 1);
     __syncthreads();
+    int claim = 0;  // thread 0: the item claimed for after this one (result needed mid-item)
     for (int item = *s_next; item < nitems && !aborted;) {
-        __syncthreads();  // every thread has read s_next
-        if (tid == 0) *s_next = atomicAdd(prm.ticket, 1);  // claimed now, so its inputs can be prefetched
-        __syncthreads();
-        const int next = *s_next;
+        if (tid == 0) claim = atomicAdd(prm.ticket, 1);
         int b, h, t0;
         item_coords(item, b, h, t0);
         uint8_t *rec = prm.ws + (size_t)item * REC_BYTES;
@@ -186,20 +184,6 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             for (int u = 0; u < SUB; ++u) al[u] = (t0 + tb + u < T && active) ? __ldg(gp + (size_t)u * H * DK) : 0.f;
         }
         if (tid < CH) s_beta[tid] = (t0 + tid < T) ? prm.beta[((size_t)b * T + t0 + tid) * H + h] : 0.f;
-        // the next item's q, k and g into L2 while this one is processed
-        if (next < nitems) {
-            int nb, nh, nt0;
-            item_coords(next, nb, nh, nt0);
-            if (tid == 0) {
-#pragma unroll
-                for (int kb = 0; kb < DK / 64; ++kb) {
-                    prefetch_tensor_4d(&tm_q, kb * 64, nh, nt0, nb);
-                    prefetch_tensor_4d(&tm_k, kb * 64, nh, nt0, nb);
-                }
-            } else if (tid >= 64 && tid < 64 + CH && nt0 + tid - 64 < T) {
-                prefetch_l2(prm.g + (((size_t)nb * T + nt0 + tid - 64) * H + nh) * DK, DK * 4);
-            }
-        }
         if (!wait_all(bar_in, ph_in, tma_pending)) { aborted = true; break; }
         ph_in ^= 1u;
 
@@ -364,8 +348,24 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 }
             }
         }
+        if (tid == 0) *s_next = claim;  // read by every thread after the barrier below
         if (!wait_all(bar_mma, ph_mma, mma_pending)) { aborted = true; break; }
         ph_mma ^= 1u;
+        const int next = *s_next;
+        // the next item's q, k and g into L2 while this one finishes
+        if (next < nitems) {
+            int nb, nh, nt0;
+            item_coords(next, nb, nh, nt0);
+            if (tid == 0) {
+#pragma unroll
+                for (int kb = 0; kb < DK / 64; ++kb) {
+                    prefetch_tensor_4d(&tm_q, kb * 64, nh, nt0, nb);
+                    prefetch_tensor_4d(&tm_k, kb * 64, nh, nt0, nb);
+                }
+            } else if (tid >= 64 && tid < 64 + CH && nt0 + tid - 64 < T) {
+                prefetch_l2(prm.g + (((size_t)nb * T + nt0 + tid - 64) * H + nh) * DK, DK * 4);
+            }
+        }
 
         // ---------------- AP: A -> fp32 scratch, P -> record ----------------
         // TMEM lane = row of [k; q]; the four warps of a lane quarter take one
