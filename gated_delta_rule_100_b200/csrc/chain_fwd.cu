@@ -20,13 +20,16 @@
 // (fp16 keeps tf32's 10-bit mantissa; K-hat, P and Vnew are bounded in
 // magnitude, T' is kept in tf32 for its range).
 //
-// Warp roles.  One issuer warp (its lane 0) issues every tensor load and every
-// product; sixteen compute warps move data between TMEM, registers and shared
-// memory.  They never meet at a CTA-wide barrier inside the loop: each hand-off
-// is an mbarrier -- the issuer's loads and product commits on one side, the
-// compute warps' arrivals (Vnew written, an output block read, V^T written,
-// S0 written) on the other -- so the tensor pipe, which executes in issue
-// order, is fed as soon as each operand is ready.  Per chunk n it runs
+// Warp roles.  One loader warp (its lane 0) issues every record load, one
+// issuer warp (its lane 0) issues every product, and sixteen compute warps move
+// data between TMEM, registers and shared memory.  They never meet at a
+// CTA-wide barrier inside the loop: each hand-off is an mbarrier -- a full/empty
+// pair per record buffer between the loader and its readers, product commits
+// and the compute warps' arrivals (Vnew written, an output block read, V^T
+// written, S0 written) between the issuer and the compute warps -- so the
+// tensor pipe, which executes in issue order, is fed as soon as each operand is
+// ready.  A TMA issue can hold its thread for hundreds of cycles while the
+// SM's copy engine is busy, which is why no load sits in the issuer's path.  Per chunk n it runs
 // 1(n), 3b(n-1), 3a(n), U(n+1): only 1 and 3a lie on the state's critical
 // path, the other two fill the pipe while the compute warps form Vnew(n) and
 // update the state.  Buffers: two output accumulators and two each of the
@@ -46,8 +49,7 @@
 namespace kda {
 
 constexpr int CHAIN_WORKERS = 512;                   // sixteen compute warps
-constexpr int CHAIN_THREADS = CHAIN_WORKERS + 32;    // plus the issuer warp
-constexpr int CHAIN_PREFETCH = 4;  // chunks between the L2 prefetch of a record and its use
+constexpr int CHAIN_THREADS = CHAIN_WORKERS + 64;    // plus the issuer and loader warps
 
 // VS value columns per CTA (64 or 128).  Every CTA of a (b, h) reads that
 // (b, h)'s whole records, so fewer, wider slices read fewer record bytes; the
@@ -104,13 +106,15 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
 
     // mbarriers (each tracks one phase at a time; the protocol never arms a
     // barrier again before its previous phase was waited for)
-    enum { B_W0, B_W1, B_P0, B_P1, B_K0, B_K1, B_T0, B_T1, B_M1, B_MB, B_M3,  // issuer loads, commits (count 1)
-           B_S0, B_VT, B_VN0, B_VN1, B_OUT0, B_OUT1,            // compute-warp arrivals
+    enum { B_W0, B_W1, B_P0, B_P1, B_K0, B_K1, B_T0, B_T1,       // record buffers full (loader, count 1)
+           B_M1, B_MB, B_M3, B_WE0, B_WE1, B_TE0, B_TE1, B_PE0, B_PE1,  // product commits (count 1)
+           B_S0, B_VT, B_VN0, B_VN1, B_OUT0, B_OUT1, B_KE0, B_KE1,  // compute-warp arrivals
            B_NEVER, NBARS };
     auto bar = [&](int i) { return smem_u32(&s_bars[i]); };
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
     const bool issuer = warp == CHAIN_WORKERS / 32;
+    const bool loader = warp == CHAIN_WORKERS / 32 + 1;
     const int slice = blockIdx.x % prm.nslices;
     const int bh = blockIdx.x / prm.nslices;
     const int h = bh % prm.H, b = bh / prm.H;
@@ -123,8 +127,9 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
 
     if (tid == 0) {
         for (int i = 0; i < NBARS; ++i) {
-            const bool group = i >= B_S0 && i <= B_OUT1;
-            const uint32_t cnt = !group ? 1u : (i == B_S0 || i == B_VT) ? 16u : 8u;  // warps that arrive
+            const bool group = i >= B_S0 && i <= B_KE1;
+            const bool all16 = i == B_S0 || i == B_VT || i == B_KE0 || i == B_KE1;
+            const uint32_t cnt = !group ? 1u : all16 ? 16u : 8u;  // warps that arrive
             mbar_init(bar(i), cnt);
         }
         *s_abort = 0;
@@ -140,12 +145,16 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
     const uint32_t tmem = *s_tmem;
 
     // Bounded wait agreed by the whole warp; false once this CTA aborts.
+    // Bounded wait of the single thread that runs the loader or the issuer.
+    auto wait1 = [&](int i, uint32_t par) -> bool {
+        if (mbar_wait(bar(i), par, polls, prm.st)) return true;
+        *s_abort = 1;
+        return false;
+    };
+    // Bounded wait agreed by the whole warp (a compute warp).
     auto wait_warp = [&](int i, uint32_t par) -> bool {
-        bool ok = *s_abort == 0;
-        if (ok) ok = mbar_wait(bar(i), par, polls, prm.st);
-        ok = __all_sync(0xffffffffu, ok);
+        const bool ok = __all_sync(0xffffffffu, mbar_wait(bar(i), par, polls, prm.st));
         if (!ok) *s_abort = 1;
-        __syncwarp();
         return ok;
     };
     auto arrive = [&](int i) {  // one arrival per warp, after all its lanes' prior work
@@ -160,145 +169,141 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
         __syncthreads();
     }
 
-    if (issuer) {
-        // ================================ issuer warp ================================
+    if (loader && lane == 0) {
+        // ====================== loader warp (lane 0; the rest idle) ======================
+        // Chunk j's records go to buffer j % WS (WQ) or j & 1 (the rest), each
+        // once its empty barrier says the readers of chunk j - WS (j - 2) are done.
+        uint32_t armed = 0, parity = 0;  // per full barrier: ever armed, count of armed completions mod 2
+        auto load_w = [&](int n) {  // WQ(n)
+            const int s = n % WS, bi = B_W0 + s;
+            mbar_expect_tx(bar(bi), TX_W);
+            for (int nb = 0; nb < 2; ++nb)
+                tma_load_3d(sbase + L::OFF_WQ + s * 32768 + nb * DK * 128, &tm_wq, bar(bi), nb * 64, 0, rec0 + n);
+            armed |= 1u << bi; parity ^= 1u << bi;
+        };
+        auto load_p = [&](int n) {  // P(n)
+            const int s = n & 1, bi = B_P0 + s;
+            mbar_expect_tx(bar(bi), TX_P);
+            tma_load_3d(sbase + L::OFF_P + s * 8192, &tm_p, bar(bi), 0, 0, rec0 + n);
+            armed |= 1u << bi; parity ^= 1u << bi;
+        };
+        auto load_k = [&](int n) {  // K-hat(n) and e^{Gamma_C}(n)
+            const int s = n & 1, bi = B_K0 + s;
+            mbar_expect_tx(bar(bi), TX_K);
+            tma_load_3d(sbase + L::OFF_KH + s * 16384, &tm_kh, bar(bi), 0, 0, rec0 + n);
+            bulk_load(sbase + L::OFF_DEC + s * 512, recs + (size_t)n * REC_BYTES + REC_DEC, 512, bar(bi));
+            armed |= 1u << bi; parity ^= 1u << bi;
+        };
+        auto load_t = [&](int n) {  // T'(n)
+            const int s = n & 1, bi = B_T0 + s;
+            mbar_expect_tx(bar(bi), TX_T);
+            for (int kb = 0; kb < 2; ++kb)
+                tma_load_3d(sbase + L::OFF_T + s * 16384 + kb * 8192, &tm_t, bar(bi), kb * 32, 0, rec0 + n);
+            armed |= 1u << bi; parity ^= 1u << bi;
+        };
+        bool ok = *s_abort == 0 && nseg > 0;
+        if (ok) {
+            prefetch_tmap(&tm_wq); prefetch_tmap(&tm_p); prefetch_tmap(&tm_kh); prefetch_tmap(&tm_t);
+        }
+        // In the order their buffers free up: T' (product U(j-2)), K-hat and
+        // e^{Gamma_C} (product 3a(j-2) and the state update of chunk j-2), WQ
+        // (product 1(j-WS)), P (product 3b(j-2)).
+        for (int j = 0; ok && j < nseg; ++j) {
+            const uint32_t ph = (uint32_t)(((j - 2) >> 1) & 1);
+            if (j >= 2 && !(ok = wait1(B_TE0 + (j & 1), ph))) break;
+            load_t(j);
+            if (j >= 2 && !(ok = wait1(B_KE0 + (j & 1), ph))) break;
+            load_k(j);
+            if (j >= WS && !(ok = wait1(B_WE0 + j % WS, (uint32_t)(((j - WS) / WS) & 1)))) break;
+            load_w(j);
+            if (j >= 2 && !(ok = wait1(B_PE0 + (j & 1), ph))) break;
+            load_p(j);
+        }
+        if (*s_abort) {
+            // Leave no copy in flight into this CTA's shared memory.  At most one
+            // phase of each barrier is in flight, so waiting for the parity of the
+            // last armed completion waits for everything on it.
+            for (int i = 0; i <= B_T1; ++i)
+                if ((armed >> i) & 1) mbar_wait(bar(i), ((parity >> i) & 1) ^ 1u, ~0ull, prm.st);
+        }
+    } else if (issuer && lane == 0) {
+        // ====================== issuer warp (lane 0; the rest idle) ======================
         const uint32_t id_tf = make_idesc(2, false, false, 128, VS);
         const uint32_t id_bf = make_idesc(1, true, true, 128, VS);
         const uint32_t id_h = make_idesc(0, false, false, 128, VS);
-        int issued[B_M3 + 1] = {0};  // completions issued per barrier
-        auto load_w = [&](int n) {  // WQ(n) -> slot n % WS
-            const int s = n % WS, bi = B_W0 + s;
-            if (lane == 0) {
-                mbar_expect_tx(bar(bi), TX_W);
-                for (int nb = 0; nb < 2; ++nb)
-                    tma_load_3d(sbase + L::OFF_WQ + s * 32768 + nb * DK * 128, &tm_wq, bar(bi), nb * 64, 0, rec0 + n);
-            }
-            ++issued[bi];
-        };
-        auto load_p = [&](int n) {  // P(n) -> slot n & 1
-            const int s = n & 1, bi = B_P0 + s;
-            if (lane == 0) {
-                mbar_expect_tx(bar(bi), TX_P);
-                tma_load_3d(sbase + L::OFF_P + s * 8192, &tm_p, bar(bi), 0, 0, rec0 + n);
-            }
-            ++issued[bi];
-        };
-        auto load_k = [&](int n) {  // K-hat(n) and e^{Gamma_C}(n) -> slot n & 1
-            const int s = n & 1, bi = B_K0 + s;
-            if (lane == 0) {
-                mbar_expect_tx(bar(bi), TX_K);
-                tma_load_3d(sbase + L::OFF_KH + s * 16384, &tm_kh, bar(bi), 0, 0, rec0 + n);
-                bulk_load(sbase + L::OFF_DEC + s * 512, recs + (size_t)n * REC_BYTES + REC_DEC, 512, bar(bi));
-            }
-            ++issued[bi];
-        };
-        auto load_t = [&](int n) {  // T'(n) -> slot n & 1
-            const int s = n & 1, bi = B_T0 + s;
-            if (lane == 0) {
-                mbar_expect_tx(bar(bi), TX_T);
-                for (int kb = 0; kb < 2; ++kb)
-                    tma_load_3d(sbase + L::OFF_T + s * 16384 + kb * 8192, &tm_t, bar(bi), kb * 32, 0, rec0 + n);
-            }
-            ++issued[bi];
-        };
+        uint32_t armed = 0, parity = 0;  // per commit barrier: ever committed, count of commits mod 2
         auto commit = [&](int bi) {
-            if (lane == 0) umma_commit(bar(bi));
-            ++issued[bi];
+            umma_commit(bar(bi));
+            armed |= 1u << bi; parity ^= 1u << bi;
         };
         auto mma_u = [&](int n) {  // U = T'(n) V(n)
-            if (lane == 0) {
-                tc_fence_after();
-                for (int kk = 0; kk < 8; ++kk)
-                    umma<1>(tmem + L::TM_U, desc_kmaj_s<128, 4>(sbase + L::OFF_T + (n & 1) * 16384, 8192, kk * 8),
-                            desc_kmaj_s<128, 4>(sbase + L::OFF_VT, VS * 128, kk * 8), id_tf, kk > 0);
-            }
+            tc_fence_after();
+            for (int kk = 0; kk < 8; ++kk)
+                umma<1>(tmem + L::TM_U, desc_kmaj_s<128, 4>(sbase + L::OFF_T + (n & 1) * 16384, 8192, kk * 8),
+                        desc_kmaj_s<128, 4>(sbase + L::OFF_VT, VS * 128, kk * 8), id_tf, kk > 0);
+            if (n + 2 < nseg) commit(B_TE0 + (n & 1));  // T'(n) read: its buffer takes T'(n+2)
         };
         auto mma_1 = [&](int n) {  // D1[n & 1] = [W; Q e^G](n) S0
-            if (lane == 0) {
-                tc_fence_after();
-                for (int kk = 0; kk < DK / 16; ++kk)
-                    umma<0>(tmem + L::TM_D1 + (n & 1) * VS, desc_mnmaj<128>(sbase + L::OFF_WQ + (n % WS) * 32768, DK, kk * 16),
-                            desc_mnmaj<128>(sbase + L::OFF_S0, DK, kk * 16), id_bf, kk > 0);
-            }
+            tc_fence_after();
+            for (int kk = 0; kk < DK / 16; ++kk)
+                umma<0>(tmem + L::TM_D1 + (n & 1) * VS, desc_mnmaj<128>(sbase + L::OFF_WQ + (n % WS) * 32768, DK, kk * 16),
+                        desc_mnmaj<128>(sbase + L::OFF_S0, DK, kk * 16), id_bf, kk > 0);
+            commit(B_M1);
+            if (n + WS < nseg) commit(B_WE0 + n % WS);  // WQ(n) read
         };
         auto mma_3a = [&](int n) {  // D3 = K-hat(n)^T Vnew(n)
-            if (lane == 0) {
-                tc_fence_after();
-                for (int kk = 0; kk < 4; ++kk)
-                    umma<0>(tmem + L::TM_D3, desc_kmaj<128, 2>(sbase + L::OFF_KH + (n & 1) * 16384, 128, kk * 16),
-                            desc_kmaj<128, 2>(sbase + L::OFF_VN + (n & 1) * VS * 128, VS, kk * 16), id_h, kk > 0);
-            }
+            tc_fence_after();
+            for (int kk = 0; kk < 4; ++kk)
+                umma<0>(tmem + L::TM_D3, desc_kmaj<128, 2>(sbase + L::OFF_KH + (n & 1) * 16384, 128, kk * 16),
+                        desc_kmaj<128, 2>(sbase + L::OFF_VN + (n & 1) * VS * 128, VS, kk * 16), id_h, kk > 0);
+            commit(B_M3);
         };
         auto mma_3b = [&](int n) {  // D1[n & 1] rows 64..127 += P(n) Vnew(n)
-            if (lane == 0) {
-                tc_fence_after();
-                for (int kk = 0; kk < 4; ++kk)
-                    umma<0>(tmem + L::TM_D1 + (n & 1) * VS,
-                            desc_kmaj<128, 2>(sbase + L::OFF_P + (n & 1) * 8192 - 8192, 128, kk * 16),
-                            desc_kmaj<128, 2>(sbase + L::OFF_VN + (n & 1) * VS * 128, VS, kk * 16), id_h, 1u);
-            }
+            tc_fence_after();
+            for (int kk = 0; kk < 4; ++kk)
+                umma<0>(tmem + L::TM_D1 + (n & 1) * VS,
+                        desc_kmaj<128, 2>(sbase + L::OFF_P + (n & 1) * 8192 - 8192, 128, kk * 16),
+                        desc_kmaj<128, 2>(sbase + L::OFF_VN + (n & 1) * VS * 128, VS, kk * 16), id_h, 1u);
+            commit(B_MB);
+            if (n + 2 < nseg) commit(B_PE0 + (n & 1));  // P(n) read
         };
 
         bool ok = *s_abort == 0 && nseg > 0;
         if (ok) {
-            if (lane == 0) {
-                prefetch_tmap(&tm_wq); prefetch_tmap(&tm_p); prefetch_tmap(&tm_kh); prefetch_tmap(&tm_t);
-                for (int n = 0; n < CHAIN_PREFETCH && n < nseg; ++n)
-                    prefetch_l2(recs + (size_t)n * REC_BYTES, REC_BYTES);
-            }
-            load_w(0); load_p(0); load_k(0); load_t(0);
-            if (nseg > 1) {
-                if (WS == 2) load_w(1);
-                load_p(1); load_k(1); load_t(1);
-            }
-            ok = wait_warp(B_VT, 0u) && wait_warp(B_T0, 0u);
+            ok = wait1(B_VT, 0u) && wait1(B_T0, 0u);
             if (ok) mma_u(0);
         }
         for (int n = 0; ok && n < nseg; ++n) {
             const bool more = n + 1 < nseg;
-            if (lane == 0 && n + CHAIN_PREFETCH < nseg)
-                prefetch_l2(recs + (size_t)(n + CHAIN_PREFETCH) * REC_BYTES, REC_BYTES);
-            if (!(ok = wait_warp(B_S0, (uint32_t)(n & 1)))) break;      // S0(n); D3, e^{Gamma_C}(n-1) consumed
-            if (n >= 1 && more) load_k(n + 1);                            // its slot held K-hat(n-1)
-            if (!(ok = wait_warp(B_W0 + (n % WS), (uint32_t)((n / WS) & 1)))) break;  // WQ(n)
-            if (n >= 2 && !(ok = wait_warp(B_OUT0 + (n & 1), (uint32_t)(((n - 2) >> 1) & 1)))) break;  // D1[n&1] free
+            if (!(ok = wait1(B_S0, (uint32_t)(n & 1)))) break;      // S0(n)
+            if (!(ok = wait1(B_W0 + (n % WS), (uint32_t)((n / WS) & 1)))) break;  // WQ(n)
+            if (n >= 2 && !(ok = wait1(B_OUT0 + (n & 1), (uint32_t)(((n - 2) >> 1) & 1)))) break;  // D1[n&1] free
             mma_1(n);
-            commit(B_M1);
             if (n >= 1) {
-                if (!(ok = wait_warp(B_P0 + ((n - 1) & 1), (uint32_t)(((n - 1) >> 1) & 1)))) break;  // P(n-1)
+                if (!(ok = wait1(B_P0 + ((n - 1) & 1), (uint32_t)(((n - 1) >> 1) & 1)))) break;  // P(n-1)
                 mma_3b(n - 1);
-                commit(B_MB);
             }
-            if (!(ok = wait_warp(B_VN0 + (n & 1), (uint32_t)((n >> 1) & 1)))) break;  // Vnew(n); U(n), WQ(n) consumed
-            // the slots of WQ(n) and T'(n): product 1(n) and U(n) are done
-            if (n + WS < nseg) load_w(n + WS);
-            if (n + 2 < nseg) load_t(n + 2);
-            if (!(ok = wait_warp(B_K0 + (n & 1), (uint32_t)((n >> 1) & 1)))) break;  // K-hat(n)
+            if (!(ok = wait1(B_VN0 + (n & 1), (uint32_t)((n >> 1) & 1)))) break;  // Vnew(n)
+            if (!(ok = wait1(B_K0 + (n & 1), (uint32_t)((n >> 1) & 1)))) break;   // K-hat(n)
             mma_3a(n);
-            commit(B_M3);
-            if (n >= 1) {
-                if (!(ok = wait_warp(B_MB, (uint32_t)((n - 1) & 1)))) break;  // 3b(n-1) has read P(n-1)
-                if (more) load_p(n + 1);                                     // into P(n-1)'s slot
-            }
             if (more) {
-                if (!(ok = wait_warp(B_VT, (uint32_t)((n + 1) & 1)))) break;                 // V^T(n+1)
-                if (!(ok = wait_warp(B_T0 + ((n + 1) & 1), (uint32_t)(((n + 1) >> 1) & 1)))) break;  // T'(n+1)
+                if (!(ok = wait1(B_VT, (uint32_t)((n + 1) & 1)))) break;                 // V^T(n+1)
+                if (!(ok = wait1(B_T0 + ((n + 1) & 1), (uint32_t)(((n + 1) >> 1) & 1)))) break;  // T'(n+1)
                 mma_u(n + 1);  // U is free: Vnew(n) has read it
             }
         }
         if (ok) {  // the last chunk's output block, once output(N-2) has been read
-            if (nseg >= 2) ok = wait_warp(B_OUT0 + (nseg & 1), (uint32_t)(((nseg - 2) >> 1) & 1));
-            if (ok) ok = wait_warp(B_P0 + ((nseg - 1) & 1), (uint32_t)(((nseg - 1) >> 1) & 1));
-            if (ok) { mma_3b(nseg - 1); commit(B_MB); }
+            if (nseg >= 2) ok = wait1(B_OUT0 + (nseg & 1), (uint32_t)(((nseg - 2) >> 1) & 1));
+            if (ok) ok = wait1(B_P0 + ((nseg - 1) & 1), (uint32_t)(((nseg - 1) >> 1) & 1));
+            if (ok) mma_3b(nseg - 1);
         }
-        if (*s_abort && lane == 0) {
-            // Leave nothing in flight that targets this CTA's shared memory or TMEM.
-            // At most one phase of each barrier is ever in flight, so waiting for the
-            // parity of its last issued completion waits for everything on it.
-            for (int i = 0; i <= B_M3; ++i)
-                if (issued[i] > 0) mbar_wait(bar(i), (uint32_t)((issued[i] - 1) & 1), ~0ull, prm.st);
+        if (*s_abort) {
+            // Leave no product in flight that writes this CTA's TMEM or arrives on
+            // its barriers (one phase in flight per barrier, as above).
+            for (int i = B_M1; i <= B_PE1; ++i)
+                if ((armed >> i) & 1) mbar_wait(bar(i), ((parity >> i) & 1) ^ 1u, ~0ull, prm.st);
         }
-    } else {
+    } else if (!loader && !issuer) {
         // =============================== compute warps ===============================
         const int lq = warp & 3;              // TMEM lane quarter of this warp
         const int cg = warp >> 2;             // value-column group of this warp
@@ -426,6 +431,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
                     for (int e = 0; e < 16; ++e) S[c16 + e] = dc * S[c16 + e] + t[e];
                 }
             }
+            if (n + 2 < nseg) arrive(B_KE0 + (n & 1));  // e^{Gamma_C}(n) read, 3a(n) done
             store_state_bf16();  // S0 is free: product 1(n) completed
             tc_fence_before();
             arrive(B_S0);
@@ -442,6 +448,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
             for (int e = 0; e < CPT / 4; ++e) dst[e] = make_float4(S[4 * e], S[4 * e + 1], S[4 * e + 2], S[4 * e + 3]);
         }
     }
+    __syncwarp();  // the idle lanes of the loader and issuer warps wait for lane 0
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
