@@ -60,22 +60,23 @@ struct ChainLayout {
     static_assert(VS_ == 64 || VS_ == 128, "value slice");
     static constexpr int VS = VS_;
     static constexpr int WS = VS == 64 ? 2 : 1;          // WQ buffers
-    static constexpr int OFF_WQ = 0;                     // bf16 MN-major [DK][128]: [W; Q e^G] (32 KB slots)
-    static constexpr int OFF_P = WS * 32768;             // two fp16 K-major [64][64] (8 KB)
-    static constexpr int OFF_KH = OFF_P + 16384;         // two fp16 K-major [128][64] (16 KB)
+    // Record tiles (32B swizzle, 32-byte rows of 16 tokens; 32 KB WQ slots):
+    static constexpr int OFF_WQ = 0;                     // bf16 MN-major [8][DK][16]: [W; Q e^G]
+    static constexpr int OFF_P = WS * 32768;             // two fp16 K-major [4][64][16] (8 KB)
+    static constexpr int OFF_KH = OFF_P + 16384;         // two fp16 K-major [4][128][16] (16 KB)
     static constexpr int OFF_T = OFF_KH + 32768;         // two tf32 K-major [64][64] (8 KB K-blocks)
     static constexpr int OFF_DEC = OFF_T + 32768;        // two 512-byte slots of e^{Gamma_C} (with K-hat)
     static constexpr int OFF_S0 = OFF_DEC + 1024;        // bf16 MN-major S0 [DK][VS], 128B swizzle
     static constexpr int OFF_VT = OFF_S0 + DK * VS * 2;  // tf32 K-major V^T [VS][64]
-    static constexpr int OFF_VN = OFF_VT + VS * 256;     // two fp16 K-major Vnew^T [VS][64]
+    static constexpr int OFF_VN = OFF_VT + VS * 256;     // two fp16 MN-major Vnew [64][VS], 128B swizzle
     static constexpr int OFF_MISC = OFF_VN + 2 * VS * 128;  // barriers, TMEM address, abort flag
     static constexpr int TOTAL = OFF_MISC + 1024;
     static constexpr int SMEM_BYTES = TOTAL + 1024;  // slack for the 1 KB base alignment
     static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
     static_assert(OFF_S0 % 1024 == 0 && OFF_VT % 1024 == 0 && OFF_VN % 1024 == 0, "1 KB aligned tiles");
-    // The 128-row views read 8 KB before each P buffer (rows 0..63, discarded)
-    // and 8 KB past T's second buffer (rows 64..127, discarded).
-    static_assert(OFF_P >= 8192 && OFF_T + 2 * 16384 + 8192 <= TOTAL, "operand views stay in bounds");
+    // The 128-row views read 2 KB before each 2 KB block of P (rows 0..63,
+    // discarded) and 8 KB past T's second buffer (rows 64..127, discarded).
+    static_assert(OFF_P >= 2048 && OFF_T + 2 * 16384 + 8192 <= TOTAL, "operand views stay in bounds");
 
     static constexpr uint32_t TM_U = 0;          // U (lane = token)
     static constexpr uint32_t TM_D1 = VS;        // two: [W; Q e^G] S0, then += P Vnew on lanes 64..127
@@ -177,20 +178,19 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
         auto load_w = [&](int n) {  // WQ(n)
             const int s = n % WS, bi = B_W0 + s;
             mbar_expect_tx(bar(bi), TX_W);
-            for (int nb = 0; nb < 2; ++nb)
-                tma_load_3d(sbase + L::OFF_WQ + s * 32768 + nb * DK * 128, &tm_wq, bar(bi), nb * 64, 0, rec0 + n);
+            tma_load_4d(sbase + L::OFF_WQ + s * 32768, &tm_wq, bar(bi), 0, 0, 0, rec0 + n);
             armed |= 1u << bi; parity ^= 1u << bi;
         };
         auto load_p = [&](int n) {  // P(n)
             const int s = n & 1, bi = B_P0 + s;
             mbar_expect_tx(bar(bi), TX_P);
-            tma_load_3d(sbase + L::OFF_P + s * 8192, &tm_p, bar(bi), 0, 0, rec0 + n);
+            tma_load_4d(sbase + L::OFF_P + s * 8192, &tm_p, bar(bi), 0, 0, 0, rec0 + n);
             armed |= 1u << bi; parity ^= 1u << bi;
         };
         auto load_k = [&](int n) {  // K-hat(n) and e^{Gamma_C}(n)
             const int s = n & 1, bi = B_K0 + s;
             mbar_expect_tx(bar(bi), TX_K);
-            tma_load_3d(sbase + L::OFF_KH + s * 16384, &tm_kh, bar(bi), 0, 0, rec0 + n);
+            tma_load_4d(sbase + L::OFF_KH + s * 16384, &tm_kh, bar(bi), 0, 0, 0, rec0 + n);
             bulk_load(sbase + L::OFF_DEC + s * 512, recs + (size_t)n * REC_BYTES + REC_DEC, 512, bar(bi));
             armed |= 1u << bi; parity ^= 1u << bi;
         };
@@ -230,7 +230,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
         // ====================== issuer warp (lane 0; the rest idle) ======================
         const uint32_t id_tf = make_idesc(2, false, false, 128, VS);
         const uint32_t id_bf = make_idesc(1, true, true, 128, VS);
-        const uint32_t id_h = make_idesc(0, false, false, 128, VS);
+        const uint32_t id_h = make_idesc(0, false, true, 128, VS);  // B = Vnew, MN-major
         uint32_t armed = 0, parity = 0;  // per commit barrier: ever committed, count of commits mod 2
         auto commit = [&](int bi) {
             umma_commit(bar(bi));
@@ -246,7 +246,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
         auto mma_1 = [&](int n) {  // D1[n & 1] = [W; Q e^G](n) S0
             tc_fence_after();
             for (int kk = 0; kk < DK / 16; ++kk)
-                umma<0>(tmem + L::TM_D1 + (n & 1) * VS, desc_mnmaj<128>(sbase + L::OFF_WQ + (n % WS) * 32768, DK, kk * 16),
+                umma<0>(tmem + L::TM_D1 + (n & 1) * VS, desc_mnmaj<32>(sbase + L::OFF_WQ + (n % WS) * 32768, DK, kk * 16),
                         desc_mnmaj<128>(sbase + L::OFF_S0, DK, kk * 16), id_bf, kk > 0);
             commit(B_M1);
             if (n + WS < nseg) commit(B_WE0 + n % WS);  // WQ(n) read
@@ -254,16 +254,16 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
         auto mma_3a = [&](int n) {  // D3 = K-hat(n)^T Vnew(n)
             tc_fence_after();
             for (int kk = 0; kk < 4; ++kk)
-                umma<0>(tmem + L::TM_D3, desc_kmaj<128, 2>(sbase + L::OFF_KH + (n & 1) * 16384, 128, kk * 16),
-                        desc_kmaj<128, 2>(sbase + L::OFF_VN + (n & 1) * VS * 128, VS, kk * 16), id_h, kk > 0);
+                umma<0>(tmem + L::TM_D3, desc_kmaj<32, 2>(sbase + L::OFF_KH + (n & 1) * 16384, 128, kk * 16),
+                        desc_mnmaj<128>(sbase + L::OFF_VN + (n & 1) * VS * 128, CH, kk * 16), id_h, kk > 0);
             commit(B_M3);
         };
         auto mma_3b = [&](int n) {  // D1[n & 1] rows 64..127 += P(n) Vnew(n)
             tc_fence_after();
             for (int kk = 0; kk < 4; ++kk)
                 umma<0>(tmem + L::TM_D1 + (n & 1) * VS,
-                        desc_kmaj<128, 2>(sbase + L::OFF_P + (n & 1) * 8192 - 8192, 128, kk * 16),
-                        desc_kmaj<128, 2>(sbase + L::OFF_VN + (n & 1) * VS * 128, VS, kk * 16), id_h, 1u);
+                        desc_kmaj<32, 2>(sbase + L::OFF_P + (n & 1) * 8192 - 2048, CH, kk * 16),
+                        desc_mnmaj<128>(sbase + L::OFF_VN + (n & 1) * VS * 128, CH, kk * 16), id_h, 1u);
             commit(B_MB);
             if (n + 2 < nseg) commit(B_PE0 + (n & 1));  // P(n) read
         };
@@ -390,7 +390,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
             const bool more = n + 1 < nseg;
             if (!(ok = wait_warp(B_M1, (uint32_t)(n & 1)))) break;  // U(n), D1[n&1] rows 0..63
             tc_fence_after();
-            if (lq < 2) {  // Vnew(n) = U - W S0 -> Vnew^T tile n & 1
+            if (lq < 2) {  // Vnew(n) = U - W S0 -> Vnew tile n & 1
                 uint8_t *vn = sm + L::OFF_VN + (n & 1) * VS * 128;
 #pragma unroll
                 for (int c16 = 0; c16 < CPT; c16 += 16) {
@@ -398,9 +398,11 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
                     tmem_ld16(tmem + lane_base + L::TM_U + cg * CPT + c16, u);
                     tmem_ld16(tmem + lane_base + L::TM_D1 + (n & 1) * VS + cg * CPT + c16, w);
                     tmem_wait_ld();
+                    float a8[8], b8[8];
 #pragma unroll
-                    for (int e = 0; e < 16; ++e)
-                        *reinterpret_cast<uint16_t *>(vn + kmaj<128, 2>(cg * CPT + c16 + e, ch, VS)) = f16_bits(u[e] - w[e]);
+                    for (int e = 0; e < 8; ++e) { a8[e] = u[e] - w[e]; b8[e] = u[8 + e] - w[8 + e]; }
+                    *reinterpret_cast<uint4 *>(vn + mnmaj<128, 2>(ch, cg * CPT + c16, CH)) = pack8_f16(a8);
+                    *reinterpret_cast<uint4 *>(vn + mnmaj<128, 2>(ch, cg * CPT + c16 + 8, CH)) = pack8_f16(b8);
                 }
                 fence_async_smem();
                 tc_fence_before();

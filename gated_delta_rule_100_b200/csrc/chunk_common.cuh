@@ -8,13 +8,17 @@
 //   chain (one CTA per (b, h), chunks in order): U = T Diag(beta) V, then the
 //         state pass Vnew = U - W S, S <- e^{Gamma_C} S + K-hat^T Vnew and the
 //         outputs (Q e^Gamma) S + P Vnew.
-// A record holds plain row-major arrays (the chain kernel's tensor loads put
-// them in the swizzled UMMA operand layouts):
-//   WQ   bf16 [dk][128]  row = key channel; columns 0..63 = W^T, 64..127 = (Q e^Gamma)^T
-//   P    fp16 [64][64]   causal q-k block (incl. diagonal), rows = queries
-//   KH   fp16 [128][64]  K-hat^T: row = key channel, column = token
-//   T'   fp32 [64][64]   T' = T Diag(beta), unit-lower times beta
-//   DEC  fp32 [128]      e^{Gamma_C} per key channel
+// A record holds these arrays (the chain kernel's tensor loads apply the UMMA
+// operand swizzle).  The first three are cut into 16-token blocks, each block a
+// row-major array of 32-byte rows, so that the prep kernel's warps, which hold
+// 16 consecutive tokens of 32 consecutive rows per thread, write them as
+// contiguous 1 KB runs:
+//   WQ   bf16 [8][dk][16]   [W; Q e^Gamma] over tokens m = 16 blk + e (blocks
+//                           0..3 = W, 4..7 = Q e^Gamma), row = key channel
+//   P    fp16 [4][64][16]   causal q-k block (incl. diagonal): [J][i][e] = P[i][16 J + e]
+//   KH   fp16 [4][128][16]  K-hat^T: [I][c][e] = K-hat[16 I + e][c]
+//   T'   fp32 [64][64]      T' = T Diag(beta), unit-lower times beta, row-major
+//   DEC  fp32 [128]         e^{Gamma_C} per key channel
 // at the offsets below (each 16-byte aligned; 72.5 KB per record).
 #pragma once
 #include <cuda_fp16.h>

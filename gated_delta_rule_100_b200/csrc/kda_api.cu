@@ -221,23 +221,31 @@ int num_sms(int dev) {
 // 128-byte swizzle of the chain kernel's operand tiles.
 int make_rec_maps(PFN_cuTensorMapEncodeTiled_v12000 enc, const uint8_t *rec, long long nrec, int dk,
                   CUtensorMap *maps) {
-    struct Part { size_t off; CUtensorMapDataType dt; int esize, cols, rows, box_cols; };
-    const Part parts[4] = {{(size_t)kda::REC_WQ, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 128, dk, 64},
-                           {(size_t)kda::REC_P, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, 64, 64, 64},
-                           {(size_t)kda::REC_KH, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, 64, 128, 64},
-                           {(size_t)kda::REC_T, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, 64, 64, 32}};
-    for (int i = 0; i < 4; ++i) {
+    // WQ, P, K-hat: [blocks][rows][16] 16-bit arrays, one box = one record's part
+    // (4-D: token-in-block, row, block, record), 32-byte swizzle
+    struct Part { size_t off; CUtensorMapDataType dt; int rows, blocks; };
+    const Part parts[3] = {{(size_t)kda::REC_WQ, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dk, 8},
+                           {(size_t)kda::REC_P, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, kda::CH, 4},
+                           {(size_t)kda::REC_KH, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 128, 4}};
+    cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+    for (int i = 0; i < 3; ++i) {
         const Part &p = parts[i];
-        cuuint64_t dims[3] = {(cuuint64_t)p.cols, (cuuint64_t)p.rows, (cuuint64_t)nrec};
-        cuuint64_t strides[2] = {(cuuint64_t)p.cols * p.esize, (cuuint64_t)kda::REC_BYTES};
-        cuuint32_t box[3] = {(cuuint32_t)p.box_cols, (cuuint32_t)p.rows, 1u};
-        cuuint32_t estr[3] = {1u, 1u, 1u};
-        CUresult r = enc(&maps[i], p.dt, 3, const_cast<uint8_t *>(rec + p.off), dims, strides, box, estr,
-                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+        cuuint64_t dims[4] = {(cuuint64_t)kda::SUB, (cuuint64_t)p.rows, (cuuint64_t)p.blocks, (cuuint64_t)nrec};
+        cuuint64_t strides[3] = {(cuuint64_t)kda::SUB * 2, (cuuint64_t)kda::SUB * 2 * p.rows, (cuuint64_t)kda::REC_BYTES};
+        cuuint32_t box[4] = {(cuuint32_t)kda::SUB, (cuuint32_t)p.rows, (cuuint32_t)p.blocks, 1u};
+        CUresult r = enc(&maps[i], p.dt, 4, const_cast<uint8_t *>(rec + p.off), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B,
                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
         if (r != CUDA_SUCCESS) return KDA_ERR_CUDA;
     }
-    return KDA_OK;
+    // T': fp32 [64][64] row-major, boxes of 32 columns, 128-byte swizzle
+    cuuint64_t dims[3] = {(cuuint64_t)kda::CH, (cuuint64_t)kda::CH, (cuuint64_t)nrec};
+    cuuint64_t strides[2] = {(cuuint64_t)kda::CH * 4, (cuuint64_t)kda::REC_BYTES};
+    cuuint32_t box[3] = {32u, (cuuint32_t)kda::CH, 1u};
+    CUresult r = enc(&maps[3], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<uint8_t *>(rec + kda::REC_T), dims, strides,
+                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? KDA_OK : KDA_ERR_CUDA;
 }
 
 // Value-column slices per (b, h) in the chain kernel.  Every CTA of a (b, h)

@@ -36,8 +36,8 @@
 //   T  (I + A)^{-1}: 16x16 diagonal blocks by substitution, off-diagonal blocks
 //      from N = D A_off as T = (I - N + N^2 - N^3) D, fp32 on CUDA cores
 //   W  T' = T Diag(beta) -> record;  W^T = (K e^G)^T T'^T  (UMMA tf32) -> record
-// Record parts are plain row-major arrays written with contiguous 16-byte
-// stores; the chain kernel's tensor loads apply the operand swizzle.
+// Each warp writes its record parts as contiguous 1 KB runs (the block layout
+// of chunk_common.cuh); the chain kernel's tensor loads apply the operand swizzle.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <stdint.h>
@@ -320,7 +320,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         {
             if (active) {
                 if (I == 0) reinterpret_cast<float *>(rec + REC_DEC)[c] = dec;
-                uint16_t *khr = reinterpret_cast<uint16_t *>(rec + REC_KH) + c * CH + tb;
+                uint16_t *khr = reinterpret_cast<uint16_t *>(rec + REC_KH) + (I * 128 + c) * SUB;
                 float r = postB;
 #pragma unroll
                 for (int hh = 1; hh >= 0; --hh) {
@@ -329,7 +329,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     for (int e = 7; e >= 0; --e) { kh[e] = kval(hh * 8 + e) * r; r *= al[hh * 8 + e]; }
                     *reinterpret_cast<uint4 *>(khr + hh * 8) = pack8_f16(kh);
                 }
-                uint16_t *qer = reinterpret_cast<uint16_t *>(rec + REC_WQ) + c * 128 + 64 + tb;
+                uint16_t *qer = reinterpret_cast<uint16_t *>(rec + REC_WQ) + ((NSUB + I) * DK + c) * SUB;
                 float p = preB;
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
@@ -406,7 +406,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     *reinterpret_cast<float4 *>(sA + i * A_LD + j0 + e) = w;
                 }
             } else {
-                uint16_t *pr = reinterpret_cast<uint16_t *>(rec + REC_P) + i * CH + j0;
+                uint16_t *pr = reinterpret_cast<uint16_t *>(rec + REC_P) + (cc * CH + i) * SUB;
 #pragma unroll
                 for (int e8 = 0; e8 < 16; e8 += 8) {
                     float p8[8];
@@ -531,7 +531,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         mma_pending = true;
         if (!wait_all(bar_mma, ph_mma, mma_pending)) { aborted = true; break; }
         ph_mma ^= 1u;
-        if ((warp & 3) < DK / 32) {  // W^T row ch -> W columns (tokens 16 qb ..) of the record's WQ
+        if ((warp & 3) < DK / 32) {  // W^T row ch, tokens 16 qb .. -> WQ block qb
             const int i0 = qb * 16;
             float t[16];
             tmem_ld16(tmem + lane_base + L::TM_W + i0, t);
@@ -539,7 +539,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             float a8[8], b8[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) { a8[e] = t[e]; b8[e] = t[8 + e]; }
-            uint16_t *wr = reinterpret_cast<uint16_t *>(rec + REC_WQ) + ch * 128 + i0;
+            uint16_t *wr = reinterpret_cast<uint16_t *>(rec + REC_WQ) + (qb * DK + ch) * SUB;
             *reinterpret_cast<uint4 *>(wr) = pack8_bf16(a8);
             *reinterpret_cast<uint4 *>(wr + 8) = pack8_bf16(b8);
         }
