@@ -1,7 +1,7 @@
 // chain_fwd.cu -- the inter-chunk (state-passing) half of the chunkwise KDA
 // prefill (sm_100a).
 //
-// One CTA owns one (b, h, slice of 64 value columns) and walks the chunks of a
+// One CTA owns one (b, h, slice of 64 or 128 value columns) and walks the chunks of a
 // segment in order, reading the per-chunk records of the prep kernel
 // (prep_fwd.cu; layout in chunk_common.cuh).  Per chunk, S0 = state at the
 // chunk start:
@@ -29,15 +29,17 @@
 // written, S0 written) between the issuer and the compute warps -- so the
 // tensor pipe, which executes in issue order, is fed as soon as each operand is
 // ready.  A TMA issue can hold its thread for hundreds of cycles while the
-// SM's copy engine is busy, which is why no load sits in the issuer's path.  Per chunk n it runs
-// 1(n), 3b(n-1), 3a(n), U(n+1): only 1 and 3a lie on the state's critical
-// path, the other two fill the pipe while the compute warps form Vnew(n) and
-// update the state.  Buffers: two output accumulators and two each of the
-// Vnew tiles, WQ, P, K-hat and T'; one V^T and one S0.
+// SM's copy engine is busy, which is why no load sits in the issuer's path.
+// Per chunk n it runs 1(n), 3b(n-1), 3a(n), U(n+1): only 1 and 3a lie on the
+// state's critical path, the other two fill the pipe while the compute warps
+// form Vnew(n) and update the state.  Buffers: two output accumulators and two
+// each of the Vnew tiles, WQ (at 64 columns), P, K-hat and T'; one V^T and one
+// S0.
 //
-// The state lives in fp32 registers (compute thread (c, g) holds row c, 16
-// columns); a bf16 copy in shared memory feeds the tensor core.  The values V
-// are read with plain coalesced loads two chunks ahead of their product.
+// The state lives in fp32 registers (compute thread (c, g) holds row c and
+// VS / 4 columns); a bf16 copy in shared memory feeds the tensor core.  The
+// values V are read with plain coalesced loads one chunk before their V^T tile
+// is built.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <stdint.h>
