@@ -382,7 +382,9 @@ int kda_chunk_fwd(const void *q, const void *k, const void *v, const float *g, c
         pp.n_begin = n0;
         pp.nseg = cnt;
         pp.st = dst;
-        cudaError_t e = timed_launch(dev, 0, sp, [&] { return kda::launch_prep(tq, tk, pp, dk, prep_ctas > 0 ? prep_ctas : 1, sp); });
+        // the first segment's prep runs alone: two CTAs on every SM
+        const int ctas = i == 0 ? 2 * sms : (prep_ctas > 0 ? prep_ctas : 1);
+        cudaError_t e = timed_launch(dev, 0, sp, [&] { return kda::launch_prep(tq, tk, pp, dk, ctas, sp); });
         if (e != cudaSuccess) return KDA_ERR_CUDA;
         if (multi && (cudaEventRecord(w->prep_done[buf], sp) != cudaSuccess ||
                       cudaStreamWaitEvent(sc, w->prep_done[buf], 0) != cudaSuccess))
