@@ -9,7 +9,8 @@ namespace kda {
 
 // Items (b, h, chunk) of chunks [n_begin, n_begin + nseg), claimed by persistent CTAs.
 struct PrepParams {
-    const float *g;      // [B, T, H, dk]
+    const float *g;      // [B, T, H, g_dk]
+    int g_dk;            // gate values per (token, head): dk (per key channel) or 1 (one, broadcast)
     const float *beta;   // [B, T, H]
     uint8_t *ws;         // records [B*H][nseg][REC_BYTES]
     int *ticket;         // item counter, zero at launch: CTAs claim items from it

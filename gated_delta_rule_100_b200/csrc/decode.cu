@@ -13,7 +13,9 @@
 // written once.  One CTA owns one (b, h): 256 threads tile the state as
 // (row groups) x (dv / 4 float4 column groups), so every warp-wide load or
 // store covers one contiguous 512-byte state row.  The two column reductions
-// (k.s' and q.s') go through shared memory across row groups.
+// (k.s' and q.s') go through shared memory across row groups.  The gate is
+// either one log-decay per key channel (g [B, H, dk]) or one per head shared by
+// all channels (g [B, H], the scalar-gate form): g_dk = dk or 1.
 #include <cuda_bf16.h>
 #include <stdint.h>
 
@@ -28,7 +30,7 @@ __global__ void __launch_bounds__(DEC_THREADS)
 decode_step_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ k,
                    const uint16_t *__restrict__ v, const float *__restrict__ g,
                    const float *__restrict__ beta, float scale, float *__restrict__ state,
-                   uint16_t *__restrict__ out) {
+                   uint16_t *__restrict__ out, int g_dk) {
     constexpr int NCG = DV / 4;              // float4 column groups
     constexpr int NRG = DEC_THREADS / NCG;   // row groups
     constexpr int RPT = DK / NRG;            // state rows per thread
@@ -45,7 +47,7 @@ decode_step_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ 
 
     const uint16_t *qh = q + (size_t)bh * DK;
     const uint16_t *kh = k + (size_t)bh * DK;
-    const float *gh = g + (size_t)bh * DK;
+    const float *gh = g + (size_t)bh * g_dk;
     float *S = state + (size_t)bh * DK * DV;
 
     // Issue the state loads first: they are the long-latency part.
@@ -58,7 +60,7 @@ decode_step_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ 
     for (int r = tid; r < DK; r += DEC_THREADS) {
         s_k[r] = bf16_bits_to_f32(kh[r]);
         s_q[r] = bf16_bits_to_f32(qh[r]);
-        s_a[r] = __expf(gh[r]);
+        s_a[r] = __expf(gh[g_dk > 1 ? r : 0]);
     }
     __syncthreads();
     if (tid < 32) {
@@ -120,23 +122,23 @@ decode_step_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ 
 template <int DK, int DV>
 static cudaError_t launch_decode_t(const void *q, const void *k, const void *v, const float *g,
                                    const float *beta, float scale, float *state, void *out,
-                                   int BH, cudaStream_t stream) {
+                                   int BH, int g_dk, cudaStream_t stream) {
     decode_step_kernel<DK, DV><<<BH, DEC_THREADS, 0, stream>>>(
         (const uint16_t *)q, (const uint16_t *)k, (const uint16_t *)v, g, beta, scale, state,
-        (uint16_t *)out);
+        (uint16_t *)out, g_dk);
     return cudaGetLastError();
 }
 
 cudaError_t launch_decode(const void *q, const void *k, const void *v, const float *g,
                           const float *beta, float scale, float *state, void *out, int BH, int dk,
-                          int dv, cudaStream_t stream) {
+                          int dv, int g_dk, cudaStream_t stream) {
     if (dk == 128 && dv == 128)
-        return launch_decode_t<128, 128>(q, k, v, g, beta, scale, state, out, BH, stream);
+        return launch_decode_t<128, 128>(q, k, v, g, beta, scale, state, out, BH, g_dk, stream);
     if (dk == 128 && dv == 64)
-        return launch_decode_t<128, 64>(q, k, v, g, beta, scale, state, out, BH, stream);
+        return launch_decode_t<128, 64>(q, k, v, g, beta, scale, state, out, BH, g_dk, stream);
     if (dk == 64 && dv == 128)
-        return launch_decode_t<64, 128>(q, k, v, g, beta, scale, state, out, BH, stream);
-    return launch_decode_t<64, 64>(q, k, v, g, beta, scale, state, out, BH, stream);
+        return launch_decode_t<64, 128>(q, k, v, g, beta, scale, state, out, BH, g_dk, stream);
+    return launch_decode_t<64, 64>(q, k, v, g, beta, scale, state, out, BH, g_dk, stream);
 }
 
 }  // namespace kda

@@ -17,7 +17,7 @@
 namespace kda {
 cudaError_t launch_decode(const void *q, const void *k, const void *v, const float *g,
                           const float *beta, float scale, float *state, void *out, int BH, int dk,
-                          int dv, cudaStream_t stream);
+                          int dv, int g_dk, cudaStream_t stream);
 }
 
 #include "chunk_common.cuh"
@@ -259,7 +259,7 @@ int chain_slices(int B, int H, int dv, int sms) { return (dv == 128 && 2LL * B *
 
 extern "C" {
 
-int kda_abi_version(void) { return 100; }
+int kda_abi_version(void) { return 101; }
 
 const char *kda_status_string(int status) {
     switch (status) {
@@ -291,14 +291,16 @@ int kda_stream_status(void *stream) {
     return (v & kda::DEV_TIMEOUT) ? KDA_ERR_TIMEOUT : KDA_OK;
 }
 
-int kda_chunk_fwd(const void *q, const void *k, const void *v, const float *g, const float *beta,
-                  float scale, const float *h0, void *out, float *hT, int B, int T, int H, int dk,
-                  int dv, void *stream) {
+// The prefill for either gate form: g_dk = dk (g [B, T, H, dk]) or 1 (g [B, T, H]).
+static int chunk_fwd_impl(const void *q, const void *k, const void *v, const float *g, const float *beta,
+                          float scale, const float *h0, void *out, float *hT, int B, int T, int H, int dk,
+                          int dv, void *stream, bool scalar_gate) {
     if (B < 1 || H < 1 || T < 0) return KDA_ERR_INVALID_ARG;
     if (T > 0 && (!q || !k || !v || !g || !beta || !out)) return KDA_ERR_INVALID_ARG;
     if ((dk != 64 && dk != 128) || (dv != 64 && dv != 128)) return KDA_ERR_UNSUPPORTED;
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(g) || !aligned4(beta) ||
-        !aligned16(out) || !aligned16(h0) || !aligned16(hT))
+    const int g_dk = scalar_gate ? 1 : dk;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !(scalar_gate ? aligned4(g) : aligned16(g)) ||
+        !aligned4(beta) || !aligned16(out) || !aligned16(h0) || !aligned16(hT))
         return KDA_ERR_ALIGNMENT;
     if ((long long)B * H * 4 > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -375,6 +377,7 @@ int kda_chunk_fwd(const void *q, const void *k, const void *v, const float *g, c
         if (cudaMemsetAsync(tickets + buf, 0, sizeof(int), sp) != cudaSuccess) return KDA_ERR_CUDA;
         kda::PrepParams pp;
         pp.g = g;
+        pp.g_dk = g_dk;
         pp.beta = beta;
         pp.ws = recs[buf];
         pp.ticket = tickets + buf;
@@ -453,18 +456,42 @@ int kda_release_workspace(void) {
     return st;
 }
 
-int kda_decode_step(const void *q, const void *k, const void *v, const float *g, const float *beta,
-                    float scale, float *state, void *out, int B, int H, int dk, int dv, void *stream) {
+// The decode step for either gate form: g [B, H, dk] or, scalar_gate, g [B, H].
+static int decode_impl(const void *q, const void *k, const void *v, const float *g, const float *beta,
+                       float scale, float *state, void *out, int B, int H, int dk, int dv, void *stream,
+                       bool scalar_gate) {
     if (!q || !k || !v || !g || !beta || !state || !out) return KDA_ERR_INVALID_ARG;
     if (B < 1 || H < 1) return KDA_ERR_INVALID_ARG;
     if ((dk != 64 && dk != 128) || (dv != 64 && dv != 128)) return KDA_ERR_UNSUPPORTED;
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(g) || !aligned4(beta) ||
-        !aligned16(state) || !aligned16(out))
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !(scalar_gate ? aligned4(g) : aligned16(g)) ||
+        !aligned4(beta) || !aligned16(state) || !aligned16(out))
         return KDA_ERR_ALIGNMENT;
     if ((long long)B * H > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
-    cudaError_t e = kda::launch_decode(q, k, v, g, beta, scale, state, out, B * H, dk, dv,
+    cudaError_t e = kda::launch_decode(q, k, v, g, beta, scale, state, out, B * H, dk, dv, scalar_gate ? 1 : dk,
                                        static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+int kda_chunk_fwd(const void *q, const void *k, const void *v, const float *g, const float *beta,
+                  float scale, const float *h0, void *out, float *hT, int B, int T, int H, int dk,
+                  int dv, void *stream) {
+    return chunk_fwd_impl(q, k, v, g, beta, scale, h0, out, hT, B, T, H, dk, dv, stream, false);
+}
+
+int kda_gdn_chunk_fwd(const void *q, const void *k, const void *v, const float *g, const float *beta,
+                      float scale, const float *h0, void *out, float *hT, int B, int T, int H, int dk,
+                      int dv, void *stream) {
+    return chunk_fwd_impl(q, k, v, g, beta, scale, h0, out, hT, B, T, H, dk, dv, stream, true);
+}
+
+int kda_decode_step(const void *q, const void *k, const void *v, const float *g, const float *beta,
+                    float scale, float *state, void *out, int B, int H, int dk, int dv, void *stream) {
+    return decode_impl(q, k, v, g, beta, scale, state, out, B, H, dk, dv, stream, false);
+}
+
+int kda_gdn_decode_step(const void *q, const void *k, const void *v, const float *g, const float *beta,
+                        float scale, float *state, void *out, int B, int H, int dk, int dv, void *stream) {
+    return decode_impl(q, k, v, g, beta, scale, state, out, B, H, dk, dv, stream, true);
 }
 
 }  // extern "C"
@@ -570,6 +597,7 @@ int kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const flo
         const bool last = n0 + cnt == nchunks;
         kda::PrepParams pp;
         pp.g = g;
+        pp.g_dk = dk;
         pp.beta = beta;
         pp.ws = recs;
         pp.ticket = ticket;

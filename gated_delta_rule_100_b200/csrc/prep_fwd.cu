@@ -89,7 +89,13 @@ __device__ __forceinline__ void prefetch_tensor_4d(const CUtensorMap *map, int c
                  : "memory");
 }
 
-template <int DK>
+// Prefetch the 128-byte line holding `p` into L2.
+__device__ __forceinline__ void prefetch_line_l2(const void *p) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<uint64_t>(p)) : "memory");
+}
+
+// SG: scalar gate, g [B, T, H] (else g [B, T, H, DK]).
+template <int DK, bool SG>
 __global__ void __launch_bounds__(PREP_THREADS, 2)
 prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
             const PrepParams prm) {
@@ -179,9 +185,11 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         tma_pending = true;
         float al[SUB];
         {
-            const float *gp = prm.g + (((size_t)b * T + t0 + tb) * H + h) * DK + c;
+            // one gate per key channel, or (SG) one per (token, head) shared by all channels
+            constexpr int gdk = SG ? 1 : DK;
+            const float *gp = prm.g + (((size_t)b * T + t0 + tb) * H + h) * gdk + (SG ? 0 : c);
 #pragma unroll
-            for (int u = 0; u < SUB; ++u) al[u] = (t0 + tb + u < T && active) ? __ldg(gp + (size_t)u * H * DK) : 0.f;
+            for (int u = 0; u < SUB; ++u) al[u] = (t0 + tb + u < T && active) ? __ldg(gp + (size_t)u * H * gdk) : 0.f;
         }
         if (tid < CH) s_beta[tid] = (t0 + tid < T) ? prm.beta[((size_t)b * T + t0 + tid) * H + h] : 0.f;
         if (!wait_all(bar_in, ph_in, tma_pending)) { aborted = true; break; }
@@ -363,7 +371,9 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     prefetch_tensor_4d(&tm_k, kb * 64, nh, nt0, nb);
                 }
             } else if (tid >= 64 && tid < 64 + CH && nt0 + tid - 64 < T) {
-                prefetch_l2(prm.g + (((size_t)nb * T + nt0 + tid - 64) * H + nh) * DK, DK * 4);
+                const float *gr = prm.g + (((size_t)nb * T + nt0 + tid - 64) * H + nh) * (SG ? 1 : DK);
+                if (SG) prefetch_line_l2(gr);
+                else prefetch_l2(gr, DK * 4);
             }
         }
 
@@ -560,24 +570,28 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     if (warp == 0) tmem_dealloc(tmem, L::TM_COLS);
 }
 
-template <int DK>
+template <int DK, bool SG>
 static cudaError_t launch_prep_t(const CUtensorMap &tq, const CUtensorMap &tk, const PrepParams &prm,
                                  int max_ctas, cudaStream_t stream) {
     using L = PrepLayout<DK>;
-    cudaError_t e = cudaFuncSetAttribute(prep_kernel<DK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(prep_kernel<DK, SG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          L::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     const long long items = (long long)prm.B * prm.H * prm.nseg;
     const int grid = (int)(items < max_ctas ? items : max_ctas);
-    prep_kernel<DK><<<grid, PREP_THREADS, L::SMEM_BYTES, stream>>>(tq, tk, prm);
+    prep_kernel<DK, SG><<<grid, PREP_THREADS, L::SMEM_BYTES, stream>>>(tq, tk, prm);
     return cudaGetLastError();
 }
 
-// At most max_ctas persistent CTAs (two fit on an SM), at most one per item.
+// At most max_ctas persistent CTAs (two fit on an SM), at most one per item;
+// prm.g_dk selects the gate form (dk: per key channel, 1: scalar).
 cudaError_t launch_prep(const CUtensorMap &tq, const CUtensorMap &tk, const PrepParams &prm, int dk,
                         int max_ctas, cudaStream_t stream) {
-    if (dk == 128) return launch_prep_t<128>(tq, tk, prm, max_ctas, stream);
-    return launch_prep_t<64>(tq, tk, prm, max_ctas, stream);
+    const bool sg = prm.g_dk == 1;
+    if (dk == 128) return sg ? launch_prep_t<128, true>(tq, tk, prm, max_ctas, stream)
+                             : launch_prep_t<128, false>(tq, tk, prm, max_ctas, stream);
+    return sg ? launch_prep_t<64, true>(tq, tk, prm, max_ctas, stream)
+              : launch_prep_t<64, false>(tq, tk, prm, max_ctas, stream);
 }
 
 }  // namespace kda

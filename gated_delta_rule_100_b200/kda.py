@@ -29,7 +29,8 @@ LIB_PATH = os.path.join(_HERE, "libkda.so")
 
 (KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_ALIGNMENT, KDA_ERR_CUDA, KDA_ERR_TIMEOUT,
  KDA_ERR_SCRATCH_LIMIT) = range(7)
-EXPORTED = ("kda_chunk_fwd", "kda_chunk_fwd_noalloc", "kda_decode_step", "kda_chunk_fwd_workspace_bytes", "kda_release_workspace",
+EXPORTED = ("kda_chunk_fwd", "kda_chunk_fwd_noalloc", "kda_decode_step", "kda_gdn_chunk_fwd", "kda_gdn_decode_step",
+            "kda_chunk_fwd_workspace_bytes", "kda_release_workspace",
             "kda_status_string", "kda_stream_status", "kda_chunk_fwd_debug_wait_limit",
             "kda_chunk_fwd_debug_inject_timeout", "kda_debug_kernel_timing", "kda_debug_kernel_times",
             "kda_abi_version")
@@ -59,6 +60,10 @@ def load():
     lib.kda_chunk_fwd_noalloc.restype = i
     lib.kda_decode_step.argtypes = [vp, vp, vp, fp, fp, f, fp, vp, i, i, i, i, vp]
     lib.kda_decode_step.restype = i
+    lib.kda_gdn_chunk_fwd.argtypes = [vp, vp, vp, fp, fp, f, fp, vp, fp, i, i, i, i, i, vp]
+    lib.kda_gdn_chunk_fwd.restype = i
+    lib.kda_gdn_decode_step.argtypes = [vp, vp, vp, fp, fp, f, fp, vp, i, i, i, i, vp]
+    lib.kda_gdn_decode_step.restype = i
     lib.kda_chunk_fwd_workspace_bytes.argtypes = [i, i, i, i, i]
     lib.kda_chunk_fwd_workspace_bytes.restype = ctypes.c_size_t
     lib.kda_release_workspace.argtypes = []
@@ -109,12 +114,22 @@ def chunk_fwd(q, k, v, g, beta, scale, h0=None, *, out=None, hT=None, final_stat
     """Chunkwise prefill.  q, k [B,T,H,dk] bf16; v [B,T,H,dv] bf16; g [B,T,H,dk] fp32;
     beta [B,T,H] fp32; h0 [B,H,dk,dv] fp32 or None.  Returns (out, hT); hT is None
     when ``final_state`` is False and no ``hT`` buffer was given."""
+    return _prefill("kda_chunk_fwd", False, q, k, v, g, beta, scale, h0, out, hT, final_state, stream)
+
+
+def gdn_chunk_fwd(q, k, v, g, beta, scale, h0=None, *, out=None, hT=None, final_state=True, stream=None):
+    """Scalar-gate (Gated DeltaNet) prefill: as ``chunk_fwd`` with g [B,T,H] fp32, one
+    log-decay per token and head shared by every key channel."""
+    return _prefill("kda_gdn_chunk_fwd", True, q, k, v, g, beta, scale, h0, out, hT, final_state, stream)
+
+
+def _prefill(symbol, scalar_gate, q, k, v, g, beta, scale, h0, out, hT, final_state, stream):
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     _check(q, "q", torch.bfloat16, (B, T, H, dk))
     _check(k, "k", torch.bfloat16, (B, T, H, dk))
     _check(v, "v", torch.bfloat16, (B, T, H, dv))
-    _check(g, "g", torch.float32, (B, T, H, dk))
+    _check(g, "g", torch.float32, (B, T, H) if scalar_gate else (B, T, H, dk))
     _check(beta, "beta", torch.float32, (B, T, H))
     if h0 is not None:
         _check(h0, "h0", torch.float32, (B, H, dk, dv))
@@ -125,10 +140,10 @@ def chunk_fwd(q, k, v, g, beta, scale, h0=None, *, out=None, hT=None, final_stat
         hT = torch.empty((B, H, dk, dv), device=q.device, dtype=torch.float32)
     if hT is not None:
         _check(hT, "hT", torch.float32, (B, H, dk, dv))
-    rc = load().kda_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale),
-                              _ptr(h0), _ptr(out), _ptr(hT), B, T, H, dk, dv, _stream(stream))
+    rc = getattr(load(), symbol)(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale),
+                                 _ptr(h0), _ptr(out), _ptr(hT), B, T, H, dk, dv, _stream(stream))
     if rc != KDA_OK:
-        raise KdaError(rc, "kda_chunk_fwd")
+        raise KdaError(rc, symbol)
     return out, hT
 
 
@@ -158,21 +173,30 @@ def chunk_fwd_noalloc(q, k, v, g, beta, scale, h0=None, *, out, hT=None, stream=
 def decode_step(q, k, v, g, beta, scale, state, *, out=None, stream=None):
     """One recurrent step.  q, k [B,H,dk] bf16; v [B,H,dv] bf16; g [B,H,dk] fp32;
     beta [B,H] fp32; state [B,H,dk,dv] fp32 (updated in place).  Returns out [B,H,dv] bf16."""
+    return _decode("kda_decode_step", False, q, k, v, g, beta, scale, state, out, stream)
+
+
+def gdn_decode_step(q, k, v, g, beta, scale, state, *, out=None, stream=None):
+    """Scalar-gate (Gated DeltaNet) decode step: as ``decode_step`` with g [B,H] fp32."""
+    return _decode("kda_gdn_decode_step", True, q, k, v, g, beta, scale, state, out, stream)
+
+
+def _decode(symbol, scalar_gate, q, k, v, g, beta, scale, state, out, stream):
     B, H, dk = q.shape
     dv = v.shape[-1]
     _check(q, "q", torch.bfloat16, (B, H, dk))
     _check(k, "k", torch.bfloat16, (B, H, dk))
     _check(v, "v", torch.bfloat16, (B, H, dv))
-    _check(g, "g", torch.float32, (B, H, dk))
+    _check(g, "g", torch.float32, (B, H) if scalar_gate else (B, H, dk))
     _check(beta, "beta", torch.float32, (B, H))
     _check(state, "state", torch.float32, (B, H, dk, dv))
     if out is None:
         out = torch.empty((B, H, dv), device=q.device, dtype=torch.bfloat16)
     _check(out, "out", torch.bfloat16, (B, H, dv))
-    rc = load().kda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale),
-                                _ptr(state), _ptr(out), B, H, dk, dv, _stream(stream))
+    rc = getattr(load(), symbol)(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale),
+                                 _ptr(state), _ptr(out), B, H, dk, dv, _stream(stream))
     if rc != KDA_OK:
-        raise KdaError(rc, "kda_decode_step")
+        raise KdaError(rc, symbol)
     return out
 
 

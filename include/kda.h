@@ -122,6 +122,28 @@ KDA_API int kda_decode_step(const void *q, const void *k, const void *v,
                     int B, int H, int dk, int dv, void *stream);
 
 /*
+ * kda_gdn_chunk_fwd, kda_gdn_decode_step -- the scalar-gate form (Gated
+ * DeltaNet): one log-decay per token and head, shared by every key channel,
+ * i.e. alpha_t = exp(g_t) * 1 in the recurrence above.
+ *
+ *   g : fp32 [B, T, H] (prefill) or [B, H] (decode), 4-byte aligned
+ *
+ * Every other argument, layout, result and error code is that of kda_chunk_fwd
+ * and kda_decode_step respectively (the prefill shares their workspace); the
+ * results are those of the per-channel entry points given g broadcast over dk.
+ * The state-independent prep reads 4 bytes of gate per token and head instead
+ * of 4 dk.
+ */
+KDA_API int kda_gdn_chunk_fwd(const void *q, const void *k, const void *v,
+                  const float *g, const float *beta, float scale,
+                  const float *h0, void *out, float *hT,
+                  int B, int T, int H, int dk, int dv, void *stream);
+KDA_API int kda_gdn_decode_step(const void *q, const void *k, const void *v,
+                    const float *g, const float *beta, float scale,
+                    float *state, void *out,
+                    int B, int H, int dk, int dv, void *stream);
+
+/*
  * kda_chunk_fwd_noalloc -- kda_chunk_fwd without any device allocation.  The
  * method itself has no counterpart: this is a deployment variant for callers
  * that cannot allocate device memory at call time (a process whose device
@@ -211,7 +233,7 @@ KDA_API void kda_chunk_fwd_debug_inject_timeout(unsigned long long polls);
 KDA_API void kda_debug_kernel_timing(int enable);
 KDA_API int kda_debug_kernel_times(double *ms, long long *launches, int nkinds);
 
-/* Version of this ABI (major * 100 + minor). */
+/* Version of this ABI (major * 100 + minor): 101 adds the scalar-gate entry points. */
 KDA_API int kda_abi_version(void);
 
 #ifdef __cplusplus
