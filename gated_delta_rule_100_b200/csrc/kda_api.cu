@@ -217,8 +217,8 @@ int num_sms(int dev) {
 }
 
 // Tensor maps over the record parts of `nrec` consecutive records at `rec`
-// (plain row-major arrays, see chunk_common.cuh), with the boxes and the
-// 128-byte swizzle of the chain kernel's operand tiles.
+// (layouts in chunk_common.cuh), with the boxes and swizzles of the chain
+// kernel's operand tiles.
 int make_rec_maps(PFN_cuTensorMapEncodeTiled_v12000 enc, const uint8_t *rec, long long nrec, int dk,
                   CUtensorMap *maps) {
     // WQ, P, K-hat: [blocks][rows][16] 16-bit arrays, one box = one record's part

@@ -55,8 +55,8 @@ def test_head_dims(dk, dv):
 
 
 def test_value_slices_are_independent():
-    """Each CTA carries 32 value columns; the columns of the state evolve
-    independently, so the first 64 columns of a dv = 128 run must equal, bit
+    """The columns of the state evolve independently (each chain CTA carries a
+    slice of them), so the first 64 columns of a dv = 128 run must equal, bit
     for bit, a dv = 64 run on those columns alone."""
     d = inputs.make_prefill(2, 200, 2, 128, 128, decay=0.05, h0_std=0.02, seed=8, device=DEV)
     out, hT = check(d, 0.1, "dv=128")
