@@ -66,6 +66,46 @@ def prefill_bytes(B, T, H, dk, dv, with_h0, with_hT):
     return B * T * H * per_token_head + (state if with_h0 else 0) + (state if with_hT else 0)
 
 
+def measure_scalar_gate(d, cfg, out, hT, stream, steps, warmup, P):
+    """The scalar-gate (Gated DeltaNet) prefill on the bench workload: the same
+    inputs with one log-decay per token and head (key channel 0 of the workload's
+    gate), timed like the step.  Device-side inputs; one process's own timing."""
+    import torch
+
+    from gated_delta_rule_100_b200 import kda
+
+    gs = d["g"][..., 0].contiguous()
+
+    def step():
+        kda.gdn_chunk_fwd(d["q"], d["k"], d["v"], gs, d["beta"], cfg.scale, d["h0"], out=out, hT=hT,
+                          stream=stream)
+
+    for _ in range(max(1, warmup)):
+        step()
+    torch.cuda.synchronize()
+    if kda.stream_status(stream) != kda.KDA_OK:
+        raise RuntimeError("device-side error during warm-up")
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if kda.stream_status(stream) != kda.KDA_OK:
+        raise RuntimeError("device-side error in the timed steps")
+    ms = e0.elapsed_time(e1) / steps
+    # the gate is 4 bytes per token-head instead of 4 dk
+    nbytes = (prefill_bytes(cfg.B, cfg.T, cfg.H, cfg.dk, cfg.dv, cfg.h0_std > 0, True)
+              - cfg.B * cfg.T * cfg.H * 4 * (cfg.dk - 1))
+    achieved = nbytes / (ms / 1e3) / 1e9
+    del gs
+    return {"metric": "scalar-gate prefill tokens/s", "value": cfg.B * cfg.T / (ms / 1e3), "unit": "tokens/s",
+            "ms_per_step": ms, "steps": steps, "entry_point": "kda_gdn_chunk_fwd",
+            "config": {"workload": cfg.name, "gate": "fp32 [B,T,H]: key channel 0 of the workload's gate"},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": P["hbm_gbs"], "unit": "GB/s",
+                         "frac": achieved / P["hbm_gbs"], "algorithmic_bytes_per_launch": nbytes}}
+
+
 def prefill_flops(B, T, H, dk, dv, C=CHUNK):
     """Algorithmic flops of the chunkwise form (triangles counted once): the three
     state contractions, A, the triangular solve, the causal q k^T and P Vnew."""
@@ -342,6 +382,14 @@ def run_ours(args):
                             "peak_tflops": P["bf16_tflops_sustained"],
                             "frac": nflops / avg_launch_s / 1e12 / P["bf16_tflops_sustained"]}}
 
+    # ---------------- scalar-gate form (after the timed steps; never fails the line) ----------------
+    gdn = None
+    if not args.no_gdn:
+        try:
+            gdn = measure_scalar_gate(d, cfg, out, hT, stream, args.steps, args.warmup, P)
+        except Exception as exc:  # noqa: BLE001 - an extra item must not cost the measurement above
+            gdn = {"error": f"{type(exc).__name__}: {exc}"[:300]}
+
     # ---------------- decode ----------------
     dec = None
     if not args.no_decode:
@@ -420,7 +468,7 @@ def run_ours(args):
                        "l2": "inputs larger than L2 (51.7 GB per step); no flush",
                        "parallelism": f"weak: one workload copy per GPU x{world}"},
             "tflops": nflops / (ms_per_step / 1e3) / 1e12 * world,
-            "roofline": roof, "decode": dec, "e2e": e2e, "cpu_baseline": cpu,
+            "roofline": roof, "decode": dec, "scalar_gate": gdn, "e2e": e2e, "cpu_baseline": cpu,
             "clocks": clk.summary(), "gpu_launches": gpu_launches,
             "launch_ms": {"mean": statistics.mean(launch_ms), "min": min(launch_ms), "max": max(launch_ms)},
         }
@@ -439,6 +487,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=WORKLOAD)
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-gdn", action="store_true", help="skip the scalar-gate prefill line")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
