@@ -16,7 +16,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 LIB_PATH = os.path.join(HERE, "libkda.so")
-SOURCES = ["kda_api.cu", "decode.cu", "prep_fwd.cu", "chain_fwd.cu"]
+SOURCES = ["kda_api.cu", "decode.cu", "prep_fwd.cu", "exact_prep.cu", "chain_fwd.cu", "varlen_setup.cu", "parts_fixup.cu"]
 HEADERS = ["kda_device.cuh", "chunk_common.cuh", "chunk_params.cuh"]
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
               "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden"]

@@ -118,14 +118,42 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
     const int warp = tid >> 5, lane = tid & 31;
     const bool issuer = warp == CHAIN_WORKERS / 32;
     const bool loader = warp == CHAIN_WORKERS / 32 + 1;
-    const int slice = blockIdx.x % prm.nslices;
-    const int bh = blockIdx.x / prm.nslices;
-    const int h = bh % prm.H, b = bh / prm.H;
-    const int T = prm.T, H = prm.H, DV = prm.DV;
-    const int col0 = slice * VS;
-    const int nseg = prm.nseg;
-    const uint8_t *recs = prm.ws + (size_t)bh * nseg * REC_BYTES;
-    const int rec0 = bh * nseg;  // index of this (b, h)'s first record in the tensor maps
+    const int slot = blockIdx.x % prm.slots;
+    const int rest = blockIdx.x / prm.slots;
+    const int part = prm.part0 + rest % prm.nparts;
+    const int bh = rest / prm.nparts;
+    const int h = bh % prm.H, seq = bh / prm.H;
+    const int H = prm.H, DV = prm.DV;
+    const int nvs = DV / VS;                       // value slices
+    const bool trans = prm.pass_a && part > 0;     // a transition of the two-level pass
+    const bool ident = trans && slot >= nvs;       // columns of the identity instead of values
+    if (!trans && slot >= nvs) return;             // pass A's part 0 needs value slices only
+    const int col0 = (ident ? slot - nvs : slot) * VS;
+    const ChainGeo geo = chain_geo(prm.gm, H, seq, h, part, prm.parts, prm.part_len);
+    const int nseg = geo.nch;  // chunks of this (sequence, head, part) in this launch
+    const uint8_t *recs = prm.ws + (size_t)geo.rec0 * REC_BYTES;
+    const int rec0 = (int)geo.rec0;  // index of its first record in the tensor maps
+    // Where the state comes from and goes to (row stride ld, this slice's column 0 at col0):
+    // the sequence's h0/hT (or the carry between segments), or the two-level pass's buffers.
+    const size_t BHn = (size_t)prm.gm.nseqs * H;
+    const float *s_in = nullptr;  // NULL: zero (or, ident, the identity)
+    float *s_out = nullptr;       // NULL: not written
+    int s_ld = DV;
+    if (trans) {
+        if (ident) {
+            s_out = prm.p_trans + ((size_t)part * BHn + bh) * DK * DK;
+            s_ld = DK;
+        } else {
+            s_out = prm.p_local + ((size_t)part * BHn + bh) * DK * DV;
+        }
+    } else {
+        const float *h0p = geo.first ? prm.h0 : prm.carry;
+        float *hTp = geo.last ? prm.hT : prm.carry;
+        s_in = part == 0 ? (h0p ? h0p + ((size_t)seq * H + h) * DK * DV : nullptr)
+                         : prm.p_start + ((size_t)part * BHn + bh) * DK * DV;
+        if (part == prm.parts - 1) s_out = hTp ? hTp + ((size_t)seq * H + h) * DK * DV : nullptr;
+        else if (prm.pass_a) s_out = prm.p_start + ((size_t)(part + 1) * BHn + bh) * DK * DV;
+    }
     const uint64_t polls = prm.st.wait_polls;
 
     if (tid == 0) {
@@ -313,11 +341,11 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
         const uint32_t lane_base = (uint32_t)(lq * 32) << 16;
         const int scol = col0 + cg * CPT;
 
-        float S[CPT];  // S[ch][scol .. scol + 15]
+        float S[CPT];  // S[ch][scol .. scol + CPT - 1]
 #pragma unroll
-        for (int e = 0; e < CPT; ++e) S[e] = 0.f;
-        if (ch < DK && prm.h0 != nullptr) {
-            const float4 *src = reinterpret_cast<const float4 *>(prm.h0 + (((size_t)b * H + h) * DK + ch) * DV + scol);
+        for (int e = 0; e < CPT; ++e) S[e] = (ident && ch == scol + e) ? 1.f : 0.f;
+        if (ch < DK && s_in != nullptr) {
+            const float4 *src = reinterpret_cast<const float4 *>(s_in + (size_t)ch * s_ld + scol);
 #pragma unroll
             for (int e = 0; e < CPT / 4; ++e) {
                 const float4 x = src[e];
@@ -340,10 +368,10 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
         const int vp = tid % NP, vtg = tid / NP;
         uint32_t vr[TPT];
         auto load_v = [&](int n) {
-            const int t0 = (prm.n_begin + n) * CH + vtg * TPT;
-            const uint32_t *src = reinterpret_cast<const uint32_t *>(prm.v + (((size_t)b * T + t0) * H + h) * DV + col0) + vp;
+            const int t0 = (geo.lc0 + n) * CH + vtg * TPT;
+            const uint32_t *src = reinterpret_cast<const uint32_t *>(prm.v + ((size_t)(geo.row0 + t0) * H + h) * DV + col0) + vp;
 #pragma unroll
-            for (int u = 0; u < TPT; ++u) vr[u] = (t0 + u < T) ? __ldg(src + (size_t)u * H * DV / 2) : 0u;
+            for (int u = 0; u < TPT; ++u) vr[u] = (!ident && t0 + u < geo.len) ? __ldg(src + (size_t)u * H * DV / 2) : 0u;
         };
         auto build_vt = [&]() {  // V^T tile: row = value column, K = token
             // a bf16 value is the top half of its fp32 (and tf32) bit pattern
@@ -361,14 +389,14 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
         // warp-collective, only the stores are guarded)
         auto write_output = [&](int n) {
             const int i = ch - 64;
-            const int t = (prm.n_begin + n) * CH + i;
-            uint16_t *dst = prm.out + (((size_t)b * T + (t < T ? t : 0)) * H + h) * DV + scol;
+            const int t = (geo.lc0 + n) * CH + i;
+            uint16_t *dst = prm.out + ((size_t)(geo.row0 + (t < geo.len ? t : 0)) * H + h) * DV + scol;
 #pragma unroll
             for (int c16 = 0; c16 < CPT; c16 += 16) {
                 float o[16];
                 tmem_ld16(tmem + lane_base + L::TM_D1 + (n & 1) * VS + cg * CPT + c16, o);
                 tmem_wait_ld();
-                if (t < T) {
+                if (t < geo.len && !trans) {
                     float a8[8], b8[8];
 #pragma unroll
                     for (int e = 0; e < 8; ++e) { a8[e] = prm.scale * o[e]; b8[e] = prm.scale * o[8 + e]; }
@@ -446,8 +474,10 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
                 write_output(nseg - 1);
             }
         }
-        if (ok && *s_abort == 0 && prm.hT != nullptr && ch < DK) {
-            float4 *dst = reinterpret_cast<float4 *>(prm.hT + (((size_t)b * H + h) * DK + ch) * DV + scol);
+        // an empty sequence passes its state through (h0, or zero) once
+        const bool write_state = nseg > 0 ? ok : (geo.first && geo.last);
+        if (write_state && *s_abort == 0 && s_out != nullptr && ch < DK) {
+            float4 *dst = reinterpret_cast<float4 *>(s_out + (size_t)ch * s_ld + scol);
 #pragma unroll
             for (int e = 0; e < CPT / 4; ++e) dst[e] = make_float4(S[4 * e], S[4 * e + 1], S[4 * e + 2], S[4 * e + 3]);
         }
@@ -465,7 +495,7 @@ static cudaError_t launch_chain_t(const CUtensorMap *maps, const ChainParams &pr
     cudaError_t e = cudaFuncSetAttribute(chain_kernel<DK, VS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          L::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    chain_kernel<DK, VS><<<prm.B * prm.H * prm.nslices, CHAIN_THREADS, L::SMEM_BYTES, stream>>>(
+    chain_kernel<DK, VS><<<prm.gm.nseqs * prm.H * prm.nparts * prm.slots, CHAIN_THREADS, L::SMEM_BYTES, stream>>>(
         maps[0], maps[1], maps[2], maps[3], prm);
     return cudaGetLastError();
 }

@@ -15,7 +15,9 @@
 // store covers one contiguous 512-byte state row.  The two column reductions
 // (k.s' and q.s') go through shared memory across row groups.  The gate is
 // either one log-decay per key channel (g [B, H, dk]) or one per head shared by
-// all channels (g [B, H], the scalar-gate form): g_dk = dk or 1.
+// all channels (g [B, H], the scalar-gate form): g_dk = dk or 1.  With the
+// gate prologue the inputs are raw projections (see gate_logdecay): the kernel
+// forms g and beta and L2-normalises q and k itself.
 #include <cuda_bf16.h>
 #include <stdint.h>
 
@@ -30,7 +32,7 @@ __global__ void __launch_bounds__(DEC_THREADS)
 decode_step_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ k,
                    const uint16_t *__restrict__ v, const float *__restrict__ g,
                    const float *__restrict__ beta, float scale, float *__restrict__ state,
-                   uint16_t *__restrict__ out, int g_dk) {
+                   uint16_t *__restrict__ out, int g_dk, int prologue, float gate_c) {
     constexpr int NCG = DV / 4;              // float4 column groups
     constexpr int NRG = DEC_THREADS / NCG;   // row groups
     constexpr int RPT = DK / NRG;            // state rows per thread
@@ -60,9 +62,23 @@ decode_step_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ 
     for (int r = tid; r < DK; r += DEC_THREADS) {
         s_k[r] = bf16_bits_to_f32(kh[r]);
         s_q[r] = bf16_bits_to_f32(qh[r]);
-        s_a[r] = __expf(gh[g_dk > 1 ? r : 0]);
+        const float gr = gh[g_dk > 1 ? r : 0];
+        s_a[r] = __expf(prologue ? gate_logdecay(gr, gate_c) : gr);
     }
     __syncthreads();
+    if (prologue) {  // raw q, k: L2-normalise each (warp 0: q, warp 1: k), as the prefill's prologue
+        if (tid < 64) {
+            float *x = tid < 32 ? s_q : s_k;
+            const int ln = tid & 31;
+            float ss = 0.f;
+            for (int r = ln; r < DK; r += 32) ss += x[r] * x[r];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+            const float rn = rsqrtf(fmaxf(ss, 1e-24f));
+            for (int r = ln; r < DK; r += 32) x[r] = bf16_bits_to_f32(to_bf16_bits(x[r] * rn));
+        }
+        __syncthreads();
+    }
     if (tid < 32) {
         float acc = 0.f;
         for (int r = tid; r < DK; r += 32) acc += s_q[r] * s_k[r];
@@ -93,7 +109,7 @@ decode_step_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ 
         p.x += a.x; p.y += a.y; p.z += a.z; p.w += a.w;
         y.x += b.x; y.y += b.y; y.z += b.z; y.w += b.w;
     }
-    const float bt = beta[bh];
+    const float bt = prologue ? gate_sigmoid(beta[bh]) : beta[bh];
     const uint16_t *vh = v + (size_t)bh * DV + cg * 4;
     float4 u;
     u.x = bt * (bf16_bits_to_f32(vh[0]) - p.x);
@@ -122,23 +138,25 @@ decode_step_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ 
 template <int DK, int DV>
 static cudaError_t launch_decode_t(const void *q, const void *k, const void *v, const float *g,
                                    const float *beta, float scale, float *state, void *out,
-                                   int BH, int g_dk, cudaStream_t stream) {
+                                   int BH, int g_dk, int prologue, float gate_c, cudaStream_t stream) {
     decode_step_kernel<DK, DV><<<BH, DEC_THREADS, 0, stream>>>(
         (const uint16_t *)q, (const uint16_t *)k, (const uint16_t *)v, g, beta, scale, state,
-        (uint16_t *)out, g_dk);
+        (uint16_t *)out, g_dk, prologue, gate_c);
     return cudaGetLastError();
 }
 
+// prologue != 0: g, beta, q and k are raw (g = -gate_c softplus(g), beta = sigmoid(beta),
+// q and k L2-normalised).
 cudaError_t launch_decode(const void *q, const void *k, const void *v, const float *g,
                           const float *beta, float scale, float *state, void *out, int BH, int dk,
-                          int dv, int g_dk, cudaStream_t stream) {
+                          int dv, int g_dk, int prologue, float gate_c, cudaStream_t stream) {
     if (dk == 128 && dv == 128)
-        return launch_decode_t<128, 128>(q, k, v, g, beta, scale, state, out, BH, g_dk, stream);
+        return launch_decode_t<128, 128>(q, k, v, g, beta, scale, state, out, BH, g_dk, prologue, gate_c, stream);
     if (dk == 128 && dv == 64)
-        return launch_decode_t<128, 64>(q, k, v, g, beta, scale, state, out, BH, g_dk, stream);
+        return launch_decode_t<128, 64>(q, k, v, g, beta, scale, state, out, BH, g_dk, prologue, gate_c, stream);
     if (dk == 64 && dv == 128)
-        return launch_decode_t<64, 128>(q, k, v, g, beta, scale, state, out, BH, g_dk, stream);
-    return launch_decode_t<64, 64>(q, k, v, g, beta, scale, state, out, BH, g_dk, stream);
+        return launch_decode_t<64, 128>(q, k, v, g, beta, scale, state, out, BH, g_dk, prologue, gate_c, stream);
+    return launch_decode_t<64, 64>(q, k, v, g, beta, scale, state, out, BH, g_dk, prologue, gate_c, stream);
 }
 
 }  // namespace kda

@@ -17,7 +17,7 @@
 namespace kda {
 cudaError_t launch_decode(const void *q, const void *k, const void *v, const float *g,
                           const float *beta, float scale, float *state, void *out, int BH, int dk,
-                          int dv, int g_dk, cudaStream_t stream);
+                          int dv, int g_dk, int prologue, float gate_c, cudaStream_t stream);
 }
 
 #include "chunk_common.cuh"
@@ -25,8 +25,13 @@ cudaError_t launch_decode(const void *q, const void *k, const void *v, const flo
 
 namespace kda {
 cudaError_t launch_prep(const CUtensorMap &tq, const CUtensorMap &tk, const PrepParams &prm, int dk,
-                        int max_ctas, cudaStream_t stream);
+                        int max_ctas, cudaStream_t stream, bool prologue);
 cudaError_t launch_chain(const CUtensorMap *maps, const ChainParams &prm, int dk, cudaStream_t stream);
+cudaError_t launch_exact(const ExactParams &prm, int dk, int ctas, cudaStream_t stream);
+cudaError_t launch_parts_fixup(float *start, const float *local, const float *trans, int BH, int dk, int dv,
+                               int parts, cudaStream_t stream);
+cudaError_t launch_varlen_setup(const int *cu, int N, int T_total, int cmax, int *cu_s, int *cc, int *chunk_seq,
+                                const DeviceStatus &st, cudaStream_t stream);
 }
 
 // Device-side status word: kernels OR error bits into it (one per device,
@@ -40,6 +45,8 @@ std::mutex g_mu;
 uint32_t *g_status_ptr[kMaxDevices] = {};
 std::atomic<unsigned long long> g_wait_polls{0};
 std::atomic<unsigned long long> g_inject_polls{0};
+std::atomic<int> g_force_exact{0};
+std::atomic<int> g_parts_override{1};  // test hook: parts of the two-level pass (0 = automatic, 1 = off)
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
 int current_status_word(uint32_t **out) {
@@ -83,13 +90,20 @@ int get_encoder(PFN_cuTensorMapEncodeTiled_v12000 *fn) {
 // of segment i: prep on a low-priority internal stream, chain on a
 // high-priority one (its few CTAs are placed first, prep fills the other SMs).
 constexpr size_t kWorkspaceCap = size_t(2) << 30;  // bytes of records
+std::atomic<unsigned long long> g_record_cap{0};   // test hook: a smaller cap (0 = kWorkspaceCap)
+size_t record_cap() {
+    const unsigned long long c = g_record_cap.load();
+    return c ? (size_t)c : kWorkspaceCap;
+}
 constexpr double kPrepCtasPerFreeSm = 2.0;         // prep density beside a chain kernel
-constexpr size_t kTicketBytes = 256;               // two item counters at the front of the records
+constexpr size_t kTicketBytes = 256;               // per record buffer: item counter, steep-item count
 struct Workspace {
-    uint8_t *base = nullptr;  // [tickets][records]
+    uint8_t *base = nullptr;  // [counters][steep-item list][records]
     size_t base_bytes = 0;
     float *state = nullptr;
     size_t state_bytes = 0;
+    float *parts = nullptr;  // the two-level pass: start, local and transition states of every part
+    size_t parts_bytes = 0;
     cudaEvent_t done = nullptr;
     cudaStream_t lo = nullptr, hi = nullptr;  // prep and chain streams of the segmented path
     cudaEvent_t fork = nullptr, prep_done[2] = {nullptr, nullptr}, chain_done[2] = {nullptr, nullptr};
@@ -97,6 +111,10 @@ struct Workspace {
 Workspace g_ws[kMaxDevices];
 
 size_t rec_row_bytes(int B, int H) { return (size_t)B * H * kda::REC_BYTES; }
+size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
+// The list of steep items of one segment (prep appends, the exact kernel reads):
+// room for every item of the segment.
+size_t steep_list_bytes(int B, int H, int seg) { return round256((size_t)B * H * seg * sizeof(int)); }
 
 struct SegPlan {
     int nchunks, seg, nbuf;  // chunks, chunks per segment, record buffers
@@ -105,20 +123,49 @@ SegPlan plan_segments(int B, int T, int H) {
     SegPlan p;
     p.nchunks = (T + kda::CH - 1) / kda::CH;
     const size_t row = rec_row_bytes(B, H);
-    if ((size_t)p.nchunks * row <= kWorkspaceCap) {
+    const size_t cap = record_cap();
+    if ((size_t)p.nchunks * row <= cap) {
         p.seg = p.nchunks;
         p.nbuf = 1;
     } else {
-        const size_t fit = kWorkspaceCap / (2 * row);
+        const size_t fit = cap / (2 * row);
         p.seg = (int)(fit < 1 ? 1 : fit);
         p.nbuf = 2;
     }
     return p;
 }
 
+// Packed batches: global chunks bounded by cmax = T_total / 64 + N + 1 (each
+// sequence adds at most one partial chunk), run in windows of W chunks.
+struct VarlenPlan {
+    int cmax, W, nwin;
+};
+VarlenPlan plan_varlen(int N, int T_total, int H) {
+    VarlenPlan p;
+    p.cmax = T_total / kda::CH + N + 1;
+    const size_t fit = record_cap() / rec_row_bytes(1, H);
+    p.W = (int)((size_t)p.cmax < fit ? (size_t)p.cmax : (fit < 1 ? 1 : fit));
+    p.nwin = (p.cmax + p.W - 1) / p.W;
+    return p;
+}
+// cu_s and cc ([N + 1] each) and chunk_seq ([cmax]), 256-byte rounded.
+size_t varlen_meta_bytes(int N, int cmax) { return round256((size_t)(2 * (N + 1) + cmax) * sizeof(int)); }
+size_t varlen_base_bytes(int N, int H, const VarlenPlan &pl) {
+    return kTicketBytes + steep_list_bytes(1, H, pl.W) + varlen_meta_bytes(N, pl.cmax) +
+           (size_t)pl.W * rec_row_bytes(1, H);
+}
+
 // Called with g_mu held.
-int reserve_workspace(int dev, size_t base_bytes, size_t state_bytes, bool streams, Workspace **out) {
+int reserve_workspace(int dev, size_t base_bytes, size_t state_bytes, bool streams, Workspace **out,
+                      size_t parts_bytes = 0) {
     Workspace &w = g_ws[dev];
+    if (w.parts_bytes < parts_bytes) {
+        if (w.parts != nullptr && cudaFree(w.parts) != cudaSuccess) return KDA_ERR_CUDA;
+        w.parts = nullptr;
+        w.parts_bytes = 0;
+        if (cudaMalloc(&w.parts, parts_bytes) != cudaSuccess) return KDA_ERR_CUDA;
+        w.parts_bytes = parts_bytes;
+    }
     if (w.base_bytes < base_bytes) {
         if (w.base != nullptr && cudaFree(w.base) != cudaSuccess) return KDA_ERR_CUDA;
         w.base = nullptr;
@@ -255,11 +302,80 @@ int make_rec_maps(PFN_cuTensorMapEncodeTiled_v12000 enc, const uint8_t *rec, lon
 // matters), the wide one otherwise (many (b, h): record traffic matters).
 int chain_slices(int B, int H, int dv, int sms) { return (dv == 128 && 2LL * B * H <= sms) ? 2 : 1; }
 
+// Parts of the two-level pass for a segment of `cnt` chunks.  The plain pass
+// keeps each (b, h)'s chain on one CTA per value slice walking every chunk in
+// order; with few (b, h) most SMs idle meanwhile.  The two-level pass runs
+// pass A on (parts - 1) x (dv + dk) / 64 CTAs per (b, h) and pass B on
+// (parts - 1) x dv / 64, so the sequential walk shrinks to two parts' worth of
+// chunks plus the short fix-up.  Parts are chosen so that pass A fits in one
+// wave and each part holds at least 4 chunks; fewer than 3 parts gain nothing
+// (the walk would not shorten), so then the plain pass runs (1 is returned).
+int plan_parts(int B, int H, int dk, int dv, int cnt, int sms) {
+    const int ov = g_parts_override.load();
+    int P;
+    if (ov >= 1) {
+        P = ov;
+    } else {
+        const long long per_part = (long long)B * H * ((dv + dk) / 64);
+        P = (int)(1 + sms / per_part);
+        if (P > cnt / 4) P = cnt / 4;
+    }
+    if (P > cnt) P = cnt;
+    if (P < 3) return 1;
+    const int len = (cnt + P - 1) / P;
+    return (cnt + len - 1) / len;  // parts actually used at that length
+}
+size_t parts_bytes(int B, int H, int dk, int dv, int P) {
+    return P < 3 ? 0 : (size_t)P * B * H * dk * (2 * dv + dk) * sizeof(float);
+}
+
+// Chain launch fields of the plain pass.
+void plain_pass(kda::ChainParams &cp, int nslices) {
+    cp.nslices = nslices;
+    cp.parts = 1;
+    cp.part_len = 0;
+    cp.part0 = 0;
+    cp.nparts = 1;
+    cp.slots = nslices;
+    cp.pass_a = 0;
+    cp.p_start = cp.p_local = cp.p_trans = nullptr;
+}
+
+// Geometry of a uniform launch: B sequences of T tokens, local chunks [n0, n0 + cnt).
+kda::SeqGeom uniform_geom(int B, int T, int n0, int cnt) {
+    kda::SeqGeom gm = {};
+    gm.cu = nullptr;
+    gm.nseqs = B;
+    gm.T = T;
+    gm.n_begin = n0;
+    gm.nseg = cnt;
+    return gm;
+}
+
+// Parameters of the exact kernel for the items of one prep launch.
+kda::ExactParams exact_params(const void *q, const void *k, const float *g, int g_dk, const float *beta,
+                              const kda::PrepParams &pp, bool prologue = false) {
+    kda::ExactParams xp;
+    xp.q = static_cast<const uint16_t *>(q);
+    xp.k = static_cast<const uint16_t *>(k);
+    xp.g = g;
+    xp.g_dk = g_dk;
+    xp.beta = beta;
+    xp.ws = pp.ws;
+    xp.steep_count = pp.steep_count;
+    xp.steep_items = pp.steep_items;
+    xp.prologue = prologue ? 1 : 0;
+    xp.gate_c = pp.gate_c;
+    xp.H = pp.H;
+    xp.gm = pp.gm;
+    return xp;
+}
+
 }  // namespace
 
 extern "C" {
 
-int kda_abi_version(void) { return 101; }
+int kda_abi_version(void) { return 102; }
 
 const char *kda_status_string(int status) {
     switch (status) {
@@ -278,6 +394,12 @@ void kda_chunk_fwd_debug_wait_limit(unsigned long long polls) { g_wait_polls.sto
 
 void kda_chunk_fwd_debug_inject_timeout(unsigned long long polls) { g_inject_polls.store(polls); }
 
+void kda_chunk_fwd_debug_force_exact(int enable) { g_force_exact.store(enable != 0); }
+
+void kda_chunk_fwd_debug_record_cap(unsigned long long bytes) { g_record_cap.store(bytes); }
+
+void kda_chunk_fwd_debug_parts(int parts) { g_parts_override.store(parts < 0 ? 0 : parts); }
+
 int kda_stream_status(void *stream) {
     if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return KDA_ERR_CUDA;
     uint32_t *word = nullptr;
@@ -288,13 +410,15 @@ int kda_stream_status(void *stream) {
         const uint32_t zero = 0;
         if (cudaMemcpy(word, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return KDA_ERR_CUDA;
     }
-    return (v & kda::DEV_TIMEOUT) ? KDA_ERR_TIMEOUT : KDA_OK;
+    if (v & kda::DEV_TIMEOUT) return KDA_ERR_TIMEOUT;
+    return (v & kda::DEV_BAD_ARG) ? KDA_ERR_INVALID_ARG : KDA_OK;
 }
 
 // The prefill for either gate form: g_dk = dk (g [B, T, H, dk]) or 1 (g [B, T, H]).
+// prologue: g, beta, q, k are raw projections (per-channel gate only), g = -gate_c softplus(g).
 static int chunk_fwd_impl(const void *q, const void *k, const void *v, const float *g, const float *beta,
                           float scale, const float *h0, void *out, float *hT, int B, int T, int H, int dk,
-                          int dv, void *stream, bool scalar_gate) {
+                          int dv, void *stream, bool scalar_gate, bool prologue = false, float gate_c = 0.f) {
     if (B < 1 || H < 1 || T < 0) return KDA_ERR_INVALID_ARG;
     if (T > 0 && (!q || !k || !v || !g || !beta || !out)) return KDA_ERR_INVALID_ARG;
     if ((dk != 64 && dk != 128) || (dv != 64 && dv != 128)) return KDA_ERR_UNSUPPORTED;
@@ -333,10 +457,14 @@ static int chunk_fwd_impl(const void *q, const void *k, const void *v, const flo
     const size_t row = rec_row_bytes(B, H);
     const size_t state_bytes = (multi && hT == nullptr) ? (size_t)B * H * dk * dv * sizeof(float) : 0;
     const int sms = num_sms(dev);
+    const int pmax = plan_parts(B, H, dk, dv, seg, sms);  // parts of a full segment (the most)
 
     std::lock_guard<std::mutex> lk(g_mu);
     Workspace *w = nullptr;
-    if (int st = reserve_workspace(dev, kTicketBytes + pl.nbuf * seg * row, state_bytes, multi, &w); st != KDA_OK)
+    const size_t list_bytes = steep_list_bytes(B, H, seg);
+    if (int st = reserve_workspace(dev, kTicketBytes + list_bytes + pl.nbuf * seg * row, state_bytes, multi, &w,
+                                   parts_bytes(B, H, dk, dv, pmax));
+        st != KDA_OK)
         return st;
     if (cudaStreamWaitEvent(s, w->done, 0) != cudaSuccess) return KDA_ERR_CUDA;
 
@@ -346,8 +474,12 @@ static int chunk_fwd_impl(const void *q, const void *k, const void *v, const flo
     dst.wait_polls = polls ? polls : ~0ull;
     // State carried between segments: the caller's hT when given, else the workspace's.
     float *carry = hT != nullptr ? hT : w->state;
-    int *tickets = reinterpret_cast<int *>(w->base);
-    uint8_t *recs[2] = {w->base + kTicketBytes, w->base + kTicketBytes + (size_t)seg * row};
+    // counters [buffer][item counter, steep count]; one steep list: the exact kernel of a
+    // segment runs on the prep stream before the next segment's prep refills it
+    int *counters = reinterpret_cast<int *>(w->base);
+    int *steep_list = reinterpret_cast<int *>(w->base + kTicketBytes);
+    uint8_t *rec0 = w->base + kTicketBytes + list_bytes;
+    uint8_t *recs[2] = {rec0, rec0 + (size_t)seg * row};
     CUtensorMap rmaps[2][4];
     for (int i = 0; i < pl.nbuf; ++i)
         if (make_rec_maps(enc, recs[i], (long long)B * H * seg, dk, rmaps[i]) != KDA_OK) return KDA_ERR_CUDA;
@@ -370,24 +502,29 @@ static int chunk_fwd_impl(const void *q, const void *k, const void *v, const flo
     int i = 0;
     for (int n0 = 0; n0 < nchunks; n0 += seg, ++i) {
         const int cnt = nchunks - n0 < seg ? nchunks - n0 : seg;
-        const bool last = n0 + cnt == nchunks;
         const int buf = multi ? (i & 1) : 0;
         // buffer reuse: the chain kernel two segments back has read it
         if (multi && i >= 2 && cudaStreamWaitEvent(sp, w->chain_done[buf], 0) != cudaSuccess) return KDA_ERR_CUDA;
-        if (cudaMemsetAsync(tickets + buf, 0, sizeof(int), sp) != cudaSuccess) return KDA_ERR_CUDA;
+        if (cudaMemsetAsync(counters + 2 * buf, 0, 2 * sizeof(int), sp) != cudaSuccess) return KDA_ERR_CUDA;
         kda::PrepParams pp;
         pp.g = g;
         pp.g_dk = g_dk;
         pp.beta = beta;
         pp.ws = recs[buf];
-        pp.ticket = tickets + buf;
-        pp.B = B; pp.T = T; pp.H = H;
-        pp.n_begin = n0;
-        pp.nseg = cnt;
+        pp.ticket = counters + 2 * buf;
+        pp.steep_count = counters + 2 * buf + 1;
+        pp.steep_items = steep_list;
+        pp.force_exact = g_force_exact.load();
+        pp.gate_c = gate_c;
+        pp.H = H;
+        pp.gm = uniform_geom(B, T, n0, cnt);
         pp.st = dst;
         // the first segment's prep runs alone: two CTAs on every SM
         const int ctas = i == 0 ? 2 * sms : (prep_ctas > 0 ? prep_ctas : 1);
-        cudaError_t e = timed_launch(dev, 0, sp, [&] { return kda::launch_prep(tq, tk, pp, dk, ctas, sp); });
+        cudaError_t e = timed_launch(dev, 0, sp, [&] { return kda::launch_prep(tq, tk, pp, dk, ctas, sp, prologue); });
+        if (e != cudaSuccess) return KDA_ERR_CUDA;
+        const kda::ExactParams xp = exact_params(q, k, g, g_dk, beta, pp, prologue);
+        e = timed_launch(dev, 2, sp, [&] { return kda::launch_exact(xp, dk, sms, sp); });
         if (e != cudaSuccess) return KDA_ERR_CUDA;
         if (multi && (cudaEventRecord(w->prep_done[buf], sp) != cudaSuccess ||
                       cudaStreamWaitEvent(sc, w->prep_done[buf], 0) != cudaSuccess))
@@ -395,19 +532,46 @@ static int chunk_fwd_impl(const void *q, const void *k, const void *v, const flo
 
         kda::ChainParams cp;
         cp.v = static_cast<const uint16_t *>(v);
-        cp.h0 = n0 == 0 ? h0 : carry;
+        cp.h0 = h0;  // read by the first segment; later ones start from carry
         cp.out = static_cast<uint16_t *>(out);
-        cp.hT = last ? hT : carry;
+        cp.hT = hT;  // written by the last segment; earlier ones end in carry
+        cp.carry = carry;
         cp.ws = recs[buf];
         cp.scale = scale;
-        cp.B = B; cp.T = T; cp.H = H; cp.DV = dv;
-        cp.n_begin = n0;
-        cp.nseg = cnt;
-        cp.nslices = chain_slices(B, H, dv, sms);
+        cp.H = H; cp.DV = dv;
+        cp.gm = pp.gm;
         cp.st = dst;
         cp.inject_wait_polls = g_inject_polls.load();
-        e = timed_launch(dev, 1, sc, [&] { return kda::launch_chain(rmaps[buf], cp, dk, sc); });
-        if (e != cudaSuccess) return KDA_ERR_CUDA;
+        const int P = plan_parts(B, H, dk, dv, cnt, sms);
+        if (P < 3) {
+            plain_pass(cp, chain_slices(B, H, dv, sms));
+            e = timed_launch(dev, 1, sc, [&] { return kda::launch_chain(rmaps[buf], cp, dk, sc); });
+            if (e != cudaSuccess) return KDA_ERR_CUDA;
+        } else {  // two-level pass: pass A, fix-up, pass B (64-column slices)
+            const size_t st_part = (size_t)B * H * dk * dv;
+            cp.nslices = dv / 64;
+            cp.parts = P;
+            cp.part_len = (cnt + P - 1) / P;
+            cp.p_start = w->parts;
+            cp.p_local = w->parts + (size_t)P * st_part;
+            cp.p_trans = w->parts + 2 * (size_t)P * st_part;
+            cp.pass_a = 1;
+            cp.part0 = 0;
+            cp.nparts = P - 1;
+            cp.slots = (dv + dk) / 64;
+            e = timed_launch(dev, 1, sc, [&] { return kda::launch_chain(rmaps[buf], cp, dk, sc); });
+            if (e != cudaSuccess) return KDA_ERR_CUDA;
+            e = timed_launch(dev, 3, sc, [&] {
+                return kda::launch_parts_fixup(cp.p_start, cp.p_local, cp.p_trans, B * H, dk, dv, P, sc);
+            });
+            if (e != cudaSuccess) return KDA_ERR_CUDA;
+            cp.pass_a = 0;
+            cp.part0 = 1;
+            cp.nparts = P - 1;
+            cp.slots = dv / 64;
+            e = timed_launch(dev, 1, sc, [&] { return kda::launch_chain(rmaps[buf], cp, dk, sc); });
+            if (e != cudaSuccess) return KDA_ERR_CUDA;
+        }
         if (multi && cudaEventRecord(w->chain_done[buf], sc) != cudaSuccess) return KDA_ERR_CUDA;
     }
     // join: the last chain kernel follows every prep kernel
@@ -421,7 +585,10 @@ size_t kda_chunk_fwd_workspace_bytes(int B, int T, int H, int dk, int dv) {
     if (T == 0) return 0;
     const SegPlan pl = plan_segments(B, T, H);
     const size_t state = pl.nbuf == 2 ? (size_t)B * H * dk * dv * sizeof(float) : 0;
-    return kTicketBytes + (size_t)pl.nbuf * pl.seg * rec_row_bytes(B, H) + state;
+    int dev = 0;
+    const int sms = cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < kMaxDevices ? num_sms(dev) : 148;
+    return kTicketBytes + steep_list_bytes(B, H, pl.seg) + (size_t)pl.nbuf * pl.seg * rec_row_bytes(B, H) + state +
+           parts_bytes(B, H, dk, dv, plan_parts(B, H, dk, dv, pl.seg, sms));
 }
 
 void kda_debug_kernel_timing(int enable) { g_timing.store(enable != 0); }
@@ -451,15 +618,17 @@ int kda_release_workspace(void) {
     int st = KDA_OK;
     if (w.base != nullptr && cudaFree(w.base) != cudaSuccess) st = KDA_ERR_CUDA;
     if (w.state != nullptr && cudaFree(w.state) != cudaSuccess) st = KDA_ERR_CUDA;
+    if (w.parts != nullptr && cudaFree(w.parts) != cudaSuccess) st = KDA_ERR_CUDA;
     w.base = nullptr; w.base_bytes = 0;
     w.state = nullptr; w.state_bytes = 0;
+    w.parts = nullptr; w.parts_bytes = 0;
     return st;
 }
 
 // The decode step for either gate form: g [B, H, dk] or, scalar_gate, g [B, H].
 static int decode_impl(const void *q, const void *k, const void *v, const float *g, const float *beta,
                        float scale, float *state, void *out, int B, int H, int dk, int dv, void *stream,
-                       bool scalar_gate) {
+                       bool scalar_gate, bool prologue = false, float gate_c = 0.f) {
     if (!q || !k || !v || !g || !beta || !state || !out) return KDA_ERR_INVALID_ARG;
     if (B < 1 || H < 1) return KDA_ERR_INVALID_ARG;
     if ((dk != 64 && dk != 128) || (dv != 64 && dv != 128)) return KDA_ERR_UNSUPPORTED;
@@ -468,7 +637,7 @@ static int decode_impl(const void *q, const void *k, const void *v, const float 
         return KDA_ERR_ALIGNMENT;
     if ((long long)B * H > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
     cudaError_t e = kda::launch_decode(q, k, v, g, beta, scale, state, out, B * H, dk, dv, scalar_gate ? 1 : dk,
-                                       static_cast<cudaStream_t>(stream));
+                                       prologue ? 1 : 0, gate_c, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
@@ -484,6 +653,126 @@ int kda_gdn_chunk_fwd(const void *q, const void *k, const void *v, const float *
     return chunk_fwd_impl(q, k, v, g, beta, scale, h0, out, hT, B, T, H, dk, dv, stream, true);
 }
 
+// Packed batch: N sequences along the token axis, cu_seqlens on the device.
+// One record buffer; the global chunks run in windows of W chunks (every head),
+// prep -> exact -> chain per window on the caller's stream; a sequence whose
+// chunks span windows carries its state between them (in hT when given).
+int kda_chunk_fwd_varlen(const void *q, const void *k, const void *v, const float *g, const float *beta,
+                         float scale, const int *cu_seqlens, int N, const float *h0, void *out, float *hT,
+                         int T_total, int H, int dk, int dv, void *stream) {
+    if (N < 1 || H < 1 || T_total < 0 || cu_seqlens == nullptr) return KDA_ERR_INVALID_ARG;
+    if (T_total > 0 && (!q || !k || !v || !g || !beta || !out)) return KDA_ERR_INVALID_ARG;
+    if ((dk != 64 && dk != 128) || (dv != 64 && dv != 128)) return KDA_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(g) || !aligned4(beta) || !aligned16(out) ||
+        !aligned16(h0) || !aligned16(hT) || !aligned4(cu_seqlens))
+        return KDA_ERR_ALIGNMENT;
+    if ((long long)N * H * 4 > 0x7fffffffLL || (long long)T_total + 64LL * (N + 1) > 0x7fffffffLL)
+        return KDA_ERR_UNSUPPORTED;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (T_total == 0) {  // every sequence is empty: hT = h0 (or zero)
+        if (hT == nullptr) return KDA_OK;
+        const size_t bytes = (size_t)N * H * dk * dv * sizeof(float);
+        cudaError_t e = h0 ? (h0 == hT ? cudaSuccess : cudaMemcpyAsync(hT, h0, bytes, cudaMemcpyDeviceToDevice, s))
+                           : cudaMemsetAsync(hT, 0, bytes, s);
+        return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+    }
+    uint32_t *word = nullptr;
+    if (current_status_word(&word) != KDA_OK) return KDA_ERR_CUDA;
+    PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
+    if (get_encoder(&enc) != KDA_OK) return KDA_ERR_CUDA;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return KDA_ERR_CUDA;
+    CUtensorMap tq, tk;  // [1][T_total][H][dk]
+    if (make_map(&tq, enc, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dk, H, T_total, 1, 64,
+                 CU_TENSOR_MAP_SWIZZLE_128B) != KDA_OK ||
+        make_map(&tk, enc, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dk, H, T_total, 1, 64,
+                 CU_TENSOR_MAP_SWIZZLE_128B) != KDA_OK)
+        return KDA_ERR_CUDA;
+
+    const VarlenPlan pl = plan_varlen(N, T_total, H);
+    const int W = pl.W;
+    const size_t row = rec_row_bytes(1, H);  // one chunk of every head
+    const size_t state_bytes = (pl.nwin > 1 && hT == nullptr) ? (size_t)N * H * dk * dv * sizeof(float) : 0;
+    const int sms = num_sms(dev);
+
+    std::lock_guard<std::mutex> lk(g_mu);
+    Workspace *w = nullptr;
+    if (int st = reserve_workspace(dev, varlen_base_bytes(N, H, pl), state_bytes, false, &w); st != KDA_OK)
+        return st;
+    if (cudaStreamWaitEvent(s, w->done, 0) != cudaSuccess) return KDA_ERR_CUDA;
+    const unsigned long long polls = g_wait_polls.load();
+    kda::DeviceStatus dst;
+    dst.word = word;
+    dst.wait_polls = polls ? polls : ~0ull;
+    // [counters][steep list][cu_s][cc][chunk_seq][records]
+    int *counters = reinterpret_cast<int *>(w->base);
+    int *steep_list = reinterpret_cast<int *>(w->base + kTicketBytes);
+    int *cu_s = reinterpret_cast<int *>(w->base + kTicketBytes + steep_list_bytes(1, H, W));
+    int *cc = cu_s + (N + 1);
+    int *chunk_seq = cc + (N + 1);
+    uint8_t *recs = w->base + kTicketBytes + steep_list_bytes(1, H, W) + varlen_meta_bytes(N, pl.cmax);
+    CUtensorMap rmaps[4];
+    if (make_rec_maps(enc, recs, (long long)H * W, dk, rmaps) != KDA_OK) return KDA_ERR_CUDA;
+    if (kda::launch_varlen_setup(cu_seqlens, N, T_total, pl.cmax, cu_s, cc, chunk_seq, dst, s) != cudaSuccess)
+        return KDA_ERR_CUDA;
+    float *carry = hT != nullptr ? hT : w->state;
+
+    for (int win = 0; win < pl.nwin; ++win) {
+        kda::SeqGeom gm = {};
+        gm.cu = cu_s;
+        gm.cc = cc;
+        gm.chunk_seq = chunk_seq;
+        gm.nseqs = N;
+        gm.T = T_total;
+        gm.c0 = win * W;
+        gm.W = W;
+        if (cudaMemsetAsync(counters, 0, 2 * sizeof(int), s) != cudaSuccess) return KDA_ERR_CUDA;
+        kda::PrepParams pp;
+        pp.g = g;
+        pp.g_dk = dk;
+        pp.beta = beta;
+        pp.ws = recs;
+        pp.ticket = counters;
+        pp.steep_count = counters + 1;
+        pp.steep_items = steep_list;
+        pp.force_exact = g_force_exact.load();
+        pp.gate_c = 0.f;
+        pp.H = H;
+        pp.gm = gm;
+        pp.st = dst;
+        cudaError_t e = timed_launch(dev, 0, s, [&] { return kda::launch_prep(tq, tk, pp, dk, 2 * sms, s, false); });
+        if (e != cudaSuccess) return KDA_ERR_CUDA;
+        const kda::ExactParams xp = exact_params(q, k, g, dk, beta, pp);
+        e = timed_launch(dev, 2, s, [&] { return kda::launch_exact(xp, dk, sms, s); });
+        if (e != cudaSuccess) return KDA_ERR_CUDA;
+        kda::ChainParams cp;
+        cp.v = static_cast<const uint16_t *>(v);
+        cp.h0 = h0;
+        cp.out = static_cast<uint16_t *>(out);
+        cp.hT = hT;
+        cp.carry = carry;
+        cp.ws = recs;
+        cp.scale = scale;
+        cp.H = H; cp.DV = dv;
+        cp.gm = gm;
+        plain_pass(cp, chain_slices(N, H, dv, sms));
+        cp.st = dst;
+        cp.inject_wait_polls = g_inject_polls.load();
+        e = timed_launch(dev, 1, s, [&] { return kda::launch_chain(rmaps, cp, dk, s); });
+        if (e != cudaSuccess) return KDA_ERR_CUDA;
+    }
+    if (cudaEventRecord(w->done, s) != cudaSuccess) return KDA_ERR_CUDA;
+    return KDA_OK;
+}
+
+size_t kda_chunk_fwd_varlen_workspace_bytes(int N, int T_total, int H, int dk, int dv) {
+    if (N < 1 || H < 1 || T_total < 0 || (dk != 64 && dk != 128) || (dv != 64 && dv != 128)) return 0;
+    if (T_total == 0) return 0;
+    const VarlenPlan pl = plan_varlen(N, T_total, H);
+    const size_t state = pl.nwin > 1 ? (size_t)N * H * dk * dv * sizeof(float) : 0;
+    return varlen_base_bytes(N, H, pl) + state;
+}
+
 int kda_decode_step(const void *q, const void *k, const void *v, const float *g, const float *beta,
                     float scale, float *state, void *out, int B, int H, int dk, int dv, void *stream) {
     return decode_impl(q, k, v, g, beta, scale, state, out, B, H, dk, dv, stream, false);
@@ -492,6 +781,21 @@ int kda_decode_step(const void *q, const void *k, const void *v, const float *g,
 int kda_gdn_decode_step(const void *q, const void *k, const void *v, const float *g, const float *beta,
                         float scale, float *state, void *out, int B, int H, int dk, int dv, void *stream) {
     return decode_impl(q, k, v, g, beta, scale, state, out, B, H, dk, dv, stream, true);
+}
+
+int kda_chunk_fwd_raw(const void *q, const void *k, const void *v, const float *g_raw, const float *beta_raw,
+                      float gate_c, float scale, const float *h0, void *out, float *hT, int B, int T, int H,
+                      int dk, int dv, void *stream) {
+    if (!(gate_c >= 0.f) || gate_c > 3.0e38f) return KDA_ERR_INVALID_ARG;  // also rejects NaN
+    return chunk_fwd_impl(q, k, v, g_raw, beta_raw, scale, h0, out, hT, B, T, H, dk, dv, stream, false, true,
+                          gate_c);
+}
+
+int kda_decode_step_raw(const void *q, const void *k, const void *v, const float *g_raw, const float *beta_raw,
+                        float gate_c, float scale, float *state, void *out, int B, int H, int dk, int dv,
+                        void *stream) {
+    if (!(gate_c >= 0.f) || gate_c > 3.0e38f) return KDA_ERR_INVALID_ARG;
+    return decode_impl(q, k, v, g_raw, beta_raw, scale, state, out, B, H, dk, dv, stream, false, true, gate_c);
 }
 
 }  // extern "C"
@@ -530,8 +834,6 @@ int scratch_base(int dev, uint8_t **out) {
     return KDA_OK;
 }
 
-size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
-
 }  // namespace
 
 extern "C" {
@@ -556,13 +858,17 @@ int kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const flo
         return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
     }
 
-    // Scratch layout: [carried state, when hT is NULL][records of one segment].
+    // Scratch layout: [counters][steep-item list][carried state, when hT is NULL][records of one
+    // segment]; a segment of n chunks needs n rows of records and n * B * H list entries.
     const int nchunks = (T + kda::CH - 1) / kda::CH;
     const size_t row = rec_row_bytes(B, H);
     const size_t state_bytes = hT == nullptr ? round256((size_t)B * H * dk * dv * sizeof(float)) : 0;
-    if (kTicketBytes + state_bytes + row > kScratchBytes) return KDA_ERR_SCRATCH_LIMIT;
-    const size_t fit = (kScratchBytes - kTicketBytes - state_bytes) / row;
+    const size_t fixed = kTicketBytes + 256 + state_bytes;  // 256: the list's rounding
+    const size_t per_chunk = row + (size_t)B * H * sizeof(int);
+    if (fixed + per_chunk > kScratchBytes) return KDA_ERR_SCRATCH_LIMIT;
+    const size_t fit = (kScratchBytes - fixed) / per_chunk;
     const int seg = fit < (size_t)nchunks ? (int)fit : nchunks;
+    const size_t list_bytes = steep_list_bytes(B, H, seg);
 
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return KDA_ERR_CUDA;
@@ -584,42 +890,46 @@ int kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const flo
     kda::DeviceStatus dst;
     dst.word = word;
     dst.wait_polls = polls ? polls : ~0ull;
-    // [the prep kernel's item counter][carried state, when hT is NULL][records]
+    // [item counter, steep count][steep list][carried state, when hT is NULL][records]
     int *ticket = reinterpret_cast<int *>(scratch);
-    float *carry = hT != nullptr ? hT : reinterpret_cast<float *>(scratch + kTicketBytes);
-    uint8_t *recs = scratch + kTicketBytes + state_bytes;
+    int *steep_list = reinterpret_cast<int *>(scratch + kTicketBytes);
+    float *carry = hT != nullptr ? hT : reinterpret_cast<float *>(scratch + kTicketBytes + list_bytes);
+    uint8_t *recs = scratch + kTicketBytes + list_bytes + state_bytes;
     const int sms = num_sms(dev);
     CUtensorMap rmaps[4];
     if (make_rec_maps(enc, recs, (long long)B * H * seg, dk, rmaps) != KDA_OK) return KDA_ERR_CUDA;
 
     for (int n0 = 0; n0 < nchunks; n0 += seg) {
         const int cnt = nchunks - n0 < seg ? nchunks - n0 : seg;
-        const bool last = n0 + cnt == nchunks;
         kda::PrepParams pp;
         pp.g = g;
         pp.g_dk = dk;
         pp.beta = beta;
         pp.ws = recs;
         pp.ticket = ticket;
-        pp.B = B; pp.T = T; pp.H = H;
-        pp.n_begin = n0;
-        pp.nseg = cnt;
+        pp.steep_count = ticket + 1;
+        pp.steep_items = steep_list;
+        pp.force_exact = g_force_exact.load();
+        pp.gate_c = 0.f;
+        pp.H = H;
+        pp.gm = uniform_geom(B, T, n0, cnt);
         pp.st = dst;
-        if (cudaMemsetAsync(ticket, 0, sizeof(int), s) != cudaSuccess ||  // the counter starts at zero
-            kda::launch_prep(tq, tk, pp, dk, 2 * sms, s) != cudaSuccess)
+        if (cudaMemsetAsync(ticket, 0, 2 * sizeof(int), s) != cudaSuccess ||  // the counters start at zero
+            kda::launch_prep(tq, tk, pp, dk, 2 * sms, s, false) != cudaSuccess ||
+            kda::launch_exact(exact_params(q, k, g, dk, beta, pp), dk, sms, s) != cudaSuccess)
             return KDA_ERR_CUDA;
 
         kda::ChainParams cp;
         cp.v = static_cast<const uint16_t *>(v);
-        cp.h0 = n0 == 0 ? h0 : carry;
+        cp.h0 = h0;
         cp.out = static_cast<uint16_t *>(out);
-        cp.hT = last ? hT : carry;
+        cp.hT = hT;
+        cp.carry = carry;
         cp.ws = recs;
         cp.scale = scale;
-        cp.B = B; cp.T = T; cp.H = H; cp.DV = dv;
-        cp.n_begin = n0;
-        cp.nseg = cnt;
-        cp.nslices = chain_slices(B, H, dv, sms);
+        cp.H = H; cp.DV = dv;
+        cp.gm = pp.gm;
+        plain_pass(cp, chain_slices(B, H, dv, sms));
         cp.st = dst;
         cp.inject_wait_polls = g_inject_polls.load();
         if (kda::launch_chain(rmaps, cp, dk, s) != cudaSuccess) return KDA_ERR_CUDA;

@@ -18,7 +18,7 @@ namespace kda {
 
 // ---------------------------------------------------------------- status ----
 // Bit flags OR-ed into the per-device status word by kernels.
-enum : uint32_t { DEV_TIMEOUT = 1u };
+enum : uint32_t { DEV_TIMEOUT = 1u, DEV_BAD_ARG = 2u };
 
 struct DeviceStatus {
     uint32_t *word;        // device-global status word (never NULL at launch)
@@ -278,6 +278,15 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
 #pragma unroll
     for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
 }
+
+// ------------------------------------------------------------ gate prologue ----
+// Raw projections in: log-decay g = -c softplus(x), with softplus(x) =
+// log(1 + e^x) written as max(x, 0) + log1p(e^-|x|) so that it neither
+// overflows nor loses small values, and beta = sigmoid(x).
+__device__ __forceinline__ float gate_logdecay(float x, float c) {
+    return -c * (fmaxf(x, 0.f) + log1pf(__expf(-fabsf(x))));
+}
+__device__ __forceinline__ float gate_sigmoid(float x) { return 1.f / (1.f + __expf(-x)); }
 
 // ------------------------------------------------------------ conversions ----
 // fp32 -> tf32 bit pattern, rounded to nearest (ties away), stored in 32 bits.

@@ -18,10 +18,16 @@
 // side of the contraction over key channels.  Rows of 16-token block I use
 // the reference m = 16 I + 8: row factor e^{Gamma_i - Gamma_m}, column factor
 // e^{Gamma_m - Gamma_j}.  For j in an earlier block both factors are <= 1; in
-// the block itself a factor can exceed 1 and is clamped at e^80, so results
-// are exact when a channel's log-decay over one aligned 16-token block is
-// >= -160.  All factors come from running products of alpha = e^g (one exp
-// per input element) plus one reciprocal per factor above 1.
+// the block itself a factor can exceed 1.  It stays below e^80 unless some key
+// channel loses more than 80 of log-decay over tokens 16 I + 1 .. 16 I + 8 or
+// 16 I + 9 .. 16 I + 15.  Such a "steep" item is flagged in phase E (its
+// factors are clamped at e^80 meanwhile, so nothing overflows) and appended to
+// a list; the exact kernel (exact_prep.cu) then rewrites its P, T' and W from
+// pairwise factors e^{Gamma_i - Gamma_j} <= 1 before the chain reads them.  So
+// results are exact up to rounding for any finite g <= 0, and only items with
+// extreme decay pay for the slow path.  All factors of this kernel come from
+// running products of alpha = e^g (one exp per input element) plus one
+// reciprocal per factor above 1.
 //
 // Persistent CTAs (two per SM, 512 threads) claim items from a counter; while
 // one item is processed the next one's q, k and g are prefetched into L2.  In the
@@ -94,8 +100,12 @@ __device__ __forceinline__ void prefetch_line_l2(const void *p) {
     asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<uint64_t>(p)) : "memory");
 }
 
-// SG: scalar gate, g [B, T, H] (else g [B, T, H, DK]).
-template <int DK, bool SG>
+// SG: scalar gate, g [B, T, H] (else g [B, T, H, DK]).  PRO: the gate prologue --
+// g, beta, q and k are raw projections: g = -c softplus(g_raw), beta =
+// sigmoid(beta_raw), and q, k are L2-normalised per token (the norms come from
+// the staged tiles; the normalised values are rounded to bf16 again, as an
+// unfused caller would store them).
+template <int DK, bool SG, bool PRO>
 __global__ void __launch_bounds__(PREP_THREADS, 2)
 prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
             const PrepParams prm) {
@@ -116,8 +126,8 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     const int warp = tid >> 5, lane = tid & 31;
     const int ch = tid & 127;        // key channel / TMEM lane of this thread
     const int qb = tid >> 7;         // 16-token block (phase E) / 16-column quarter (elsewhere)
-    const int T = prm.T, H = prm.H;
-    const int nitems = prm.B * prm.H * prm.nseg;  // (b, h) major, chunk minor
+    const int H = prm.H;
+    const int nitems = geom_items(prm.gm, H);
     const uint64_t polls = prm.st.wait_polls;
 
     if (tid == 0) {
@@ -153,14 +163,6 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         __syncthreads();
         tc_fence_after();
     };
-    // first token, batch and head of an item
-    auto item_coords = [&](int it, int &b, int &h, int &t0) {
-        const int ni = it % prm.nseg, bh = it / prm.nseg;
-        h = bh % H;
-        b = bh / H;
-        t0 = (prm.n_begin + ni) * CH;
-    };
-
     const int c = ch, I = qb, tb = SUB * I;
     const bool active = c < DK;
 
@@ -169,17 +171,17 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     int claim = 0;  // thread 0: the item claimed for after this one (result needed mid-item)
     for (int item = *s_next; item < nitems && !aborted;) {
         if (tid == 0) claim = atomicAdd(prm.ticket, 1);
-        int b, h, t0;
-        item_coords(item, b, h, t0);
-        uint8_t *rec = prm.ws + (size_t)item * REC_BYTES;
+        const ItemGeo gi = item_geo(prm.gm, H, item);
+        const int h = gi.h;
+        uint8_t *rec = prm.ws + (size_t)gi.rec * REC_BYTES;
 
         // ---------------- inputs: q, k by TMA; g (this thread's 16 tokens) and beta by plain loads
         if (tid == 0) {
             mbar_expect_tx(bar_in, (uint32_t)(2 * CH * DK * 2));
 #pragma unroll
             for (int kb = 0; kb < DK / 64; ++kb) {
-                tma_load_4d(sbase + L::OFF_QIN + kb * CH * 128, &tm_q, bar_in, kb * 64, h, t0, b);
-                tma_load_4d(sbase + L::OFF_KIN + kb * CH * 128, &tm_k, bar_in, kb * 64, h, t0, b);
+                tma_load_4d(sbase + L::OFF_QIN + kb * CH * 128, &tm_q, bar_in, kb * 64, h, gi.tok0, gi.bcoord);
+                tma_load_4d(sbase + L::OFF_KIN + kb * CH * 128, &tm_k, bar_in, kb * 64, h, gi.tok0, gi.bcoord);
             }
         }
         tma_pending = true;
@@ -187,13 +189,36 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         {
             // one gate per key channel, or (SG) one per (token, head) shared by all channels
             constexpr int gdk = SG ? 1 : DK;
-            const float *gp = prm.g + (((size_t)b * T + t0 + tb) * H + h) * gdk + (SG ? 0 : c);
+            const float *gp = prm.g + ((size_t)(gi.row0 + tb) * H + h) * gdk + (SG ? 0 : c);
 #pragma unroll
-            for (int u = 0; u < SUB; ++u) al[u] = (t0 + tb + u < T && active) ? __ldg(gp + (size_t)u * H * gdk) : 0.f;
+            for (int u = 0; u < SUB; ++u) al[u] = (tb + u < gi.nvalid && active) ? __ldg(gp + (size_t)u * H * gdk) : 0.f;
         }
-        if (tid < CH) s_beta[tid] = (t0 + tid < T) ? prm.beta[((size_t)b * T + t0 + tid) * H + h] : 0.f;
+        if (tid < CH) {
+            const float braw = (tid < gi.nvalid) ? prm.beta[(size_t)(gi.row0 + tid) * H + h] : 0.f;
+            s_beta[tid] = (PRO && tid < gi.nvalid) ? gate_sigmoid(braw) : braw;
+        }
         if (!wait_all(bar_in, ph_in, tma_pending)) { aborted = true; break; }
         ph_in ^= 1u;
+        float *s_rn = reinterpret_cast<float *>(sm + L::OFF_MISC + 256);  // PRO: 1 / |q_t|, then 1 / |k_t|
+        if constexpr (PRO) {
+#pragma unroll
+            for (int u = 0; u < SUB; ++u) al[u] = (tb + u < gi.nvalid && active) ? gate_logdecay(al[u], prm.gate_c) : 0.f;
+            // warp w: rows 8 w .. 8 w + 7 of [q; k]; each lane sums DK / 32 squares
+            for (int rr = 0; rr < 8; ++rr) {
+                const int row = warp * 8 + rr;
+                const uint8_t *tile = sm + (row < CH ? L::OFF_QIN : L::OFF_KIN);
+                float ss = 0.f;
+#pragma unroll
+                for (int cc = lane; cc < DK; cc += 32) {
+                    const float x = bf16_bits_to_f32(*reinterpret_cast<const uint16_t *>(tile + kmaj<128, 2>(row & (CH - 1), cc, CH)));
+                    ss += x * x;
+                }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+                if (lane == 0) s_rn[row] = rsqrtf(fmaxf(ss, 1e-24f));
+            }
+            __syncthreads();
+        }
 
         // ---------------- E: decay factors and operand tiles ----------------
         // This thread's 16 key and query values, kept as bf16 pairs (tokens 2e, 2e + 1).
@@ -202,10 +227,17 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             const uint8_t *qs = sm + L::OFF_QIN, *ks = sm + L::OFF_KIN;
 #pragma unroll
             for (int e = 0; e < SUB / 2; ++e) {
-                const uint32_t k0 = *reinterpret_cast<const uint16_t *>(ks + kmaj<128, 2>(tb + 2 * e, c, CH));
-                const uint32_t k1 = *reinterpret_cast<const uint16_t *>(ks + kmaj<128, 2>(tb + 2 * e + 1, c, CH));
-                const uint32_t q0 = *reinterpret_cast<const uint16_t *>(qs + kmaj<128, 2>(tb + 2 * e, c, CH));
-                const uint32_t q1 = *reinterpret_cast<const uint16_t *>(qs + kmaj<128, 2>(tb + 2 * e + 1, c, CH));
+                uint32_t k0 = *reinterpret_cast<const uint16_t *>(ks + kmaj<128, 2>(tb + 2 * e, c, CH));
+                uint32_t k1 = *reinterpret_cast<const uint16_t *>(ks + kmaj<128, 2>(tb + 2 * e + 1, c, CH));
+                uint32_t q0 = *reinterpret_cast<const uint16_t *>(qs + kmaj<128, 2>(tb + 2 * e, c, CH));
+                uint32_t q1 = *reinterpret_cast<const uint16_t *>(qs + kmaj<128, 2>(tb + 2 * e + 1, c, CH));
+                if constexpr (PRO) {
+                    const int t = tb + 2 * e;
+                    k0 = to_bf16_bits(bf16_bits_to_f32((uint16_t)k0) * s_rn[CH + t]);
+                    k1 = to_bf16_bits(bf16_bits_to_f32((uint16_t)k1) * s_rn[CH + t + 1]);
+                    q0 = to_bf16_bits(bf16_bits_to_f32((uint16_t)q0) * s_rn[t]);
+                    q1 = to_bf16_bits(bf16_bits_to_f32((uint16_t)q1) * s_rn[t + 1]);
+                }
                 kp[e] = k0 | (k1 << 16);
                 qp[e] = q0 | (q1 << 16);
             }
@@ -248,6 +280,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         auto xput = [&](int col, const float (&v8)[8]) {
             *reinterpret_cast<uint4 *>(sm + L::OFF_X + mnmaj<128, 2>(c, col, DK)) = pack8_bf16(v8);
         };
+        bool steep = false;  // a split factor of this thread's block would pass e^80
         if (active) {
             // Own block, reference m = tb + 8:
             //   u >= 8: f_u = prod_{s=9..u} alpha     X = k f,   Y^(I) = k / f
@@ -257,6 +290,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 float ff = 1.f;
 #pragma unroll
                 for (int e = 0; e < 8; ++e) { if (e > 0) ff *= al[8 + e]; f[e] = ff; }
+                steep = f[7] < EXP_CLAMP_LO;  // prod of alpha over tokens 9..15, the smallest f
 #pragma unroll
                 for (int e = 0; e < 8; ++e) v8[e] = kval(8 + e) * f[e];
                 xput(tb + 8, v8);
@@ -272,6 +306,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 float yy = 1.f;
 #pragma unroll
                 for (int e = 7; e >= 0; --e) { yy *= al[e + 1]; y[e] = yy; }
+                steep = steep || y[0] < EXP_CLAMP_LO;  // prod over tokens 1..8, the smallest y
 #pragma unroll
                 for (int e = 0; e < 8; ++e) v8[e] = kval(e) * y[e];
                 yput(I, tb, v8);
@@ -311,7 +346,11 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 }
             }
         }
-        sync_for_mma();
+        fence_async_smem();
+        tc_fence_before();
+        const bool exact_item = __syncthreads_or(steep) || prm.force_exact;
+        tc_fence_after();
+        if (exact_item && tid == 0) prm.steep_items[atomicAdd(prm.steep_count, 1)] = item;
 
         // ---------------- F: formation products (bf16), overlapped with the rest of E ----------------
         if (tid == 0) {  // X [Y^(0) | .. | Y^(3)]^T: 128 x 160, column block I' = D^(I')
@@ -362,16 +401,15 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         const int next = *s_next;
         // the next item's q, k and g into L2 while this one finishes
         if (next < nitems) {
-            int nb, nh, nt0;
-            item_coords(next, nb, nh, nt0);
+            const ItemGeo ng = item_geo(prm.gm, H, next);
             if (tid == 0) {
 #pragma unroll
                 for (int kb = 0; kb < DK / 64; ++kb) {
-                    prefetch_tensor_4d(&tm_q, kb * 64, nh, nt0, nb);
-                    prefetch_tensor_4d(&tm_k, kb * 64, nh, nt0, nb);
+                    prefetch_tensor_4d(&tm_q, kb * 64, ng.h, ng.tok0, ng.bcoord);
+                    prefetch_tensor_4d(&tm_k, kb * 64, ng.h, ng.tok0, ng.bcoord);
                 }
-            } else if (tid >= 64 && tid < 64 + CH && nt0 + tid - 64 < T) {
-                const float *gr = prm.g + (((size_t)nb * T + nt0 + tid - 64) * H + nh) * (SG ? 1 : DK);
+            } else if (tid >= 64 && tid < 64 + CH && tid - 64 < ng.nvalid) {
+                const float *gr = prm.g + ((size_t)(ng.row0 + tid - 64) * H + ng.h) * (SG ? 1 : DK);
                 if (SG) prefetch_line_l2(gr);
                 else prefetch_l2(gr, DK * 4);
             }
@@ -570,28 +608,36 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     if (warp == 0) tmem_dealloc(tmem, L::TM_COLS);
 }
 
-template <int DK, bool SG>
+template <int DK, bool SG, bool PRO>
 static cudaError_t launch_prep_t(const CUtensorMap &tq, const CUtensorMap &tk, const PrepParams &prm,
                                  int max_ctas, cudaStream_t stream) {
     using L = PrepLayout<DK>;
-    cudaError_t e = cudaFuncSetAttribute(prep_kernel<DK, SG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(prep_kernel<DK, SG, PRO>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          L::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    const long long items = (long long)prm.B * prm.H * prm.nseg;
+    // items of the launch (packed: an upper bound, the kernel reads the exact count)
+    const long long items = prm.gm.cu == nullptr ? (long long)prm.gm.nseqs * prm.H * prm.gm.nseg
+                                                 : (long long)prm.gm.W * prm.H;
     const int grid = (int)(items < max_ctas ? items : max_ctas);
-    prep_kernel<DK, SG><<<grid, PREP_THREADS, L::SMEM_BYTES, stream>>>(tq, tk, prm);
+    prep_kernel<DK, SG, PRO><<<grid, PREP_THREADS, L::SMEM_BYTES, stream>>>(tq, tk, prm);
     return cudaGetLastError();
 }
 
 // At most max_ctas persistent CTAs (two fit on an SM), at most one per item;
-// prm.g_dk selects the gate form (dk: per key channel, 1: scalar).
+// prm.g_dk selects the gate form (dk: per key channel, 1: scalar); `prologue`
+// the raw-input form (per key channel only).
 cudaError_t launch_prep(const CUtensorMap &tq, const CUtensorMap &tk, const PrepParams &prm, int dk,
-                        int max_ctas, cudaStream_t stream) {
+                        int max_ctas, cudaStream_t stream, bool prologue) {
     const bool sg = prm.g_dk == 1;
-    if (dk == 128) return sg ? launch_prep_t<128, true>(tq, tk, prm, max_ctas, stream)
-                             : launch_prep_t<128, false>(tq, tk, prm, max_ctas, stream);
-    return sg ? launch_prep_t<64, true>(tq, tk, prm, max_ctas, stream)
-              : launch_prep_t<64, false>(tq, tk, prm, max_ctas, stream);
+    if (prologue) {
+        if (sg) return cudaErrorInvalidValue;
+        return dk == 128 ? launch_prep_t<128, false, true>(tq, tk, prm, max_ctas, stream)
+                         : launch_prep_t<64, false, true>(tq, tk, prm, max_ctas, stream);
+    }
+    if (dk == 128) return sg ? launch_prep_t<128, true, false>(tq, tk, prm, max_ctas, stream)
+                             : launch_prep_t<128, false, false>(tq, tk, prm, max_ctas, stream);
+    return sg ? launch_prep_t<64, true, false>(tq, tk, prm, max_ctas, stream)
+              : launch_prep_t<64, false, false>(tq, tk, prm, max_ctas, stream);
 }
 
 }  // namespace kda

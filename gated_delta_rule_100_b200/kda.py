@@ -6,7 +6,10 @@ The entry points mirror ``include/kda.h``:
 * ``chunk_fwd``   -> ``kda_chunk_fwd``   (chunkwise prefill)
 * ``chunk_fwd_noalloc`` -> ``kda_chunk_fwd_noalloc`` (the same prefill over a fixed
   scratch array: no device allocation)
+* ``chunk_fwd_varlen`` -> ``kda_chunk_fwd_varlen`` (packed batch of sequences, cu_seqlens)
 * ``decode_step`` -> ``kda_decode_step`` (one recurrent step, state in place)
+* ``chunk_fwd_raw`` / ``decode_step_raw`` -> ``kda_chunk_fwd_raw`` / ``kda_decode_step_raw``
+  (raw projections in: the gate prologue and the q/k normalisation run in the kernels)
 * ``stream_status`` -> ``kda_stream_status``
 * ``workspace_bytes`` / ``release_workspace`` -> ``kda_chunk_fwd_workspace_bytes`` /
   ``kda_release_workspace``
@@ -29,10 +32,12 @@ LIB_PATH = os.path.join(_HERE, "libkda.so")
 
 (KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_ALIGNMENT, KDA_ERR_CUDA, KDA_ERR_TIMEOUT,
  KDA_ERR_SCRATCH_LIMIT) = range(7)
-EXPORTED = ("kda_chunk_fwd", "kda_chunk_fwd_noalloc", "kda_decode_step", "kda_gdn_chunk_fwd", "kda_gdn_decode_step",
-            "kda_chunk_fwd_workspace_bytes", "kda_release_workspace",
+EXPORTED = ("kda_chunk_fwd", "kda_chunk_fwd_noalloc", "kda_chunk_fwd_varlen", "kda_decode_step",
+            "kda_gdn_chunk_fwd", "kda_gdn_decode_step", "kda_chunk_fwd_raw", "kda_decode_step_raw",
+            "kda_chunk_fwd_workspace_bytes", "kda_chunk_fwd_varlen_workspace_bytes", "kda_release_workspace",
             "kda_status_string", "kda_stream_status", "kda_chunk_fwd_debug_wait_limit",
-            "kda_chunk_fwd_debug_inject_timeout", "kda_debug_kernel_timing", "kda_debug_kernel_times",
+            "kda_chunk_fwd_debug_inject_timeout", "kda_chunk_fwd_debug_force_exact", "kda_chunk_fwd_debug_record_cap",
+            "kda_debug_kernel_timing", "kda_debug_kernel_times",
             "kda_abi_version")
 
 _lib = None
@@ -58,6 +63,14 @@ def load():
     lib.kda_chunk_fwd.restype = i
     lib.kda_chunk_fwd_noalloc.argtypes = [vp, vp, vp, fp, fp, f, fp, vp, fp, i, i, i, i, i, vp]
     lib.kda_chunk_fwd_noalloc.restype = i
+    lib.kda_chunk_fwd_raw.argtypes = [vp, vp, vp, fp, fp, f, f, fp, vp, fp, i, i, i, i, i, vp]
+    lib.kda_chunk_fwd_raw.restype = i
+    lib.kda_decode_step_raw.argtypes = [vp, vp, vp, fp, fp, f, f, fp, vp, i, i, i, i, vp]
+    lib.kda_decode_step_raw.restype = i
+    lib.kda_chunk_fwd_varlen.argtypes = [vp, vp, vp, fp, fp, f, vp, i, fp, vp, fp, i, i, i, i, vp]
+    lib.kda_chunk_fwd_varlen.restype = i
+    lib.kda_chunk_fwd_varlen_workspace_bytes.argtypes = [i, i, i, i, i]
+    lib.kda_chunk_fwd_varlen_workspace_bytes.restype = ctypes.c_size_t
     lib.kda_decode_step.argtypes = [vp, vp, vp, fp, fp, f, fp, vp, i, i, i, i, vp]
     lib.kda_decode_step.restype = i
     lib.kda_gdn_chunk_fwd.argtypes = [vp, vp, vp, fp, fp, f, fp, vp, fp, i, i, i, i, i, vp]
@@ -76,6 +89,10 @@ def load():
     lib.kda_chunk_fwd_debug_wait_limit.restype = None
     lib.kda_chunk_fwd_debug_inject_timeout.argtypes = [ctypes.c_ulonglong]
     lib.kda_chunk_fwd_debug_inject_timeout.restype = None
+    lib.kda_chunk_fwd_debug_record_cap.argtypes = [ctypes.c_ulonglong]
+    lib.kda_chunk_fwd_debug_record_cap.restype = None
+    lib.kda_chunk_fwd_debug_force_exact.argtypes = [i]
+    lib.kda_chunk_fwd_debug_force_exact.restype = None
     lib.kda_debug_kernel_timing.argtypes = [i]
     lib.kda_debug_kernel_timing.restype = None
     lib.kda_debug_kernel_times.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_longlong), i]
@@ -147,6 +164,53 @@ def _prefill(symbol, scalar_gate, q, k, v, g, beta, scale, h0, out, hT, final_st
     return out, hT
 
 
+def chunk_fwd_raw(q, k, v, g_raw, beta_raw, gate_c, scale, h0=None, *, out=None, hT=None, final_state=True,
+                  stream=None):
+    """Prefill from raw projections: g = -gate_c softplus(g_raw), beta = sigmoid(beta_raw),
+    q and k L2-normalised, all inside the kernels.  Shapes and dtypes as ``chunk_fwd``."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    _check(q, "q", torch.bfloat16, (B, T, H, dk))
+    _check(k, "k", torch.bfloat16, (B, T, H, dk))
+    _check(v, "v", torch.bfloat16, (B, T, H, dv))
+    _check(g_raw, "g_raw", torch.float32, (B, T, H, dk))
+    _check(beta_raw, "beta_raw", torch.float32, (B, T, H))
+    if h0 is not None:
+        _check(h0, "h0", torch.float32, (B, H, dk, dv))
+    if out is None:
+        out = torch.empty((B, T, H, dv), device=q.device, dtype=torch.bfloat16)
+    _check(out, "out", torch.bfloat16, (B, T, H, dv))
+    if hT is None and final_state:
+        hT = torch.empty((B, H, dk, dv), device=q.device, dtype=torch.float32)
+    if hT is not None:
+        _check(hT, "hT", torch.float32, (B, H, dk, dv))
+    rc = load().kda_chunk_fwd_raw(_ptr(q), _ptr(k), _ptr(v), _ptr(g_raw), _ptr(beta_raw), float(gate_c),
+                                  float(scale), _ptr(h0), _ptr(out), _ptr(hT), B, T, H, dk, dv, _stream(stream))
+    if rc != KDA_OK:
+        raise KdaError(rc, "kda_chunk_fwd_raw")
+    return out, hT
+
+
+def decode_step_raw(q, k, v, g_raw, beta_raw, gate_c, scale, state, *, out=None, stream=None):
+    """One recurrent step from raw projections (see ``chunk_fwd_raw``); shapes as ``decode_step``."""
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    _check(q, "q", torch.bfloat16, (B, H, dk))
+    _check(k, "k", torch.bfloat16, (B, H, dk))
+    _check(v, "v", torch.bfloat16, (B, H, dv))
+    _check(g_raw, "g_raw", torch.float32, (B, H, dk))
+    _check(beta_raw, "beta_raw", torch.float32, (B, H))
+    _check(state, "state", torch.float32, (B, H, dk, dv))
+    if out is None:
+        out = torch.empty((B, H, dv), device=q.device, dtype=torch.bfloat16)
+    _check(out, "out", torch.bfloat16, (B, H, dv))
+    rc = load().kda_decode_step_raw(_ptr(q), _ptr(k), _ptr(v), _ptr(g_raw), _ptr(beta_raw), float(gate_c),
+                                    float(scale), _ptr(state), _ptr(out), B, H, dk, dv, _stream(stream))
+    if rc != KDA_OK:
+        raise KdaError(rc, "kda_decode_step_raw")
+    return out
+
+
 def chunk_fwd_noalloc(q, k, v, g, beta, scale, h0=None, *, out, hT=None, stream=None):
     """``chunk_fwd`` through ``kda_chunk_fwd_noalloc``: the caller passes ``out``
     (and ``hT`` unless the final state is not wanted); the library allocates
@@ -168,6 +232,50 @@ def chunk_fwd_noalloc(q, k, v, g, beta, scale, h0=None, *, out, hT=None, stream=
     if rc != KDA_OK:
         raise KdaError(rc, "kda_chunk_fwd_noalloc")
     return out, hT
+
+
+def chunk_fwd_varlen(q, k, v, g, beta, scale, cu_seqlens, h0=None, *, out=None, hT=None, final_state=True,
+                     stream=None):
+    """Prefill of a packed batch.  q, k [T_total,H,dk] bf16; v [T_total,H,dv] bf16;
+    g [T_total,H,dk] fp32; beta [T_total,H] fp32; cu_seqlens int32 [N+1] on the
+    device; h0 [N,H,dk,dv] fp32 or None.  Returns (out [T_total,H,dv], hT [N,H,dk,dv]);
+    hT is None when ``final_state`` is False and no ``hT`` buffer was given."""
+    T, H, dk = q.shape
+    dv = v.shape[-1]
+    _check(q, "q", torch.bfloat16, (T, H, dk))
+    _check(k, "k", torch.bfloat16, (T, H, dk))
+    _check(v, "v", torch.bfloat16, (T, H, dv))
+    _check(g, "g", torch.float32, (T, H, dk))
+    _check(beta, "beta", torch.float32, (T, H))
+    if cu_seqlens.dim() != 1 or cu_seqlens.numel() < 2:
+        raise ValueError("cu_seqlens must be a 1-D tensor of N + 1 >= 2 offsets")
+    N = cu_seqlens.numel() - 1
+    _check(cu_seqlens, "cu_seqlens", torch.int32, (N + 1,))
+    if h0 is not None:
+        _check(h0, "h0", torch.float32, (N, H, dk, dv))
+    if out is None:
+        out = torch.empty((T, H, dv), device=q.device, dtype=torch.bfloat16)
+    _check(out, "out", torch.bfloat16, (T, H, dv))
+    if hT is None and final_state:
+        hT = torch.empty((N, H, dk, dv), device=q.device, dtype=torch.float32)
+    if hT is not None:
+        _check(hT, "hT", torch.float32, (N, H, dk, dv))
+    rc = load().kda_chunk_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale),
+                                     _ptr(cu_seqlens), N, _ptr(h0), _ptr(out), _ptr(hT), T, H, dk, dv,
+                                     _stream(stream))
+    if rc != KDA_OK:
+        raise KdaError(rc, "kda_chunk_fwd_varlen")
+    return out, hT
+
+
+def varlen_workspace_bytes(N: int, T_total: int, H: int, dk: int, dv: int) -> int:
+    """Device memory ``chunk_fwd_varlen`` holds for these sizes (0 when unsupported)."""
+    return int(load().kda_chunk_fwd_varlen_workspace_bytes(int(N), int(T_total), int(H), int(dk), int(dv)))
+
+
+def set_record_cap(nbytes: int) -> None:
+    """Test hook: cap the chunk records the prefill workspace holds (0 = default)."""
+    load().kda_chunk_fwd_debug_record_cap(int(nbytes))
 
 
 def decode_step(q, k, v, g, beta, scale, state, *, out=None, stream=None):
@@ -228,7 +336,12 @@ def inject_timeout(polls: int) -> None:
     load().kda_chunk_fwd_debug_inject_timeout(int(polls))
 
 
-KERNEL_KINDS = ("prep", "chain")
+def force_exact(enable: bool) -> None:
+    """Test hook: every prefill chunk takes the exact path (see ``kda.h``)."""
+    load().kda_chunk_fwd_debug_force_exact(1 if enable else 0)
+
+
+KERNEL_KINDS = ("prep", "chain", "exact")
 
 
 def kernel_timing(enable: bool) -> None:

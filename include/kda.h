@@ -35,10 +35,20 @@
  *   and NULL required pointers) without enqueueing work.
  * - Value domain: g <= 0 and finite, beta in [0, 1].  Keys are used as given
  *   (the caller L2-normalises them if the model does).  Results are exact up
- *   to rounding when, for every key channel, the log-decay summed over any
- *   16-token block aligned to a multiple of 16 within the sequence is >= -160;
- *   beyond that the kernel stays finite but the within-block decay factors of
- *   that channel are clamped.
+ *   to rounding for every such g.  A 64-token chunk in which some key channel
+ *   loses more than 80 of log-decay over 8 consecutive tokens (in an aligned
+ *   16-token block: tokens 1..8 or 9..15 of it) takes a slower exact path for
+ *   its intra-chunk terms (about one such chunk in a million at the decays of
+ *   trained models; none in the workloads here).
+ * - Operand range of the prefill.  Three intermediate operands of the tensor
+ *   contractions are fp16 (10-bit mantissa, largest finite value 65504): the
+ *   causal block P (entries bounded by |q_i| |k_j|), the decayed keys
+ *   k * e^{Gamma_C - Gamma} (bounded by |k|), and the corrected values
+ *   v_new = beta (v - (decayed S)^T k)-combinations, bounded by about
+ *   max|v| + |k| max|S column|.  So the prefill needs |q|, |k| <= ~1 (unit
+ *   keys and queries, as the model uses) and |v| and the state's entries well
+ *   below 6.5e4; within that, its relative error does not depend on the scale
+ *   of v and h0 (the method is linear in them).  Decode has no such limit.
  */
 #ifndef KDA_H_
 #define KDA_H_
@@ -144,6 +154,90 @@ KDA_API int kda_gdn_decode_step(const void *q, const void *k, const void *v,
                     int B, int H, int dk, int dv, void *stream);
 
 /*
+ * kda_chunk_fwd_raw, kda_decode_step_raw -- the prefill and the decode step
+ * with the gate prologue fused: they take the raw projections a KDA layer
+ * produces and form the recurrence's inputs themselves, per token and head:
+ *
+ *   g     = -gate_c * softplus(g_raw)      per key channel (so g <= 0)
+ *   beta  = sigmoid(beta_raw)
+ *   q, k  = q_raw / |q_raw|, k_raw / |k_raw|  (L2 over dk, norms floored at
+ *           1e-12; the normalised values are rounded to bf16 as stored inputs)
+ *
+ * gate_c = 1 gives alpha = e^g = sigmoid(-g_raw): the channel-wise sigmoid gate
+ * of the "Kimi Linear" explainer (math.kryvik.com), "Step 2: Per-Channel
+ * Decay", with the sign folded into the projection; the decay is the
+ * fine-grained gate of section 3.2 of "Kimi Linear's Hybrid Linear Attention
+ * Architecture: A Technical Breakdown".  The kernels apply it where they load
+ * g, beta, q and k, so the unfused values never go through memory.
+ *
+ *   q, k, v, g_raw, beta_raw: the layouts and dtypes of kda_chunk_fwd
+ *           (prefill) and kda_decode_step (decode); q and k need not be
+ *           normalised, g_raw and beta_raw are any finite fp32 values
+ *   gate_c: >= 0 and finite, else KDA_ERR_INVALID_ARG
+ *
+ * Everything else (arguments, workspace, errors, value range) is that of
+ * kda_chunk_fwd and kda_decode_step; the results are theirs given the
+ * prologue's values.  Per key channel gates only.
+ */
+KDA_API int kda_chunk_fwd_raw(const void *q, const void *k, const void *v,
+                  const float *g_raw, const float *beta_raw, float gate_c, float scale,
+                  const float *h0, void *out, float *hT,
+                  int B, int T, int H, int dk, int dv, void *stream);
+KDA_API int kda_decode_step_raw(const void *q, const void *k, const void *v,
+                  const float *g_raw, const float *beta_raw, float gate_c, float scale,
+                  float *state, void *out,
+                  int B, int H, int dk, int dv, void *stream);
+
+/*
+ * kda_chunk_fwd_varlen -- chunkwise prefill over a packed batch of N sequences
+ * of different lengths, each with its own initial and final state.  This is
+ * the serving form of the prefill: a batch of requests concatenated along the
+ * token axis, each continuing from its cached recurrent state (the state cache
+ * that takes the place of a KV cache in serving, paragraph on vLLM and LMCache
+ * in "Kimi Linear: How Moonshot AI Built a Hybrid Attention Architecture That
+ * Beats Full Attention").  Per sequence the result is exactly kda_chunk_fwd's.
+ *
+ *   q, k       : bf16 [T_total, H, dk]   the sequences back to back
+ *   v          : bf16 [T_total, H, dv]
+ *   g          : fp32 [T_total, H, dk]
+ *   beta       : fp32 [T_total, H]
+ *   cu_seqlens : int32 [N + 1], DEVICE memory, 4-byte aligned: sequence n
+ *                holds tokens cu_seqlens[n] .. cu_seqlens[n+1] - 1; must
+ *                start at 0, never decrease and end at T_total.  Empty
+ *                sequences are allowed (their hT is their h0).
+ *   h0         : fp32 [N, H, dk, dv] or NULL (zero states)
+ *   out        : bf16 [T_total, H, dv]
+ *   hT         : fp32 [N, H, dk, dv] or NULL; may alias h0
+ *
+ * Every sequence starts a new 64-token chunk, so chunks never mix sequences.
+ * The library checks cu_seqlens on the device (the host never reads it):
+ * offsets are clamped into a non-decreasing sequence within [0, T_total]
+ * before any kernel uses them, so a bad array cannot make a kernel read or
+ * write outside the buffers; the call then computes on the clamped offsets
+ * and kda_stream_status() reports KDA_ERR_INVALID_ARG.  Uses the prefill
+ * workspace (see kda_chunk_fwd_varlen_workspace_bytes); when the records of
+ * all chunks do not fit in it, the chunks run in windows of kernel launches
+ * and a state spanning windows is carried in hT (or in the workspace).
+ * Other arguments, alignment rules and errors as kda_chunk_fwd (N < 1 or a
+ * NULL cu_seqlens: KDA_ERR_INVALID_ARG).
+ */
+KDA_API int kda_chunk_fwd_varlen(const void *q, const void *k, const void *v,
+                  const float *g, const float *beta, float scale,
+                  const int *cu_seqlens, int N,
+                  const float *h0, void *out, float *hT,
+                  int T_total, int H, int dk, int dv, void *stream);
+
+/*
+ * kda_chunk_fwd_varlen_workspace_bytes -- device memory kda_chunk_fwd_varlen
+ * holds for these sizes: counters, the steep-chunk list, the chunk geometry
+ * (2 (N + 1) + T_total / 64 + N + 1 ints) and the records of one window of
+ * chunks of every head (all chunks when they fit in 2 GiB), plus an fp32
+ * state buffer [N, H, dk, dv] when there are several windows.  0 for
+ * unsupported sizes or T_total == 0.
+ */
+KDA_API size_t kda_chunk_fwd_varlen_workspace_bytes(int N, int T_total, int H, int dk, int dv);
+
+/*
  * kda_chunk_fwd_noalloc -- kda_chunk_fwd without any device allocation.  The
  * method itself has no counterpart: this is a deployment variant for callers
  * that cannot allocate device memory at call time (a process whose device
@@ -153,12 +247,13 @@ KDA_API int kda_gdn_decode_step(const void *q, const void *k, const void *v,
  * Same arguments, layouts, results and error codes as kda_chunk_fwd; the
  * outputs are bit-identical to it.  The chunk records live in a fixed 64 MiB
  * array per device that is part of the library's module image, so a long
- * sequence runs in several segments of two kernel launches each.  Limit: the
- * records of one 64-token chunk of every (b, h) (B * H * 74,240 bytes), plus,
- * when hT is NULL, the fp32 state [B, H, dk, dv] carried between segments,
- * must fit in 64 MiB (B * H <= 903 with hT given); a larger problem returns
- * KDA_ERR_SCRATCH_LIMIT without enqueueing work.  The only part of the
- * scratch that must start at zero, an item counter, is cleared by each call.
+ * sequence runs in several segments of a few kernel launches each.  Limit:
+ * the records of one 64-token chunk of every (b, h) with their list entries
+ * (B * H * 74,244 bytes), plus, when hT is NULL, the fp32 state [B, H, dk, dv]
+ * carried between segments, must fit in 64 MiB (B * H <= 903 with hT given,
+ * B * H <= 480 without, at dk = dv = 128); a larger problem returns
+ * KDA_ERR_SCRATCH_LIMIT without enqueueing work.  The only parts of the
+ * scratch that must start at zero, two counters, are cleared by each call.
  *
  * The first call on a device looks up the array's device address (with that
  * device current) and caches it: make that first call before any stream
@@ -220,6 +315,24 @@ KDA_API void kda_chunk_fwd_debug_wait_limit(unsigned long long polls);
 KDA_API void kda_chunk_fwd_debug_inject_timeout(unsigned long long polls);
 
 /*
+ * kda_chunk_fwd_debug_force_exact -- test hook.  While enabled (enable != 0),
+ * every chunk of every prefill launched afterwards takes the exact path that
+ * otherwise only chunks with extreme decay take (see "Value domain" above), so
+ * a test can compare the two paths on the same inputs.  Process-wide; off by
+ * default.
+ */
+KDA_API void kda_chunk_fwd_debug_force_exact(int enable);
+
+/*
+ * kda_chunk_fwd_debug_record_cap -- test hook.  Caps the bytes of chunk
+ * records the prefill workspace holds at once (0 restores the default,
+ * 2 GiB), so that small problems exercise the paths long ones take: segments
+ * on two streams (kda_chunk_fwd) and windows (kda_chunk_fwd_varlen).
+ * Applies to calls made afterwards; process-wide.
+ */
+KDA_API void kda_chunk_fwd_debug_record_cap(unsigned long long bytes);
+
+/*
  * kda_debug_kernel_timing -- measurement hook.  While enabled (enable != 0),
  * every kda_chunk_fwd records a pair of CUDA events on its stream around each
  * kernel it launches (kind 0 = the per-chunk prep kernel, kind 1 = the state
@@ -233,7 +346,9 @@ KDA_API void kda_chunk_fwd_debug_inject_timeout(unsigned long long polls);
 KDA_API void kda_debug_kernel_timing(int enable);
 KDA_API int kda_debug_kernel_times(double *ms, long long *launches, int nkinds);
 
-/* Version of this ABI (major * 100 + minor): 101 adds the scalar-gate entry points. */
+/* Version of this ABI (major * 100 + minor): 101 adds the scalar-gate entry
+ * points, 102 the packed-batch prefill, the raw-input (fused gate prologue)
+ * entry points and the exact-path test hooks. */
 KDA_API int kda_abi_version(void);
 
 #ifdef __cplusplus

@@ -11,3 +11,18 @@ if HERE not in sys.path:
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
+
+
+def pytest_sessionfinish(session, exitstatus):
+    """Write the parity margins recorded by kda_testlib.assert_close when
+    KDA_PARITY_LOG names a file."""
+    path = os.environ.get("KDA_PARITY_LOG")
+    if not path:
+        return
+    try:
+        import kda_testlib
+    except ImportError:
+        return
+    import json
+    with open(path, "w") as f:
+        json.dump(kda_testlib.PARITY_LOG, f, indent=1)

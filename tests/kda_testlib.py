@@ -28,8 +28,15 @@ def max_abs(x, ref):
     return float(np.max(np.abs(x - ref))) if x.size else 0.0
 
 
+# Every comparison made by assert_close, in order: (what, rel-L2, max-abs, rel tol,
+# max-abs tol).  conftest.py writes them to $KDA_PARITY_LOG (JSON) at the end of
+# the session, so the precision margin of each check can be read off a run.
+PARITY_LOG = []
+
+
 def assert_close(x, ref, what, rel=REL_L2_TOL, mabs=MAX_ABS_TOL):
     r, m = rel_l2(x, ref), max_abs(x, ref)
+    PARITY_LOG.append({"what": what, "rel_l2": r, "max_abs": m, "rel_tol": rel, "max_abs_tol": mabs})
     assert np.all(np.isfinite(np.asarray(x, np.float64))), f"{what}: non-finite values"
     assert r <= rel and m <= mabs, f"{what}: rel-L2 {r:.3e} (tol {rel:.1e}), max-abs {m:.3e} (tol {mabs:.1e})"
     return r, m

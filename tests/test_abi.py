@@ -33,7 +33,7 @@ def test_header_declares_the_boundary():
 def test_library_exports_every_declared_symbol(lib):
     for name in declared_symbols():
         assert hasattr(lib, name), name
-    assert lib.kda_abi_version() == 101
+    assert lib.kda_abi_version() == 102
 
 
 def test_status_strings(lib):
@@ -101,14 +101,18 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
 
 def test_workspace_bytes(lib):
     rec = 74240  # bytes of one chunk record of one (b, h)
-    tick = 256   # the prep kernel's item counters
+    tick = 256   # the prep kernel's item and steep-item counters
+
+    def lst(items):  # the list of steep items: one int per item of a segment, 256-byte rounded
+        return (4 * items + 255) // 256 * 256
+
     # one segment: all chunks' records, no state buffer
-    assert kda.workspace_bytes(1, 256, 1, 128, 128) == tick + 4 * rec
-    assert kda.workspace_bytes(2, 65, 3, 64, 64) == tick + 2 * 6 * rec
+    assert kda.workspace_bytes(1, 256, 1, 128, 128) == tick + lst(4) + 4 * rec
+    assert kda.workspace_bytes(2, 65, 3, 64, 64) == tick + lst(12) + 2 * 6 * rec
     # long sequence: two buffers of as many chunks as fit in 1 GiB each, plus the carried state
     row = 32 * rec
     seg = (1 << 30) // row
-    assert kda.workspace_bytes(1, 1 << 20, 32, 128, 128) == tick + 2 * seg * row + 32 * 128 * 128 * 4
+    assert kda.workspace_bytes(1, 1 << 20, 32, 128, 128) == tick + lst(32 * seg) + 2 * seg * row + 32 * 128 * 128 * 4
     # unsupported or empty
     assert kda.workspace_bytes(1, 0, 1, 128, 128) == 0
     assert kda.workspace_bytes(1, 64, 1, 96, 128) == 0
@@ -170,3 +174,56 @@ def test_gate_alignment_rule_differs_by_form(lib):
     # (T == 0, no h0/hT: validation only, nothing enqueued); the per-channel gate needs 16
     assert gdn_chunk(lib, g=FOUR, T=0) == kda.KDA_OK
     assert chunk(lib, g=FOUR, T=0) == kda.KDA_ERR_ALIGNMENT
+
+
+def varlen(lib, q=A, k=A, v=A, g=A, beta=A, cu=A, N=2, h0=None, out=A, hT=None, T=100, H=1, dk=64, dv=64):
+    return lib.kda_chunk_fwd_varlen(q, k, v, g, beta, 1.0, cu, N, h0, out, hT, T, H, dk, dv, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(cu=None), kda.KDA_ERR_INVALID_ARG),
+    (dict(N=0), kda.KDA_ERR_INVALID_ARG),
+    (dict(q=None), kda.KDA_ERR_INVALID_ARG),
+    (dict(T=-1), kda.KDA_ERR_INVALID_ARG),
+    (dict(H=0), kda.KDA_ERR_INVALID_ARG),
+    (dict(dk=96), kda.KDA_ERR_UNSUPPORTED),
+    (dict(cu=ODD), kda.KDA_ERR_ALIGNMENT),
+    (dict(g=MIS), kda.KDA_ERR_ALIGNMENT),
+    (dict(hT=MIS), kda.KDA_ERR_ALIGNMENT),
+])
+def test_varlen_rejects(lib, kw, code):
+    assert varlen(lib, **kw) == code
+
+
+def test_varlen_zero_tokens_accepts_null_inputs(lib):
+    # T_total == 0 with no h0/hT: every sequence is empty, nothing to read or write
+    assert varlen(lib, q=None, k=None, v=None, g=None, beta=None, out=None, T=0) == kda.KDA_OK
+
+
+def test_varlen_workspace_bytes(lib):
+    rec, tick = 74240, 256
+
+    def r256(x):
+        return (x + 255) // 256 * 256
+
+    N, T, H = 3, 1000, 4
+    cmax = T // 64 + N + 1  # chunks: at most one partial chunk per sequence
+    assert kda.varlen_workspace_bytes(N, T, H, 128, 128) == \
+        tick + r256(4 * H * cmax) + r256(4 * (2 * (N + 1) + cmax)) + cmax * H * rec
+    assert kda.varlen_workspace_bytes(N, 0, H, 128, 128) == 0
+    assert kda.varlen_workspace_bytes(0, 10, H, 128, 128) == 0
+
+
+def test_raw_entry_points_validate_gate_scale(lib):
+    def raw(c, **kw):
+        a = dict(q=A, k=A, v=A, g=A, beta=A, h0=None, out=A, hT=None, B=1, T=64, H=1, dk=64, dv=64)
+        a.update(kw)
+        return lib.kda_chunk_fwd_raw(a["q"], a["k"], a["v"], a["g"], a["beta"], c, 1.0, a["h0"], a["out"], a["hT"],
+                                     a["B"], a["T"], a["H"], a["dk"], a["dv"], None)
+    assert raw(-0.5) == kda.KDA_ERR_INVALID_ARG
+    assert raw(float("nan")) == kda.KDA_ERR_INVALID_ARG
+    assert raw(0.5, q=None) == kda.KDA_ERR_INVALID_ARG
+    assert raw(0.5, dk=96) == kda.KDA_ERR_UNSUPPORTED
+    assert raw(0.5, k=MIS) == kda.KDA_ERR_ALIGNMENT
+    assert lib.kda_decode_step_raw(A, A, A, A, A, -1.0, 1.0, A, A, 1, 1, 64, 64, None) == kda.KDA_ERR_INVALID_ARG
+    assert lib.kda_decode_step_raw(A, A, A, A, A, 1.0, 1.0, None, A, 1, 1, 64, 64, None) == kda.KDA_ERR_INVALID_ARG

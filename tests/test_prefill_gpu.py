@@ -15,9 +15,11 @@ DEV = "cuda:0"
 def _reset_hooks():
     kda.inject_timeout(0)
     kda.set_wait_limit(0)
+    kda.force_exact(False)
     yield
     kda.inject_timeout(0)
     kda.set_wait_limit(0)
+    kda.force_exact(False)
     assert kda.stream_status() == kda.KDA_OK
 
 
@@ -182,3 +184,89 @@ def test_long_context_sampled():
     assert_close(f64(out[:, :65536, 0:2]), o_ref, "long-context out (heads 0-1, 64k tokens)")
     _, s_ref = oracle_prefill(d, cfg.scale, heads=slice(0, 1))
     assert_close(f64(hT[:, 0:1]), s_ref, "long-context hT (head 0)")
+
+
+def steep_gate(d, pattern):
+    """Decays far beyond the workloads': every chunk (constant -12), isolated
+    spikes (-30 on every 7th token), or one burst of four -25 tokens inside the
+    second half of a 16-token block (one steep chunk among ordinary ones)."""
+    g = d["g"]
+    if pattern == "const_m12":
+        g.fill_(-12.0)
+    elif pattern == "every7_m30":
+        g[:, 6::7] = -30.0
+    elif pattern == "burst_m25":
+        g[:, 41:45] = -25.0
+    return d
+
+
+@pytest.mark.parametrize("gate", ["per_channel", "scalar"])
+@pytest.mark.parametrize("pattern", ["const_m12", "every7_m30", "burst_m25"])
+@pytest.mark.parametrize("T", [64, 1000])
+def test_steep_decay(T, pattern, gate):
+    """Any finite g <= 0: chunks whose decay would push a split factor past e^80
+    take the exact path; the result must match the oracle either way, on both
+    gate forms (the scalar gate is channel 0 of the gate, broadcast for the oracle)."""
+    d = steep_gate(inputs.make_prefill(1, T, 2, 128, 128, decay=0.05, h0_std=0.02, seed=500 + T, device=DEV),
+                   pattern)
+    scale = 128 ** -0.5
+    if gate == "scalar":
+        gs = d["g"][..., 0].contiguous()
+        d["g"] = gs.unsqueeze(-1).expand_as(d["g"]).contiguous()
+        out, hT = kda.gdn_chunk_fwd(d["q"], d["k"], d["v"], gs, d["beta"], scale, d["h0"])
+    else:
+        out, hT = kda.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], scale, d["h0"])
+    torch.cuda.synchronize()
+    o_ref, s_ref = oracle_prefill(d, scale)
+    assert_close(f64(out), o_ref, f"{pattern} T={T} {gate} out")
+    assert_close(f64(hT), s_ref, f"{pattern} T={T} {gate} hT")
+
+
+@pytest.mark.parametrize("dk,dv", [(64, 64), (128, 128)])
+def test_exact_path_matches_fast_path(dk, dv):
+    """The exact path (forced on every chunk) and the tensor-core path agree with
+    the oracle and with each other on ordinary inputs."""
+    d = inputs.make_prefill(2, 300, 2, dk, dv, decay=0.1, h0_std=0.02, seed=600 + dk, device=DEV)
+    fast_o, fast_s = check(d, dk ** -0.5, f"fast path dk={dk}")
+    kda.force_exact(True)
+    ex_o, ex_s = check(d, dk ** -0.5, f"exact path dk={dk}")
+    kda.force_exact(False)
+    assert_close(f64(ex_o), f64(fast_o), "exact vs fast out")
+    assert_close(f64(ex_s), f64(fast_s), "exact vs fast hT")
+
+
+def test_large_values_and_state():
+    """|v| ~ 100 and h0 ~ N(0, 1): the fp16 operands (P, decayed keys, corrected
+    values) stay in range.  The method is linear in (v, h0), so this is the base
+    problem scaled by ~100: rel-L2 keeps its bar and the max-abs bar scales by 100."""
+    d = inputs.make_prefill(2, 1000, 2, 128, 128, decay=0.05, h0_std=1.0, seed=700, device=DEV)
+    d["v"] = (d["v"].float() * 100.0).to(torch.bfloat16)
+    out, hT = run(d, 128 ** -0.5)
+    o_ref, s_ref = oracle_prefill(d, 128 ** -0.5)
+    assert_close(f64(out), o_ref, "|v|~100 out", mabs=100 * 2e-2)
+    assert_close(f64(hT), s_ref, "|v|~100 hT", mabs=100 * 2e-2)
+
+
+@pytest.mark.parametrize("pieces", [(16,), (32,), (1, 17, 50, 64, 23)])
+def test_chunk_boundaries_do_not_matter(pieces):
+    """The chunkwise form equals the recurrence whatever the blocking.  Feeding the
+    same sequence through chunk_fwd in pieces (state carried through hT -> h0) puts
+    the chunk boundaries every 16 or 32 tokens (chunk sizes 16 and 32 of the same
+    kernels: each call holds one partial chunk) or at irregular offsets; all must
+    match one whole-sequence call (chunk size 64) and the oracle."""
+    T = 448
+    d = inputs.make_prefill(1, T, 2, 128, 128, decay=0.1, h0_std=0.02, seed=800, device=DEV)
+    whole_o, whole_s = check(d, 0.2, "whole sequence")
+    outs, state, t0, n = [], d["h0"], 0, 0
+    while t0 < T:
+        L = min(pieces[n % len(pieces)], T - t0)
+        part = {k: (v[:, t0:t0 + L].contiguous() if k != "h0" else state) for k, v in d.items()}
+        o, state = run(part, 0.2)
+        outs.append(o)
+        t0, n = t0 + L, n + 1
+    o_ref, s_ref = oracle_prefill(d, 0.2)
+    pieced = torch.cat(outs, dim=1)
+    assert_close(f64(pieced), o_ref, f"pieces {pieces} out")
+    assert_close(f64(state), s_ref, f"pieces {pieces} hT")
+    assert_close(f64(pieced), f64(whole_o), f"pieces {pieces} vs whole out")
+    assert_close(f64(state), f64(whole_s), f"pieces {pieces} vs whole hT")

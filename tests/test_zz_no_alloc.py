@@ -53,6 +53,29 @@ def test_noalloc_matches_chunk_fwd_twice(B, T, H, dk, dv, with_hT):
             assert torch.equal(hT, ref_hT)
 
 
+def test_noalloc_allocates_nothing():
+    """With the prefill workspace released, a warmed-up kda_chunk_fwd_noalloc call
+    must leave the device's free memory unchanged: no cudaMalloc of a workspace
+    (which would be at least the 64 MiB of records this problem needs), nothing
+    else either."""
+    lib = kda.load()
+    dev = torch.device("cuda", 0)
+    d = inputs.make_prefill(2, 1000, 64, 128, 128, decay=0.05, h0_std=0.02, seed=12, device=dev)
+    out = torch.empty((2, 1000, 64, 128), dtype=torch.bfloat16, device=dev)
+    hT = torch.empty((2, 64, 128, 128), dtype=torch.float32, device=dev)
+    assert _noalloc(lib, d, 128 ** -0.5, out, hT) == kda.KDA_OK  # first call: symbol lookup, lazy loading
+    torch.cuda.synchronize()
+    kda.release_workspace()
+    assert kda.workspace_bytes(2, 1000, 64, 128, 128) >= 64 << 20
+    free0, _ = torch.cuda.mem_get_info(dev)
+    for _ in range(2):
+        assert _noalloc(lib, d, 128 ** -0.5, out, hT) == kda.KDA_OK
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info(dev)
+    assert kda.stream_status() == kda.KDA_OK
+    assert free1 == free0, f"free device memory changed by {free0 - free1} bytes"
+
+
 def test_noalloc_zero_length_and_limit():
     lib = kda.load()
     dev = torch.device("cuda", 0)
