@@ -18,11 +18,15 @@ Also measured and reported in the same line:
            512 MiB fp32 state (GB/s of algorithmic traffic);
   e2e      the same prefill metric through the public API with pinned host
            buffers: H2D of the inputs, the kernel, D2H of out and hT per step;
-  roofline achieved algorithmic GB/s of the prefill call (its two kernels) vs
-           measured HBM peak, with each kernel's device time from one extra
-           instrumented step (CUDA events around every launch, on its stream);
+  roofline achieved algorithmic GB/s of the prefill call (its kernels) vs
+           measured HBM peak, with each kernel's busy time from one extra step
+           whose launches the kernels stamp themselves (%globaltimer);
+  training the training-shape prefill (B8 H32 T4096) timed the same way;
   cpu_baseline  the fp64 oracle on a bounded sample of the workload (rank 0,
-           N = 1 only).
+           N = 1 only), plus every workload's recipe on 1 thread and all cores.
+
+--record-traffic CSV writes profiles/traffic.json from an ncu capture of the
+DRAM-bytes counters (taken on --workload) and exits.
 
 --impl reference times the fp64 oracle (the only reference that exists for
 this method) on the host cores, on bounded samples of the same workload.
@@ -136,18 +140,90 @@ def kernel_source_hash():
     return h.hexdigest()[:16]
 
 
-def measured_traffic(kernel):
-    """Per-launch DRAM bytes from the committed ncu summary, if it was taken on
-    the current kernel sources (else None)."""
+REC_BYTES = 74240            # one chunk record of one (b, h)
+RECORD_CAP = 2 << 30         # bytes of records the prefill workspace holds at once
+TRAFFIC_KERNELS = ("prep_kernel", "chain_kernel", "exact_prep_kernel", "decode_step_kernel")
+
+
+def prep_launch_token_heads(B, T, H):
+    """Token-heads (and chunks) of each prep/chain launch of kda_chunk_fwd on
+    [B, T, H] (the library's segmentation: all chunks when their records fit the
+    cap, else segments of as many chunks as fit in half of it)."""
+    nch = -(-T // CHUNK)
+    row = B * H * REC_BYTES
+    seg = nch if nch * row <= RECORD_CAP else max(1, RECORD_CAP // (2 * row))
+    out = []
+    for n0 in range(0, nch, seg):
+        cnt = min(seg, nch - n0)
+        out.append(B * H * min(cnt * CHUNK, T - n0 * CHUNK))
+    return out
+
+
+def record_traffic(csv_path, workload, out_path=None):
+    """Turn an ncu --csv log of dram__bytes_read.sum / dram__bytes_write.sum
+    (one or more kernels, each launch complete) into profiles/traffic.json, keyed
+    to the current kernel sources.  Per kernel: the mean bytes per launch and, for
+    the prefill kernels, per token-head of the captured launches (the launches are
+    in issue order, so the n-th prep or chain launch is segment n)."""
+    import csv
+
+    from gated_delta_rule_100_b200 import inputs
+
+    launches = {}  # launch id -> (kernel, bytes)
+    order = []
+    with open(csv_path) as f:
+        rows = [r for r in csv.reader(f) if r and not r[0].startswith("==")]
+    head = rows[0]
+    idx = {k: head.index(k) for k in ("ID", "Kernel Name", "Metric Name", "Metric Unit", "Metric Value")}
+    scale_of = {"byte": 1.0, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9, "KB": 1e3, "MB": 1e6, "GB": 1e9}
+    for r in rows[1:]:
+        if r[idx["Metric Name"]] not in ("dram__bytes_read.sum", "dram__bytes_write.sum"):
+            continue
+        lid = r[idx["ID"]]
+        name = next((k for k in TRAFFIC_KERNELS if k in r[idx["Kernel Name"]]), None)
+        if name is None:
+            continue
+        val = float(r[idx["Metric Value"]].replace(",", "")) * scale_of.get(r[idx["Metric Unit"]], 1.0)
+        if lid not in launches:
+            launches[lid] = [name, 0.0]
+            order.append(lid)
+        launches[lid][1] += val
+    cfg = inputs.CONFIGS.get(workload)
+    per_launch_th = prep_launch_token_heads(cfg.B, cfg.T, cfg.H) if cfg is not None else []
+    kernels = {}
+    for name in TRAFFIC_KERNELS:
+        ids = [i for i in order if launches[i][0] == name]
+        if not ids:
+            continue
+        e = {"launches_captured": len(ids), "bytes_per_launch": [launches[i][1] for i in ids]}
+        e["mean_bytes_per_launch"] = sum(e["bytes_per_launch"]) / len(ids)
+        if name in ("prep_kernel", "chain_kernel") and per_launch_th:
+            th = [per_launch_th[n % len(per_launch_th)] for n in range(len(ids))]
+            e["bytes_per_token_head"] = sum(e["bytes_per_launch"]) / sum(th)
+        kernels[name] = e
+    t = {"source_hash": kernel_source_hash(), "captured_on": workload, "kernels": kernels,
+         "source_key": "sha256 of the csrc .cu/.cuh files with comments removed and whitespace collapsed"}
+    out_path = out_path or os.path.join(ROOT, "profiles", "traffic.json")
+    with open(out_path, "w") as f:
+        json.dump(t, f, indent=1)
+    return t
+
+
+def measured_traffic(kernel, field="mean_bytes_per_launch"):
+    """A kernel's DRAM-traffic figure from profiles/traffic.json, if that capture
+    was taken on the current kernel sources (else None), with the workload it was
+    captured on."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
-        return None
+        return None, None
     with open(path) as f:
         t = json.load(f)
-    e = t.get(kernel)
-    if not e or e.get("source_hash") != kernel_source_hash():
-        return None
-    return e.get("bytes_per_launch_full_workload")
+    if t.get("source_hash") != kernel_source_hash():
+        return None, None
+    e = t.get("kernels", {}).get(kernel)
+    if not e or field not in e:
+        return None, None
+    return e[field], t.get("captured_on")
 
 
 class ClockSampler:
@@ -270,6 +346,109 @@ def cpu_baseline(d, cfg, budget_s):
                       f"({n} token-heads, {dt:.1f} s, {heads} threads); tokens/s = token-heads/s / {cfg.H}"}
 
 
+def measure_training(P, peak_src, stream, steps, warmup, dev):
+    """The training-shape prefill (B8 H32 T4096 d128, 1.65 GB of inputs: above L2,
+    no flush) through kda_chunk_fwd, timed like the step, with its own roofline."""
+    import torch
+
+    from gated_delta_rule_100_b200 import inputs, kda
+
+    cfg = inputs.CONFIGS["training_B8_H32_T4096_d128"]
+    d = inputs.make_config(cfg, device=dev)
+    out = torch.empty((cfg.B, cfg.T, cfg.H, cfg.dv), dtype=torch.bfloat16, device=dev)
+    hT = torch.empty((cfg.B, cfg.H, cfg.dk, cfg.dv), dtype=torch.float32, device=dev)
+
+    def step():
+        kda.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], cfg.scale, d["h0"], out=out, hT=hT,
+                      stream=stream)
+
+    for _ in range(max(3, warmup)):
+        step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if kda.stream_status(stream) != kda.KDA_OK:
+        raise RuntimeError("device-side error in the training-shape steps")
+    ms = e0.elapsed_time(e1) / steps
+    kda.kernel_times()
+    kda.kernel_timing(True)
+    step()
+    torch.cuda.synchronize()
+    kda.kernel_timing(False)
+    kt = kda.kernel_times()
+    nbytes = prefill_bytes(cfg.B, cfg.T, cfg.H, cfg.dk, cfg.dv, cfg.h0_std > 0, True)
+    nflops = prefill_flops(cfg.B, cfg.T, cfg.H, cfg.dk, cfg.dv)
+    achieved = nbytes / (ms / 1e3) / 1e9
+    return {"metric": "training-shape prefill tokens/s", "value": cfg.B * cfg.T / (ms / 1e3), "unit": "tokens/s",
+            "ms_per_step": ms, "steps": steps, "tflops": nflops / (ms / 1e3) / 1e12,
+            "config": {"workload": cfg.name, "B": cfg.B, "H": cfg.H, "T": cfg.T, "dk": cfg.dk, "dv": cfg.dv,
+                       "l2": "inputs 1.65 GB, larger than L2; no flush"},
+            "kernels": {k: {"ms": t, "launches": n} for k, (t, n) in kt.items() if n > 0},
+            "roofline": {"kernel": "kda_chunk_fwd (prep_kernel + chain_kernel)", "bound": "hbm",
+                         "achieved": achieved, "peak": P["hbm_gbs"], "unit": "GB/s",
+                         "frac": achieved / P["hbm_gbs"], "peak_source": peak_src,
+                         "algorithmic_bytes_per_launch": nbytes,
+                         "tensor_view": {"achieved_tflops": nflops / (ms / 1e3) / 1e12,
+                                         "peak_tflops": P["bf16_tflops_sustained"],
+                                         "frac": nflops / (ms / 1e3) / 1e12 / P["bf16_tflops_sustained"]}}}
+
+
+def cpu_baseline_table(budget_s=3.0):
+    """The fp64 oracle on each workload's recipe, on 1 thread and on all host
+    cores: the first two workloads in full, the training shape and the decode
+    workload on samples sized to about `budget_s` each.  Prefill in tokens/s of
+    the full workload's head count (token-heads/s / H), decode in GB/s of the
+    decode step's algorithmic traffic."""
+    import numpy as np
+
+    import oracle
+    from gated_delta_rule_100_b200 import inputs
+
+    cores = os.cpu_count() or 1
+    rows = []
+
+    def f64(t):
+        return t.to("cpu", dtype=__import__("torch").float64).numpy()
+
+    for name in ("oracle_scale_B1_H1_T256_d64", "prefill_B1_H4_T2048_d128", "training_B8_H32_T4096_d128"):
+        cfg = inputs.CONFIGS[name]
+        for threads in (1, cores):
+            full = name != "training_B8_H32_T4096_d128"
+            heads = cfg.H if full else min(cfg.H, max(1, threads))
+            T = cfg.T
+            d = inputs.make_prefill(1 if not full else cfg.B, T, heads, cfg.dk, cfg.dv, decay=cfg.decay,
+                                    h0_std=cfg.h0_std, seed=cfg.seed)
+            t0 = time.perf_counter()
+            oracle.kda_fwd(*(f64(d[k]) for k in ("q", "k", "v", "g", "beta")), cfg.scale,
+                           None if d["h0"] is None else f64(d["h0"]), threads=threads)
+            dt = time.perf_counter() - t0
+            th = d["q"].shape[0] * T * heads
+            rows.append({"workload": name, "threads": threads, "seconds": dt,
+                         "sample": "full" if full else f"{heads} heads x {T} tokens (batch 1)",
+                         "tokens_per_s": th / dt / cfg.H})
+    dcfg = inputs.DECODE_CONFIG
+    for threads in (1, cores):
+        nbh = min(dcfg.B, 8 * max(1, threads))  # sequences of the sample (all heads of each)
+        d = inputs.make_decode(nbh, dcfg.H, dcfg.dk, dcfg.dv, decay=dcfg.decay, state_std=dcfg.state_std,
+                               steps=8, seed=dcfg.seed)
+        S = f64(d["state"])
+        t0 = time.perf_counter()
+        for s_ in range(8):
+            _, S = oracle.kda_decode_step(*(f64(d[k][s_]) for k in ("q", "k", "v", "g", "beta")), dcfg.scale, S,
+                                          threads=threads)
+        dt = time.perf_counter() - t0
+        gbs = decode_bytes(nbh, dcfg.H, dcfg.dk, dcfg.dv) * 8 / dt / 1e9
+        rows.append({"workload": dcfg.name, "threads": threads, "seconds": dt,
+                     "sample": f"{nbh} of {dcfg.B} sequences x {dcfg.H} heads x 8 steps", "state_gbs": gbs})
+    del np
+    return {"kind": "oracle", "cores": cores, "rows": rows,
+            "note": "fp64 oracle; OpenMP over (b, h), so a workload with fewer (b, h) than threads uses fewer"}
+
+
 # -------------------------------------------------------------------- arms ----
 def run_reference(args):
     """The fp64 oracle on the host cores (rank 0 only)."""
@@ -350,8 +529,7 @@ def run_ours(args):
         raise RuntimeError("device-side error in the timed region")
     launch_ms = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
     # Per-kernel split and launch count: one more step, outside the timed region,
-    # with each kernel launch bracketed by CUDA events on its stream (the events
-    # slow the two-stream step, so they stay out of the timed steps).
+    # with every launch's busy interval stamped by its own CTAs (%globaltimer).
     kda.kernel_times()
     kda.kernel_timing(True)
     step()
@@ -368,15 +546,22 @@ def run_ours(args):
     nflops = prefill_flops(cfg.B, cfg.T, cfg.H, cfg.dk, cfg.dv)
     avg_launch_s = statistics.mean(launch_ms) / 1e3
     achieved = nbytes / avg_launch_s / 1e9
-    kernel_ms = sum(t for t, _ in ktimes.values())
-    kernels = {k: {"ms_per_step": t, "launches_per_step": n, "share": t / kernel_ms if kernel_ms > 0 else None}
-               for k, (t, n) in ktimes.items()}
-    kernels["note"] = ("device time summed per kernel over one instrumented step; the two kernels overlap "
-                       "on two streams when the sequence spans several segments")
+    kernels = {k: {"ms_per_step": t, "launches_per_step": n, "busy_fraction_of_step": t / ms_per_step}
+               for k, (t, n) in ktimes.items() if n > 0}
+    kernels["note"] = ("per kind: the launches' busy intervals (first CTA start to last CTA end, stamped by the "
+                       "kernels) summed over one extra step; prep and chain launches overlap on two streams")
     gpu_launches = sum(n for _, n in ktimes.values()) * args.steps
+    th_step = cfg.B * cfg.T * cfg.H
+    bpth = [measured_traffic(k, "bytes_per_token_head") for k in ("prep_kernel", "chain_kernel")]
+    traffic = traffic_note = None
+    if all(b is not None for b, _ in bpth):
+        traffic = sum(b for b, _ in bpth) * th_step
+        traffic_note = (f"DRAM bytes of prep_kernel + chain_kernel per token-head, captured by ncu on "
+                        f"{bpth[0][1]} (the same segmented two-stream code path), times this workload's "
+                        f"token-heads: a scaled estimate, not a capture of this workload")
     roof = {"kernel": "kda_chunk_fwd (prep_kernel + chain_kernel)", "bound": "hbm", "achieved": achieved,
             "peak": P["hbm_gbs"], "unit": "GB/s", "frac": achieved / P["hbm_gbs"], "peak_source": peak_src,
-            "traffic": measured_traffic("kda_chunk_fwd"),
+            "traffic": traffic, "traffic_note": traffic_note,
             "algorithmic_bytes_per_launch": nbytes, "kernels": kernels,
             "tensor_view": {"achieved_tflops": nflops / avg_launch_s / 1e12,
                             "peak_tflops": P["bf16_tflops_sustained"],
@@ -389,6 +574,14 @@ def run_ours(args):
             gdn = measure_scalar_gate(d, cfg, out, hT, stream, args.steps, args.warmup, P)
         except Exception as exc:  # noqa: BLE001 - an extra item must not cost the measurement above
             gdn = {"error": f"{type(exc).__name__}: {exc}"[:300]}
+
+    # ---------------- training shape (after the timed steps; never fails the line) ----------------
+    training = None
+    if not args.no_training:
+        try:
+            training = measure_training(P, peak_src, stream, args.steps, args.warmup, dev)
+        except Exception as exc:  # noqa: BLE001 - an extra item must not cost the measurement above
+            training = {"error": f"{type(exc).__name__}: {exc}"[:300]}
 
     # ---------------- decode ----------------
     dec = None
@@ -419,7 +612,10 @@ def run_ours(args):
                "gpu_launches": dcfg.steps,
                "roofline": {"kernel": "decode_step_kernel", "bound": "hbm", "achieved": gbs,
                             "peak": P["hbm_gbs"], "unit": "GB/s", "frac": gbs / P["hbm_gbs"],
-                            "peak_source": peak_src, "traffic": measured_traffic("decode_step_kernel"),
+                            "peak_source": peak_src,
+                            "traffic": measured_traffic("decode_step_kernel")[0],
+                            "traffic_note": "ncu dram__bytes_read.sum + dram__bytes_write.sum per launch, "
+                                            "captured on this workload",
                             "algorithmic_bytes_per_launch": db}}
         del dd, state
 
@@ -456,6 +652,10 @@ def run_ours(args):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(d, cfg, args.cpu_seconds)
+        try:
+            cpu["per_workload"] = cpu_baseline_table()
+        except Exception as exc:  # noqa: BLE001
+            cpu["per_workload"] = {"error": f"{type(exc).__name__}: {exc}"[:300]}
 
     if rank == 0:
         line = {
@@ -468,7 +668,8 @@ def run_ours(args):
                        "l2": "inputs larger than L2 (51.7 GB per step); no flush",
                        "parallelism": f"weak: one workload copy per GPU x{world}"},
             "tflops": nflops / (ms_per_step / 1e3) / 1e12 * world,
-            "roofline": roof, "decode": dec, "scalar_gate": gdn, "e2e": e2e, "cpu_baseline": cpu,
+            "roofline": roof, "decode": dec, "scalar_gate": gdn, "training": training, "e2e": e2e,
+            "cpu_baseline": cpu,
             "clocks": clk.summary(), "gpu_launches": gpu_launches,
             "launch_ms": {"mean": statistics.mean(launch_ms), "min": min(launch_ms), "max": max(launch_ms)},
         }
@@ -489,9 +690,15 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-gdn", action="store_true", help="skip the scalar-gate prefill line")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-training", action="store_true", help="skip the training-shape prefill line")
+    ap.add_argument("--record-traffic", metavar="CSV",
+                    help="write profiles/traffic.json from an ncu dram-bytes CSV and exit")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     args = ap.parse_args()
+    if args.record_traffic:
+        print(json.dumps(record_traffic(args.record_traffic, args.workload), indent=1))
+        return 0
     args.warmup = max(3, args.warmup)  # at least three untimed warm-up steps
     return run_reference(args) if args.impl == "reference" else run_ours(args)
 

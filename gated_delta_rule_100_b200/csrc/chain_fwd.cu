@@ -157,6 +157,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
     const uint64_t polls = prm.st.wait_polls;
 
     if (tid == 0) {
+        stamp_start(prm.stamp);
         for (int i = 0; i < NBARS; ++i) {
             const bool group = i >= B_S0 && i <= B_KE1;
             const bool all16 = i == B_S0 || i == B_VT || i == B_KE0 || i == B_KE1;
@@ -487,6 +488,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
     __syncthreads();
     tc_fence_after();
     if (warp == 0) tmem_dealloc(tmem, L::TM_COLS);
+    if (tid == 0) stamp_end(prm.stamp);
 }
 
 template <int DK, int VS>

@@ -135,6 +135,7 @@ struct PrepParams {
     int H;
     SeqGeom gm;
     DeviceStatus st;
+    unsigned long long *stamp;  // measurement hook: this launch's timing slot, or NULL
 };
 
 // The exact kernel (exact_prep.cu): rewrites P, T' and W of the listed items.
@@ -149,6 +150,7 @@ struct ExactParams {
     float gate_c;
     int H;
     SeqGeom gm;
+    unsigned long long *stamp;
 };
 
 // One CTA per (sequence, head, part, slot); walks its chunks of the launch in order.
@@ -180,6 +182,7 @@ struct ChainParams {
     SeqGeom gm;
     DeviceStatus st;
     uint64_t inject_wait_polls;  // test hook: nonzero = first wait on a barrier nothing signals
+    unsigned long long *stamp;
 };
 
 }  // namespace kda

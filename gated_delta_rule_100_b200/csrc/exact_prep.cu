@@ -57,6 +57,7 @@ __global__ void __launch_bounds__(EXACT_THREADS, 1) exact_prep_kernel(const Exac
     const int tid = threadIdx.x;
     const int H = prm.H;
     constexpr int gdk = SG ? 1 : DK;
+    if (tid == 0) stamp_start(prm.stamp);
     const int count = *prm.steep_count;
 
     for (int idx = blockIdx.x; idx < count; idx += gridDim.x) {
@@ -172,6 +173,7 @@ __global__ void __launch_bounds__(EXACT_THREADS, 1) exact_prep_kernel(const Exac
         }
         __syncthreads();  // the tiles are reused by the next item
     }
+    if (tid == 0) stamp_end(prm.stamp);
 }
 
 template <int DK, bool SG>

@@ -29,7 +29,7 @@ cudaError_t launch_prep(const CUtensorMap &tq, const CUtensorMap &tk, const Prep
 cudaError_t launch_chain(const CUtensorMap *maps, const ChainParams &prm, int dk, cudaStream_t stream);
 cudaError_t launch_exact(const ExactParams &prm, int dk, int ctas, cudaStream_t stream);
 cudaError_t launch_parts_fixup(float *start, const float *local, const float *trans, int BH, int dk, int dv,
-                               int parts, cudaStream_t stream);
+                               int parts, cudaStream_t stream, unsigned long long *stamp);
 cudaError_t launch_varlen_setup(const int *cu, int N, int T_total, int cmax, int *cu_s, int *cc, int *chunk_seq,
                                 const DeviceStatus &st, cudaStream_t stream);
 }
@@ -46,7 +46,7 @@ uint32_t *g_status_ptr[kMaxDevices] = {};
 std::atomic<unsigned long long> g_wait_polls{0};
 std::atomic<unsigned long long> g_inject_polls{0};
 std::atomic<int> g_force_exact{0};
-std::atomic<int> g_parts_override{1};  // test hook: parts of the two-level pass (0 = automatic, 1 = off)
+std::atomic<int> g_parts_override{0};  // test hook: parts of the two-level pass (0 = automatic, 1 = off)
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
 int current_status_word(uint32_t **out) {
@@ -196,39 +196,45 @@ int reserve_workspace(int dev, size_t base_bytes, size_t state_bytes, bool strea
     return KDA_OK;
 }
 
-// Per-kernel timing hook (measurement only): CUDA events recorded on the
-// launching stream around every prefill kernel while enabled.
+// Per-kernel timing hook (measurement only).  While enabled, every prefill
+// kernel launch gets a slot in the device's stamp array, set to all ones on the
+// launching stream just before the launch; the kernel's CTAs fold their
+// %globaltimer start and end into it (see stamp_start / stamp_end), so a slot
+// ends as the launch's busy interval on the device.  The kernels' own stamps
+// add two atomics per CTA and nothing to the streams' ordering, unlike events
+// around each launch.
+constexpr int kMaxStamps = 8192;  // launches timed between two reads, per device
 struct TimedLaunch {
-    int dev, kind;
-    cudaEvent_t start, stop;
+    int dev, kind, slot;
 };
 std::atomic<int> g_timing{0};
-std::vector<TimedLaunch> g_timed;            // recorded, not yet read
-std::vector<std::pair<int, cudaEvent_t>> g_event_pool;  // (device, event)
+std::vector<TimedLaunch> g_timed;  // recorded, not yet read
+int g_stamp_next[kMaxDevices] = {};
+unsigned long long *g_stamp_ptr[kMaxDevices] = {};
 
-cudaEvent_t pooled_event(int dev) {  // called with g_mu held
-    for (size_t i = 0; i < g_event_pool.size(); ++i) {
-        if (g_event_pool[i].first == dev) {
-            cudaEvent_t e = g_event_pool[i].second;
-            g_event_pool.erase(g_event_pool.begin() + i);
-            return e;
-        }
-    }
-    cudaEvent_t e = nullptr;
-    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
-    return e;
-}
+}  // namespace
 
-// Launch `fn` on `s`, bracketed by timing events when the hook is on.
+__device__ unsigned long long g_kda_stamps[2 * kMaxStamps];
+
+namespace {
+
+// Launch `fn(stamp)` on `s`; stamp is the launch's timing slot, or NULL when
+// the hook is off (or every slot is taken).  Called with g_mu held.
 template <class F>
 cudaError_t timed_launch(int dev, int kind, cudaStream_t s, F &&fn) {
-    if (!g_timing.load()) return fn();
-    cudaEvent_t a = pooled_event(dev), b = pooled_event(dev);
-    if (a == nullptr || b == nullptr) return cudaErrorMemoryAllocation;
-    cudaError_t e = cudaEventRecord(a, s);
-    if (e == cudaSuccess) e = fn();
-    if (e == cudaSuccess) e = cudaEventRecord(b, s);
-    g_timed.push_back({dev, kind, a, b});
+    if (!g_timing.load()) return fn(nullptr);
+    if (g_stamp_ptr[dev] == nullptr) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_kda_stamps) != cudaSuccess) return cudaErrorUnknown;
+        g_stamp_ptr[dev] = static_cast<unsigned long long *>(p);
+    }
+    if (g_stamp_next[dev] >= kMaxStamps) return fn(nullptr);
+    const int slot = g_stamp_next[dev]++;
+    unsigned long long *st = g_stamp_ptr[dev] + 2 * slot;
+    cudaError_t e = cudaMemsetAsync(st, 0xFF, 2 * sizeof(unsigned long long), s);
+    if (e != cudaSuccess) return e;
+    e = fn(st);
+    g_timed.push_back({dev, kind, slot});
     return e;
 }
 
@@ -308,8 +314,11 @@ int chain_slices(int B, int H, int dv, int sms) { return (dv == 128 && 2LL * B *
 // pass A on (parts - 1) x (dv + dk) / 64 CTAs per (b, h) and pass B on
 // (parts - 1) x dv / 64, so the sequential walk shrinks to two parts' worth of
 // chunks plus the short fix-up.  Parts are chosen so that pass A fits in one
-// wave and each part holds at least 4 chunks; fewer than 3 parts gain nothing
-// (the walk would not shorten), so then the plain pass runs (1 is returned).
+// wave and each part holds at least kMinPartChunks chunks (below that the two
+// extra launches and the fix-up cost more than the walk saves: on the B200,
+// B1 H4 T2048 took 0.158 ms in 8 parts of 4 chunks against 0.113 ms plain);
+// fewer than 3 parts gain nothing, so then the plain pass runs (1 is returned).
+constexpr int kMinPartChunks = 16;
 int plan_parts(int B, int H, int dk, int dv, int cnt, int sms) {
     const int ov = g_parts_override.load();
     int P;
@@ -318,7 +327,7 @@ int plan_parts(int B, int H, int dk, int dv, int cnt, int sms) {
     } else {
         const long long per_part = (long long)B * H * ((dv + dk) / 64);
         P = (int)(1 + sms / per_part);
-        if (P > cnt / 4) P = cnt / 4;
+        if (P > cnt / kMinPartChunks) P = cnt / kMinPartChunks;
     }
     if (P > cnt) P = cnt;
     if (P < 3) return 1;
@@ -339,6 +348,7 @@ void plain_pass(kda::ChainParams &cp, int nslices) {
     cp.slots = nslices;
     cp.pass_a = 0;
     cp.p_start = cp.p_local = cp.p_trans = nullptr;
+    cp.stamp = nullptr;
 }
 
 // Geometry of a uniform launch: B sequences of T tokens, local chunks [n0, n0 + cnt).
@@ -365,6 +375,7 @@ kda::ExactParams exact_params(const void *q, const void *k, const float *g, int 
     xp.steep_count = pp.steep_count;
     xp.steep_items = pp.steep_items;
     xp.prologue = prologue ? 1 : 0;
+    xp.stamp = nullptr;
     xp.gate_c = pp.gate_c;
     xp.H = pp.H;
     xp.gm = pp.gm;
@@ -521,10 +532,16 @@ static int chunk_fwd_impl(const void *q, const void *k, const void *v, const flo
         pp.st = dst;
         // the first segment's prep runs alone: two CTAs on every SM
         const int ctas = i == 0 ? 2 * sms : (prep_ctas > 0 ? prep_ctas : 1);
-        cudaError_t e = timed_launch(dev, 0, sp, [&] { return kda::launch_prep(tq, tk, pp, dk, ctas, sp, prologue); });
+        cudaError_t e = timed_launch(dev, 0, sp, [&](unsigned long long *t) {
+            pp.stamp = t;
+            return kda::launch_prep(tq, tk, pp, dk, ctas, sp, prologue);
+        });
         if (e != cudaSuccess) return KDA_ERR_CUDA;
-        const kda::ExactParams xp = exact_params(q, k, g, g_dk, beta, pp, prologue);
-        e = timed_launch(dev, 2, sp, [&] { return kda::launch_exact(xp, dk, sms, sp); });
+        kda::ExactParams xp = exact_params(q, k, g, g_dk, beta, pp, prologue);
+        e = timed_launch(dev, 2, sp, [&](unsigned long long *t) {
+            xp.stamp = t;
+            return kda::launch_exact(xp, dk, sms, sp);
+        });
         if (e != cudaSuccess) return KDA_ERR_CUDA;
         if (multi && (cudaEventRecord(w->prep_done[buf], sp) != cudaSuccess ||
                       cudaStreamWaitEvent(sc, w->prep_done[buf], 0) != cudaSuccess))
@@ -545,7 +562,10 @@ static int chunk_fwd_impl(const void *q, const void *k, const void *v, const flo
         const int P = plan_parts(B, H, dk, dv, cnt, sms);
         if (P < 3) {
             plain_pass(cp, chain_slices(B, H, dv, sms));
-            e = timed_launch(dev, 1, sc, [&] { return kda::launch_chain(rmaps[buf], cp, dk, sc); });
+            e = timed_launch(dev, 1, sc, [&](unsigned long long *t) {
+                cp.stamp = t;
+                return kda::launch_chain(rmaps[buf], cp, dk, sc);
+            });
             if (e != cudaSuccess) return KDA_ERR_CUDA;
         } else {  // two-level pass: pass A, fix-up, pass B (64-column slices)
             const size_t st_part = (size_t)B * H * dk * dv;
@@ -559,17 +579,23 @@ static int chunk_fwd_impl(const void *q, const void *k, const void *v, const flo
             cp.part0 = 0;
             cp.nparts = P - 1;
             cp.slots = (dv + dk) / 64;
-            e = timed_launch(dev, 1, sc, [&] { return kda::launch_chain(rmaps[buf], cp, dk, sc); });
+            e = timed_launch(dev, 1, sc, [&](unsigned long long *t) {
+                cp.stamp = t;
+                return kda::launch_chain(rmaps[buf], cp, dk, sc);
+            });
             if (e != cudaSuccess) return KDA_ERR_CUDA;
-            e = timed_launch(dev, 3, sc, [&] {
-                return kda::launch_parts_fixup(cp.p_start, cp.p_local, cp.p_trans, B * H, dk, dv, P, sc);
+            e = timed_launch(dev, 3, sc, [&](unsigned long long *t) {
+                return kda::launch_parts_fixup(cp.p_start, cp.p_local, cp.p_trans, B * H, dk, dv, P, sc, t);
             });
             if (e != cudaSuccess) return KDA_ERR_CUDA;
             cp.pass_a = 0;
             cp.part0 = 1;
             cp.nparts = P - 1;
             cp.slots = dv / 64;
-            e = timed_launch(dev, 1, sc, [&] { return kda::launch_chain(rmaps[buf], cp, dk, sc); });
+            e = timed_launch(dev, 1, sc, [&](unsigned long long *t) {
+                cp.stamp = t;
+                return kda::launch_chain(rmaps[buf], cp, dk, sc);
+            });
             if (e != cudaSuccess) return KDA_ERR_CUDA;
         }
         if (multi && cudaEventRecord(w->chain_done[buf], sc) != cudaSuccess) return KDA_ERR_CUDA;
@@ -597,16 +623,27 @@ int kda_debug_kernel_times(double *ms, long long *launches, int nkinds) {
     if (ms == nullptr || launches == nullptr || nkinds < 0) return KDA_ERR_INVALID_ARG;
     for (int i = 0; i < nkinds; ++i) { ms[i] = 0.0; launches[i] = 0; }
     std::lock_guard<std::mutex> lk(g_mu);
-    int st = KDA_OK;
-    for (const TimedLaunch &t : g_timed) {
-        float e_ms = 0.f;
-        if (cudaEventSynchronize(t.stop) != cudaSuccess || cudaEventElapsedTime(&e_ms, t.start, t.stop) != cudaSuccess)
+    int st = KDA_OK, cur = 0;
+    if (cudaGetDevice(&cur) != cudaSuccess) return KDA_ERR_CUDA;
+    std::vector<unsigned long long> host;
+    for (int dev = 0; dev < kMaxDevices; ++dev) {
+        const int n = g_stamp_next[dev];
+        if (n == 0) continue;
+        host.assign(2 * (size_t)n, 0ull);
+        if (cudaSetDevice(dev) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess ||
+            cudaMemcpy(host.data(), g_stamp_ptr[dev], host.size() * sizeof(unsigned long long),
+                       cudaMemcpyDeviceToHost) != cudaSuccess)
             st = KDA_ERR_CUDA;
-        if (t.kind < nkinds) { ms[t.kind] += e_ms; launches[t.kind] += 1; }
-        g_event_pool.push_back({t.dev, t.start});
-        g_event_pool.push_back({t.dev, t.stop});
+        for (const TimedLaunch &t : g_timed) {
+            if (t.dev != dev || t.kind < 0 || t.kind >= nkinds) continue;
+            const unsigned long long a = host[2 * t.slot], e = ~host[2 * t.slot + 1];
+            if (st == KDA_OK && a != ~0ull && e >= a) ms[t.kind] += (double)(e - a) * 1e-6;
+            launches[t.kind] += 1;
+        }
+        g_stamp_next[dev] = 0;
     }
     g_timed.clear();
+    if (cudaSetDevice(cur) != cudaSuccess) st = KDA_ERR_CUDA;
     return st;
 }
 
@@ -740,10 +777,16 @@ int kda_chunk_fwd_varlen(const void *q, const void *k, const void *v, const floa
         pp.H = H;
         pp.gm = gm;
         pp.st = dst;
-        cudaError_t e = timed_launch(dev, 0, s, [&] { return kda::launch_prep(tq, tk, pp, dk, 2 * sms, s, false); });
+        cudaError_t e = timed_launch(dev, 0, s, [&](unsigned long long *t) {
+            pp.stamp = t;
+            return kda::launch_prep(tq, tk, pp, dk, 2 * sms, s, false);
+        });
         if (e != cudaSuccess) return KDA_ERR_CUDA;
-        const kda::ExactParams xp = exact_params(q, k, g, dk, beta, pp);
-        e = timed_launch(dev, 2, s, [&] { return kda::launch_exact(xp, dk, sms, s); });
+        kda::ExactParams xp = exact_params(q, k, g, dk, beta, pp);
+        e = timed_launch(dev, 2, s, [&](unsigned long long *t) {
+            xp.stamp = t;
+            return kda::launch_exact(xp, dk, sms, s);
+        });
         if (e != cudaSuccess) return KDA_ERR_CUDA;
         kda::ChainParams cp;
         cp.v = static_cast<const uint16_t *>(v);
@@ -758,7 +801,10 @@ int kda_chunk_fwd_varlen(const void *q, const void *k, const void *v, const floa
         plain_pass(cp, chain_slices(N, H, dv, sms));
         cp.st = dst;
         cp.inject_wait_polls = g_inject_polls.load();
-        e = timed_launch(dev, 1, s, [&] { return kda::launch_chain(rmaps, cp, dk, s); });
+        e = timed_launch(dev, 1, s, [&](unsigned long long *t) {
+            cp.stamp = t;
+            return kda::launch_chain(rmaps, cp, dk, s);
+        });
         if (e != cudaSuccess) return KDA_ERR_CUDA;
     }
     if (cudaEventRecord(w->done, s) != cudaSuccess) return KDA_ERR_CUDA;
@@ -914,6 +960,7 @@ int kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const flo
         pp.H = H;
         pp.gm = uniform_geom(B, T, n0, cnt);
         pp.st = dst;
+        pp.stamp = nullptr;
         if (cudaMemsetAsync(ticket, 0, 2 * sizeof(int), s) != cudaSuccess ||  // the counters start at zero
             kda::launch_prep(tq, tk, pp, dk, 2 * sms, s, false) != cudaSuccess ||
             kda::launch_exact(exact_params(q, k, g, dk, beta, pp), dk, sms, s) != cudaSuccess)

@@ -144,6 +144,16 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
     return t;
 }
 
+// Launch timing (measurement hook): a launch's slot holds {start, ~end}, both
+// initialised to all ones; every CTA folds in its own start and end with
+// atomicMin, so the slot ends as {first CTA start, ~(last CTA end)}.
+__device__ __forceinline__ void stamp_start(unsigned long long *slot) {
+    if (slot != nullptr) atomicMin(slot, (unsigned long long)globaltimer_ns());
+}
+__device__ __forceinline__ void stamp_end(unsigned long long *slot) {
+    if (slot != nullptr) atomicMin(slot + 1, ~(unsigned long long)globaltimer_ns());
+}
+
 // Longest a bounded wait polls before giving up, whatever the poll budget.
 constexpr uint64_t WAIT_TIMEOUT_NS = 1000000000ull;
 

@@ -17,6 +17,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "kda_device.cuh"
+
 namespace kda {
 
 constexpr int FIX_THREADS = 256;
@@ -24,7 +26,8 @@ constexpr int FIX_COLS = 32;
 
 template <int DK>
 __global__ void __launch_bounds__(FIX_THREADS, 1)
-parts_fixup_kernel(float *start, const float *local, const float *trans, int BH, int DV, int parts) {
+parts_fixup_kernel(float *start, const float *local, const float *trans, int BH, int DV, int parts,
+                   unsigned long long *stamp) {
     constexpr int TPR = FIX_THREADS / DK;  // threads per state row
     constexpr int CPT = FIX_COLS / TPR;    // columns per thread
     extern __shared__ float fsm[];
@@ -35,6 +38,7 @@ parts_fixup_kernel(float *start, const float *local, const float *trans, int BH,
     const int tid = threadIdx.x;
     const int r = tid / TPR, c0 = (tid % TPR) * CPT;
     const size_t sst = (size_t)BH * DK * DV, mst = (size_t)BH * DK * DK;  // per-part strides
+    if (tid == 0) stamp_start(stamp);
     for (int p = 1; p + 1 < parts; ++p) {
         const float *Sp = start + p * sst + (size_t)bh * DK * DV + cb * FIX_COLS;
         const float *Mp = trans + p * mst + (size_t)bh * DK * DK;
@@ -58,22 +62,23 @@ parts_fixup_kernel(float *start, const float *local, const float *trans, int BH,
         for (int c = 0; c < CPT; ++c) Sn[c] = acc[c];
         __syncthreads();  // the next step restages; its start block is this step's output
     }
+    if (tid == 0) stamp_end(stamp);
 }
 
 // start/local: [parts][BH][dk][dv], trans: [parts][BH][dk][dk], dv a multiple of 32.
 cudaError_t launch_parts_fixup(float *start, const float *local, const float *trans, int BH, int dk, int dv,
-                               int parts, cudaStream_t stream) {
+                               int parts, cudaStream_t stream, unsigned long long *stamp) {
     const int grid = BH * (dv / FIX_COLS);
     if (dk == 128) {
         const int smem = (128 * 129 + 128 * (FIX_COLS + 1)) * 4;
         cudaError_t e = cudaFuncSetAttribute(parts_fixup_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
-        parts_fixup_kernel<128><<<grid, FIX_THREADS, smem, stream>>>(start, local, trans, BH, dv, parts);
+        parts_fixup_kernel<128><<<grid, FIX_THREADS, smem, stream>>>(start, local, trans, BH, dv, parts, stamp);
     } else {
         const int smem = (64 * 65 + 64 * (FIX_COLS + 1)) * 4;
         cudaError_t e = cudaFuncSetAttribute(parts_fixup_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
-        parts_fixup_kernel<64><<<grid, FIX_THREADS, smem, stream>>>(start, local, trans, BH, dv, parts);
+        parts_fixup_kernel<64><<<grid, FIX_THREADS, smem, stream>>>(start, local, trans, BH, dv, parts, stamp);
     }
     return cudaGetLastError();
 }

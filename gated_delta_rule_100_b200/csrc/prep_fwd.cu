@@ -131,6 +131,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     const uint64_t polls = prm.st.wait_polls;
 
     if (tid == 0) {
+        stamp_start(prm.stamp);
         mbar_init(bar_in, 1);
         mbar_init(bar_mma, 1);
         fence_mbar_init();
@@ -606,6 +607,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     __syncthreads();
     tc_fence_after();
     if (warp == 0) tmem_dealloc(tmem, L::TM_COLS);
+    if (tid == 0) stamp_end(prm.stamp);
 }
 
 template <int DK, bool SG, bool PRO>

@@ -73,6 +73,10 @@ CONFIGS = {
     # the training shape at a quarter of the batch: inputs (0.34 GB) above L2, small enough for
     # multi-pass counter captures
     "profile_B2_H32_T4096_d128": PrefillConfig("profile_B2_H32_T4096_d128", 2, 32, 4096, 128, 128, 0.05, 0.0, 4),
+    # the long-context recipe on its first 65,536 tokens: 3.2 GB of inputs and records beyond the
+    # 2 GiB workspace cap, so it runs the long-context code path (segments on two streams)
+    "long_context_slice_B1_H32_T65536_d128": PrefillConfig("long_context_slice_B1_H32_T65536_d128", 1, 32, 65536,
+                                                           128, 128, 0.01, 0.0, 3),
 }
 DECODE_CONFIG = DecodeConfig("decode_B256_H32_d128_64steps", 256, 32, 128, 128, 0.05, 0.02, 64, 4)
 

@@ -36,7 +36,7 @@ EXPORTED = ("kda_chunk_fwd", "kda_chunk_fwd_noalloc", "kda_chunk_fwd_varlen", "k
             "kda_gdn_chunk_fwd", "kda_gdn_decode_step", "kda_chunk_fwd_raw", "kda_decode_step_raw",
             "kda_chunk_fwd_workspace_bytes", "kda_chunk_fwd_varlen_workspace_bytes", "kda_release_workspace",
             "kda_status_string", "kda_stream_status", "kda_chunk_fwd_debug_wait_limit",
-            "kda_chunk_fwd_debug_inject_timeout", "kda_chunk_fwd_debug_force_exact", "kda_chunk_fwd_debug_record_cap",
+            "kda_chunk_fwd_debug_inject_timeout", "kda_chunk_fwd_debug_force_exact", "kda_chunk_fwd_debug_record_cap", "kda_chunk_fwd_debug_parts",
             "kda_debug_kernel_timing", "kda_debug_kernel_times",
             "kda_abi_version")
 
@@ -89,6 +89,8 @@ def load():
     lib.kda_chunk_fwd_debug_wait_limit.restype = None
     lib.kda_chunk_fwd_debug_inject_timeout.argtypes = [ctypes.c_ulonglong]
     lib.kda_chunk_fwd_debug_inject_timeout.restype = None
+    lib.kda_chunk_fwd_debug_parts.argtypes = [i]
+    lib.kda_chunk_fwd_debug_parts.restype = None
     lib.kda_chunk_fwd_debug_record_cap.argtypes = [ctypes.c_ulonglong]
     lib.kda_chunk_fwd_debug_record_cap.restype = None
     lib.kda_chunk_fwd_debug_force_exact.argtypes = [i]
@@ -273,6 +275,11 @@ def varlen_workspace_bytes(N: int, T_total: int, H: int, dk: int, dv: int) -> in
     return int(load().kda_chunk_fwd_varlen_workspace_bytes(int(N), int(T_total), int(H), int(dk), int(dv)))
 
 
+def set_parts(parts: int) -> None:
+    """Test hook: parts of the two-level pass (0 = automatic, 1 = off, P >= 3 = forced)."""
+    load().kda_chunk_fwd_debug_parts(int(parts))
+
+
 def set_record_cap(nbytes: int) -> None:
     """Test hook: cap the chunk records the prefill workspace holds (0 = default)."""
     load().kda_chunk_fwd_debug_record_cap(int(nbytes))
@@ -341,7 +348,7 @@ def force_exact(enable: bool) -> None:
     load().kda_chunk_fwd_debug_force_exact(1 if enable else 0)
 
 
-KERNEL_KINDS = ("prep", "chain", "exact")
+KERNEL_KINDS = ("prep", "chain", "exact", "fixup")
 
 
 def kernel_timing(enable: bool) -> None:

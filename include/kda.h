@@ -90,12 +90,17 @@ typedef enum {
  *   stream: cudaStream_t
  *
  * Internally each sequence is cut into chunks of 64 tokens; the last chunk of
- * a sequence may be partial.  Two kernels run per segment of chunks: one
- * builds every chunk's state-independent pieces in parallel (decay-scaled
- * operands, the intra-chunk blocks, the inverse of the unit-lower system and
- * the WY factors) into the workspace; the other walks the chunks of each
- * (b, h) in order, carrying the state in fp32.  The chunk contractions run on
- * the tcgen05 tensor cores with fp32 accumulation.  T == 0 copies h0 to hT
+ * a sequence may be partial.  Per segment of chunks, one kernel builds every
+ * chunk's state-independent pieces in parallel (decay-scaled operands, the
+ * intra-chunk blocks, the inverse of the unit-lower system and the WY
+ * factors) into the workspace; another walks the chunks of each (b, h) in
+ * order, carrying the state in fp32.  With few (b, h) and enough chunks the
+ * walk is two-level: the segment is cut into parts, every part's transition
+ * (dk x dk) and zero-start state are formed in parallel, a short sequential
+ * fix-up gives each part its start state, and the parts then produce their
+ * outputs in parallel (the "chunked parallel" scheme of the "Kimi Linear"
+ * explainer, math.kryvik.com).  The chunk contractions run on the tcgen05
+ * tensor cores with fp32 accumulation.  T == 0 copies h0 to hT
  * (or zeroes hT) and writes no output; q, k, v, g, beta and out are then not
  * read and may be NULL.
  *
@@ -331,6 +336,15 @@ KDA_API void kda_chunk_fwd_debug_force_exact(int enable);
  * Applies to calls made afterwards; process-wide.
  */
 KDA_API void kda_chunk_fwd_debug_record_cap(unsigned long long bytes);
+
+/*
+ * kda_chunk_fwd_debug_parts -- test hook for the two-level pass of
+ * kda_chunk_fwd (long sequences with few (b, h)): 0 chooses the number of
+ * parts per segment automatically (the default), 1 turns the two-level pass
+ * off, P >= 3 forces P parts wherever a segment has at least P chunks.
+ * Applies to calls made afterwards; process-wide.
+ */
+KDA_API void kda_chunk_fwd_debug_parts(int parts);
 
 /*
  * kda_debug_kernel_timing -- measurement hook.  While enabled (enable != 0),

@@ -23,17 +23,55 @@ def test_source_key_sees_code_changes():
 
 
 def test_traffic_figure_is_tied_to_its_sources(tmp_path, monkeypatch):
-    """bench.py reports the committed traffic figure only for the sources it was
+    """bench.py reports a committed traffic figure only for the sources it was
     taken on: a key that does not match gives None."""
     prof = tmp_path / "profiles"
     prof.mkdir()
-    entry = {"source_hash": bench.kernel_source_hash(), "bytes_per_launch_full_workload": 123.0}
-    (prof / "traffic.json").write_text(json.dumps({"kda_chunk_fwd": entry}))
+    t = {"source_hash": bench.kernel_source_hash(), "captured_on": "w",
+         "kernels": {"prep_kernel": {"mean_bytes_per_launch": 123.0, "bytes_per_token_head": 7.0}}}
+    (prof / "traffic.json").write_text(json.dumps(t))
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
-    monkeypatch.setattr(bench, "kernel_source_hash", lambda: entry["source_hash"])
-    assert bench.measured_traffic("kda_chunk_fwd") == 123.0
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda: t["source_hash"])
+    assert bench.measured_traffic("prep_kernel") == (123.0, "w")
+    assert bench.measured_traffic("prep_kernel", "bytes_per_token_head") == (7.0, "w")
+    assert bench.measured_traffic("chain_kernel") == (None, None)
     monkeypatch.setattr(bench, "kernel_source_hash", lambda: "another")
-    assert bench.measured_traffic("kda_chunk_fwd") is None
+    assert bench.measured_traffic("prep_kernel") == (None, None)
+
+
+def test_record_traffic_from_ncu_csv(tmp_path, monkeypatch):
+    """The ncu CSV of two prep and one chain launch on the long-context slice
+    becomes per-kernel bytes per launch and per token-head, keyed to the sources."""
+    rows = [
+        ["ID", "Process ID", "Process Name", "Host Name", "Kernel Name", "Context", "Stream", "Block Size",
+         "Grid Size", "Device", "CC", "Section Name", "Metric Name", "Metric Unit", "Metric Value"],
+    ]
+    def add(i, kern, name, unit, val):
+        rows.append([str(i), "1", "python", "h", kern, "1", "7", "(512,1,1)", "(296,1,1)", "0", "10.0", "",
+                     name, unit, val])
+    add(0, "void kda::prep_kernel<128, false, false>(CUtensorMap, CUtensorMap, kda::PrepParams)",
+        "dram__bytes_read.sum", "Gbyte", "1.5")
+    add(0, "void kda::prep_kernel<128, false, false>(CUtensorMap, CUtensorMap, kda::PrepParams)",
+        "dram__bytes_write.sum", "Mbyte", "500")
+    add(1, "void kda::chain_kernel<128, 64>(...)", "dram__bytes_read.sum", "Gbyte", "2.0")
+    add(1, "void kda::chain_kernel<128, 64>(...)", "dram__bytes_write.sum", "byte", "1,000")
+    add(2, "void kda::prep_kernel<128, false, false>(CUtensorMap, CUtensorMap, kda::PrepParams)",
+        "dram__bytes_read.sum", "Gbyte", "1.0")
+    add(2, "void kda::prep_kernel<128, false, false>(CUtensorMap, CUtensorMap, kda::PrepParams)",
+        "dram__bytes_write.sum", "Gbyte", "1.0")
+    import csv
+    path = tmp_path / "t.csv"
+    with open(path, "w", newline="") as f:
+        csv.writer(f).writerows(rows)
+    out = tmp_path / "traffic.json"
+    t = bench.record_traffic(str(path), "long_context_slice_B1_H32_T65536_d128", str(out))
+    assert t["source_hash"] == bench.kernel_source_hash()
+    prep = t["kernels"]["prep_kernel"]
+    assert prep["launches_captured"] == 2 and prep["bytes_per_launch"] == [2.0e9, 2.0e9]
+    th = bench.prep_launch_token_heads(1, 65536, 32)
+    assert th[:2] == [32 * 451 * 64] * 2 and sum(th) == 32 * 65536
+    assert abs(prep["bytes_per_token_head"] - 4.0e9 / (2 * 32 * 451 * 64)) < 1e-9
+    assert t["kernels"]["chain_kernel"]["mean_bytes_per_launch"] == 2.0e9 + 1000
 
 
 def test_scalar_gate_line_with_stand_in_device(monkeypatch):

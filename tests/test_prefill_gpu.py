@@ -270,3 +270,24 @@ def test_chunk_boundaries_do_not_matter(pieces):
     assert_close(f64(state), s_ref, f"pieces {pieces} hT")
     assert_close(f64(pieced), f64(whole_o), f"pieces {pieces} vs whole out")
     assert_close(f64(state), f64(whole_s), f"pieces {pieces} vs whole hT")
+
+
+def test_kernel_timing_hook_stamps_every_launch():
+    """The measurement hook: every prefill launch stamps its busy interval; each
+    kind's summed time is positive and within the call's wall time on the device."""
+    d = inputs.make_prefill(2, 2000, 4, 128, 128, decay=0.05, h0_std=0.02, seed=18, device=DEV)
+    run(d, 0.1)
+    kda.kernel_times()  # forget anything recorded before
+    kda.kernel_timing(True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    run(d, 0.1)
+    e1.record()
+    torch.cuda.synchronize()
+    kda.kernel_timing(False)
+    t = kda.kernel_times()
+    wall = e0.elapsed_time(e1)
+    assert t["prep"][1] >= 1 and t["chain"][1] >= 1 and t["exact"][1] >= 1
+    for kind in ("prep", "chain"):
+        assert 0.0 < t[kind][0] <= wall * 1.05 + 0.01, (kind, t[kind], wall)
+    assert kda.kernel_times() == {k: (0.0, 0) for k in kda.KERNEL_KINDS}  # read once
