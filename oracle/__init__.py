@@ -55,6 +55,8 @@ def _bind(path):
     lib.kda_oracle_fwd.restype = ctypes.c_int
     lib.kda_oracle_bruteforce.argtypes = [dp] * 6 + [ctypes.c_double, dp, dp, dp] + [L] * 5
     lib.kda_oracle_bruteforce.restype = ctypes.c_int
+    lib.kda_oracle_bwd.argtypes = [dp] * 6 + [ctypes.c_double, dp, dp, dp] + [dp] * 7 + [L] * 5 + [ctypes.c_int]
+    lib.kda_oracle_bwd.restype = ctypes.c_int
     lib.kda_oracle_max_threads.restype = ctypes.c_int
     return lib
 
@@ -143,6 +145,35 @@ def kda_bruteforce(q, k, v, g, beta, scale, h0=None, *, erase=None, write=None, 
     if rc != 0:
         raise RuntimeError("kda_oracle_bruteforce failed")
     return out, hT
+
+
+def kda_bwd(q, k, v, g, beta, scale, h0=None, dout=None, dhT=None, *, erase=None, write=None,
+            threads: int | None = None, lib=None):
+    """Gradients of sum(dout * out) + sum(dhT * hT) with respect to the inputs of
+    ``kda_fwd``, by reverse-mode differentiation of the token loop.  Returns a
+    dict with dq, dk, dv, dg, dbeta (= derase + dwrite), derase, dwrite, dh0
+    (float64, the inputs' layouts).  Keeps every state of a (b, h): small T only."""
+    q, k, v, g, e, w, h0, (B, T, H, dk, dv) = _prep(q, k, v, g, beta, h0, erase, write)
+    dout = None if dout is None else _f64(dout)
+    dhT = None if dhT is None else _f64(dhT)
+    if dout is not None and dout.shape != (B, T, H, dv):
+        raise ValueError("dout must be [B,T,H,dv]")
+    if dhT is not None and dhT.shape != (B, H, dk, dv):
+        raise ValueError("dhT must be [B,H,dk,dv]")
+    r = {n: np.zeros((B, T, H, dk)) for n in ("dq", "dk", "dg")}
+    r["dv"] = np.zeros((B, T, H, dv))
+    r["derase"] = np.zeros((B, T, H))
+    r["dwrite"] = np.zeros((B, T, H))
+    r["dh0"] = np.zeros((B, H, dk, dv))
+    lib = _load(lib)
+    nt = int(lib.kda_oracle_max_threads()) if threads is None else int(threads)
+    rc = lib.kda_oracle_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(e), _ptr(w), float(scale), _ptr(h0),
+                            _ptr(dout), _ptr(dhT), _ptr(r["dq"]), _ptr(r["dk"]), _ptr(r["dv"]), _ptr(r["dg"]),
+                            _ptr(r["derase"]), _ptr(r["dwrite"]), _ptr(r["dh0"]), B, T, H, dk, dv, nt)
+    if rc != 0:
+        raise RuntimeError("kda_oracle_bwd failed")
+    r["dbeta"] = r["derase"] + r["dwrite"]
+    return r
 
 
 def kda_decode_step(q, k, v, g, beta, scale, state, threads: int | None = None, lib=None):
