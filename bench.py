@@ -22,6 +22,7 @@ Also measured and reported in the same line:
            measured HBM peak, with each kernel's busy time from one extra step
            whose launches the kernels stamp themselves (%globaltimer);
   training the training-shape prefill (B8 H32 T4096) timed the same way;
+  backward kda_chunk_bwd on the training shape (fp32 CUDA cores, "alu" roofline);
   cpu_baseline  the fp64 oracle on a bounded sample of the workload (rank 0,
            N = 1 only), plus every workload's recipe on 1 thread and all cores.
 
@@ -130,13 +131,27 @@ def source_code_tokens(text):
     return " ".join(text.split())
 
 
-def kernel_source_hash():
+# The device sources each captured kernel is built from (its file and the headers
+# it includes): a traffic figure stays valid while these are unchanged.
+COMMON_HEADERS = ("chunk_common.cuh", "chunk_params.cuh", "kda_device.cuh")
+KERNEL_SOURCES = {
+    "prep_kernel": ("prep_fwd.cu",) + COMMON_HEADERS,
+    "exact_prep_kernel": ("exact_prep.cu",) + COMMON_HEADERS,
+    "chain_kernel": ("chain_fwd.cu",) + COMMON_HEADERS,
+    "decode_step_kernel": ("decode.cu", "kda_device.cuh"),
+}
+
+
+def kernel_source_hash(kernel=None):
+    """sha256 (first 16 hex digits) of a kernel's device sources (all of csrc when
+    kernel is None), comments removed and whitespace collapsed."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "gated_delta_rule_100_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, name), encoding="utf-8") as f:
-                h.update(name.encode() + source_code_tokens(f.read()).encode())
+    names = sorted(KERNEL_SOURCES[kernel]) if kernel else sorted(
+        n for n in os.listdir(csrc) if n.endswith((".cu", ".cuh")))
+    for name in names:
+        with open(os.path.join(csrc, name), encoding="utf-8") as f:
+            h.update(name.encode() + source_code_tokens(f.read()).encode())
     return h.hexdigest()[:16]
 
 
@@ -180,7 +195,9 @@ def record_traffic(csv_path, workload, out_path=None):
         if r[idx["Metric Name"]] not in ("dram__bytes_read.sum", "dram__bytes_write.sum"):
             continue
         lid = r[idx["ID"]]
-        name = next((k for k in TRAFFIC_KERNELS if k in r[idx["Kernel Name"]]), None)
+        # the function's own name: "void ns::name<...>(args)" -> "name"
+        base = r[idx["Kernel Name"]].split("(")[0].split("<")[0].split()[-1].split("::")[-1]
+        name = base if base in TRAFFIC_KERNELS else None
         if name is None:
             continue
         val = float(r[idx["Metric Value"]].replace(",", "")) * scale_of.get(r[idx["Metric Unit"]], 1.0)
@@ -195,15 +212,23 @@ def record_traffic(csv_path, workload, out_path=None):
         ids = [i for i in order if launches[i][0] == name]
         if not ids:
             continue
-        e = {"launches_captured": len(ids), "bytes_per_launch": [launches[i][1] for i in ids]}
+        e = {"source_hash": kernel_source_hash(name), "launches_captured": len(ids),
+             "bytes_per_launch": [launches[i][1] for i in ids]}
         e["mean_bytes_per_launch"] = sum(e["bytes_per_launch"]) / len(ids)
         if name in ("prep_kernel", "chain_kernel") and per_launch_th:
             th = [per_launch_th[n % len(per_launch_th)] for n in range(len(ids))]
             e["bytes_per_token_head"] = sum(e["bytes_per_launch"]) / sum(th)
         kernels[name] = e
-    t = {"source_hash": kernel_source_hash(), "captured_on": workload, "kernels": kernels,
-         "source_key": "sha256 of the csrc .cu/.cuh files with comments removed and whitespace collapsed"}
     out_path = out_path or os.path.join(ROOT, "profiles", "traffic.json")
+    t = {"kernels": {}}
+    if os.path.exists(out_path):  # captures of other kernels stay
+        with open(out_path) as f:
+            t = json.load(f)
+    for name, e in kernels.items():
+        e["captured_on"] = workload
+        t.setdefault("kernels", {})[name] = e
+    t["source_key"] = ("per kernel: sha256 of its device sources (bench.KERNEL_SOURCES) with comments removed "
+                       "and whitespace collapsed")
     with open(out_path, "w") as f:
         json.dump(t, f, indent=1)
     return t
@@ -211,19 +236,17 @@ def record_traffic(csv_path, workload, out_path=None):
 
 def measured_traffic(kernel, field="mean_bytes_per_launch"):
     """A kernel's DRAM-traffic figure from profiles/traffic.json, if that capture
-    was taken on the current kernel sources (else None), with the workload it was
-    captured on."""
+    was taken on the kernel's current device sources (else None), with the
+    workload it was captured on."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None, None
     with open(path) as f:
         t = json.load(f)
-    if t.get("source_hash") != kernel_source_hash():
-        return None, None
     e = t.get("kernels", {}).get(kernel)
-    if not e or field not in e:
+    if not e or field not in e or e.get("source_hash") != kernel_source_hash(kernel):
         return None, None
-    return e[field], t.get("captured_on")
+    return e[field], e.get("captured_on")
 
 
 class ClockSampler:
@@ -395,6 +418,71 @@ def measure_training(P, peak_src, stream, steps, warmup, dev):
                          "tensor_view": {"achieved_tflops": nflops / (ms / 1e3) / 1e12,
                                          "peak_tflops": P["bf16_tflops_sustained"],
                                          "frac": nflops / (ms / 1e3) / 1e12 / P["bf16_tflops_sustained"]}}}
+
+
+# fp32 CUDA-core peak of the B200, from its unit counts and clock: 148 SMs x 128
+# fp32 lanes x 2 flops (FMA) x the measured maximum SM clock.
+def fp32_alu_peak_tflops(P):
+    return 148 * 128 * 2 * P.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+
+
+def backward_flops(B, T, H, dk, dv):
+    """Algorithmic flops of the recurrence's backward, once per token: the
+    forward step it differentiates (decay, p = S'^T k, the write: ~5 dk dv) and
+    the reverse step (S', p, S_t, dq, dS += q do, du, dk (two terms), dS', dalpha,
+    dS_{t-1}: ~20 dk dv).  Recomputation from checkpoints is not counted."""
+    return B * T * H * 25 * dk * dv
+
+
+def backward_bytes(B, T, H, dk, dv):
+    """Algorithmic HBM bytes: q, k, v, dout (bf16), g, beta read; dq, dk, dv (bf16),
+    dg, dbeta (fp32) written."""
+    return B * T * H * (2 * (2 * dk + 2 * dv) + 4 * dk + 4 + 2 * (2 * dk + dv) + 4 * dk + 4)
+
+
+def measure_backward(P, stream, steps, dev):
+    """kda_chunk_bwd on the training shape with a random dL/dout, timed like the
+    step (3 warm-ups), with its roofline: the recurrent form is bound by fp32
+    CUDA-core arithmetic ("alu"), against the unit-count peak."""
+    import torch
+
+    from gated_delta_rule_100_b200 import inputs, kda
+
+    cfg = inputs.CONFIGS["training_B8_H32_T4096_d128"]
+    d = inputs.make_config(cfg, device=dev)
+    gen = torch.Generator(device=dev).manual_seed(cfg.seed + 100)
+    dout = torch.randn((cfg.B, cfg.T, cfg.H, cfg.dv), generator=gen, device=dev).to(torch.bfloat16)
+
+    def step():
+        return kda.chunk_bwd(d["q"], d["k"], d["v"], d["g"], d["beta"], cfg.scale, d["h0"], dout, None,
+                             stream=stream)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n = max(1, min(steps, 3))
+    e0.record(stream)
+    for _ in range(n):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if kda.stream_status(stream) != kda.KDA_OK:
+        raise RuntimeError("device-side error in the backward steps")
+    ms = e0.elapsed_time(e1) / n
+    fl = backward_flops(cfg.B, cfg.T, cfg.H, cfg.dk, cfg.dv)
+    peak = fp32_alu_peak_tflops(P)
+    return {"metric": "training-shape backward tokens/s", "value": cfg.B * cfg.T / (ms / 1e3), "unit": "tokens/s",
+            "ms_per_step": ms, "steps": n, "entry_point": "kda_chunk_bwd",
+            "config": {"workload": cfg.name, "cotangents": "dL/dout ~ N(0, 1) bf16, dL/dhT = 0"},
+            "roofline": {"kernel": "kda_chunk_bwd (recurrent form: checkpoint pass + reverse pass)", "bound": "alu",
+                         "achieved": fl / (ms / 1e3) / 1e12, "peak": peak, "unit": "TFLOP/s",
+                         "frac": fl / (ms / 1e3) / 1e12 / peak,
+                         "peak_source": "148 SMs x 128 fp32 lanes x 2 x max SM clock",
+                         "algorithmic_flops_per_launch": fl,
+                         "hbm_view": {"algorithmic_bytes": backward_bytes(cfg.B, cfg.T, cfg.H, cfg.dk, cfg.dv),
+                                      "achieved_gbs": backward_bytes(cfg.B, cfg.T, cfg.H, cfg.dk, cfg.dv)
+                                      / (ms / 1e3) / 1e9}}}
 
 
 def cpu_baseline_table(budget_s=3.0):
@@ -583,6 +671,13 @@ def run_ours(args):
         except Exception as exc:  # noqa: BLE001 - an extra item must not cost the measurement above
             training = {"error": f"{type(exc).__name__}: {exc}"[:300]}
 
+    backward = None
+    if not args.no_backward:
+        try:
+            backward = measure_backward(P, stream, args.steps, dev)
+        except Exception as exc:  # noqa: BLE001
+            backward = {"error": f"{type(exc).__name__}: {exc}"[:300]}
+
     # ---------------- decode ----------------
     dec = None
     if not args.no_decode:
@@ -668,7 +763,8 @@ def run_ours(args):
                        "l2": "inputs larger than L2 (51.7 GB per step); no flush",
                        "parallelism": f"weak: one workload copy per GPU x{world}"},
             "tflops": nflops / (ms_per_step / 1e3) / 1e12 * world,
-            "roofline": roof, "decode": dec, "scalar_gate": gdn, "training": training, "e2e": e2e,
+            "roofline": roof, "decode": dec, "scalar_gate": gdn, "training": training, "backward": backward,
+            "e2e": e2e,
             "cpu_baseline": cpu,
             "clocks": clk.summary(), "gpu_launches": gpu_launches,
             "launch_ms": {"mean": statistics.mean(launch_ms), "min": min(launch_ms), "max": max(launch_ms)},
@@ -691,6 +787,7 @@ def main():
     ap.add_argument("--no-gdn", action="store_true", help="skip the scalar-gate prefill line")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-training", action="store_true", help="skip the training-shape prefill line")
+    ap.add_argument("--no-backward", action="store_true", help="skip the training-shape backward line")
     ap.add_argument("--record-traffic", metavar="CSV",
                     help="write profiles/traffic.json from an ncu dram-bytes CSV and exit")
     ap.add_argument("--no-cpu-baseline", action="store_true")

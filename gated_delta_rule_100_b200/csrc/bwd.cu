@@ -1,0 +1,366 @@
+// bwd.cu -- the backward pass of the KDA prefill: gradients of a loss through
+// kda_chunk_fwd's outputs (out and hT) with respect to q, k, v, g, beta and h0
+// (sm_100a, fp32 on CUDA cores).
+//
+// Reverse-mode differentiation of the recurrence (per (b, h), state S, dk x dv)
+//   S' = Diag(alpha) S_{t-1},  p = S'^T k,  u = beta (v - p),  S_t = S' + k u^T,
+//   o_t = scale S_t^T q
+// (the combined update of section 3.3 of "Kimi Linear's Hybrid Linear
+// Attention Architecture: A Technical Breakdown"), walking the tokens
+// backwards with the adjoint dS of the state:
+//   dq = scale S_t do,  dS += scale q do^T,  du = dS^T k,  dk = dS u + S' dp,
+//   dbeta = du . (v - p),  dv = beta du,  dp = -beta du,  dS' = dS + k dp^T,
+//   dg = alpha * rowsum(dS' * S_{t-1}),  dS_{t-1} = Diag(alpha) dS'.
+// This is the recurrent form: exact, and every step is column-local except
+// for dq, dk, dg and dbeta, which sum over the dv columns.
+//
+// Layout: one CTA of 512 threads per (b, h).  Warp w owns state columns
+// w CW .. w CW + CW - 1, lane l owns rows l + 32 i; so the column reductions
+// (p, du) are warp shuffles, and the sums over columns go through
+// shared-memory atomics per token.
+//   Pass 1 (bwd_ckpt_kernel): the forward recurrence from h0, storing S every
+//          CK1 = 64 tokens (level-1 checkpoints, fp32, in the workspace).
+//   Pass 2 (bwd_kernel): chunks of CK1 tokens from the last to the first.  Per
+//          chunk, the forward is re-run from its level-1 checkpoint to leave a
+//          state every CK = 8 tokens in a per-(b, h) scratch (level 2); then
+//          blocks of CK tokens from the last to the first: for token t of a
+//          block, the state before t is recomputed from the block's checkpoint
+//          (kept in shared memory), then the reverse step.  After each block
+//          its tokens' dq, dk (bf16), dg and dbeta (fp32) are written; dv per
+//          column as it is formed; dh0 at the end.
+// Memory: (ceil(T / 64) + 8) dk dv fp32 per (b, h); forward steps per token:
+// one in pass 1, one for level 2, 3.5 on average for the per-token states.
+// Inputs are staged in shared memory per block of tokens.  Level-2 states go
+// through global memory (the scratch), read back after a block barrier.
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "bwd_params.cuh"
+#include "kda_device.cuh"
+
+namespace kda {
+
+constexpr int BWD_THREADS = 512;
+constexpr int BWD_CK1 = 64;  // tokens per level-1 checkpoint
+constexpr int BWD_CK = 8;    // tokens per level-2 checkpoint (per block)
+constexpr int BWD_FT = 32;   // tokens staged at a time in pass 1
+
+// This lane's CW consecutive state columns of row r (CW a multiple of 4, 16-byte aligned).
+template <int CW>
+__device__ __forceinline__ void load_row(const float *src, float (&x)[CW]) {
+#pragma unroll
+    for (int c = 0; c < CW; c += 4) {
+        const float4 v = *reinterpret_cast<const float4 *>(src + c);
+        x[c] = v.x; x[c + 1] = v.y; x[c + 2] = v.z; x[c + 3] = v.w;
+    }
+}
+template <int CW>
+__device__ __forceinline__ void store_row(float *dst, const float (&x)[CW]) {
+#pragma unroll
+    for (int c = 0; c < CW; c += 4) *reinterpret_cast<float4 *>(dst + c) = make_float4(x[c], x[c + 1], x[c + 2], x[c + 3]);
+}
+
+// One forward step on this warp's columns: S <- Diag(a) S + k (beta (v - k^T Diag(a) S))^T.
+template <int RI, int CW>
+__device__ __forceinline__ void fwd_step(float (&S)[RI][CW], const float *sk, const float *sa, const float *sv,
+                                         float beta, int lane, int col0) {
+    float kr[RI], p[CW];
+#pragma unroll
+    for (int i = 0; i < RI; ++i) kr[i] = sk[lane + 32 * i];
+#pragma unroll
+    for (int c = 0; c < CW; ++c) p[c] = 0.f;
+#pragma unroll
+    for (int i = 0; i < RI; ++i) {
+        const float a = sa[lane + 32 * i];
+#pragma unroll
+        for (int c = 0; c < CW; ++c) {
+            S[i][c] *= a;
+            p[c] += kr[i] * S[i][c];
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+        for (int c = 0; c < CW; ++c) p[c] += __shfl_xor_sync(0xffffffffu, p[c], o);
+#pragma unroll
+    for (int c = 0; c < CW; ++c) {
+        const float u = beta * (sv[col0 + c] - p[c]);
+#pragma unroll
+        for (int i = 0; i < RI; ++i) S[i][c] += kr[i] * u;
+    }
+}
+
+template <int DK, int DV>
+__global__ void __launch_bounds__(BWD_THREADS, 1) bwd_ckpt_kernel(const BwdParams prm) {
+    constexpr int RI = DK / 32, CW = DV / 16;
+    extern __shared__ __align__(16) float fsm[];
+    float *sk = fsm;                      // [FT][DK]
+    float *sa = sk + BWD_FT * DK;         // [FT][DK] alpha
+    float *sv = sa + BWD_FT * DK;         // [FT][DV]
+    float *sb = sv + BWD_FT * DV;         // [FT]
+    const int bh = blockIdx.x, b = bh / prm.H, h = bh % prm.H;
+    const int T = prm.T, H = prm.H;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, col0 = warp * CW;
+    const int nck = (T + BWD_CK1 - 1) / BWD_CK1;
+    if (tid == 0) stamp_start(prm.stamp);
+    float S[RI][CW];
+#pragma unroll
+    for (int i = 0; i < RI; ++i) {
+        if (prm.h0) {
+            load_row<CW>(prm.h0 + ((size_t)bh * DK + lane + 32 * i) * DV + col0, S[i]);
+        } else {
+#pragma unroll
+            for (int c = 0; c < CW; ++c) S[i][c] = 0.f;
+        }
+    }
+    for (int t0 = 0; t0 < T; t0 += BWD_FT) {
+        const int nt = T - t0 < BWD_FT ? T - t0 : BWD_FT;
+        __syncthreads();  // the previous block's inputs are no longer read
+        for (int e = tid; e < nt * DK; e += BWD_THREADS) {
+            const int t = e / DK, r = e % DK;
+            const size_t row = ((size_t)b * T + t0 + t) * H + h;
+            sk[t * DK + r] = bf16_bits_to_f32(prm.k[row * DK + r]);
+            sa[t * DK + r] = __expf(prm.g[row * DK + r]);
+        }
+        for (int e = tid; e < nt * DV; e += BWD_THREADS) {
+            const int t = e / DV, c = e % DV;
+            sv[t * DV + c] = bf16_bits_to_f32(prm.v[(((size_t)b * T + t0 + t) * H + h) * DV + c]);
+        }
+        if (tid < nt) sb[tid] = prm.beta[((size_t)b * T + t0 + tid) * H + h];
+        __syncthreads();
+        for (int t = 0; t < nt; ++t) {
+            if ((t0 + t) % BWD_CK1 == 0) {  // the state before token t0 + t
+                float *dst = prm.ckpt + ((size_t)bh * nck + (t0 + t) / BWD_CK1) * DK * DV;
+#pragma unroll
+                for (int i = 0; i < RI; ++i) store_row<CW>(dst + (size_t)(lane + 32 * i) * DV + col0, S[i]);
+            }
+            fwd_step<RI, CW>(S, sk + t * DK, sa + t * DK, sv + t * DV, sb[t], lane, col0);
+        }
+    }
+    if (tid == 0) stamp_end(prm.stamp);
+}
+
+template <int DK, int DV>
+__global__ void __launch_bounds__(BWD_THREADS, 1) bwd_kernel(const BwdParams prm) {
+    constexpr int RI = DK / 32, CW = DV / 16, CK = BWD_CK;
+    constexpr int LD0 = DV + 1;      // row stride of the checkpoint tile (lanes own rows)
+    extern __shared__ __align__(16) float fsm[];
+    float *s0 = fsm;                 // [DK][LD0] the block's checkpoint
+    float *sk = s0 + DK * LD0;       // [CK][DK]
+    float *sq = sk + CK * DK;        // [CK][DK]
+    float *sa = sq + CK * DK;        // [CK][DK] alpha
+    float *sv = sa + CK * DK;        // [CK][DV]
+    float *sd = sv + CK * DV;        // [CK][DV] dout
+    float *sb = sd + CK * DV;        // [CK] beta
+    float *acq = sb + CK;            // [CK][DK] sums over columns: dq
+    float *ack = acq + CK * DK;      //                             dk
+    float *aca = ack + CK * DK;      //                             d alpha
+    float *acb = aca + CK * DK;      // [CK]                        dbeta
+    const int bh = blockIdx.x, b = bh / prm.H, h = bh % prm.H;
+    const int T = prm.T, H = prm.H;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, col0 = warp * CW;
+    const int nck1 = (T + BWD_CK1 - 1) / BWD_CK1;
+    const float scale = prm.scale;
+
+    float dS[RI][CW];
+#pragma unroll
+    for (int i = 0; i < RI; ++i) {
+        if (prm.dhT) {
+            load_row<CW>(prm.dhT + ((size_t)bh * DK + lane + 32 * i) * DV + col0, dS[i]);
+        } else {
+#pragma unroll
+            for (int c = 0; c < CW; ++c) dS[i][c] = 0.f;
+        }
+    }
+
+    // the inputs a forward step needs, for the CK tokens from t0 (nt of them)
+    auto stage_fwd = [&](int t0, int nt) {
+        for (int e = tid; e < nt * DK; e += BWD_THREADS) {
+            const int t = e / DK, r = e % DK;
+            const size_t row = ((size_t)b * T + t0 + t) * H + h;
+            sk[t * DK + r] = bf16_bits_to_f32(prm.k[row * DK + r]);
+            sa[t * DK + r] = __expf(prm.g[row * DK + r]);
+        }
+        for (int e = tid; e < nt * DV; e += BWD_THREADS) {
+            const int t = e / DV, c = e % DV;
+            sv[t * DV + c] = bf16_bits_to_f32(prm.v[(((size_t)b * T + t0 + t) * H + h) * DV + c]);
+        }
+        if (tid < nt) sb[tid] = prm.beta[((size_t)b * T + t0 + tid) * H + h];
+    };
+    float *scratch = prm.ckpt + ((size_t)prm.B * H * nck1 + (size_t)bh * (BWD_CK1 / CK)) * DK * DV;
+
+    for (int n = nck1 - 1; n >= 0; --n) {
+        const int c0 = n * BWD_CK1;
+        const int nb = ((T - c0 < BWD_CK1 ? T - c0 : BWD_CK1) + CK - 1) / CK;  // blocks of the chunk
+        {  // level 2: run the chunk forward from its level-1 checkpoint, leaving a state per block
+            float S[RI][CW];
+            const float *ck = prm.ckpt + ((size_t)bh * nck1 + n) * DK * DV;
+#pragma unroll
+            for (int i = 0; i < RI; ++i) load_row<CW>(ck + (size_t)(lane + 32 * i) * DV + col0, S[i]);
+            for (int jb = 0; jb < nb; ++jb) {
+                const int t0 = c0 + jb * CK;
+                const int nt = T - t0 < CK ? T - t0 : CK;
+                float *dst = scratch + (size_t)jb * DK * DV;
+#pragma unroll
+                for (int i = 0; i < RI; ++i) store_row<CW>(dst + (size_t)(lane + 32 * i) * DV + col0, S[i]);
+                if (jb + 1 == nb) break;  // the last block's state is not needed past its start
+                __syncthreads();          // the previous block's inputs are no longer read
+                stage_fwd(t0, nt);
+                __syncthreads();
+                for (int t = 0; t < nt; ++t)
+                    fwd_step<RI, CW>(S, sk + t * DK, sa + t * DK, sv + t * DV, sb[t], lane, col0);
+            }
+        }
+    for (int j = nb - 1; j >= 0; --j) {
+        const int t0 = c0 + j * CK;
+        const int nt = T - t0 < CK ? T - t0 : CK;
+        __syncthreads();  // the previous block's tiles and sums have been read; level 2 is written
+        const float *ck = scratch + (size_t)j * DK * DV;
+        for (int e = tid; e < DK * DV; e += BWD_THREADS) s0[(e / DV) * LD0 + e % DV] = ck[e];
+        for (int e = tid; e < nt * DK; e += BWD_THREADS) {
+            const int t = e / DK, r = e % DK;
+            const size_t row = ((size_t)b * T + t0 + t) * H + h;
+            sk[t * DK + r] = bf16_bits_to_f32(prm.k[row * DK + r]);
+            sq[t * DK + r] = bf16_bits_to_f32(prm.q[row * DK + r]);
+            sa[t * DK + r] = __expf(prm.g[row * DK + r]);
+        }
+        for (int e = tid; e < nt * DV; e += BWD_THREADS) {
+            const int t = e / DV, c = e % DV;
+            const size_t row = ((size_t)b * T + t0 + t) * H + h;
+            sv[t * DV + c] = bf16_bits_to_f32(prm.v[row * DV + c]);
+            sd[t * DV + c] = prm.dout ? bf16_bits_to_f32(prm.dout[row * DV + c]) : 0.f;
+        }
+        if (tid < nt) sb[tid] = prm.beta[((size_t)b * T + t0 + tid) * H + h];
+        for (int e = tid; e < CK * DK; e += BWD_THREADS) { acq[e] = 0.f; ack[e] = 0.f; aca[e] = 0.f; }
+        if (tid < CK) acb[tid] = 0.f;
+        __syncthreads();
+
+        for (int tt = nt - 1; tt >= 0; --tt) {
+            // the state before token t0 + tt, from the checkpoint
+            float S[RI][CW];
+#pragma unroll
+            for (int i = 0; i < RI; ++i)
+#pragma unroll
+                for (int c = 0; c < CW; ++c) S[i][c] = s0[(lane + 32 * i) * LD0 + col0 + c];
+            for (int s = 0; s < tt; ++s) fwd_step<RI, CW>(S, sk + s * DK, sa + s * DK, sv + s * DV, sb[s], lane, col0);
+
+            const float *kt = sk + tt * DK, *qt = sq + tt * DK, *at = sa + tt * DK;
+            const float *vt = sv + tt * DV, *dot = sd + tt * DV;
+            const float bt = sb[tt];
+            float kr[RI], qr[RI], ar[RI];
+#pragma unroll
+            for (int i = 0; i < RI; ++i) {
+                kr[i] = kt[lane + 32 * i];
+                qr[i] = qt[lane + 32 * i];
+                ar[i] = at[lane + 32 * i];
+            }
+            // forward quantities of the token: p = (Diag(a) S)^T k, u = beta (v - p)
+            float p[CW];
+#pragma unroll
+            for (int c = 0; c < CW; ++c) {
+                float acc = 0.f;
+#pragma unroll
+                for (int i = 0; i < RI; ++i) acc += kr[i] * ar[i] * S[i][c];
+                p[c] = acc;
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+                for (int c = 0; c < CW; ++c) p[c] += __shfl_xor_sync(0xffffffffu, p[c], o);
+            float dqp[RI], dkp[RI], dap[RI], du[CW];
+#pragma unroll
+            for (int i = 0; i < RI; ++i) { dqp[i] = 0.f; dkp[i] = 0.f; dap[i] = 0.f; }
+            // readout: dq = scale S_t do, dS += scale q do^T; then du = dS^T k
+#pragma unroll
+            for (int c = 0; c < CW; ++c) {
+                const float u = bt * (vt[col0 + c] - p[c]);
+                const float d = dot[col0 + c];
+                float acc = 0.f;
+#pragma unroll
+                for (int i = 0; i < RI; ++i) {
+                    const float snew = ar[i] * S[i][c] + kr[i] * u;
+                    dqp[i] += scale * snew * d;
+                    dS[i][c] += scale * qr[i] * d;
+                    acc += dS[i][c] * kr[i];
+                    dkp[i] += dS[i][c] * u;
+                }
+                du[c] = acc;
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+                for (int c = 0; c < CW; ++c) du[c] += __shfl_xor_sync(0xffffffffu, du[c], o);
+            float dbp = 0.f;
+            const size_t row = ((size_t)b * T + t0 + tt) * H + h;
+#pragma unroll
+            for (int c = 0; c < CW; ++c) {
+                dbp += du[c] * (vt[col0 + c] - p[c]);
+                const float dp = -bt * du[c];
+#pragma unroll
+                for (int i = 0; i < RI; ++i) {
+                    const float sdv = ar[i] * S[i][c];
+                    dkp[i] += sdv * dp;
+                    const float dsd = dS[i][c] + kr[i] * dp;
+                    dap[i] += dsd * S[i][c];
+                    dS[i][c] = ar[i] * dsd;
+                }
+            }
+            if (lane == 0) {
+#pragma unroll
+                for (int c = 0; c < CW; ++c) prm.dv[row * DV + col0 + c] = to_bf16_bits(bt * du[c]);
+                atomicAdd(&acb[tt], dbp);
+            }
+#pragma unroll
+            for (int i = 0; i < RI; ++i) {
+                atomicAdd(&acq[tt * DK + lane + 32 * i], dqp[i]);
+                atomicAdd(&ack[tt * DK + lane + 32 * i], dkp[i]);
+                atomicAdd(&aca[tt * DK + lane + 32 * i], dap[i]);
+            }
+        }
+        __syncthreads();
+        for (int e = tid; e < nt * DK; e += BWD_THREADS) {
+            const int t = e / DK, r = e % DK;
+            const size_t row = ((size_t)b * T + t0 + t) * H + h;
+            prm.dq[row * DK + r] = to_bf16_bits(acq[e]);
+            prm.dk[row * DK + r] = to_bf16_bits(ack[e]);
+            prm.dg[row * DK + r] = sa[e] * aca[e];
+        }
+        if (tid < nt) prm.dbeta[((size_t)b * T + t0 + tid) * H + h] = acb[tid];
+    }
+    }
+    if (prm.dh0) {
+#pragma unroll
+        for (int i = 0; i < RI; ++i) store_row<CW>(prm.dh0 + ((size_t)bh * DK + lane + 32 * i) * DV + col0, dS[i]);
+    }
+    __syncthreads();
+    if (tid == 0) stamp_end(prm.stamp);
+}
+
+template <int DK, int DV>
+static cudaError_t launch_bwd_t(const BwdParams &prm, cudaStream_t stream) {
+    const int BH = prm.B * prm.H;
+    const int s1 = (2 * BWD_FT * DK + BWD_FT * DV + BWD_FT) * 4;
+    const int s2 = (DK * (DV + 1) + 3 * BWD_CK * DK + 2 * BWD_CK * DV + BWD_CK + 3 * BWD_CK * DK + BWD_CK) * 4;
+    cudaError_t e = cudaFuncSetAttribute(bwd_ckpt_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, s1);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(bwd_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, s2);
+    if (e != cudaSuccess) return e;
+    bwd_ckpt_kernel<DK, DV><<<BH, BWD_THREADS, s1, stream>>>(prm);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    bwd_kernel<DK, DV><<<BH, BWD_THREADS, s2, stream>>>(prm);
+    return cudaGetLastError();
+}
+
+// Level-1 checkpoints [B H][ceil(T / CK1)] and level-2 scratch [B H][CK1 / CK], each dk x dv fp32.
+size_t bwd_ckpt_bytes(int B, int T, int H, int dk, int dv) {
+    return (size_t)B * H * ((T + BWD_CK1 - 1) / BWD_CK1 + BWD_CK1 / BWD_CK) * dk * dv * sizeof(float);
+}
+
+cudaError_t launch_bwd(const BwdParams &prm, int dk, int dv, cudaStream_t stream) {
+    if (dk == 128 && dv == 128) return launch_bwd_t<128, 128>(prm, stream);
+    if (dk == 128 && dv == 64) return launch_bwd_t<128, 64>(prm, stream);
+    if (dk == 64 && dv == 128) return launch_bwd_t<64, 128>(prm, stream);
+    return launch_bwd_t<64, 64>(prm, stream);
+}
+
+}  // namespace kda

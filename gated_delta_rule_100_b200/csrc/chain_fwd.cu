@@ -155,6 +155,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
         else if (prm.pass_a) s_out = prm.p_start + ((size_t)(part + 1) * BHn + bh) * DK * DV;
     }
     const uint64_t polls = prm.st.wait_polls;
+    const long long rows = geom_rows(prm.gm);  // token rows of v and out (debug-build checks)
 
     if (tid == 0) {
         stamp_start(prm.stamp);
@@ -222,7 +223,10 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
             const int s = n & 1, bi = B_K0 + s;
             mbar_expect_tx(bar(bi), TX_K);
             tma_load_4d(sbase + L::OFF_KH + s * 16384, &tm_kh, bar(bi), 0, 0, 0, rec0 + n);
-            bulk_load(sbase + L::OFF_DEC + s * 512, recs + (size_t)n * REC_BYTES + REC_DEC, 512, bar(bi));
+            // debug build: a record past the tensor maps' extent is reported, and the
+            // plain bulk copy then reads record 0 instead (the barrier still completes)
+            const bool in = KDA_CHECK(prm.st, rec0 + n < prm.nrec);
+            bulk_load(sbase + L::OFF_DEC + s * 512, (in ? recs + (size_t)n * REC_BYTES : prm.ws) + REC_DEC, 512, bar(bi));
             armed |= 1u << bi; parity ^= 1u << bi;
         };
         auto load_t = [&](int n) {  // T'(n)
@@ -267,8 +271,15 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
             umma_commit(bar(bi));
             armed |= 1u << bi; parity ^= 1u << bi;
         };
+        // debug build: an operand view [lo, hi) (bytes from the tile base) inside the layout;
+        // a view that is not skips its instructions (the commits still arrive)
+        auto views_ok = [&](int alo, int ahi, int blo, int bhi) {
+            return KDA_CHECK(prm.st, alo >= 0 && ahi <= L::TOTAL && blo >= 0 && bhi <= L::TOTAL);
+        };
         auto mma_u = [&](int n) {  // U = T'(n) V(n)
             tc_fence_after();
+            const int ta = L::OFF_T + (n & 1) * 16384;
+            if (views_ok(ta, ta + 8192 + 16384, L::OFF_VT, L::OFF_VT + VS * 256))
             for (int kk = 0; kk < 8; ++kk)
                 umma<1>(tmem + L::TM_U, desc_kmaj_s<128, 4>(sbase + L::OFF_T + (n & 1) * 16384, 8192, kk * 8),
                         desc_kmaj_s<128, 4>(sbase + L::OFF_VT, VS * 128, kk * 8), id_tf, kk > 0);
@@ -276,6 +287,8 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
         };
         auto mma_1 = [&](int n) {  // D1[n & 1] = [W; Q e^G](n) S0
             tc_fence_after();
+            const int wa = L::OFF_WQ + (n % WS) * 32768;
+            if (views_ok(wa, wa + DK * 256, L::OFF_S0, L::OFF_S0 + DK * VS * 2))
             for (int kk = 0; kk < DK / 16; ++kk)
                 umma<0>(tmem + L::TM_D1 + (n & 1) * VS, desc_mnmaj<32>(sbase + L::OFF_WQ + (n % WS) * 32768, DK, kk * 16),
                         desc_mnmaj<128>(sbase + L::OFF_S0, DK, kk * 16), id_bf, kk > 0);
@@ -284,6 +297,8 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
         };
         auto mma_3a = [&](int n) {  // D3 = K-hat(n)^T Vnew(n)
             tc_fence_after();
+            const int ka = L::OFF_KH + (n & 1) * 16384, vb = L::OFF_VN + (n & 1) * VS * 128;
+            if (views_ok(ka, ka + 16384, vb, vb + VS * 128))
             for (int kk = 0; kk < 4; ++kk)
                 umma<0>(tmem + L::TM_D3, desc_kmaj<32, 2>(sbase + L::OFF_KH + (n & 1) * 16384, 128, kk * 16),
                         desc_mnmaj<128>(sbase + L::OFF_VN + (n & 1) * VS * 128, CH, kk * 16), id_h, kk > 0);
@@ -291,6 +306,9 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
         };
         auto mma_3b = [&](int n) {  // D1[n & 1] rows 64..127 += P(n) Vnew(n)
             tc_fence_after();
+            // the 128-row view of P starts 2 KB before the buffer (rows 0..63, discarded)
+            const int pa = L::OFF_P + (n & 1) * 8192 - 2048, vb = L::OFF_VN + (n & 1) * VS * 128;
+            if (views_ok(pa, pa + 10240, vb, vb + VS * 128))
             for (int kk = 0; kk < 4; ++kk)
                 umma<0>(tmem + L::TM_D1 + (n & 1) * VS,
                         desc_kmaj<32, 2>(sbase + L::OFF_P + (n & 1) * 8192 - 2048, CH, kk * 16),
@@ -345,7 +363,9 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
         float S[CPT];  // S[ch][scol .. scol + CPT - 1]
 #pragma unroll
         for (int e = 0; e < CPT; ++e) S[e] = (ident && ch == scol + e) ? 1.f : 0.f;
-        if (ch < DK && s_in != nullptr) {
+        // debug build: the state slice this CTA reads and writes
+        const bool slice_in = KDA_CHECK(prm.st, seq < prm.gm.nseqs && part < prm.parts && scol + CPT <= s_ld);
+        if (ch < DK && s_in != nullptr && slice_in) {
             const float4 *src = reinterpret_cast<const float4 *>(s_in + (size_t)ch * s_ld + scol);
 #pragma unroll
             for (int e = 0; e < CPT / 4; ++e) {
@@ -372,7 +392,9 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
             const int t0 = (geo.lc0 + n) * CH + vtg * TPT;
             const uint32_t *src = reinterpret_cast<const uint32_t *>(prm.v + ((size_t)(geo.row0 + t0) * H + h) * DV + col0) + vp;
 #pragma unroll
-            for (int u = 0; u < TPT; ++u) vr[u] = (!ident && t0 + u < geo.len) ? __ldg(src + (size_t)u * H * DV / 2) : 0u;
+            for (int u = 0; u < TPT; ++u)
+                vr[u] = (!ident && t0 + u < geo.len && KDA_CHECK(prm.st, geo.row0 + t0 + u < rows))
+                            ? __ldg(src + (size_t)u * H * DV / 2) : 0u;
         };
         auto build_vt = [&]() {  // V^T tile: row = value column, K = token
             // a bf16 value is the top half of its fp32 (and tf32) bit pattern
@@ -397,7 +419,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
                 float o[16];
                 tmem_ld16(tmem + lane_base + L::TM_D1 + (n & 1) * VS + cg * CPT + c16, o);
                 tmem_wait_ld();
-                if (t < geo.len && !trans) {
+                if (t < geo.len && !trans && KDA_CHECK(prm.st, geo.row0 + t < rows && scol + c16 + 16 <= DV)) {
                     float a8[8], b8[8];
 #pragma unroll
                     for (int e = 0; e < 8; ++e) { a8[e] = prm.scale * o[e]; b8[e] = prm.scale * o[8 + e]; }
@@ -477,7 +499,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
         }
         // an empty sequence passes its state through (h0, or zero) once
         const bool write_state = nseg > 0 ? ok : (geo.first && geo.last);
-        if (write_state && *s_abort == 0 && s_out != nullptr && ch < DK) {
+        if (write_state && *s_abort == 0 && s_out != nullptr && ch < DK && slice_in) {
             float4 *dst = reinterpret_cast<float4 *>(s_out + (size_t)ch * s_ld + scol);
 #pragma unroll
             for (int e = 0; e < CPT / 4; ++e) dst[e] = make_float4(S[4 * e], S[4 * e + 1], S[4 * e + 2], S[4 * e + 3]);

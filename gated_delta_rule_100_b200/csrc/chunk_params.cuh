@@ -43,16 +43,25 @@ struct ItemGeo {
 
 __device__ __forceinline__ bool geom_packed(const SeqGeom &gm) { return gm.cu != nullptr; }
 
+// Token rows of the launch's tensors ([rows, H, *]).
+__device__ __forceinline__ long long geom_rows(const SeqGeom &gm) {
+    return geom_packed(gm) ? (long long)gm.T : (long long)gm.nseqs * gm.T;
+}
+
 // Items of the launch (packed: read from the device-side chunk offsets).
+// PACKED: the launch's geometry form, known at compile time (kernels that take
+// both forms pass the runtime test).
+template <bool PACKED>
 __device__ __forceinline__ int geom_items(const SeqGeom &gm, int H) {
-    if (!geom_packed(gm)) return gm.nseqs * H * gm.nseg;
+    if (!PACKED) return gm.nseqs * H * gm.nseg;
     const int left = gm.cc[gm.nseqs] - gm.c0;
     return (left < gm.W ? (left > 0 ? left : 0) : gm.W) * H;
 }
 
+template <bool PACKED>
 __device__ __forceinline__ ItemGeo item_geo(const SeqGeom &gm, int H, int it) {
     ItemGeo r;
-    if (!geom_packed(gm)) {
+    if (!PACKED) {
         const int ni = it % gm.nseg, bh = it / gm.nseg;
         r.h = bh % H;
         r.seq = bh / H;
@@ -127,6 +136,7 @@ struct PrepParams {
     int g_dk;            // gate values per (token, head): dk (per key channel) or 1 (one, broadcast)
     const float *beta;   // [tokens, H]
     uint8_t *ws;         // records, REC_BYTES each, at their record index
+    long long nrec;      // records in ws (the debug build checks record indices against it)
     int *ticket;         // item counter, zero at launch: CTAs claim items from it
     int *steep_count;    // zero at launch: items appended to steep_items
     int *steep_items;    // items whose decay needs the exact kernel (room for every item)
@@ -145,11 +155,13 @@ struct ExactParams {
     int g_dk;
     const float *beta;      // [tokens, H]
     uint8_t *ws;            // records, as in PrepParams
+    long long nrec;
     const int *steep_count, *steep_items;
     int prologue;           // raw g, beta, q, k: apply the gate prologue and normalise q, k
     float gate_c;
     int H;
     SeqGeom gm;
+    DeviceStatus st;
     unsigned long long *stamp;
 };
 
@@ -172,6 +184,7 @@ struct ChainParams {
     float *hT;           // [nseqs, H, dk, dv] or NULL: the state after the sequence's last chunk
     float *carry;        // packed: [nseqs, H, dk, dv], the state between windows (may be hT)
     const uint8_t *ws;   // records written by the prep kernel
+    long long nrec;      // records in ws (tensor-map extent)
     float scale;
     int H, DV, nslices;
     int parts, part_len;  // the segment's parts (1: the plain pass)

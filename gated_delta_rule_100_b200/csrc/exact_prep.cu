@@ -61,9 +61,14 @@ __global__ void __launch_bounds__(EXACT_THREADS, 1) exact_prep_kernel(const Exac
     const int count = *prm.steep_count;
 
     for (int idx = blockIdx.x; idx < count; idx += gridDim.x) {
-        const ItemGeo gi = item_geo(prm.gm, H, prm.steep_items[idx]);
+        const ItemGeo gi = geom_packed(prm.gm) ? item_geo<true>(prm.gm, H, prm.steep_items[idx])
+                                               : item_geo<false>(prm.gm, H, prm.steep_items[idx]);
         const int h = gi.h;
         uint8_t *rec = prm.ws + (size_t)gi.rec * REC_BYTES;
+        // debug build: the record and rows of the item (a bad one is reported and skipped)
+        if (!KDA_CHECK(prm.st, gi.rec >= 0 && gi.rec < prm.nrec && gi.row0 >= 0 &&
+                                   gi.row0 + (gi.nvalid < CH ? gi.nvalid : CH) <= geom_rows(prm.gm)))
+            continue;
 
         // ---- inputs (tokens past the sequence's end read as zero, with beta = 0) ----
         for (int e = tid; e < CH * DK; e += EXACT_THREADS) {

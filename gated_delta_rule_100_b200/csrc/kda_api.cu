@@ -20,16 +20,19 @@ cudaError_t launch_decode(const void *q, const void *k, const void *v, const flo
                           int dv, int g_dk, int prologue, float gate_c, cudaStream_t stream);
 }
 
+#include "bwd_params.cuh"
 #include "chunk_common.cuh"
 #include "chunk_params.cuh"
 
 namespace kda {
-cudaError_t launch_prep(const CUtensorMap &tq, const CUtensorMap &tk, const PrepParams &prm, int dk,
-                        int max_ctas, cudaStream_t stream, bool prologue);
+cudaError_t launch_prep(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tg, const PrepParams &prm,
+                        int dk, int max_ctas, cudaStream_t stream, bool prologue);
 cudaError_t launch_chain(const CUtensorMap *maps, const ChainParams &prm, int dk, cudaStream_t stream);
 cudaError_t launch_exact(const ExactParams &prm, int dk, int ctas, cudaStream_t stream);
 cudaError_t launch_parts_fixup(float *start, const float *local, const float *trans, int BH, int dk, int dv,
                                int parts, cudaStream_t stream, unsigned long long *stamp);
+cudaError_t launch_bwd(const BwdParams &prm, int dk, int dv, cudaStream_t stream);
+size_t bwd_ckpt_bytes(int B, int T, int H, int dk, int dv);
 cudaError_t launch_varlen_setup(const int *cu, int N, int T_total, int cmax, int *cu_s, int *cc, int *chunk_seq,
                                 const DeviceStatus &st, cudaStream_t stream);
 }
@@ -104,6 +107,8 @@ struct Workspace {
     size_t state_bytes = 0;
     float *parts = nullptr;  // the two-level pass: start, local and transition states of every part
     size_t parts_bytes = 0;
+    float *ckpt = nullptr;   // the backward pass: state checkpoints
+    size_t ckpt_bytes = 0;
     cudaEvent_t done = nullptr;
     cudaStream_t lo = nullptr, hi = nullptr;  // prep and chain streams of the segmented path
     cudaEvent_t fork = nullptr, prep_done[2] = {nullptr, nullptr}, chain_done[2] = {nullptr, nullptr};
@@ -372,6 +377,8 @@ kda::ExactParams exact_params(const void *q, const void *k, const float *g, int 
     xp.g_dk = g_dk;
     xp.beta = beta;
     xp.ws = pp.ws;
+    xp.nrec = pp.nrec;
+    xp.st = pp.st;
     xp.steep_count = pp.steep_count;
     xp.steep_items = pp.steep_items;
     xp.prologue = prologue ? 1 : 0;
@@ -397,6 +404,7 @@ const char *kda_status_string(int status) {
         case KDA_ERR_CUDA: return "KDA_ERR_CUDA";
         case KDA_ERR_TIMEOUT: return "KDA_ERR_TIMEOUT";
         case KDA_ERR_SCRATCH_LIMIT: return "KDA_ERR_SCRATCH_LIMIT";
+        case KDA_ERR_BOUNDS: return "KDA_ERR_BOUNDS";
         default: return "KDA_ERR_UNKNOWN";
     }
 }
@@ -422,6 +430,7 @@ int kda_stream_status(void *stream) {
         if (cudaMemcpy(word, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return KDA_ERR_CUDA;
     }
     if (v & kda::DEV_TIMEOUT) return KDA_ERR_TIMEOUT;
+    if (v & kda::DEV_BOUNDS) return KDA_ERR_BOUNDS;
     return (v & kda::DEV_BAD_ARG) ? KDA_ERR_INVALID_ARG : KDA_OK;
 }
 
@@ -455,11 +464,15 @@ static int chunk_fwd_impl(const void *q, const void *k, const void *v, const flo
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return KDA_ERR_CUDA;
 
-    CUtensorMap tq, tk;
+    CUtensorMap tq, tk, tg;  // tg: the per-channel gate, 32 channels x 64 tokens per box
     if (make_map(&tq, enc, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dk, H, T, B, 64,
                  CU_TENSOR_MAP_SWIZZLE_128B) != KDA_OK ||
         make_map(&tk, enc, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dk, H, T, B, 64,
                  CU_TENSOR_MAP_SWIZZLE_128B) != KDA_OK)
+        return KDA_ERR_CUDA;
+    if (scalar_gate) tg = tq;  // not read
+    else if (make_map(&tg, enc, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dk, H, T, B, 32,
+                      CU_TENSOR_MAP_SWIZZLE_NONE) != KDA_OK)
         return KDA_ERR_CUDA;
 
     const SegPlan pl = plan_segments(B, T, H);
@@ -522,6 +535,7 @@ static int chunk_fwd_impl(const void *q, const void *k, const void *v, const flo
         pp.g_dk = g_dk;
         pp.beta = beta;
         pp.ws = recs[buf];
+        pp.nrec = (long long)B * H * seg;
         pp.ticket = counters + 2 * buf;
         pp.steep_count = counters + 2 * buf + 1;
         pp.steep_items = steep_list;
@@ -534,7 +548,7 @@ static int chunk_fwd_impl(const void *q, const void *k, const void *v, const flo
         const int ctas = i == 0 ? 2 * sms : (prep_ctas > 0 ? prep_ctas : 1);
         cudaError_t e = timed_launch(dev, 0, sp, [&](unsigned long long *t) {
             pp.stamp = t;
-            return kda::launch_prep(tq, tk, pp, dk, ctas, sp, prologue);
+            return kda::launch_prep(tq, tk, tg, pp, dk, ctas, sp, prologue);
         });
         if (e != cudaSuccess) return KDA_ERR_CUDA;
         kda::ExactParams xp = exact_params(q, k, g, g_dk, beta, pp, prologue);
@@ -554,6 +568,7 @@ static int chunk_fwd_impl(const void *q, const void *k, const void *v, const flo
         cp.hT = hT;  // written by the last segment; earlier ones end in carry
         cp.carry = carry;
         cp.ws = recs[buf];
+        cp.nrec = (long long)B * H * seg;
         cp.scale = scale;
         cp.H = H; cp.DV = dv;
         cp.gm = pp.gm;
@@ -656,6 +671,8 @@ int kda_release_workspace(void) {
     if (w.base != nullptr && cudaFree(w.base) != cudaSuccess) st = KDA_ERR_CUDA;
     if (w.state != nullptr && cudaFree(w.state) != cudaSuccess) st = KDA_ERR_CUDA;
     if (w.parts != nullptr && cudaFree(w.parts) != cudaSuccess) st = KDA_ERR_CUDA;
+    if (w.ckpt != nullptr && cudaFree(w.ckpt) != cudaSuccess) st = KDA_ERR_CUDA;
+    w.ckpt = nullptr; w.ckpt_bytes = 0;
     w.base = nullptr; w.base_bytes = 0;
     w.state = nullptr; w.state_bytes = 0;
     w.parts = nullptr; w.parts_bytes = 0;
@@ -719,11 +736,13 @@ int kda_chunk_fwd_varlen(const void *q, const void *k, const void *v, const floa
     if (get_encoder(&enc) != KDA_OK) return KDA_ERR_CUDA;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return KDA_ERR_CUDA;
-    CUtensorMap tq, tk;  // [1][T_total][H][dk]
+    CUtensorMap tq, tk, tg;  // [1][T_total][H][dk]
     if (make_map(&tq, enc, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dk, H, T_total, 1, 64,
                  CU_TENSOR_MAP_SWIZZLE_128B) != KDA_OK ||
         make_map(&tk, enc, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dk, H, T_total, 1, 64,
-                 CU_TENSOR_MAP_SWIZZLE_128B) != KDA_OK)
+                 CU_TENSOR_MAP_SWIZZLE_128B) != KDA_OK ||
+        make_map(&tg, enc, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dk, H, T_total, 1, 32,
+                 CU_TENSOR_MAP_SWIZZLE_NONE) != KDA_OK)
         return KDA_ERR_CUDA;
 
     const VarlenPlan pl = plan_varlen(N, T_total, H);
@@ -769,6 +788,7 @@ int kda_chunk_fwd_varlen(const void *q, const void *k, const void *v, const floa
         pp.g_dk = dk;
         pp.beta = beta;
         pp.ws = recs;
+        pp.nrec = (long long)H * W;
         pp.ticket = counters;
         pp.steep_count = counters + 1;
         pp.steep_items = steep_list;
@@ -779,7 +799,7 @@ int kda_chunk_fwd_varlen(const void *q, const void *k, const void *v, const floa
         pp.st = dst;
         cudaError_t e = timed_launch(dev, 0, s, [&](unsigned long long *t) {
             pp.stamp = t;
-            return kda::launch_prep(tq, tk, pp, dk, 2 * sms, s, false);
+            return kda::launch_prep(tq, tk, tg, pp, dk, 2 * sms, s, false);
         });
         if (e != cudaSuccess) return KDA_ERR_CUDA;
         kda::ExactParams xp = exact_params(q, k, g, dk, beta, pp);
@@ -795,6 +815,7 @@ int kda_chunk_fwd_varlen(const void *q, const void *k, const void *v, const floa
         cp.hT = hT;
         cp.carry = carry;
         cp.ws = recs;
+        cp.nrec = (long long)H * W;
         cp.scale = scale;
         cp.H = H; cp.DV = dv;
         cp.gm = gm;
@@ -817,6 +838,73 @@ size_t kda_chunk_fwd_varlen_workspace_bytes(int N, int T_total, int H, int dk, i
     const VarlenPlan pl = plan_varlen(N, T_total, H);
     const size_t state = pl.nwin > 1 ? (size_t)N * H * dk * dv * sizeof(float) : 0;
     return varlen_base_bytes(N, H, pl) + state;
+}
+
+// Backward of the prefill (recurrent form, bwd.cu): checkpoints of the state
+// every few tokens in the workspace, then the reverse walk.
+int kda_chunk_bwd(const void *q, const void *k, const void *v, const float *g, const float *beta, float scale,
+                  const float *h0, const void *dout, const float *dhT, void *dq, void *dk_, void *dv_, float *dg,
+                  float *dbeta, float *dh0, int B, int T, int H, int dk, int dv, void *stream) {
+    if (B < 1 || H < 1 || T < 0) return KDA_ERR_INVALID_ARG;
+    if (T > 0 && (!q || !k || !v || !g || !beta || !dq || !dk_ || !dv_ || !dg || !dbeta)) return KDA_ERR_INVALID_ARG;
+    if ((dk != 64 && dk != 128) || (dv != 64 && dv != 128)) return KDA_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(g) || !aligned4(beta) || !aligned16(h0) ||
+        !aligned16(dout) || !aligned16(dhT) || !aligned16(dq) || !aligned16(dk_) || !aligned16(dv_) ||
+        !aligned16(dg) || !aligned4(dbeta) || !aligned16(dh0))
+        return KDA_ERR_ALIGNMENT;
+    if ((long long)B * H > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (T == 0) {  // hT = h0, so dh0 = dhT
+        if (dh0 == nullptr) return KDA_OK;
+        const size_t bytes = (size_t)B * H * dk * dv * sizeof(float);
+        cudaError_t e = dhT ? (dhT == dh0 ? cudaSuccess : cudaMemcpyAsync(dh0, dhT, bytes, cudaMemcpyDeviceToDevice, s))
+                            : cudaMemsetAsync(dh0, 0, bytes, s);
+        return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+    }
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return KDA_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_mu);
+    Workspace *w = nullptr;
+    if (int st = reserve_workspace(dev, 0, 0, false, &w); st != KDA_OK) return st;
+    const size_t need = kda::bwd_ckpt_bytes(B, T, H, dk, dv);
+    if (w->ckpt_bytes < need) {
+        if (w->ckpt != nullptr && cudaFree(w->ckpt) != cudaSuccess) return KDA_ERR_CUDA;
+        w->ckpt = nullptr;
+        w->ckpt_bytes = 0;
+        if (cudaMalloc(&w->ckpt, need) != cudaSuccess) return KDA_ERR_CUDA;
+        w->ckpt_bytes = need;
+    }
+    if (cudaStreamWaitEvent(s, w->done, 0) != cudaSuccess) return KDA_ERR_CUDA;
+    kda::BwdParams bp;
+    bp.q = static_cast<const uint16_t *>(q);
+    bp.k = static_cast<const uint16_t *>(k);
+    bp.v = static_cast<const uint16_t *>(v);
+    bp.g = g;
+    bp.beta = beta;
+    bp.h0 = h0;
+    bp.dout = static_cast<const uint16_t *>(dout);
+    bp.dhT = dhT;
+    bp.dq = static_cast<uint16_t *>(dq);
+    bp.dk = static_cast<uint16_t *>(dk_);
+    bp.dv = static_cast<uint16_t *>(dv_);
+    bp.dg = dg;
+    bp.dbeta = dbeta;
+    bp.dh0 = dh0;
+    bp.ckpt = w->ckpt;
+    bp.scale = scale;
+    bp.B = B; bp.T = T; bp.H = H;
+    if (timed_launch(dev, 4, s, [&](unsigned long long *t) {
+            bp.stamp = t;
+            return kda::launch_bwd(bp, dk, dv, s);
+        }) != cudaSuccess)
+        return KDA_ERR_CUDA;
+    if (cudaEventRecord(w->done, s) != cudaSuccess) return KDA_ERR_CUDA;
+    return KDA_OK;
+}
+
+size_t kda_chunk_bwd_workspace_bytes(int B, int T, int H, int dk, int dv) {
+    if (B < 1 || H < 1 || T <= 0 || (dk != 64 && dk != 128) || (dv != 64 && dv != 128)) return 0;
+    return kda::bwd_ckpt_bytes(B, T, H, dk, dv);
 }
 
 int kda_decode_step(const void *q, const void *k, const void *v, const float *g, const float *beta,
@@ -925,11 +1013,13 @@ int kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const flo
     PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
     if (get_encoder(&enc) != KDA_OK) return KDA_ERR_CUDA;
 
-    CUtensorMap tq, tk;
+    CUtensorMap tq, tk, tg;
     if (make_map(&tq, enc, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dk, H, T, B, 64,
                  CU_TENSOR_MAP_SWIZZLE_128B) != KDA_OK ||
         make_map(&tk, enc, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dk, H, T, B, 64,
-                 CU_TENSOR_MAP_SWIZZLE_128B) != KDA_OK)
+                 CU_TENSOR_MAP_SWIZZLE_128B) != KDA_OK ||
+        make_map(&tg, enc, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dk, H, T, B, 32,
+                 CU_TENSOR_MAP_SWIZZLE_NONE) != KDA_OK)
         return KDA_ERR_CUDA;
 
     const unsigned long long polls = g_wait_polls.load();
@@ -952,6 +1042,7 @@ int kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const flo
         pp.g_dk = dk;
         pp.beta = beta;
         pp.ws = recs;
+        pp.nrec = (long long)B * H * seg;
         pp.ticket = ticket;
         pp.steep_count = ticket + 1;
         pp.steep_items = steep_list;
@@ -962,7 +1053,7 @@ int kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const flo
         pp.st = dst;
         pp.stamp = nullptr;
         if (cudaMemsetAsync(ticket, 0, 2 * sizeof(int), s) != cudaSuccess ||  // the counters start at zero
-            kda::launch_prep(tq, tk, pp, dk, 2 * sms, s, false) != cudaSuccess ||
+            kda::launch_prep(tq, tk, tg, pp, dk, 2 * sms, s, false) != cudaSuccess ||
             kda::launch_exact(exact_params(q, k, g, dk, beta, pp), dk, sms, s) != cudaSuccess)
             return KDA_ERR_CUDA;
 
@@ -973,6 +1064,7 @@ int kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const flo
         cp.hT = hT;
         cp.carry = carry;
         cp.ws = recs;
+        cp.nrec = (long long)B * H * seg;
         cp.scale = scale;
         cp.H = H; cp.DV = dv;
         cp.gm = pp.gm;

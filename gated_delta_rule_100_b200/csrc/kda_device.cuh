@@ -18,7 +18,7 @@ namespace kda {
 
 // ---------------------------------------------------------------- status ----
 // Bit flags OR-ed into the per-device status word by kernels.
-enum : uint32_t { DEV_TIMEOUT = 1u, DEV_BAD_ARG = 2u };
+enum : uint32_t { DEV_TIMEOUT = 1u, DEV_BAD_ARG = 2u, DEV_BOUNDS = 4u };
 
 struct DeviceStatus {
     uint32_t *word;        // device-global status word (never NULL at launch)
@@ -28,6 +28,21 @@ struct DeviceStatus {
 __device__ __forceinline__ void report(const DeviceStatus &st, uint32_t bits) {
     atomicOr(st.word, bits);
 }
+
+// Index checks of the debug build (KDA_DEBUG, libkda_debug.so): before an
+// access whose bounds follow from layout constants and launch geometry rather
+// than from the code in front of it, KDA_CHECK(st, cond) tests the bound; a
+// failed check records DEV_BOUNDS in the status word and the caller skips the
+// access (no trap).  In the release build it is the constant true.
+__device__ __forceinline__ bool bounds_ok(const DeviceStatus &st, bool ok) {
+    if (!ok) report(st, DEV_BOUNDS);
+    return ok;
+}
+#ifdef KDA_DEBUG
+#define KDA_CHECK(st, cond) ::kda::bounds_ok((st), (cond))
+#else
+#define KDA_CHECK(st, cond) true
+#endif
 
 // ------------------------------------------------------------- addressing ----
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {

@@ -78,6 +78,10 @@ struct PrepLayout {
     static constexpr int OFF_QIN = OFF_BK;                   // bf16 [64][DK], 128B swizzle
     static constexpr int OFF_KIN = OFF_BK + CH * DK * 2;
     static constexpr int OFF_MISC = OFF_BK + 128 * 64 * 4;   // beta, barriers, TMEM address
+    // g (per key channel) by TMA during the inputs: fp32 [DK / 32][64 tokens][32 channels],
+    // after the block-products exchange in R_form (free until phase E writes X)
+    static constexpr int OFF_GIN = OFF_F + 4096;
+    static_assert(OFF_GIN + CH * DK * 4 <= OFF_F + RF_B, "g tile fits in R_form");
     static constexpr int TOTAL = OFF_MISC + 1024;
     static constexpr int SMEM_BYTES = TOTAL + 1024;          // slack for the 1 KB base alignment
     static_assert(SMEM_BYTES <= 113 * 1024, "two CTAs per SM");
@@ -104,11 +108,12 @@ __device__ __forceinline__ void prefetch_line_l2(const void *p) {
 // g, beta, q and k are raw projections: g = -c softplus(g_raw), beta =
 // sigmoid(beta_raw), and q, k are L2-normalised per token (the norms come from
 // the staged tiles; the normalised values are rounded to bf16 again, as an
-// unfused caller would store them).
-template <int DK, bool SG, bool PRO>
+// unfused caller would store them).  PACKED: the packed-batch geometry (see
+// SeqGeom), else uniform.
+template <int DK, bool SG, bool PRO, bool PACKED>
 __global__ void __launch_bounds__(PREP_THREADS, 2)
 prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-            const PrepParams prm) {
+            const __grid_constant__ CUtensorMap tm_g, const PrepParams prm) {
     using L = PrepLayout<DK>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -127,7 +132,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     const int ch = tid & 127;        // key channel / TMEM lane of this thread
     const int qb = tid >> 7;         // 16-token block (phase E) / 16-column quarter (elsewhere)
     const int H = prm.H;
-    const int nitems = geom_items(prm.gm, H);
+    const int nitems = geom_items<PACKED>(prm.gm, H);
     const uint64_t polls = prm.st.wait_polls;
 
     if (tid == 0) {
@@ -137,6 +142,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         fence_mbar_init();
         prefetch_tmap(&tm_q);
         prefetch_tmap(&tm_k);
+        if (!SG) prefetch_tmap(&tm_g);
     }
     if (warp == 0) {
         tmem_alloc(smem_u32(s_tmem), L::TM_COLS);
@@ -172,34 +178,49 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     int claim = 0;  // thread 0: the item claimed for after this one (result needed mid-item)
     for (int item = *s_next; item < nitems && !aborted;) {
         if (tid == 0) claim = atomicAdd(prm.ticket, 1);
-        const ItemGeo gi = item_geo(prm.gm, H, item);
+        const ItemGeo gi = item_geo<PACKED>(prm.gm, H, item);
         const int h = gi.h;
         uint8_t *rec = prm.ws + (size_t)gi.rec * REC_BYTES;
+        // debug build: the record and the token rows this item touches
+        const bool rec_in = KDA_CHECK(prm.st, gi.rec >= 0 && gi.rec < prm.nrec);
+        const long long rows = geom_rows(prm.gm);
+        (void)KDA_CHECK(prm.st, h < H && gi.tok0 >= 0 && gi.row0 >= 0);
 
         // ---------------- inputs: q, k by TMA; g (this thread's 16 tokens) and beta by plain loads
         if (tid == 0) {
-            mbar_expect_tx(bar_in, (uint32_t)(2 * CH * DK * 2));
+            mbar_expect_tx(bar_in, (uint32_t)(2 * CH * DK * 2 + (SG ? 0 : CH * DK * 4)));
 #pragma unroll
             for (int kb = 0; kb < DK / 64; ++kb) {
                 tma_load_4d(sbase + L::OFF_QIN + kb * CH * 128, &tm_q, bar_in, kb * 64, h, gi.tok0, gi.bcoord);
                 tma_load_4d(sbase + L::OFF_KIN + kb * CH * 128, &tm_k, bar_in, kb * 64, h, gi.tok0, gi.bcoord);
             }
+            if (!SG) {
+#pragma unroll
+                for (int kb = 0; kb < DK / 32; ++kb)
+                    tma_load_4d(sbase + L::OFF_GIN + kb * CH * 128, &tm_g, bar_in, kb * 32, h, gi.tok0, gi.bcoord);
+            }
         }
         tma_pending = true;
         float al[SUB];
-        {
-            // one gate per key channel, or (SG) one per (token, head) shared by all channels
-            constexpr int gdk = SG ? 1 : DK;
-            const float *gp = prm.g + ((size_t)(gi.row0 + tb) * H + h) * gdk + (SG ? 0 : c);
+        if constexpr (SG) {  // one gate per (token, head), shared by all channels: plain loads
+            const float *gp = prm.g + (size_t)(gi.row0 + tb) * H + h;
 #pragma unroll
-            for (int u = 0; u < SUB; ++u) al[u] = (tb + u < gi.nvalid && active) ? __ldg(gp + (size_t)u * H * gdk) : 0.f;
+            for (int u = 0; u < SUB; ++u)
+                al[u] = (tb + u < gi.nvalid && active && KDA_CHECK(prm.st, gi.row0 + tb + u < rows))
+                            ? __ldg(gp + (size_t)u * H) : 0.f;
         }
         if (tid < CH) {
-            const float braw = (tid < gi.nvalid) ? prm.beta[(size_t)(gi.row0 + tid) * H + h] : 0.f;
+            const float braw = (tid < gi.nvalid && KDA_CHECK(prm.st, gi.row0 + tid < rows))
+                                   ? prm.beta[(size_t)(gi.row0 + tid) * H + h] : 0.f;
             s_beta[tid] = (PRO && tid < gi.nvalid) ? gate_sigmoid(braw) : braw;
         }
         if (!wait_all(bar_in, ph_in, tma_pending)) { aborted = true; break; }
         ph_in ^= 1u;
+        if constexpr (!SG) {  // one gate per key channel, from the g tile (TMA; zero past the tensor)
+            const float *gs = reinterpret_cast<const float *>(sm + L::OFF_GIN) + ((c >> 5) * CH + tb) * 32 + (c & 31);
+#pragma unroll
+            for (int u = 0; u < SUB; ++u) al[u] = (tb + u < gi.nvalid && active) ? gs[u * 32] : 0.f;
+        }
         float *s_rn = reinterpret_cast<float *>(sm + L::OFF_MISC + 256);  // PRO: 1 / |q_t|, then 1 / |k_t|
         if constexpr (PRO) {
 #pragma unroll
@@ -276,10 +297,14 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         __syncthreads();  // the exchange area becomes X
 
         auto yput = [&](int Iy, int j0, const float (&v8)[8]) {
-            *reinterpret_cast<uint4 *>(sm + L::OFF_Y + mnmaj<64, 2>(c, yoff(Iy) + j0, DK)) = pack8_bf16(v8);
+            const uint32_t off = mnmaj<64, 2>(c, yoff(Iy) + j0, DK);
+            if (KDA_CHECK(prm.st, off + 16 <= (uint32_t)(DK * 320)))
+                *reinterpret_cast<uint4 *>(sm + L::OFF_Y + off) = pack8_bf16(v8);
         };
         auto xput = [&](int col, const float (&v8)[8]) {
-            *reinterpret_cast<uint4 *>(sm + L::OFF_X + mnmaj<128, 2>(c, col, DK)) = pack8_bf16(v8);
+            const uint32_t off = mnmaj<128, 2>(c, col, DK);
+            if (KDA_CHECK(prm.st, off + 16 <= (uint32_t)(DK * 256)))
+                *reinterpret_cast<uint4 *>(sm + L::OFF_X + off) = pack8_bf16(v8);
         };
         bool steep = false;  // a split factor of this thread's block would pass e^80
         if (active) {
@@ -351,7 +376,10 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         tc_fence_before();
         const bool exact_item = __syncthreads_or(steep) || prm.force_exact;
         tc_fence_after();
-        if (exact_item && tid == 0) prm.steep_items[atomicAdd(prm.steep_count, 1)] = item;
+        if (exact_item && tid == 0) {
+            const int pos = atomicAdd(prm.steep_count, 1);
+            if (KDA_CHECK(prm.st, pos < nitems)) prm.steep_items[pos] = item;
+        }
 
         // ---------------- F: formation products (bf16), overlapped with the rest of E ----------------
         if (tid == 0) {  // X [Y^(0) | .. | Y^(3)]^T: 128 x 160, column block I' = D^(I')
@@ -367,17 +395,20 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         // e^{Gamma_C - Gamma_t}: K-hat^T (record);  e^{Gamma_t}: Q e^G (record) and (K e^G)^T (smem)
         {
             if (active) {
-                if (I == 0) reinterpret_cast<float *>(rec + REC_DEC)[c] = dec;
+                if (I == 0 && rec_in && KDA_CHECK(prm.st, REC_DEC + 4 * c + 4 <= REC_BYTES))
+                    reinterpret_cast<float *>(rec + REC_DEC)[c] = dec;
                 uint16_t *khr = reinterpret_cast<uint16_t *>(rec + REC_KH) + (I * 128 + c) * SUB;
+                const bool kh_in = rec_in && KDA_CHECK(prm.st, ((I * 128 + c) * SUB + 16) * 2 <= REC_T - REC_KH);
                 float r = postB;
 #pragma unroll
                 for (int hh = 1; hh >= 0; --hh) {
                     float kh[8];
 #pragma unroll
                     for (int e = 7; e >= 0; --e) { kh[e] = kval(hh * 8 + e) * r; r *= al[hh * 8 + e]; }
-                    *reinterpret_cast<uint4 *>(khr + hh * 8) = pack8_f16(kh);
+                    if (kh_in) *reinterpret_cast<uint4 *>(khr + hh * 8) = pack8_f16(kh);
                 }
                 uint16_t *qer = reinterpret_cast<uint16_t *>(rec + REC_WQ) + ((NSUB + I) * DK + c) * SUB;
+                const bool qe_in = rec_in && KDA_CHECK(prm.st, (((NSUB + I) * DK + c) * SUB + 16) * 2 <= REC_P - REC_WQ);
                 float p = preB;
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
@@ -388,11 +419,12 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                         qe[e] = qval(hh * 8 + e) * p;
                         bk[e] = kval(hh * 8 + e) * p;
                     }
-                    *reinterpret_cast<uint4 *>(qer + hh * 8) = pack8_bf16(qe);
-                    *reinterpret_cast<uint4 *>(sm + L::OFF_BK + kmaj<128, 4>(c, tb + hh * 8, 128)) =
-                        pack4_tf32(bk[0], bk[1], bk[2], bk[3]);
-                    *reinterpret_cast<uint4 *>(sm + L::OFF_BK + kmaj<128, 4>(c, tb + hh * 8 + 4, 128)) =
-                        pack4_tf32(bk[4], bk[5], bk[6], bk[7]);
+                    if (qe_in) *reinterpret_cast<uint4 *>(qer + hh * 8) = pack8_bf16(qe);
+                    const uint32_t o0 = kmaj<128, 4>(c, tb + hh * 8, 128), o1 = kmaj<128, 4>(c, tb + hh * 8 + 4, 128);
+                    if (KDA_CHECK(prm.st, o0 + 16 <= 128 * 64 * 4 && o1 + 16 <= 128 * 64 * 4)) {
+                        *reinterpret_cast<uint4 *>(sm + L::OFF_BK + o0) = pack4_tf32(bk[0], bk[1], bk[2], bk[3]);
+                        *reinterpret_cast<uint4 *>(sm + L::OFF_BK + o1) = pack4_tf32(bk[4], bk[5], bk[6], bk[7]);
+                    }
                 }
             }
         }
@@ -402,17 +434,19 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         const int next = *s_next;
         // the next item's q, k and g into L2 while this one finishes
         if (next < nitems) {
-            const ItemGeo ng = item_geo(prm.gm, H, next);
+            const ItemGeo ng = item_geo<PACKED>(prm.gm, H, next);
             if (tid == 0) {
 #pragma unroll
                 for (int kb = 0; kb < DK / 64; ++kb) {
                     prefetch_tensor_4d(&tm_q, kb * 64, ng.h, ng.tok0, ng.bcoord);
                     prefetch_tensor_4d(&tm_k, kb * 64, ng.h, ng.tok0, ng.bcoord);
                 }
-            } else if (tid >= 64 && tid < 64 + CH && tid - 64 < ng.nvalid) {
-                const float *gr = prm.g + ((size_t)(ng.row0 + tid - 64) * H + ng.h) * (SG ? 1 : DK);
-                if (SG) prefetch_line_l2(gr);
-                else prefetch_l2(gr, DK * 4);
+                if (!SG) {
+#pragma unroll
+                    for (int kb = 0; kb < DK / 32; ++kb) prefetch_tensor_4d(&tm_g, kb * 32, ng.h, ng.tok0, ng.bcoord);
+                }
+            } else if (SG && tid >= 64 && tid < 64 + CH && tid - 64 < ng.nvalid) {
+                prefetch_line_l2(prm.g + (size_t)(ng.row0 + tid - 64) * H + ng.h);
             }
         }
 
@@ -456,12 +490,13 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 }
             } else {
                 uint16_t *pr = reinterpret_cast<uint16_t *>(rec + REC_P) + (cc * CH + i) * SUB;
+                const bool p_in = rec_in && KDA_CHECK(prm.st, ((cc * CH + i) * SUB + 16) * 2 <= REC_KH - REC_P);
 #pragma unroll
                 for (int e8 = 0; e8 < 16; e8 += 8) {
                     float p8[8];
 #pragma unroll
                     for (int e = 0; e < 8; ++e) p8[e] = (j0 + e8 + e <= i) ? v16[e8 + e] : 0.f;
-                    *reinterpret_cast<uint4 *>(pr + e8) = pack8_f16(p8);
+                    if (p_in) *reinterpret_cast<uint4 *>(pr + e8) = pack8_f16(p8);
                 }
             }
         }
@@ -562,8 +597,11 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 const float4 bj = *reinterpret_cast<const float4 *>(s_beta + j);
                 const float4 w = make_float4(j + 0 <= i ? src[0] * bj.x : 0.f, j + 1 <= i ? src[1] * bj.y : 0.f,
                                              j + 2 <= i ? src[2] * bj.z : 0.f, j + 3 <= i ? src[3] * bj.w : 0.f);
-                *reinterpret_cast<uint4 *>(sm + L::OFF_T + kmaj_s<128, 4>(i, j, 8192)) = pack4_tf32(w.x, w.y, w.z, w.w);
-                *reinterpret_cast<float4 *>(rec + REC_T + (i * CH + j) * 4) = w;
+                const uint32_t ot = kmaj_s<128, 4>(i, j, 8192);
+                if (KDA_CHECK(prm.st, ot + 16 <= 16384))
+                    *reinterpret_cast<uint4 *>(sm + L::OFF_T + ot) = pack4_tf32(w.x, w.y, w.z, w.w);
+                if (rec_in && KDA_CHECK(prm.st, (i * CH + j) * 4 + 16 <= REC_DEC - REC_T))
+                    *reinterpret_cast<float4 *>(rec + REC_T + (i * CH + j) * 4) = w;
             }
         }
         sync_for_mma();
@@ -589,8 +627,10 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 #pragma unroll
             for (int e = 0; e < 8; ++e) { a8[e] = t[e]; b8[e] = t[8 + e]; }
             uint16_t *wr = reinterpret_cast<uint16_t *>(rec + REC_WQ) + (qb * DK + ch) * SUB;
-            *reinterpret_cast<uint4 *>(wr) = pack8_bf16(a8);
-            *reinterpret_cast<uint4 *>(wr + 8) = pack8_bf16(b8);
+            if (rec_in && KDA_CHECK(prm.st, ((qb * DK + ch) * SUB + 16) * 2 <= NSUB * DK * SUB * 2)) {
+                *reinterpret_cast<uint4 *>(wr) = pack8_bf16(a8);
+                *reinterpret_cast<uint4 *>(wr + 8) = pack8_bf16(b8);
+            }
         }
         tc_fence_before();
         __syncthreads();  // this item's shared memory and TMEM are free for the next one
@@ -610,36 +650,41 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     if (tid == 0) stamp_end(prm.stamp);
 }
 
-template <int DK, bool SG, bool PRO>
-static cudaError_t launch_prep_t(const CUtensorMap &tq, const CUtensorMap &tk, const PrepParams &prm,
-                                 int max_ctas, cudaStream_t stream) {
+template <int DK, bool SG, bool PRO, bool PACKED = false>
+static cudaError_t launch_prep_t(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tg,
+                                 const PrepParams &prm, int max_ctas, cudaStream_t stream) {
     using L = PrepLayout<DK>;
-    cudaError_t e = cudaFuncSetAttribute(prep_kernel<DK, SG, PRO>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(prep_kernel<DK, SG, PRO, PACKED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          L::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     // items of the launch (packed: an upper bound, the kernel reads the exact count)
     const long long items = prm.gm.cu == nullptr ? (long long)prm.gm.nseqs * prm.H * prm.gm.nseg
                                                  : (long long)prm.gm.W * prm.H;
     const int grid = (int)(items < max_ctas ? items : max_ctas);
-    prep_kernel<DK, SG, PRO><<<grid, PREP_THREADS, L::SMEM_BYTES, stream>>>(tq, tk, prm);
+    prep_kernel<DK, SG, PRO, PACKED><<<grid, PREP_THREADS, L::SMEM_BYTES, stream>>>(tq, tk, tg, prm);
     return cudaGetLastError();
 }
 
 // At most max_ctas persistent CTAs (two fit on an SM), at most one per item;
-// prm.g_dk selects the gate form (dk: per key channel, 1: scalar); `prologue`
-// the raw-input form (per key channel only).
-cudaError_t launch_prep(const CUtensorMap &tq, const CUtensorMap &tk, const PrepParams &prm, int dk,
-                        int max_ctas, cudaStream_t stream, bool prologue) {
+// prm.g_dk selects the gate form (dk: per key channel, read through tg; 1:
+// scalar, tg unused); `prologue` the raw-input form (per key channel only).
+cudaError_t launch_prep(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tg, const PrepParams &prm,
+                        int dk, int max_ctas, cudaStream_t stream, bool prologue) {
     const bool sg = prm.g_dk == 1;
+    if (prm.gm.cu != nullptr) {  // packed batches: per-channel gate, inputs as given
+        if (sg || prologue) return cudaErrorInvalidValue;
+        return dk == 128 ? launch_prep_t<128, false, false, true>(tq, tk, tg, prm, max_ctas, stream)
+                         : launch_prep_t<64, false, false, true>(tq, tk, tg, prm, max_ctas, stream);
+    }
     if (prologue) {
         if (sg) return cudaErrorInvalidValue;
-        return dk == 128 ? launch_prep_t<128, false, true>(tq, tk, prm, max_ctas, stream)
-                         : launch_prep_t<64, false, true>(tq, tk, prm, max_ctas, stream);
+        return dk == 128 ? launch_prep_t<128, false, true>(tq, tk, tg, prm, max_ctas, stream)
+                         : launch_prep_t<64, false, true>(tq, tk, tg, prm, max_ctas, stream);
     }
-    if (dk == 128) return sg ? launch_prep_t<128, true, false>(tq, tk, prm, max_ctas, stream)
-                             : launch_prep_t<128, false, false>(tq, tk, prm, max_ctas, stream);
-    return sg ? launch_prep_t<64, true, false>(tq, tk, prm, max_ctas, stream)
-              : launch_prep_t<64, false, false>(tq, tk, prm, max_ctas, stream);
+    if (dk == 128) return sg ? launch_prep_t<128, true, false>(tq, tk, tg, prm, max_ctas, stream)
+                             : launch_prep_t<128, false, false>(tq, tk, tg, prm, max_ctas, stream);
+    return sg ? launch_prep_t<64, true, false>(tq, tk, tg, prm, max_ctas, stream)
+              : launch_prep_t<64, false, false>(tq, tk, tg, prm, max_ctas, stream);
 }
 
 }  // namespace kda

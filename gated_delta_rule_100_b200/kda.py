@@ -29,18 +29,21 @@ import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libkda.so")
+DEBUG_LIB_PATH = os.path.join(_HERE, "libkda_debug.so")
 
 (KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_ALIGNMENT, KDA_ERR_CUDA, KDA_ERR_TIMEOUT,
- KDA_ERR_SCRATCH_LIMIT) = range(7)
+ KDA_ERR_SCRATCH_LIMIT, KDA_ERR_BOUNDS) = range(8)
 EXPORTED = ("kda_chunk_fwd", "kda_chunk_fwd_noalloc", "kda_chunk_fwd_varlen", "kda_decode_step",
             "kda_gdn_chunk_fwd", "kda_gdn_decode_step", "kda_chunk_fwd_raw", "kda_decode_step_raw",
+            "kda_chunk_bwd", "kda_chunk_bwd_workspace_bytes",
             "kda_chunk_fwd_workspace_bytes", "kda_chunk_fwd_varlen_workspace_bytes", "kda_release_workspace",
             "kda_status_string", "kda_stream_status", "kda_chunk_fwd_debug_wait_limit",
             "kda_chunk_fwd_debug_inject_timeout", "kda_chunk_fwd_debug_force_exact", "kda_chunk_fwd_debug_record_cap", "kda_chunk_fwd_debug_parts",
             "kda_debug_kernel_timing", "kda_debug_kernel_times",
             "kda_abi_version")
 
-_lib = None
+_lib = None          # the library the calls below go through
+_libs = {}           # path -> loaded library
 
 
 class KdaError(RuntimeError):
@@ -50,19 +53,38 @@ class KdaError(RuntimeError):
 
 
 def load():
-    """Load libkda.so (built in-tree by ``gated_delta_rule_100_b200.build``)."""
+    """The library the binding's calls go through: libkda.so (built in-tree by
+    ``gated_delta_rule_100_b200.build``) unless ``use_debug_library(True)``."""
     global _lib
-    if _lib is not None:
-        return _lib
-    if not os.path.exists(LIB_PATH):
-        raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+    if _lib is None:
+        _lib = _open(LIB_PATH)
+    return _lib
+
+
+def use_debug_library(enable: bool) -> None:
+    """Route every call through libkda_debug.so (device-side index checks that
+    report KDA_ERR_BOUNDS) or back through libkda.so.  The two libraries have
+    separate device state (status word, workspace)."""
+    global _lib
+    _lib = _open(DEBUG_LIB_PATH if enable else LIB_PATH)
+
+
+def _open(path):
+    if path in _libs:
+        return _libs[path]
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with "
                            "`python -m gated_delta_rule_100_b200.build`")
-    lib = ctypes.CDLL(LIB_PATH)
+    lib = ctypes.CDLL(path)
     vp, fp, i, f = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_float
     lib.kda_chunk_fwd.argtypes = [vp, vp, vp, fp, fp, f, fp, vp, fp, i, i, i, i, i, vp]
     lib.kda_chunk_fwd.restype = i
     lib.kda_chunk_fwd_noalloc.argtypes = [vp, vp, vp, fp, fp, f, fp, vp, fp, i, i, i, i, i, vp]
     lib.kda_chunk_fwd_noalloc.restype = i
+    lib.kda_chunk_bwd.argtypes = [vp, vp, vp, fp, fp, f, fp, vp, fp, vp, vp, vp, fp, fp, fp, i, i, i, i, i, vp]
+    lib.kda_chunk_bwd.restype = i
+    lib.kda_chunk_bwd_workspace_bytes.argtypes = [i, i, i, i, i]
+    lib.kda_chunk_bwd_workspace_bytes.restype = ctypes.c_size_t
     lib.kda_chunk_fwd_raw.argtypes = [vp, vp, vp, fp, fp, f, f, fp, vp, fp, i, i, i, i, i, vp]
     lib.kda_chunk_fwd_raw.restype = i
     lib.kda_decode_step_raw.argtypes = [vp, vp, vp, fp, fp, f, f, fp, vp, i, i, i, i, vp]
@@ -100,7 +122,7 @@ def load():
     lib.kda_debug_kernel_times.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_longlong), i]
     lib.kda_debug_kernel_times.restype = i
     lib.kda_abi_version.restype = i
-    _lib = lib
+    _libs[path] = lib
     return lib
 
 
@@ -164,6 +186,38 @@ def _prefill(symbol, scalar_gate, q, k, v, g, beta, scale, h0, out, hT, final_st
     if rc != KDA_OK:
         raise KdaError(rc, symbol)
     return out, hT
+
+
+def chunk_bwd(q, k, v, g, beta, scale, h0=None, dout=None, dhT=None, *, want_dh0=True, stream=None):
+    """Backward of ``chunk_fwd``: gradients of L given dL/dout (bf16 [B,T,H,dv]) and
+    dL/dhT (fp32 [B,H,dk,dv]); either may be None (zero).  Returns a dict with dq, dk,
+    dv (bf16), dg, dbeta and dh0 (fp32; None when ``want_dh0`` is False)."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    _check(q, "q", torch.bfloat16, (B, T, H, dk))
+    _check(k, "k", torch.bfloat16, (B, T, H, dk))
+    _check(v, "v", torch.bfloat16, (B, T, H, dv))
+    _check(g, "g", torch.float32, (B, T, H, dk))
+    _check(beta, "beta", torch.float32, (B, T, H))
+    if h0 is not None:
+        _check(h0, "h0", torch.float32, (B, H, dk, dv))
+    if dout is not None:
+        _check(dout, "dout", torch.bfloat16, (B, T, H, dv))
+    if dhT is not None:
+        _check(dhT, "dhT", torch.float32, (B, H, dk, dv))
+    z = dict(device=q.device)
+    r = dict(dq=torch.empty((B, T, H, dk), dtype=torch.bfloat16, **z),
+             dk=torch.empty((B, T, H, dk), dtype=torch.bfloat16, **z),
+             dv=torch.empty((B, T, H, dv), dtype=torch.bfloat16, **z),
+             dg=torch.empty((B, T, H, dk), dtype=torch.float32, **z),
+             dbeta=torch.empty((B, T, H), dtype=torch.float32, **z),
+             dh0=torch.empty((B, H, dk, dv), dtype=torch.float32, **z) if want_dh0 else None)
+    rc = load().kda_chunk_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale), _ptr(h0), _ptr(dout),
+                              _ptr(dhT), _ptr(r["dq"]), _ptr(r["dk"]), _ptr(r["dv"]), _ptr(r["dg"]), _ptr(r["dbeta"]),
+                              _ptr(r["dh0"]), B, T, H, dk, dv, _stream(stream))
+    if rc != KDA_OK:
+        raise KdaError(rc, "kda_chunk_bwd")
+    return r
 
 
 def chunk_fwd_raw(q, k, v, g_raw, beta_raw, gate_c, scale, h0=None, *, out=None, hT=None, final_state=True,
@@ -348,7 +402,7 @@ def force_exact(enable: bool) -> None:
     load().kda_chunk_fwd_debug_force_exact(1 if enable else 0)
 
 
-KERNEL_KINDS = ("prep", "chain", "exact", "fixup")
+KERNEL_KINDS = ("prep", "chain", "exact", "fixup", "bwd")
 
 
 def kernel_timing(enable: bool) -> None:

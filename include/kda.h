@@ -72,7 +72,8 @@ typedef enum {
     KDA_ERR_ALIGNMENT = 3,   /* a pointer below its required alignment        */
     KDA_ERR_CUDA = 4,        /* a CUDA runtime/driver call or launch failed    */
     KDA_ERR_TIMEOUT = 5,     /* a device-side bounded wait gave up             */
-    KDA_ERR_SCRATCH_LIMIT = 6 /* kda_chunk_fwd_noalloc: problem exceeds its fixed scratch */
+    KDA_ERR_SCRATCH_LIMIT = 6, /* kda_chunk_fwd_noalloc: problem exceeds its fixed scratch */
+    KDA_ERR_BOUNDS = 7       /* debug build (libkda_debug.so): an index check failed */
 } kda_status;
 
 /*
@@ -194,6 +195,40 @@ KDA_API int kda_decode_step_raw(const void *q, const void *k, const void *v,
                   int B, int H, int dk, int dv, void *stream);
 
 /*
+ * kda_chunk_bwd -- the backward pass of kda_chunk_fwd: the gradients of a
+ * loss L with respect to q, k, v, g, beta and h0, given dL/dout and dL/dhT.
+ * The pages describe training ("Kimi Linear" explainer, "Chunked
+ * Processing": training speed comparable to FlashAttention) but print no
+ * backward; this is reverse-mode differentiation of the recurrence of section
+ * 3.3 of the Baidu breakdown, evaluated in its recurrent form: a forward walk
+ * that stores the state every 8 tokens, then a backward walk over the tokens
+ * that recomputes each token's state from checkpoints (two levels: a state
+ * every 64 tokens from the forward walk, then per 64-token chunk a state every
+ * 8 tokens).  fp32 arithmetic on CUDA cores, one CTA per (b, h).
+ *
+ *   q, k, v, g, beta, scale, h0 : the forward's inputs (layouts of kda_chunk_fwd)
+ *   dout  : bf16 [B, T, H, dv]   dL/dout, or NULL (zero)
+ *   dhT   : fp32 [B, H, dk, dv]  dL/dhT, or NULL (zero)
+ *   dq, dk: bf16 [B, T, H, dk]   (written)
+ *   dv    : bf16 [B, T, H, dv]
+ *   dg    : fp32 [B, T, H, dk]   gradient of the log-decay
+ *   dbeta : fp32 [B, T, H]
+ *   dh0   : fp32 [B, H, dk, dv]  or NULL (not written)
+ *
+ * Workspace: the checkpoints, B H (ceil(T / 64) + 8) dk dv fp32
+ * (kda_chunk_bwd_workspace_bytes: 1.1 GB for B8 H32 T4096 d128, 34 GB for
+ * B1 H32 T1M), held like the prefill's workspace (grown with cudaMalloc,
+ * freed by kda_release_workspace).  T == 0 sets dh0 = dhT.
+ * Errors as kda_chunk_fwd.
+ */
+KDA_API int kda_chunk_bwd(const void *q, const void *k, const void *v,
+                  const float *g, const float *beta, float scale, const float *h0,
+                  const void *dout, const float *dhT,
+                  void *dq, void *dk, void *dv, float *dg, float *dbeta, float *dh0,
+                  int B, int T, int H, int dk_, int dv_, void *stream);
+KDA_API size_t kda_chunk_bwd_workspace_bytes(int B, int T, int H, int dk, int dv);
+
+/*
  * kda_chunk_fwd_varlen -- chunkwise prefill over a packed batch of N sequences
  * of different lengths, each with its own initial and final state.  This is
  * the serving form of the prefill: a batch of requests concatenated along the
@@ -296,7 +331,16 @@ KDA_API const char *kda_status_string(int status);
  * kda_stream_status -- synchronise `stream`, then read and clear the current
  * device's status word.  Returns KDA_OK, KDA_ERR_TIMEOUT when a kernel's
  * bounded wait gave up since the last call (that kernel's outputs are then
- * unspecified), or KDA_ERR_CUDA when the synchronisation itself failed.
+ * unspecified), KDA_ERR_INVALID_ARG when kda_chunk_fwd_varlen found bad
+ * offsets, KDA_ERR_BOUNDS when (debug build only) an index check failed, or
+ * KDA_ERR_CUDA when the synchronisation itself failed.
+ *
+ * Debug build.  libkda_debug.so is this library compiled with KDA_DEBUG: the
+ * kernels check, before each access whose bounds rest on layout constants and
+ * launch geometry (record indices and offsets, shared-memory tiles and tensor
+ * operand views, token rows, state slices), that it stays in bounds; a failed
+ * check skips the access and sets the status reported as KDA_ERR_BOUNDS.  It
+ * exports the same symbols and is for testing; it is slower.
  */
 KDA_API int kda_stream_status(void *stream);
 
@@ -348,21 +392,28 @@ KDA_API void kda_chunk_fwd_debug_parts(int parts);
 
 /*
  * kda_debug_kernel_timing -- measurement hook.  While enabled (enable != 0),
- * every kda_chunk_fwd records a pair of CUDA events on its stream around each
- * kernel it launches (kind 0 = the per-chunk prep kernel, kind 1 = the state
- * chain kernel).  Process-wide; off by default.
+ * every kernel launch of the prefill and backward entry points gets a timing
+ * slot: the kernel's own CTAs record, with %globaltimer, when the first of
+ * them started and the last of them ended (two atomics per CTA; nothing is
+ * added to the streams' ordering).  Kinds: 0 = the per-chunk prep kernel,
+ * 1 = the state chain kernel, 2 = the exact kernel of steep chunks, 3 = the
+ * two-level pass's fix-up, 4 = the backward pass (both of its kernels).
+ * At most 8192 launches per device are timed between two reads.
+ * Process-wide; off by default.
  *
- * kda_debug_kernel_times -- waits for the events recorded so far, writes per
- * kind the summed device time in ms (ms[kind]) and the number of launches
- * (launches[kind]) for kinds < nkinds, and forgets them.  The host arrays are
- * the caller's.  KDA_OK, KDA_ERR_INVALID_ARG for NULL arrays, or KDA_ERR_CUDA.
+ * kda_debug_kernel_times -- waits for the device(s), writes per kind the
+ * summed busy time of the launches timed so far in ms (ms[kind]) and their
+ * number (launches[kind]) for kinds < nkinds, and forgets them.  The host
+ * arrays are the caller's.  KDA_OK, KDA_ERR_INVALID_ARG for NULL arrays, or
+ * KDA_ERR_CUDA.
  */
 KDA_API void kda_debug_kernel_timing(int enable);
 KDA_API int kda_debug_kernel_times(double *ms, long long *launches, int nkinds);
 
 /* Version of this ABI (major * 100 + minor): 101 adds the scalar-gate entry
  * points, 102 the packed-batch prefill, the raw-input (fused gate prologue)
- * entry points and the exact-path test hooks. */
+ * entry points, the backward pass and the exact-path and two-level test
+ * hooks. */
 KDA_API int kda_abi_version(void);
 
 #ifdef __cplusplus

@@ -227,3 +227,35 @@ def test_raw_entry_points_validate_gate_scale(lib):
     assert raw(0.5, k=MIS) == kda.KDA_ERR_ALIGNMENT
     assert lib.kda_decode_step_raw(A, A, A, A, A, -1.0, 1.0, A, A, 1, 1, 64, 64, None) == kda.KDA_ERR_INVALID_ARG
     assert lib.kda_decode_step_raw(A, A, A, A, A, 1.0, 1.0, None, A, 1, 1, 64, 64, None) == kda.KDA_ERR_INVALID_ARG
+
+
+def test_backward_rejects(lib):
+    def bwd(**kw):
+        a = dict(q=A, k=A, v=A, g=A, beta=A, h0=None, dout=A, dhT=None, dq=A, dk=A, dv=A, dg=A, db=A, dh0=None,
+                 B=1, T=64, H=1, dk_=64, dv_=64)
+        a.update(kw)
+        return lib.kda_chunk_bwd(a["q"], a["k"], a["v"], a["g"], a["beta"], 1.0, a["h0"], a["dout"], a["dhT"],
+                                 a["dq"], a["dk"], a["dv"], a["dg"], a["db"], a["dh0"], a["B"], a["T"], a["H"],
+                                 a["dk_"], a["dv_"], None)
+    assert bwd(q=None) == kda.KDA_ERR_INVALID_ARG
+    assert bwd(dg=None) == kda.KDA_ERR_INVALID_ARG
+    assert bwd(B=0) == kda.KDA_ERR_INVALID_ARG
+    assert bwd(dk_=96) == kda.KDA_ERR_UNSUPPORTED
+    assert bwd(dq=MIS) == kda.KDA_ERR_ALIGNMENT
+    assert bwd(db=ODD) == kda.KDA_ERR_ALIGNMENT
+    # T == 0 with no dh0 wanted: nothing to do
+    assert bwd(q=None, k=None, v=None, g=None, beta=None, dq=None, dk=None, dv=None, dg=None, db=None, T=0) == \
+        kda.KDA_OK
+    # a state every 64 tokens and a scratch of 8 states, per (b, h)
+    assert lib.kda_chunk_bwd_workspace_bytes(2, 100, 3, 128, 64) == 2 * 3 * (2 + 8) * 128 * 64 * 4
+
+
+def test_debug_library_exports_the_same_symbols(lib):
+    """libkda_debug.so (KDA_DEBUG: device-side index checks) is a separate build
+    of the same sources with the same C ABI."""
+    from gated_delta_rule_100_b200 import kda as k
+    dbg = ctypes.CDLL(k.DEBUG_LIB_PATH)
+    for name in declared_symbols():
+        assert hasattr(dbg, name), name
+    assert os.path.getsize(k.DEBUG_LIB_PATH) != os.path.getsize(k.LIB_PATH)
+    assert kda.status_string(kda.KDA_ERR_BOUNDS) == "KDA_ERR_BOUNDS"

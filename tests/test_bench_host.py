@@ -23,55 +23,64 @@ def test_source_key_sees_code_changes():
 
 
 def test_traffic_figure_is_tied_to_its_sources(tmp_path, monkeypatch):
-    """bench.py reports a committed traffic figure only for the sources it was
-    taken on: a key that does not match gives None."""
+    """bench.py reports a committed traffic figure only while the kernel's device
+    sources are those it was taken on: a key that does not match gives None."""
     prof = tmp_path / "profiles"
     prof.mkdir()
-    t = {"source_hash": bench.kernel_source_hash(), "captured_on": "w",
-         "kernels": {"prep_kernel": {"mean_bytes_per_launch": 123.0, "bytes_per_token_head": 7.0}}}
+    t = {"kernels": {"prep_kernel": {"source_hash": "abc", "captured_on": "w",
+                                     "mean_bytes_per_launch": 123.0, "bytes_per_token_head": 7.0}}}
     (prof / "traffic.json").write_text(json.dumps(t))
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
-    monkeypatch.setattr(bench, "kernel_source_hash", lambda: t["source_hash"])
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda kernel=None: "abc")
     assert bench.measured_traffic("prep_kernel") == (123.0, "w")
     assert bench.measured_traffic("prep_kernel", "bytes_per_token_head") == (7.0, "w")
     assert bench.measured_traffic("chain_kernel") == (None, None)
-    monkeypatch.setattr(bench, "kernel_source_hash", lambda: "another")
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda kernel=None: "another")
     assert bench.measured_traffic("prep_kernel") == (None, None)
 
 
-def test_record_traffic_from_ncu_csv(tmp_path, monkeypatch):
-    """The ncu CSV of two prep and one chain launch on the long-context slice
-    becomes per-kernel bytes per launch and per token-head, keyed to the sources."""
-    rows = [
-        ["ID", "Process ID", "Process Name", "Host Name", "Kernel Name", "Context", "Stream", "Block Size",
-         "Grid Size", "Device", "CC", "Section Name", "Metric Name", "Metric Unit", "Metric Value"],
-    ]
+def test_kernel_source_keys_cover_their_files():
+    """Each kernel's key changes with its own sources only."""
+    assert bench.kernel_source_hash("prep_kernel") != bench.kernel_source_hash("chain_kernel")
+    assert bench.kernel_source_hash("decode_step_kernel") != bench.kernel_source_hash()
+    for files in bench.KERNEL_SOURCES.values():
+        for name in files:
+            assert os.path.exists(os.path.join(ROOT, "gated_delta_rule_100_b200", "csrc", name)), name
+
+
+def test_record_traffic_from_ncu_csv(tmp_path):
+    """The ncu CSV of prep, exact and chain launches on the long-context slice
+    becomes per-kernel bytes per launch and per token-head, each keyed to that
+    kernel's sources (an exact_prep_kernel launch is not taken for prep_kernel)."""
+    import csv
+    rows = [["ID", "Process ID", "Process Name", "Host Name", "Kernel Name", "Context", "Stream", "Block Size",
+             "Grid Size", "Device", "CC", "Section Name", "Metric Name", "Metric Unit", "Metric Value"]]
+
     def add(i, kern, name, unit, val):
         rows.append([str(i), "1", "python", "h", kern, "1", "7", "(512,1,1)", "(296,1,1)", "0", "10.0", "",
                      name, unit, val])
-    add(0, "void kda::prep_kernel<128, false, false>(CUtensorMap, CUtensorMap, kda::PrepParams)",
-        "dram__bytes_read.sum", "Gbyte", "1.5")
-    add(0, "void kda::prep_kernel<128, false, false>(CUtensorMap, CUtensorMap, kda::PrepParams)",
-        "dram__bytes_write.sum", "Mbyte", "500")
+    prep = "void prep_kernel<128, 0, 0>(CUtensorMap_st, CUtensorMap_st, PrepParams)"
+    add(0, prep, "dram__bytes_read.sum", "Gbyte", "1.5")
+    add(0, prep, "dram__bytes_write.sum", "Mbyte", "500")
+    add(9, "void exact_prep_kernel<128, 0>(ExactParams)", "dram__bytes_read.sum", "byte", "24576")
     add(1, "void kda::chain_kernel<128, 64>(...)", "dram__bytes_read.sum", "Gbyte", "2.0")
     add(1, "void kda::chain_kernel<128, 64>(...)", "dram__bytes_write.sum", "byte", "1,000")
-    add(2, "void kda::prep_kernel<128, false, false>(CUtensorMap, CUtensorMap, kda::PrepParams)",
-        "dram__bytes_read.sum", "Gbyte", "1.0")
-    add(2, "void kda::prep_kernel<128, false, false>(CUtensorMap, CUtensorMap, kda::PrepParams)",
-        "dram__bytes_write.sum", "Gbyte", "1.0")
-    import csv
+    add(2, prep, "dram__bytes_read.sum", "Gbyte", "1.0")
+    add(2, prep, "dram__bytes_write.sum", "Gbyte", "1.0")
     path = tmp_path / "t.csv"
     with open(path, "w", newline="") as f:
+        f.write("==PROF== Connected to process 1\n")
         csv.writer(f).writerows(rows)
     out = tmp_path / "traffic.json"
     t = bench.record_traffic(str(path), "long_context_slice_B1_H32_T65536_d128", str(out))
-    assert t["source_hash"] == bench.kernel_source_hash()
-    prep = t["kernels"]["prep_kernel"]
-    assert prep["launches_captured"] == 2 and prep["bytes_per_launch"] == [2.0e9, 2.0e9]
+    p = t["kernels"]["prep_kernel"]
+    assert p["source_hash"] == bench.kernel_source_hash("prep_kernel")
+    assert p["launches_captured"] == 2 and p["bytes_per_launch"] == [2.0e9, 2.0e9]
     th = bench.prep_launch_token_heads(1, 65536, 32)
     assert th[:2] == [32 * 451 * 64] * 2 and sum(th) == 32 * 65536
-    assert abs(prep["bytes_per_token_head"] - 4.0e9 / (2 * 32 * 451 * 64)) < 1e-9
+    assert abs(p["bytes_per_token_head"] - 4.0e9 / (2 * 32 * 451 * 64)) < 1e-9
     assert t["kernels"]["chain_kernel"]["mean_bytes_per_launch"] == 2.0e9 + 1000
+    assert t["kernels"]["exact_prep_kernel"]["launches_captured"] == 1
 
 
 def test_scalar_gate_line_with_stand_in_device(monkeypatch):
