@@ -22,14 +22,15 @@
 //          CK1 = 64 tokens (level-1 checkpoints, fp32, in the workspace).
 //   Pass 2 (bwd_kernel): chunks of CK1 tokens from the last to the first.  Per
 //          chunk, the forward is re-run from its level-1 checkpoint to leave a
-//          state every CK = 8 tokens in a per-(b, h) scratch (level 2); then
+//          state every CK = 4 tokens in a per-(b, h) scratch (level 2); then
 //          blocks of CK tokens from the last to the first: for token t of a
 //          block, the state before t is recomputed from the block's checkpoint
 //          (kept in shared memory), then the reverse step.  After each block
 //          its tokens' dq, dk (bf16), dg and dbeta (fp32) are written; dv per
 //          column as it is formed; dh0 at the end.
-// Memory: (ceil(T / 64) + 8) dk dv fp32 per (b, h); forward steps per token:
-// one in pass 1, one for level 2, 3.5 on average for the per-token states.
+// Memory: (ceil(T / 64) + 16) dk dv fp32 per (b, h); forward steps per token:
+// one in pass 1, one for level 2, 1.5 on average for the per-token states
+// (blocks of 8 took 56 ms on B8 H32 T4096, 3.5 recomputed steps per token).
 // Inputs are staged in shared memory per block of tokens.  Level-2 states go
 // through global memory (the scratch), read back after a block barrier.
 #include <cuda_bf16.h>
@@ -42,7 +43,7 @@ namespace kda {
 
 constexpr int BWD_THREADS = 512;
 constexpr int BWD_CK1 = 64;  // tokens per level-1 checkpoint
-constexpr int BWD_CK = 8;    // tokens per level-2 checkpoint (per block)
+constexpr int BWD_CK = 4;    // tokens per level-2 checkpoint (per block)
 constexpr int BWD_FT = 32;   // tokens staged at a time in pass 1
 
 // This lane's CW consecutive state columns of row r (CW a multiple of 4, 16-byte aligned).

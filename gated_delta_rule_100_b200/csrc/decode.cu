@@ -27,12 +27,14 @@ namespace kda {
 
 constexpr int DEC_THREADS = 256;
 
-template <int DK, int DV>
+// PRO: the gate prologue (raw g, beta, q, k), a separate instantiation so that
+// the plain kernel carries none of it.
+template <int DK, int DV, bool PRO>
 __global__ void __launch_bounds__(DEC_THREADS)
 decode_step_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ k,
                    const uint16_t *__restrict__ v, const float *__restrict__ g,
                    const float *__restrict__ beta, float scale, float *__restrict__ state,
-                   uint16_t *__restrict__ out, int g_dk, int prologue, float gate_c) {
+                   uint16_t *__restrict__ out, int g_dk, float gate_c) {
     constexpr int NCG = DV / 4;              // float4 column groups
     constexpr int NRG = DEC_THREADS / NCG;   // row groups
     constexpr int RPT = DK / NRG;            // state rows per thread
@@ -63,10 +65,10 @@ decode_step_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ 
         s_k[r] = bf16_bits_to_f32(kh[r]);
         s_q[r] = bf16_bits_to_f32(qh[r]);
         const float gr = gh[g_dk > 1 ? r : 0];
-        s_a[r] = __expf(prologue ? gate_logdecay(gr, gate_c) : gr);
+        s_a[r] = __expf(PRO ? gate_logdecay(gr, gate_c) : gr);
     }
     __syncthreads();
-    if (prologue) {  // raw q, k: L2-normalise each (warp 0: q, warp 1: k), as the prefill's prologue
+    if constexpr (PRO) {  // raw q, k: L2-normalise each (warp 0: q, warp 1: k), as the prefill's prologue
         if (tid < 64) {
             float *x = tid < 32 ? s_q : s_k;
             const int ln = tid & 31;
@@ -109,7 +111,7 @@ decode_step_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ 
         p.x += a.x; p.y += a.y; p.z += a.z; p.w += a.w;
         y.x += b.x; y.y += b.y; y.z += b.z; y.w += b.w;
     }
-    const float bt = prologue ? gate_sigmoid(beta[bh]) : beta[bh];
+    const float bt = PRO ? gate_sigmoid(beta[bh]) : beta[bh];
     const uint16_t *vh = v + (size_t)bh * DV + cg * 4;
     float4 u;
     u.x = bt * (bf16_bits_to_f32(vh[0]) - p.x);
@@ -139,9 +141,14 @@ template <int DK, int DV>
 static cudaError_t launch_decode_t(const void *q, const void *k, const void *v, const float *g,
                                    const float *beta, float scale, float *state, void *out,
                                    int BH, int g_dk, int prologue, float gate_c, cudaStream_t stream) {
-    decode_step_kernel<DK, DV><<<BH, DEC_THREADS, 0, stream>>>(
-        (const uint16_t *)q, (const uint16_t *)k, (const uint16_t *)v, g, beta, scale, state,
-        (uint16_t *)out, g_dk, prologue, gate_c);
+    if (prologue)
+        decode_step_kernel<DK, DV, true><<<BH, DEC_THREADS, 0, stream>>>(
+            (const uint16_t *)q, (const uint16_t *)k, (const uint16_t *)v, g, beta, scale, state,
+            (uint16_t *)out, g_dk, gate_c);
+    else
+        decode_step_kernel<DK, DV, false><<<BH, DEC_THREADS, 0, stream>>>(
+            (const uint16_t *)q, (const uint16_t *)k, (const uint16_t *)v, g, beta, scale, state,
+            (uint16_t *)out, g_dk, gate_c);
     return cudaGetLastError();
 }
 

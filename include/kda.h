@@ -204,7 +204,7 @@ KDA_API int kda_decode_step_raw(const void *q, const void *k, const void *v,
  * that stores the state every 8 tokens, then a backward walk over the tokens
  * that recomputes each token's state from checkpoints (two levels: a state
  * every 64 tokens from the forward walk, then per 64-token chunk a state every
- * 8 tokens).  fp32 arithmetic on CUDA cores, one CTA per (b, h).
+ * 4 tokens).  fp32 arithmetic on CUDA cores, one CTA per (b, h).
  *
  *   q, k, v, g, beta, scale, h0 : the forward's inputs (layouts of kda_chunk_fwd)
  *   dout  : bf16 [B, T, H, dv]   dL/dout, or NULL (zero)
@@ -215,8 +215,8 @@ KDA_API int kda_decode_step_raw(const void *q, const void *k, const void *v,
  *   dbeta : fp32 [B, T, H]
  *   dh0   : fp32 [B, H, dk, dv]  or NULL (not written)
  *
- * Workspace: the checkpoints, B H (ceil(T / 64) + 8) dk dv fp32
- * (kda_chunk_bwd_workspace_bytes: 1.1 GB for B8 H32 T4096 d128, 34 GB for
+ * Workspace: the checkpoints, B H (ceil(T / 64) + 16) dk dv fp32
+ * (kda_chunk_bwd_workspace_bytes: 1.3 GB for B8 H32 T4096 d128, 34 GB for
  * B1 H32 T1M), held like the prefill's workspace (grown with cudaMalloc,
  * freed by kda_release_workspace).  T == 0 sets dh0 = dhT.
  * Errors as kda_chunk_fwd.
