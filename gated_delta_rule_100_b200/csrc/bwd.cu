@@ -189,6 +189,53 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_kernel(const BwdParams prm
         if (tid < nt) sb[tid] = prm.beta[((size_t)b * T + t0 + tid) * H + h];
     };
     float *scratch = prm.ckpt + ((size_t)prm.B * H * nck1 + (size_t)bh * (BWD_CK1 / CK)) * DK * DV;
+    // The reverse walk's inputs for a block of CK tokens: loaded into registers one
+    // block ahead (fetch), converted into the shared tiles at the block's start (put).
+    constexpr int PK = (CK * DK + BWD_THREADS - 1) / BWD_THREADS, PV = (CK * DV + BWD_THREADS - 1) / BWD_THREADS;
+    uint16_t rk[PK], rq[PK], rv[PV], rd[PV];
+    float rg[PK], rb = 0.f;
+    int pf_t0 = -1;  // first token of the block held in the registers
+    auto fetch = [&](int t0, int nt) {
+#pragma unroll
+        for (int x = 0; x < PK; ++x) {
+            const int e = tid + x * BWD_THREADS, t = e / DK, r = e % DK;
+            const bool in = t < nt;
+            const size_t row = ((size_t)b * T + (in ? t0 + t : 0)) * H + h;
+            rk[x] = in ? prm.k[row * DK + r] : (uint16_t)0;
+            rq[x] = in ? prm.q[row * DK + r] : (uint16_t)0;
+            rg[x] = in ? prm.g[row * DK + r] : 0.f;
+        }
+#pragma unroll
+        for (int x = 0; x < PV; ++x) {
+            const int e = tid + x * BWD_THREADS, t = e / DV, c = e % DV;
+            const bool in = t < nt;
+            const size_t row = ((size_t)b * T + (in ? t0 + t : 0)) * H + h;
+            rv[x] = in ? prm.v[row * DV + c] : (uint16_t)0;
+            rd[x] = (in && prm.dout) ? prm.dout[row * DV + c] : (uint16_t)0;
+        }
+        rb = tid < nt ? prm.beta[((size_t)b * T + t0 + tid) * H + h] : 0.f;
+        pf_t0 = t0;
+    };
+    auto put = [&](int nt) {
+#pragma unroll
+        for (int x = 0; x < PK; ++x) {
+            const int e = tid + x * BWD_THREADS;
+            if (e < nt * DK) {
+                sk[e] = bf16_bits_to_f32(rk[x]);
+                sq[e] = bf16_bits_to_f32(rq[x]);
+                sa[e] = __expf(rg[x]);
+            }
+        }
+#pragma unroll
+        for (int x = 0; x < PV; ++x) {
+            const int e = tid + x * BWD_THREADS;
+            if (e < nt * DV) {
+                sv[e] = bf16_bits_to_f32(rv[x]);
+                sd[e] = bf16_bits_to_f32(rd[x]);
+            }
+        }
+        if (tid < nt) sb[tid] = rb;
+    };
 
     for (int n = nck1 - 1; n >= 0; --n) {
         const int c0 = n * BWD_CK1;
@@ -218,23 +265,12 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_kernel(const BwdParams prm
         __syncthreads();  // the previous block's tiles and sums have been read; level 2 is written
         const float *ck = scratch + (size_t)j * DK * DV;
         for (int e = tid; e < DK * DV; e += BWD_THREADS) s0[(e / DV) * LD0 + e % DV] = ck[e];
-        for (int e = tid; e < nt * DK; e += BWD_THREADS) {
-            const int t = e / DK, r = e % DK;
-            const size_t row = ((size_t)b * T + t0 + t) * H + h;
-            sk[t * DK + r] = bf16_bits_to_f32(prm.k[row * DK + r]);
-            sq[t * DK + r] = bf16_bits_to_f32(prm.q[row * DK + r]);
-            sa[t * DK + r] = __expf(prm.g[row * DK + r]);
-        }
-        for (int e = tid; e < nt * DV; e += BWD_THREADS) {
-            const int t = e / DV, c = e % DV;
-            const size_t row = ((size_t)b * T + t0 + t) * H + h;
-            sv[t * DV + c] = bf16_bits_to_f32(prm.v[row * DV + c]);
-            sd[t * DV + c] = prm.dout ? bf16_bits_to_f32(prm.dout[row * DV + c]) : 0.f;
-        }
-        if (tid < nt) sb[tid] = prm.beta[((size_t)b * T + t0 + tid) * H + h];
+        if (pf_t0 != t0) fetch(t0, nt);  // the first block walked: nothing was prefetched
+        put(nt);
         for (int e = tid; e < CK * DK; e += BWD_THREADS) { acq[e] = 0.f; ack[e] = 0.f; aca[e] = 0.f; }
         if (tid < CK) acb[tid] = 0.f;
         __syncthreads();
+        if (t0 > 0) fetch(t0 - CK, CK);  // the next block's inputs, in flight during this one
 
         for (int tt = nt - 1; tt >= 0; --tt) {
             // the state before token t0 + tt, from the checkpoint
@@ -255,52 +291,46 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_kernel(const BwdParams prm
                 qr[i] = qt[lane + 32 * i];
                 ar[i] = at[lane + 32 * i];
             }
-            // forward quantities of the token: p = (Diag(a) S)^T k, u = beta (v - p)
-            float p[CW];
+            // The readout's share of dS first (it needs no forward quantity), then the two
+            // column reductions together: p = (Diag(a) S)^T k and du = dS^T k.
+            float p[CW], du[CW];
 #pragma unroll
             for (int c = 0; c < CW; ++c) {
-                float acc = 0.f;
-#pragma unroll
-                for (int i = 0; i < RI; ++i) acc += kr[i] * ar[i] * S[i][c];
-                p[c] = acc;
-            }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1)
-#pragma unroll
-                for (int c = 0; c < CW; ++c) p[c] += __shfl_xor_sync(0xffffffffu, p[c], o);
-            float dqp[RI], dkp[RI], dap[RI], du[CW];
-#pragma unroll
-            for (int i = 0; i < RI; ++i) { dqp[i] = 0.f; dkp[i] = 0.f; dap[i] = 0.f; }
-            // readout: dq = scale S_t do, dS += scale q do^T; then du = dS^T k
-#pragma unroll
-            for (int c = 0; c < CW; ++c) {
-                const float u = bt * (vt[col0 + c] - p[c]);
-                const float d = dot[col0 + c];
-                float acc = 0.f;
+                const float d = scale * dot[col0 + c];
+                float pa = 0.f, ua = 0.f;
 #pragma unroll
                 for (int i = 0; i < RI; ++i) {
-                    const float snew = ar[i] * S[i][c] + kr[i] * u;
-                    dqp[i] += scale * snew * d;
-                    dS[i][c] += scale * qr[i] * d;
-                    acc += dS[i][c] * kr[i];
-                    dkp[i] += dS[i][c] * u;
+                    dS[i][c] += qr[i] * d;
+                    pa += kr[i] * ar[i] * S[i][c];
+                    ua += dS[i][c] * kr[i];
                 }
-                du[c] = acc;
+                p[c] = pa;
+                du[c] = ua;
             }
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1)
 #pragma unroll
-                for (int c = 0; c < CW; ++c) du[c] += __shfl_xor_sync(0xffffffffu, du[c], o);
+                for (int c = 0; c < CW; ++c) {
+                    p[c] += __shfl_xor_sync(0xffffffffu, p[c], o);
+                    du[c] += __shfl_xor_sync(0xffffffffu, du[c], o);
+                }
+            float dqp[RI], dkp[RI], dap[RI];
+#pragma unroll
+            for (int i = 0; i < RI; ++i) { dqp[i] = 0.f; dkp[i] = 0.f; dap[i] = 0.f; }
             float dbp = 0.f;
             const size_t row = ((size_t)b * T + t0 + tt) * H + h;
 #pragma unroll
             for (int c = 0; c < CW; ++c) {
-                dbp += du[c] * (vt[col0 + c] - p[c]);
+                const float vmp = vt[col0 + c] - p[c];
+                const float u = bt * vmp;                 // u = beta (v - p)
+                const float d = scale * dot[col0 + c];
+                dbp += du[c] * vmp;
                 const float dp = -bt * du[c];
 #pragma unroll
                 for (int i = 0; i < RI; ++i) {
-                    const float sdv = ar[i] * S[i][c];
-                    dkp[i] += sdv * dp;
+                    const float sdv = ar[i] * S[i][c];    // S' = Diag(a) S_{t-1}
+                    dqp[i] += (sdv + kr[i] * u) * d;      // dq = scale S_t do
+                    dkp[i] += dS[i][c] * u + sdv * dp;    // dk = dS u + S' dp
                     const float dsd = dS[i][c] + kr[i] * dp;
                     dap[i] += dsd * S[i][c];
                     dS[i][c] = ar[i] * dsd;

@@ -514,22 +514,40 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
 }
 
 template <int DK, int VS>
-static cudaError_t launch_chain_t(const CUtensorMap *maps, const ChainParams &prm, cudaStream_t stream) {
+static cudaError_t launch_chain_t(const CUtensorMap *maps, const ChainParams &prm, cudaStream_t stream,
+                                  cudaEvent_t started) {
     using L = ChainLayout<DK, VS>;
     cudaError_t e = cudaFuncSetAttribute(chain_kernel<DK, VS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          L::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    chain_kernel<DK, VS><<<prm.gm.nseqs * prm.H * prm.nparts * prm.slots, CHAIN_THREADS, L::SMEM_BYTES, stream>>>(
-        maps[0], maps[1], maps[2], maps[3], prm);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(prm.gm.nseqs * prm.H * prm.nparts * prm.slots);
+    cfg.blockDim = dim3(CHAIN_THREADS);
+    cfg.dynamicSmemBytes = L::SMEM_BYTES;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    if (started != nullptr) {
+        attr[0].id = cudaLaunchAttributeLaunchCompletionEvent;
+        attr[0].val.launchCompletionEvent.event = started;
+        attr[0].val.launchCompletionEvent.flags = 0;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    }
+    return cudaLaunchKernelEx(&cfg, chain_kernel<DK, VS>, maps[0], maps[1], maps[2], maps[3], prm);
 }
 
 // maps: the record parts WQ, P, K-hat, T' (see chunk_common.cuh); the value
-// slice of a CTA is DV / nslices columns (64 or 128).
-cudaError_t launch_chain(const CUtensorMap *maps, const ChainParams &prm, int dk, cudaStream_t stream) {
+// slice of a CTA is DV / nslices columns (64 or 128).  `started`, when given,
+// is recorded once every CTA of the launch has begun (a launch-completion
+// event; the runtime may fire it later, at the kernel's end).
+cudaError_t launch_chain(const CUtensorMap *maps, const ChainParams &prm, int dk, cudaStream_t stream,
+                         cudaEvent_t started) {
     const int vs = prm.DV / prm.nslices;
-    if (dk == 128) return vs == 128 ? launch_chain_t<128, 128>(maps, prm, stream) : launch_chain_t<128, 64>(maps, prm, stream);
-    return vs == 128 ? launch_chain_t<64, 128>(maps, prm, stream) : launch_chain_t<64, 64>(maps, prm, stream);
+    if (dk == 128)
+        return vs == 128 ? launch_chain_t<128, 128>(maps, prm, stream, started)
+                         : launch_chain_t<128, 64>(maps, prm, stream, started);
+    return vs == 128 ? launch_chain_t<64, 128>(maps, prm, stream, started)
+                     : launch_chain_t<64, 64>(maps, prm, stream, started);
 }
 
 }  // namespace kda

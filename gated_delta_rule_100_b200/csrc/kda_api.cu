@@ -27,7 +27,8 @@ cudaError_t launch_decode(const void *q, const void *k, const void *v, const flo
 namespace kda {
 cudaError_t launch_prep(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tg, const PrepParams &prm,
                         int dk, int max_ctas, cudaStream_t stream, bool prologue);
-cudaError_t launch_chain(const CUtensorMap *maps, const ChainParams &prm, int dk, cudaStream_t stream);
+cudaError_t launch_chain(const CUtensorMap *maps, const ChainParams &prm, int dk, cudaStream_t stream,
+                         cudaEvent_t started = nullptr);
 cudaError_t launch_exact(const ExactParams &prm, int dk, int ctas, cudaStream_t stream);
 cudaError_t launch_parts_fixup(float *start, const float *local, const float *trans, int BH, int dk, int dv,
                                int parts, cudaStream_t stream, unsigned long long *stamp);
@@ -112,6 +113,7 @@ struct Workspace {
     cudaEvent_t done = nullptr;
     cudaStream_t lo = nullptr, hi = nullptr;  // prep and chain streams of the segmented path
     cudaEvent_t fork = nullptr, prep_done[2] = {nullptr, nullptr}, chain_done[2] = {nullptr, nullptr};
+    cudaEvent_t chain_go = nullptr;  // every CTA of a segment's first chain launch has begun
 };
 Workspace g_ws[kMaxDevices];
 
@@ -193,7 +195,8 @@ int reserve_workspace(int dev, size_t base_bytes, size_t state_bytes, bool strea
             cudaStreamCreateWithPriority(&w.lo, cudaStreamNonBlocking, least) != cudaSuccess ||
             cudaStreamCreateWithPriority(&w.hi, cudaStreamNonBlocking, greatest) != cudaSuccess)
             return KDA_ERR_CUDA;
-        cudaEvent_t *evs[5] = {&w.fork, &w.prep_done[0], &w.prep_done[1], &w.chain_done[0], &w.chain_done[1]};
+        cudaEvent_t *evs[6] = {&w.fork, &w.prep_done[0], &w.prep_done[1], &w.chain_done[0], &w.chain_done[1],
+                               &w.chain_go};
         for (cudaEvent_t *e : evs)
             if (cudaEventCreateWithFlags(e, cudaEventDisableTiming) != cudaSuccess) return KDA_ERR_CUDA;
     }
@@ -529,6 +532,10 @@ static int chunk_fwd_impl(const void *q, const void *k, const void *v, const flo
         const int buf = multi ? (i & 1) : 0;
         // buffer reuse: the chain kernel two segments back has read it
         if (multi && i >= 2 && cudaStreamWaitEvent(sp, w->chain_done[buf], 0) != cudaSuccess) return KDA_ERR_CUDA;
+        // and the previous segment's chain CTAs are all placed: a prep kernel placed
+        // before them spreads its persistent CTAs over every SM and keeps the chain off
+        // until it ends (the first segments; later ones are ordered by the wait above)
+        if (multi && i >= 1 && cudaStreamWaitEvent(sp, w->chain_go, 0) != cudaSuccess) return KDA_ERR_CUDA;
         if (cudaMemsetAsync(counters + 2 * buf, 0, 2 * sizeof(int), sp) != cudaSuccess) return KDA_ERR_CUDA;
         kda::PrepParams pp;
         pp.g = g;
@@ -575,11 +582,12 @@ static int chunk_fwd_impl(const void *q, const void *k, const void *v, const flo
         cp.st = dst;
         cp.inject_wait_polls = g_inject_polls.load();
         const int P = plan_parts(B, H, dk, dv, cnt, sms);
+        cudaEvent_t go = multi ? w->chain_go : nullptr;
         if (P < 3) {
             plain_pass(cp, chain_slices(B, H, dv, sms));
             e = timed_launch(dev, 1, sc, [&](unsigned long long *t) {
                 cp.stamp = t;
-                return kda::launch_chain(rmaps[buf], cp, dk, sc);
+                return kda::launch_chain(rmaps[buf], cp, dk, sc, go);
             });
             if (e != cudaSuccess) return KDA_ERR_CUDA;
         } else {  // two-level pass: pass A, fix-up, pass B (64-column slices)
@@ -596,7 +604,7 @@ static int chunk_fwd_impl(const void *q, const void *k, const void *v, const flo
             cp.slots = (dv + dk) / 64;
             e = timed_launch(dev, 1, sc, [&](unsigned long long *t) {
                 cp.stamp = t;
-                return kda::launch_chain(rmaps[buf], cp, dk, sc);
+                return kda::launch_chain(rmaps[buf], cp, dk, sc, go);
             });
             if (e != cudaSuccess) return KDA_ERR_CUDA;
             e = timed_launch(dev, 3, sc, [&](unsigned long long *t) {
@@ -634,10 +642,13 @@ size_t kda_chunk_fwd_workspace_bytes(int B, int T, int H, int dk, int dv) {
 
 void kda_debug_kernel_timing(int enable) { g_timing.store(enable != 0); }
 
-int kda_debug_kernel_times(double *ms, long long *launches, int nkinds) {
-    if (ms == nullptr || launches == nullptr || nkinds < 0) return KDA_ERR_INVALID_ARG;
-    for (int i = 0; i < nkinds; ++i) { ms[i] = 0.0; launches[i] = 0; }
-    std::lock_guard<std::mutex> lk(g_mu);
+// Every launch timed since the last read, in launch order: (kind, start, end) in
+// globaltimer nanoseconds, end < start when the kernel left no stamp.  Forgets them.
+struct StampRec {
+    int kind;
+    unsigned long long start, end;
+};
+static int collect_stamps(std::vector<StampRec> *out) {
     int st = KDA_OK, cur = 0;
     if (cudaGetDevice(&cur) != cudaSuccess) return KDA_ERR_CUDA;
     std::vector<unsigned long long> host;
@@ -650,15 +661,45 @@ int kda_debug_kernel_times(double *ms, long long *launches, int nkinds) {
                        cudaMemcpyDeviceToHost) != cudaSuccess)
             st = KDA_ERR_CUDA;
         for (const TimedLaunch &t : g_timed) {
-            if (t.dev != dev || t.kind < 0 || t.kind >= nkinds) continue;
+            if (t.dev != dev) continue;
             const unsigned long long a = host[2 * t.slot], e = ~host[2 * t.slot + 1];
-            if (st == KDA_OK && a != ~0ull && e >= a) ms[t.kind] += (double)(e - a) * 1e-6;
-            launches[t.kind] += 1;
+            const bool ok = st == KDA_OK && a != ~0ull && e >= a;
+            out->push_back({t.kind, ok ? a : 1ull, ok ? e : 0ull});
         }
         g_stamp_next[dev] = 0;
     }
     g_timed.clear();
     if (cudaSetDevice(cur) != cudaSuccess) st = KDA_ERR_CUDA;
+    return st;
+}
+
+int kda_debug_kernel_times(double *ms, long long *launches, int nkinds) {
+    if (ms == nullptr || launches == nullptr || nkinds < 0) return KDA_ERR_INVALID_ARG;
+    for (int i = 0; i < nkinds; ++i) { ms[i] = 0.0; launches[i] = 0; }
+    std::lock_guard<std::mutex> lk(g_mu);
+    std::vector<StampRec> recs;
+    const int st = collect_stamps(&recs);
+    for (const StampRec &r : recs) {
+        if (r.kind < 0 || r.kind >= nkinds) continue;
+        if (r.end >= r.start) ms[r.kind] += (double)(r.end - r.start) * 1e-6;
+        launches[r.kind] += 1;
+    }
+    return st;
+}
+
+int kda_debug_kernel_launches(int *kind, long long *start_ns, long long *end_ns, int cap, int *count) {
+    if (kind == nullptr || start_ns == nullptr || end_ns == nullptr || count == nullptr || cap < 0)
+        return KDA_ERR_INVALID_ARG;
+    std::lock_guard<std::mutex> lk(g_mu);
+    std::vector<StampRec> recs;
+    const int st = collect_stamps(&recs);
+    const int n = (int)recs.size() < cap ? (int)recs.size() : cap;
+    for (int i = 0; i < n; ++i) {
+        kind[i] = recs[i].kind;
+        start_ns[i] = (long long)recs[i].start;
+        end_ns[i] = (long long)recs[i].end;
+    }
+    *count = n;
     return st;
 }
 

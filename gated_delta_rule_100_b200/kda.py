@@ -39,7 +39,7 @@ EXPORTED = ("kda_chunk_fwd", "kda_chunk_fwd_noalloc", "kda_chunk_fwd_varlen", "k
             "kda_chunk_fwd_workspace_bytes", "kda_chunk_fwd_varlen_workspace_bytes", "kda_release_workspace",
             "kda_status_string", "kda_stream_status", "kda_chunk_fwd_debug_wait_limit",
             "kda_chunk_fwd_debug_inject_timeout", "kda_chunk_fwd_debug_force_exact", "kda_chunk_fwd_debug_record_cap", "kda_chunk_fwd_debug_parts",
-            "kda_debug_kernel_timing", "kda_debug_kernel_times",
+            "kda_debug_kernel_timing", "kda_debug_kernel_times", "kda_debug_kernel_launches",
             "kda_abi_version")
 
 _lib = None          # the library the calls below go through
@@ -121,6 +121,9 @@ def _open(path):
     lib.kda_debug_kernel_timing.restype = None
     lib.kda_debug_kernel_times.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_longlong), i]
     lib.kda_debug_kernel_times.restype = i
+    ll = ctypes.POINTER(ctypes.c_longlong)
+    lib.kda_debug_kernel_launches.argtypes = [ctypes.POINTER(ctypes.c_int), ll, ll, i, ctypes.POINTER(ctypes.c_int)]
+    lib.kda_debug_kernel_launches.restype = i
     lib.kda_abi_version.restype = i
     _libs[path] = lib
     return lib
@@ -406,7 +409,8 @@ KERNEL_KINDS = ("prep", "chain", "exact", "fixup", "bwd")
 
 
 def kernel_timing(enable: bool) -> None:
-    """Measurement hook: time every prefill kernel launch with CUDA events."""
+    """Measurement hook: every prefill and backward launch stamps its first CTA's
+    start and last CTA's end (device globaltimer)."""
     load().kda_debug_kernel_timing(1 if enable else 0)
 
 
@@ -419,6 +423,21 @@ def kernel_times() -> dict:
     if rc != KDA_OK:
         raise KdaError(rc, "kda_debug_kernel_times")
     return {k: (ms[i], int(cnt[i])) for i, k in enumerate(KERNEL_KINDS)}
+
+
+def kernel_launches(cap: int = 8192) -> list:
+    """[(kind, start_ms, end_ms)] of the launches timed since the last read, in launch
+    order, times relative to the first start (end < start: no stamp)."""
+    kind = (ctypes.c_int * cap)()
+    st, en = (ctypes.c_longlong * cap)(), (ctypes.c_longlong * cap)()
+    cnt = ctypes.c_int(0)
+    rc = load().kda_debug_kernel_launches(kind, st, en, cap, ctypes.byref(cnt))
+    if rc != KDA_OK:
+        raise KdaError(rc, "kda_debug_kernel_launches")
+    n = cnt.value
+    t0 = min((st[i] for i in range(n) if en[i] >= st[i]), default=0)
+    return [(KERNEL_KINDS[kind[i]] if 0 <= kind[i] < len(KERNEL_KINDS) else kind[i],
+             (st[i] - t0) * 1e-6, (en[i] - t0) * 1e-6) for i in range(n)]
 
 
 class DeviceBuffers:

@@ -410,6 +410,18 @@ KDA_API void kda_chunk_fwd_debug_parts(int parts);
 KDA_API void kda_debug_kernel_timing(int enable);
 KDA_API int kda_debug_kernel_times(double *ms, long long *launches, int nkinds);
 
+/*
+ * kda_debug_kernel_launches -- the same timed launches one by one, in the
+ * order they were launched: kind[i], and start_ns[i] / end_ns[i], the
+ * %globaltimer readings (nanoseconds, one clock per device) of the first CTA's
+ * start and the last CTA's end; end_ns[i] < start_ns[i] for a launch that left
+ * no stamp.  Writes at most `cap` entries (host arrays of the caller), the
+ * number written to *count, and forgets every timed launch, like
+ * kda_debug_kernel_times.  KDA_OK, KDA_ERR_INVALID_ARG for a NULL pointer or
+ * cap < 0, or KDA_ERR_CUDA.
+ */
+KDA_API int kda_debug_kernel_launches(int *kind, long long *start_ns, long long *end_ns, int cap, int *count);
+
 /* Version of this ABI (major * 100 + minor): 101 adds the scalar-gate entry
  * points, 102 the packed-batch prefill, the raw-input (fused gate prologue)
  * entry points, the backward pass and the exact-path and two-level test
