@@ -467,14 +467,14 @@ static int chunk_fwd_impl(const void *q, const void *k, const void *v, const flo
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return KDA_ERR_CUDA;
 
-    CUtensorMap tq, tk, tg;  // tg: the per-channel gate, 32 channels x 64 tokens per box
+    CUtensorMap tq, tk, tg;  // tg: the per-channel gate, dk channels x 64 tokens per box
     if (make_map(&tq, enc, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dk, H, T, B, 64,
                  CU_TENSOR_MAP_SWIZZLE_128B) != KDA_OK ||
         make_map(&tk, enc, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dk, H, T, B, 64,
                  CU_TENSOR_MAP_SWIZZLE_128B) != KDA_OK)
         return KDA_ERR_CUDA;
     if (scalar_gate) tg = tq;  // not read
-    else if (make_map(&tg, enc, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dk, H, T, B, 32,
+    else if (make_map(&tg, enc, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dk, H, T, B, dk,
                       CU_TENSOR_MAP_SWIZZLE_NONE) != KDA_OK)
         return KDA_ERR_CUDA;
 
@@ -782,7 +782,7 @@ int kda_chunk_fwd_varlen(const void *q, const void *k, const void *v, const floa
                  CU_TENSOR_MAP_SWIZZLE_128B) != KDA_OK ||
         make_map(&tk, enc, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dk, H, T_total, 1, 64,
                  CU_TENSOR_MAP_SWIZZLE_128B) != KDA_OK ||
-        make_map(&tg, enc, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dk, H, T_total, 1, 32,
+        make_map(&tg, enc, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dk, H, T_total, 1, dk,
                  CU_TENSOR_MAP_SWIZZLE_NONE) != KDA_OK)
         return KDA_ERR_CUDA;
 
@@ -1059,7 +1059,7 @@ int kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const flo
                  CU_TENSOR_MAP_SWIZZLE_128B) != KDA_OK ||
         make_map(&tk, enc, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dk, H, T, B, 64,
                  CU_TENSOR_MAP_SWIZZLE_128B) != KDA_OK ||
-        make_map(&tg, enc, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dk, H, T, B, 32,
+        make_map(&tg, enc, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dk, H, T, B, dk,
                  CU_TENSOR_MAP_SWIZZLE_NONE) != KDA_OK)
         return KDA_ERR_CUDA;
 

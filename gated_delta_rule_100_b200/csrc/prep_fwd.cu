@@ -78,8 +78,8 @@ struct PrepLayout {
     static constexpr int OFF_QIN = OFF_BK;                   // bf16 [64][DK], 128B swizzle
     static constexpr int OFF_KIN = OFF_BK + CH * DK * 2;
     static constexpr int OFF_MISC = OFF_BK + 128 * 64 * 4;   // beta, barriers, TMEM address
-    // g (per key channel) by TMA during the inputs: fp32 [DK / 32][64 tokens][32 channels],
-    // after the block-products exchange in R_form (free until phase E writes X)
+    // g (per key channel) by TMA during the inputs: fp32 [64 tokens][DK channels], after
+    // the block-products exchange in R_form (free until phase E writes X)
     static constexpr int OFF_GIN = OFF_F + 4096;
     static_assert(OFF_GIN + CH * DK * 4 <= OFF_F + RF_B, "g tile fits in R_form");
     static constexpr int TOTAL = OFF_MISC + 1024;
@@ -186,7 +186,10 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         const long long rows = geom_rows(prm.gm);
         (void)KDA_CHECK(prm.st, h < H && gi.tok0 >= 0 && gi.row0 >= 0);
 
-        // ---------------- inputs: q, k by TMA; g (this thread's 16 tokens) and beta by plain loads
+        // ---------------- inputs: q, k (thread 0) and g (thread 32) by TMA; beta by plain loads.
+        // Thread 0's arrival carries every byte of the phase, so the phase cannot complete
+        // before it even if thread 32's load lands first (the count of pending bytes may dip
+        // below zero meanwhile); a TMA issue can hold its thread for a while, hence two issuers.
         if (tid == 0) {
             mbar_expect_tx(bar_in, (uint32_t)(2 * CH * DK * 2 + (SG ? 0 : CH * DK * 4)));
 #pragma unroll
@@ -194,12 +197,8 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 tma_load_4d(sbase + L::OFF_QIN + kb * CH * 128, &tm_q, bar_in, kb * 64, h, gi.tok0, gi.bcoord);
                 tma_load_4d(sbase + L::OFF_KIN + kb * CH * 128, &tm_k, bar_in, kb * 64, h, gi.tok0, gi.bcoord);
             }
-            if (!SG) {
-#pragma unroll
-                for (int kb = 0; kb < DK / 32; ++kb)
-                    tma_load_4d(sbase + L::OFF_GIN + kb * CH * 128, &tm_g, bar_in, kb * 32, h, gi.tok0, gi.bcoord);
-            }
         }
+        if (!SG && tid == 32) tma_load_4d(sbase + L::OFF_GIN, &tm_g, bar_in, 0, h, gi.tok0, gi.bcoord);
         tma_pending = true;
         float al[SUB];
         if constexpr (SG) {  // one gate per (token, head), shared by all channels: plain loads
@@ -217,9 +216,9 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         if (!wait_all(bar_in, ph_in, tma_pending)) { aborted = true; break; }
         ph_in ^= 1u;
         if constexpr (!SG) {  // one gate per key channel, from the g tile (TMA; zero past the tensor)
-            const float *gs = reinterpret_cast<const float *>(sm + L::OFF_GIN) + ((c >> 5) * CH + tb) * 32 + (c & 31);
+            const float *gs = reinterpret_cast<const float *>(sm + L::OFF_GIN) + tb * DK + c;
 #pragma unroll
-            for (int u = 0; u < SUB; ++u) al[u] = (tb + u < gi.nvalid && active) ? gs[u * 32] : 0.f;
+            for (int u = 0; u < SUB; ++u) al[u] = (tb + u < gi.nvalid && active) ? gs[u * DK] : 0.f;
         }
         float *s_rn = reinterpret_cast<float *>(sm + L::OFF_MISC + 256);  // PRO: 1 / |q_t|, then 1 / |k_t|
         if constexpr (PRO) {
@@ -441,10 +440,8 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     prefetch_tensor_4d(&tm_q, kb * 64, ng.h, ng.tok0, ng.bcoord);
                     prefetch_tensor_4d(&tm_k, kb * 64, ng.h, ng.tok0, ng.bcoord);
                 }
-                if (!SG) {
-#pragma unroll
-                    for (int kb = 0; kb < DK / 32; ++kb) prefetch_tensor_4d(&tm_g, kb * 32, ng.h, ng.tok0, ng.bcoord);
-                }
+            } else if (!SG && tid == 32) {
+                prefetch_tensor_4d(&tm_g, 0, ng.h, ng.tok0, ng.bcoord);
             } else if (SG && tid >= 64 && tid < 64 + CH && tid - 64 < ng.nvalid) {
                 prefetch_line_l2(prm.g + (size_t)(ng.row0 + tid - 64) * H + ng.h);
             }
