@@ -25,11 +25,13 @@
 //          state every CK = 4 tokens in a per-(b, h) scratch (level 2); then
 //          blocks of CK tokens from the last to the first: for token t of a
 //          block, the state before t is recomputed from the block's checkpoint
-//          (kept in shared memory), then the reverse step.  After each block
+//          (kept in shared memory) or, past the block's second token, from a
+//          thread-private copy of the state before its third token (stored on
+//          the way to the last token), then the reverse step.  After each block
 //          its tokens' dq, dk (bf16), dg and dbeta (fp32) are written; dv per
 //          column as it is formed; dh0 at the end.
 // Memory: (ceil(T / 64) + 16) dk dv fp32 per (b, h); forward steps per token:
-// one in pass 1, one for level 2, 1.5 on average for the per-token states
+// one in pass 1, one for level 2, one on average for the per-token states
 // (blocks of 8 took 56 ms on B8 H32 T4096, 3.5 recomputed steps per token).
 // Inputs are staged in shared memory per block of tokens.  Level-2 states go
 // through global memory (the scratch), read back after a block barrier.
@@ -157,6 +159,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_kernel(const BwdParams prm
     float *ack = acq + CK * DK;      //                             dk
     float *aca = ack + CK * DK;      //                             d alpha
     float *acb = aca + CK * DK;      // [CK]                        dbeta
+    float *sst = acb + CK;           // [RI CW][threads] each thread's state before token 2 of the block
     const int bh = blockIdx.x, b = bh / prm.H, h = bh % prm.H;
     const int T = prm.T, H = prm.H;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, col0 = warp * CW;
@@ -272,14 +275,34 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_kernel(const BwdParams prm
         __syncthreads();
         if (t0 > 0) fetch(t0 - CK, CK);  // the next block's inputs, in flight during this one
 
+        constexpr int SP = 2;  // the stashed state is the one before the block's token SP
+        bool stashed = false;
         for (int tt = nt - 1; tt >= 0; --tt) {
-            // the state before token t0 + tt, from the checkpoint
+            // the state before token t0 + tt, from the stash or the checkpoint
             float S[RI][CW];
+            int s = 0;
+            if (tt >= SP && stashed) {
 #pragma unroll
-            for (int i = 0; i < RI; ++i)
+                for (int i = 0; i < RI; ++i)
 #pragma unroll
-                for (int c = 0; c < CW; ++c) S[i][c] = s0[(lane + 32 * i) * LD0 + col0 + c];
-            for (int s = 0; s < tt; ++s) fwd_step<RI, CW>(S, sk + s * DK, sa + s * DK, sv + s * DV, sb[s], lane, col0);
+                    for (int c = 0; c < CW; ++c) S[i][c] = sst[(i * CW + c) * BWD_THREADS + tid];
+                s = SP;
+            } else {
+#pragma unroll
+                for (int i = 0; i < RI; ++i)
+#pragma unroll
+                    for (int c = 0; c < CW; ++c) S[i][c] = s0[(lane + 32 * i) * LD0 + col0 + c];
+            }
+            for (; s < tt; ++s) {
+                fwd_step<RI, CW>(S, sk + s * DK, sa + s * DK, sv + s * DV, sb[s], lane, col0);
+                if (s + 1 == SP && tt > SP) {  // on the way to a later token: keep the state before SP
+#pragma unroll
+                    for (int i = 0; i < RI; ++i)
+#pragma unroll
+                        for (int c = 0; c < CW; ++c) sst[(i * CW + c) * BWD_THREADS + tid] = S[i][c];
+                    stashed = true;
+                }
+            }
 
             const float *kt = sk + tt * DK, *qt = sq + tt * DK, *at = sa + tt * DK;
             const float *vt = sv + tt * DV, *dot = sd + tt * DV;
@@ -371,7 +394,7 @@ template <int DK, int DV>
 static cudaError_t launch_bwd_t(const BwdParams &prm, cudaStream_t stream) {
     const int BH = prm.B * prm.H;
     const int s1 = (2 * BWD_FT * DK + BWD_FT * DV + BWD_FT) * 4;
-    const int s2 = (DK * (DV + 1) + 3 * BWD_CK * DK + 2 * BWD_CK * DV + BWD_CK + 3 * BWD_CK * DK + BWD_CK) * 4;
+    const int s2 = (DK * (DV + 1) + 3 * BWD_CK * DK + 2 * BWD_CK * DV + BWD_CK + 3 * BWD_CK * DK + BWD_CK + DK * DV) * 4;
     cudaError_t e = cudaFuncSetAttribute(bwd_ckpt_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, s1);
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(bwd_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, s2);

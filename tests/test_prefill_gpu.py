@@ -291,3 +291,23 @@ def test_kernel_timing_hook_stamps_every_launch():
     for kind in ("prep", "chain"):
         assert 0.0 < t[kind][0] <= wall * 1.05 + 0.01, (kind, t[kind], wall)
     assert kda.kernel_times() == {k: (0.0, 0) for k in kda.KERNEL_KINDS}  # read once
+
+
+def test_kernel_launch_timeline():
+    """The hook's per-launch form: one entry per launch in launch order, each with
+    start <= end; prep precedes the chain it feeds, and the list is read once."""
+    d = inputs.make_prefill(1, 3000, 2, 128, 128, decay=0.05, seed=19, device=DEV)
+    run(d, 0.1)
+    kda.kernel_launches()
+    kda.kernel_timing(True)
+    run(d, 0.1)
+    torch.cuda.synchronize()
+    kda.kernel_timing(False)
+    L = kda.kernel_launches()
+    kinds = [k for k, _, _ in L]
+    assert kinds[:2] == ["prep", "exact"] and "chain" in kinds, kinds
+    assert all(e >= s for _, s, e in L), L
+    p = next(x for x in L if x[0] == "prep")
+    c = next(x for x in L if x[0] == "chain")
+    assert c[1] >= p[2] - 1e-6  # the chain starts after its records are written
+    assert kda.kernel_launches() == []
