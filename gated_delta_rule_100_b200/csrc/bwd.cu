@@ -33,8 +33,10 @@
 // Memory: (ceil(T / 64) + 16) dk dv fp32 per (b, h); forward steps per token:
 // one in pass 1, one for level 2, one on average for the per-token states
 // (blocks of 8 took 56 ms on B8 H32 T4096, 3.5 recomputed steps per token).
-// Inputs are staged in shared memory per block of tokens.  Level-2 states go
-// through global memory (the scratch), read back after a block barrier.
+// Inputs are staged in shared memory per block of tokens, loaded into registers
+// one block ahead.  Level-2 states go through global memory (the scratch); the
+// reverse walk copies each block's state into one of two shared buffers with
+// cp.async while the block before it (in walk order) runs.
 #include <cuda_bf16.h>
 #include <stdint.h>
 
@@ -57,6 +59,16 @@ __device__ __forceinline__ void load_row(const float *src, float (&x)[CW]) {
         x[c] = v.x; x[c + 1] = v.y; x[c + 2] = v.z; x[c + 3] = v.w;
     }
 }
+// 16-byte asynchronous global -> shared copy (L2 only), and its group fences.
+__device__ __forceinline__ void cp_async16(float *dst, const float *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)),
+                 "l"(reinterpret_cast<uint64_t>(src))
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
 template <int CW>
 __device__ __forceinline__ void store_row(float *dst, const float (&x)[CW]) {
 #pragma unroll
@@ -146,10 +158,12 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_ckpt_kernel(const BwdParam
 template <int DK, int DV>
 __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_kernel(const BwdParams prm) {
     constexpr int RI = DK / 32, CW = DV / 16, CK = BWD_CK;
-    constexpr int LD0 = DV + 1;      // row stride of the checkpoint tile (lanes own rows)
+    // Row stride of a checkpoint tile: lanes own rows, and 16-byte reads of a row
+    // by 8 lanes at a time cover all 32 banks once.
+    constexpr int LD0 = DV + 4;
     extern __shared__ __align__(16) float fsm[];
-    float *s0 = fsm;                 // [DK][LD0] the block's checkpoint
-    float *sk = s0 + DK * LD0;       // [CK][DK]
+    float *s0b = fsm;                // [2][DK][LD0] block checkpoints (double buffer)
+    float *sk = s0b + 2 * DK * LD0;  // [CK][DK]
     float *sq = sk + CK * DK;        // [CK][DK]
     float *sa = sq + CK * DK;        // [CK][DK] alpha
     float *sv = sa + CK * DK;        // [CK][DV]
@@ -177,20 +191,6 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_kernel(const BwdParams prm
         }
     }
 
-    // the inputs a forward step needs, for the CK tokens from t0 (nt of them)
-    auto stage_fwd = [&](int t0, int nt) {
-        for (int e = tid; e < nt * DK; e += BWD_THREADS) {
-            const int t = e / DK, r = e % DK;
-            const size_t row = ((size_t)b * T + t0 + t) * H + h;
-            sk[t * DK + r] = bf16_bits_to_f32(prm.k[row * DK + r]);
-            sa[t * DK + r] = __expf(prm.g[row * DK + r]);
-        }
-        for (int e = tid; e < nt * DV; e += BWD_THREADS) {
-            const int t = e / DV, c = e % DV;
-            sv[t * DV + c] = bf16_bits_to_f32(prm.v[(((size_t)b * T + t0 + t) * H + h) * DV + c]);
-        }
-        if (tid < nt) sb[tid] = prm.beta[((size_t)b * T + t0 + tid) * H + h];
-    };
     float *scratch = prm.ckpt + ((size_t)prm.B * H * nck1 + (size_t)bh * (BWD_CK1 / CK)) * DK * DV;
     // The reverse walk's inputs for a block of CK tokens: loaded into registers one
     // block ahead (fetch), converted into the shared tiles at the block's start (put).
@@ -239,6 +239,15 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_kernel(const BwdParams prm
         }
         if (tid < nt) sb[tid] = rb;
     };
+    // a level-2 state from the scratch into a checkpoint tile (this thread's share)
+    auto copy_state = [&](float *dst, const float *src) {
+#pragma unroll
+        for (int x = 0; x < DK * DV / 4 / BWD_THREADS; ++x) {
+            const int e = (tid + x * BWD_THREADS) * 4;
+            cp_async16(dst + (e / DV) * LD0 + e % DV, src + e);
+        }
+        cp_async_commit();
+    };
 
     for (int n = nck1 - 1; n >= 0; --n) {
         const int c0 = n * BWD_CK1;
@@ -256,8 +265,13 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_kernel(const BwdParams prm
                 for (int i = 0; i < RI; ++i) store_row<CW>(dst + (size_t)(lane + 32 * i) * DV + col0, S[i]);
                 if (jb + 1 == nb) break;  // the last block's state is not needed past its start
                 __syncthreads();          // the previous block's inputs are no longer read
-                stage_fwd(t0, nt);
+                if (pf_t0 != t0) fetch(t0, nt);
+                put(nt);
                 __syncthreads();
+                {  // the next block's inputs (it exists: jb + 1 < nb), in flight during this one
+                    const int t1 = t0 + CK;
+                    fetch(t1, T - t1 < CK ? T - t1 : CK);
+                }
                 for (int t = 0; t < nt; ++t)
                     fwd_step<RI, CW>(S, sk + t * DK, sa + t * DK, sv + t * DV, sb[t], lane, col0);
             }
@@ -266,14 +280,23 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_kernel(const BwdParams prm
         const int t0 = c0 + j * CK;
         const int nt = T - t0 < CK ? T - t0 : CK;
         __syncthreads();  // the previous block's tiles and sums have been read; level 2 is written
-        const float *ck = scratch + (size_t)j * DK * DV;
-        for (int e = tid; e < DK * DV; e += BWD_THREADS) s0[(e / DV) * LD0 + e % DV] = ck[e];
+        const float *s0 = s0b + (j & 1) * DK * LD0;
+        if (j == nb - 1) copy_state(s0b + (j & 1) * DK * LD0, scratch + (size_t)j * DK * DV);
+        if (j > 0) {  // the next block's state, into the other buffer (last read two blocks ago)
+            copy_state(s0b + ((j - 1) & 1) * DK * LD0, scratch + (size_t)(j - 1) * DK * DV);
+            cp_async_wait<1>();
+        } else {
+            cp_async_wait<0>();
+        }
         if (pf_t0 != t0) fetch(t0, nt);  // the first block walked: nothing was prefetched
         put(nt);
         for (int e = tid; e < CK * DK; e += BWD_THREADS) { acq[e] = 0.f; ack[e] = 0.f; aca[e] = 0.f; }
         if (tid < CK) acb[tid] = 0.f;
         __syncthreads();
-        if (t0 > 0) fetch(t0 - CK, CK);  // the next block's inputs, in flight during this one
+        // the inputs of the next block walked, or of the previous chunk's first block
+        // (its level-2 pass comes next), in flight during this one
+        if (j > 0) fetch(t0 - CK, CK);
+        else if (c0 > 0) fetch(c0 - BWD_CK1, CK);
 
         constexpr int SP = 2;  // the stashed state is the one before the block's token SP
         bool stashed = false;
@@ -289,9 +312,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_kernel(const BwdParams prm
                 s = SP;
             } else {
 #pragma unroll
-                for (int i = 0; i < RI; ++i)
-#pragma unroll
-                    for (int c = 0; c < CW; ++c) S[i][c] = s0[(lane + 32 * i) * LD0 + col0 + c];
+                for (int i = 0; i < RI; ++i) load_row<CW>(s0 + (lane + 32 * i) * LD0 + col0, S[i]);
             }
             for (; s < tt; ++s) {
                 fwd_step<RI, CW>(S, sk + s * DK, sa + s * DK, sv + s * DV, sb[s], lane, col0);
@@ -394,7 +415,7 @@ template <int DK, int DV>
 static cudaError_t launch_bwd_t(const BwdParams &prm, cudaStream_t stream) {
     const int BH = prm.B * prm.H;
     const int s1 = (2 * BWD_FT * DK + BWD_FT * DV + BWD_FT) * 4;
-    const int s2 = (DK * (DV + 1) + 3 * BWD_CK * DK + 2 * BWD_CK * DV + BWD_CK + 3 * BWD_CK * DK + BWD_CK + DK * DV) * 4;
+    const int s2 = (2 * DK * (DV + 4) + 3 * BWD_CK * DK + 2 * BWD_CK * DV + BWD_CK + 3 * BWD_CK * DK + BWD_CK + DK * DV) * 4;
     cudaError_t e = cudaFuncSetAttribute(bwd_ckpt_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, s1);
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(bwd_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, s2);
