@@ -721,20 +721,17 @@ def run_ours(args):
                 for k, v in d.items()}
         h_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
         h_hT = torch.empty(hT.shape, dtype=hT.dtype, pin_memory=True)
-        bufs = kda.DeviceBuffers.__new__(kda.DeviceBuffers)
-        bufs.q, bufs.k, bufs.v, bufs.g, bufs.beta, bufs.h0 = d["q"], d["k"], d["v"], d["g"], d["beta"], d["h0"]
-        bufs.out, bufs.hT = out, hT
         e2e_steps = max(1, min(args.steps, 3))
         nin = nout = 0
         kda.chunk_fwd_host(host["q"], host["k"], host["v"], host["g"], host["beta"], cfg.scale, host["h0"],
-                           out=h_out, hT=h_hT, bufs=bufs, stream=stream)
+                           out=h_out, hT=h_hT, stream=stream)
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         barrier(world)
         e0.record(stream)
         for _ in range(e2e_steps):
             nin, nout = kda.chunk_fwd_host(host["q"], host["k"], host["v"], host["g"], host["beta"], cfg.scale,
-                                           host["h0"], out=h_out, hT=h_hT, bufs=bufs, stream=stream)
+                                           host["h0"], out=h_out, hT=h_hT, stream=stream)
         e1.record(stream)
         torch.cuda.synchronize()
         barrier(world)

@@ -19,7 +19,7 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 LIB_PATH = os.path.join(HERE, "libkda.so")
 DEBUG_LIB_PATH = os.path.join(HERE, "libkda_debug.so")
-SOURCES = ["kda_api.cu", "decode.cu", "prep_fwd.cu", "exact_prep.cu", "chain_fwd.cu", "varlen_setup.cu", "parts_fixup.cu", "bwd.cu"]
+SOURCES = ["kda_api.cu", "decode.cu", "prep_fwd.cu", "exact_prep.cu", "chain_fwd.cu", "varlen_setup.cu", "parts_fixup.cu", "bwd.cu", "host_fwd.cu"]
 HEADERS = ["kda_device.cuh", "chunk_common.cuh", "chunk_params.cuh", "bwd_params.cuh"]
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
               "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden"]

@@ -396,7 +396,7 @@ kda::ExactParams exact_params(const void *q, const void *k, const float *g, int 
 
 extern "C" {
 
-int kda_abi_version(void) { return 102; }
+int kda_abi_version(void) { return 103; }
 
 const char *kda_status_string(int status) {
     switch (status) {
@@ -703,9 +703,12 @@ int kda_debug_kernel_launches(int *kind, long long *start_ns, long long *end_ns,
     return st;
 }
 
+extern "C" int kda_release_host_staging(int dev);  // host_fwd.cu
+
 int kda_release_workspace(void) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return KDA_ERR_CUDA;
+    const int hs = kda_release_host_staging(dev);
     std::lock_guard<std::mutex> lk(g_mu);
     Workspace &w = g_ws[dev];
     int st = KDA_OK;
@@ -717,7 +720,7 @@ int kda_release_workspace(void) {
     w.base = nullptr; w.base_bytes = 0;
     w.state = nullptr; w.state_bytes = 0;
     w.parts = nullptr; w.parts_bytes = 0;
-    return st;
+    return st != KDA_OK ? st : hs;
 }
 
 // The decode step for either gate form: g [B, H, dk] or, scalar_gate, g [B, H].

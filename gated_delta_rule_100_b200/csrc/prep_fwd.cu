@@ -629,9 +629,10 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 *reinterpret_cast<uint4 *>(wr + 8) = pack8_bf16(b8);
             }
         }
-        tc_fence_before();
-        __syncthreads();  // this item's shared memory and TMEM are free for the next one
-        tc_fence_after();
+        // This item's shared memory and TMEM are free for the next one.  No tcgen05
+        // fences: the W rows' TMEM loads completed (wait::ld), and the next tcgen05
+        // operation (the formation product) follows its own fenced barrier.
+        __syncthreads();
         item = next;
     }
 

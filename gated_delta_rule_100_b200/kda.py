@@ -14,9 +14,8 @@ The entry points mirror ``include/kda.h``:
 * ``workspace_bytes`` / ``release_workspace`` -> ``kda_chunk_fwd_workspace_bytes`` /
   ``kda_release_workspace``
 
-plus ``chunk_fwd_host``, the same prefill for host (pinned) tensors: it copies
-the inputs to the device, runs ``kda_chunk_fwd`` and copies the results back,
-all on one stream.
+* ``chunk_fwd_host`` -> ``kda_chunk_fwd_host`` (the prefill on host tensors, pinned for
+  overlap: the library streams pieces of the token axis up, through the prefill and back)
 
 If ``libkda.so`` is missing the calls raise; there is no fallback.
 """
@@ -33,7 +32,7 @@ DEBUG_LIB_PATH = os.path.join(_HERE, "libkda_debug.so")
 
 (KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_ALIGNMENT, KDA_ERR_CUDA, KDA_ERR_TIMEOUT,
  KDA_ERR_SCRATCH_LIMIT, KDA_ERR_BOUNDS) = range(8)
-EXPORTED = ("kda_chunk_fwd", "kda_chunk_fwd_noalloc", "kda_chunk_fwd_varlen", "kda_decode_step",
+EXPORTED = ("kda_chunk_fwd", "kda_chunk_fwd_noalloc", "kda_chunk_fwd_host", "kda_chunk_fwd_host_debug_piece", "kda_chunk_fwd_varlen", "kda_decode_step",
             "kda_gdn_chunk_fwd", "kda_gdn_decode_step", "kda_chunk_fwd_raw", "kda_decode_step_raw",
             "kda_chunk_bwd", "kda_chunk_bwd_workspace_bytes",
             "kda_chunk_fwd_workspace_bytes", "kda_chunk_fwd_varlen_workspace_bytes", "kda_release_workspace",
@@ -81,6 +80,10 @@ def _open(path):
     lib.kda_chunk_fwd.restype = i
     lib.kda_chunk_fwd_noalloc.argtypes = [vp, vp, vp, fp, fp, f, fp, vp, fp, i, i, i, i, i, vp]
     lib.kda_chunk_fwd_noalloc.restype = i
+    lib.kda_chunk_fwd_host.argtypes = [vp, vp, vp, fp, fp, f, fp, vp, fp, i, i, i, i, i, vp]
+    lib.kda_chunk_fwd_host.restype = i
+    lib.kda_chunk_fwd_host_debug_piece.argtypes = [i]
+    lib.kda_chunk_fwd_host_debug_piece.restype = None
     lib.kda_chunk_bwd.argtypes = [vp, vp, vp, fp, fp, f, fp, vp, fp, vp, vp, vp, fp, fp, fp, i, i, i, i, i, vp]
     lib.kda_chunk_bwd.restype = i
     lib.kda_chunk_bwd_workspace_bytes.argtypes = [i, i, i, i, i]
@@ -440,36 +443,42 @@ def kernel_launches(cap: int = 8192) -> list:
              (st[i] - t0) * 1e-6, (en[i] - t0) * 1e-6) for i in range(n)]
 
 
-class DeviceBuffers:
-    """Device copies of one prefill problem, allocated once and reused."""
-
-    def __init__(self, B, T, H, dk, dv, device, with_h0):
-        z = dict(device=device)
-        self.q = torch.empty((B, T, H, dk), dtype=torch.bfloat16, **z)
-        self.k = torch.empty((B, T, H, dk), dtype=torch.bfloat16, **z)
-        self.v = torch.empty((B, T, H, dv), dtype=torch.bfloat16, **z)
-        self.g = torch.empty((B, T, H, dk), dtype=torch.float32, **z)
-        self.beta = torch.empty((B, T, H), dtype=torch.float32, **z)
-        self.h0 = torch.empty((B, H, dk, dv), dtype=torch.float32, **z) if with_h0 else None
-        self.out = torch.empty((B, T, H, dv), dtype=torch.bfloat16, **z)
-        self.hT = torch.empty((B, H, dk, dv), dtype=torch.float32, **z)
+def _check_host(t, name, dtype, shape):
+    if t.is_cuda:
+        raise ValueError(f"{name} must be a host tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
 
 
-def chunk_fwd_host(q, k, v, g, beta, scale, h0=None, *, out, hT, bufs: DeviceBuffers, stream=None):
-    """Prefill from host tensors (pinned for asynchronous copies): H2D of the inputs,
-    ``kda_chunk_fwd`` on the device copies, D2H of out and hT, all enqueued on
-    ``stream``.  Returns the (bytes_h2d, bytes_d2h) it moved."""
-    st = torch.cuda.current_stream() if stream is None else stream
-    with torch.cuda.stream(st):
-        nin = 0
-        for src, dst in ((q, bufs.q), (k, bufs.k), (v, bufs.v), (g, bufs.g), (beta, bufs.beta),
-                         (h0, bufs.h0)):
-            if src is not None:
-                dst.copy_(src, non_blocking=True)
-                nin += src.numel() * src.element_size()
-        chunk_fwd(bufs.q, bufs.k, bufs.v, bufs.g, bufs.beta, scale,
-                  bufs.h0 if h0 is not None else None, out=bufs.out, hT=bufs.hT, stream=st)
-        out.copy_(bufs.out, non_blocking=True)
-        hT.copy_(bufs.hT, non_blocking=True)
-    nout = out.numel() * out.element_size() + hT.numel() * hT.element_size()
+def chunk_fwd_host(q, k, v, g, beta, scale, h0=None, *, out, hT=None, stream=None):
+    """``kda_chunk_fwd_host``: the prefill on HOST tensors (pinned, for overlapped copies),
+    shapes and dtypes as ``chunk_fwd``; writes ``out`` (and ``hT`` when given) once
+    ``stream`` reaches the end of the call's work.  Returns (bytes_h2d, bytes_d2h)."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    _check_host(q, "q", torch.bfloat16, (B, T, H, dk))
+    _check_host(k, "k", torch.bfloat16, (B, T, H, dk))
+    _check_host(v, "v", torch.bfloat16, (B, T, H, dv))
+    _check_host(g, "g", torch.float32, (B, T, H, dk))
+    _check_host(beta, "beta", torch.float32, (B, T, H))
+    _check_host(out, "out", torch.bfloat16, (B, T, H, dv))
+    if h0 is not None:
+        _check_host(h0, "h0", torch.float32, (B, H, dk, dv))
+    if hT is not None:
+        _check_host(hT, "hT", torch.float32, (B, H, dk, dv))
+    rc = load().kda_chunk_fwd_host(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale), _ptr(h0),
+                                   _ptr(out), _ptr(hT), B, T, H, dk, dv, _stream(stream))
+    if rc != KDA_OK:
+        raise KdaError(rc, "kda_chunk_fwd_host")
+    nin = sum(t.numel() * t.element_size() for t in (q, k, v, g, beta, h0) if t is not None)
+    nout = sum(t.numel() * t.element_size() for t in (out, hT) if t is not None)
     return nin, nout
+
+
+def set_host_piece(tokens: int) -> None:
+    """Test hook: pieces of ``tokens`` tokens for ``chunk_fwd_host`` (0 = automatic)."""
+    load().kda_chunk_fwd_host_debug_piece(int(tokens))

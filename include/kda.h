@@ -19,7 +19,8 @@
  * Conventions shared by every entry point
  * ---------------------------------------
  * - All pointers are DEVICE pointers (cudaMalloc / torch CUDA tensors) on the
- *   current device, row-major and contiguous, 16-byte aligned (beta: 4-byte).
+ *   current device, row-major and contiguous, 16-byte aligned (beta: 4-byte);
+ *   kda_chunk_fwd_host alone takes host pointers.
  * - bf16 tensors are passed as void* holding IEEE bfloat16 (uint16 bits).
  * - The caller owns every buffer it passes.  The library keeps no pointer to
  *   them after a call returns.  Library-owned device memory: one 4-byte status
@@ -307,6 +308,42 @@ KDA_API int kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v,
                   int B, int T, int H, int dk, int dv, void *stream);
 
 /*
+ * kda_chunk_fwd_host -- kda_chunk_fwd on HOST buffers: the one entry point
+ * whose tensor pointers are host memory (q, k, v, g, beta, out as for
+ * kda_chunk_fwd, h0 and hT fp32 [B, H, dk, dv] or NULL; any alignment).
+ * Page-locked (pinned) buffers let the copies run asynchronously; pageable
+ * ones work, with each copy staged synchronously by the runtime.
+ *
+ * The token axis runs in pieces of a multiple of 64 tokens (about 256 MB of
+ * inputs each): the upload of a piece, the prefill of the one before it
+ * (kda_chunk_fwd on device copies, continued from the previous piece's final
+ * state: the recurrence of section 3.3 of the Baidu breakdown is exact across
+ * any token boundary) and the download of the one before that overlap, on
+ * two internal copy streams and `stream`.  Results equal those of
+ * kda_chunk_fwd on the same inputs up to rounding at the piece boundaries
+ * (identical chunks; the state passes through memory in fp32).
+ *
+ * Work is enqueued and the call returns: the host buffers must stay valid and
+ * unchanged, and out / hT must not be read, until `stream` reaches the end of
+ * this call's work (cudaStreamSynchronize or an event on it).  The library
+ * holds device staging for two pieces and the state (grown on demand, freed
+ * by kda_release_workspace) besides kda_chunk_fwd's own workspace; calls on a
+ * device are ordered one after another.  T == 0 synchronises `stream` and sets
+ * hT = h0 (or zero) on the host.  Return codes as kda_chunk_fwd.
+ */
+KDA_API int kda_chunk_fwd_host(const void *q, const void *k, const void *v,
+                 const float *g, const float *beta, float scale,
+                 const float *h0, void *out, float *hT,
+                 int B, int T, int H, int dk, int dv, void *stream);
+
+/*
+ * kda_chunk_fwd_host_debug_piece -- test hook: pieces of `tokens` tokens for
+ * kda_chunk_fwd_host (any positive count, not only multiples of 64); 0
+ * restores the automatic size.  Process-wide.
+ */
+KDA_API void kda_chunk_fwd_host_debug_piece(int tokens);
+
+/*
  * kda_chunk_fwd_workspace_bytes -- device memory kda_chunk_fwd holds for these
  * sizes: the per-chunk records (72.5 KB per 64-token chunk and (b, h)) of
  * the whole sequence when they fit in 2 GiB, else of two segments of as many
@@ -318,8 +355,8 @@ KDA_API int kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v,
 KDA_API size_t kda_chunk_fwd_workspace_bytes(int B, int T, int H, int dk, int dv);
 
 /*
- * kda_release_workspace -- free the current device's prefill workspace (the
- * next kda_chunk_fwd allocates it again).  cudaFree synchronises the device,
+ * kda_release_workspace -- free the current device's prefill workspace and
+ * kda_chunk_fwd_host's staging (the next call allocates them again).  cudaFree synchronises the device,
  * so no launched work still uses it.  KDA_OK, or KDA_ERR_CUDA.
  */
 KDA_API int kda_release_workspace(void);
@@ -425,7 +462,7 @@ KDA_API int kda_debug_kernel_launches(int *kind, long long *start_ns, long long 
 /* Version of this ABI (major * 100 + minor): 101 adds the scalar-gate entry
  * points, 102 the packed-batch prefill, the raw-input (fused gate prologue)
  * entry points, the backward pass and the exact-path and two-level test
- * hooks. */
+ * hooks, 103 the host-buffer prefill and the per-launch timing list. */
 KDA_API int kda_abi_version(void);
 
 #ifdef __cplusplus

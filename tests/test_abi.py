@@ -33,7 +33,7 @@ def test_header_declares_the_boundary():
 def test_library_exports_every_declared_symbol(lib):
     for name in declared_symbols():
         assert hasattr(lib, name), name
-    assert lib.kda_abi_version() == 102
+    assert lib.kda_abi_version() == 103
 
 
 def test_status_strings(lib):
@@ -85,6 +85,25 @@ def test_chunk_fwd_rejects(lib, kw, code):
 ])
 def test_decode_step_rejects(lib, kw, code):
     assert decode(lib, **kw) == code
+
+
+def host_chunk(lib, q=A, k=A, v=A, g=A, beta=A, h0=None, out=A, hT=None, B=1, T=64, H=1, dk=64, dv=64):
+    return lib.kda_chunk_fwd_host(q, k, v, g, beta, 1.0, h0, out, hT, B, T, H, dk, dv, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), kda.KDA_ERR_INVALID_ARG),
+    (dict(g=None), kda.KDA_ERR_INVALID_ARG),
+    (dict(out=None), kda.KDA_ERR_INVALID_ARG),
+    (dict(B=0), kda.KDA_ERR_INVALID_ARG),
+    (dict(H=0), kda.KDA_ERR_INVALID_ARG),
+    (dict(T=-1), kda.KDA_ERR_INVALID_ARG),
+    (dict(dk=96), kda.KDA_ERR_UNSUPPORTED),
+    (dict(dv=32), kda.KDA_ERR_UNSUPPORTED),
+])
+def test_chunk_fwd_host_rejects(lib, kw, code):
+    # validated before any CUDA call (host pointers need no alignment)
+    assert host_chunk(lib, **kw) == code
 
 
 def test_zero_length_accepts_null_inputs(lib):
