@@ -19,7 +19,11 @@
 // (p, du) are warp shuffles, and the sums over columns go through
 // shared-memory atomics per token.
 //   Pass 1 (bwd_ckpt_kernel): the forward recurrence from h0, storing S every
-//          CK1 = 64 tokens (level-1 checkpoints, fp32, in the workspace).
+//          CK1 = 64 tokens (level-1 checkpoints, fp32, in the workspace) and
+//          every token's p = S'^T k (fp32 [T][dv] per (b, h)).  Every later
+//          forward step re-runs from a state this pass produced, so it finds
+//          the same p and reads it instead of reducing over the rows again:
+//          one column reduction per token is left (du), not four.
 //   Pass 2 (bwd_kernel): chunks of CK1 tokens from the last to the first.  Per
 //          chunk, the forward is re-run from its level-1 checkpoint to leave a
 //          state every CK = 4 tokens in a per-(b, h) scratch (level 2); then
@@ -30,7 +34,7 @@
 //          the way to the last token), then the reverse step.  After each block
 //          its tokens' dq, dk (bf16), dg and dbeta (fp32) are written; dv per
 //          column as it is formed; dh0 at the end.
-// Memory: (ceil(T / 64) + 16) dk dv fp32 per (b, h); forward steps per token:
+// Memory: (ceil(T / 64) + 16) dk dv + T dv fp32 per (b, h); forward steps per token:
 // one in pass 1, one for level 2, one on average for the per-token states
 // (blocks of 8 took 56 ms on B8 H32 T4096, 3.5 recomputed steps per token).
 // Inputs are staged in shared memory per block of tokens, loaded into registers
@@ -75,10 +79,11 @@ __device__ __forceinline__ void store_row(float *dst, const float (&x)[CW]) {
     for (int c = 0; c < CW; c += 4) *reinterpret_cast<float4 *>(dst + c) = make_float4(x[c], x[c + 1], x[c + 2], x[c + 3]);
 }
 
-// One forward step on this warp's columns: S <- Diag(a) S + k (beta (v - k^T Diag(a) S))^T.
+// One forward step on this warp's columns: S <- Diag(a) S + k (beta (v - k^T Diag(a) S))^T;
+// lane 0 writes p = k^T Diag(a) S of the columns to p_out (global, 16-byte aligned).
 template <int RI, int CW>
 __device__ __forceinline__ void fwd_step(float (&S)[RI][CW], const float *sk, const float *sa, const float *sv,
-                                         float beta, int lane, int col0) {
+                                         float beta, int lane, int col0, float *p_out) {
     float kr[RI], p[CW];
 #pragma unroll
     for (int i = 0; i < RI; ++i) kr[i] = sk[lane + 32 * i];
@@ -97,9 +102,32 @@ __device__ __forceinline__ void fwd_step(float (&S)[RI][CW], const float *sk, co
     for (int o = 16; o > 0; o >>= 1)
 #pragma unroll
         for (int c = 0; c < CW; ++c) p[c] += __shfl_xor_sync(0xffffffffu, p[c], o);
+    if (lane == 0) store_row<CW>(p_out + col0, p);
 #pragma unroll
     for (int c = 0; c < CW; ++c) {
         const float u = beta * (sv[col0 + c] - p[c]);
+#pragma unroll
+        for (int i = 0; i < RI; ++i) S[i][c] += kr[i] * u;
+    }
+}
+
+// The same step with p known (sp: the token's p, staged in shared memory): the
+// same operations in the same order, so the same state, without the reduction.
+template <int RI, int CW>
+__device__ __forceinline__ void fwd_step_p(float (&S)[RI][CW], const float *sk, const float *sa, const float *sv,
+                                           const float *sp, float beta, int lane, int col0) {
+    float kr[RI];
+#pragma unroll
+    for (int i = 0; i < RI; ++i) kr[i] = sk[lane + 32 * i];
+#pragma unroll
+    for (int i = 0; i < RI; ++i) {
+        const float a = sa[lane + 32 * i];
+#pragma unroll
+        for (int c = 0; c < CW; ++c) S[i][c] *= a;
+    }
+#pragma unroll
+    for (int c = 0; c < CW; ++c) {
+        const float u = beta * (sv[col0 + c] - sp[col0 + c]);
 #pragma unroll
         for (int i = 0; i < RI; ++i) S[i][c] += kr[i] * u;
     }
@@ -117,6 +145,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_ckpt_kernel(const BwdParam
     const int T = prm.T, H = prm.H;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, col0 = warp * CW;
     const int nck = (T + BWD_CK1 - 1) / BWD_CK1;
+    float *pbuf = prm.ckpt + (size_t)prm.B * H * (nck + BWD_CK1 / BWD_CK) * DK * DV + (size_t)bh * T * DV;
     if (tid == 0) stamp_start(prm.stamp);
     float S[RI][CW];
 #pragma unroll
@@ -149,7 +178,8 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_ckpt_kernel(const BwdParam
 #pragma unroll
                 for (int i = 0; i < RI; ++i) store_row<CW>(dst + (size_t)(lane + 32 * i) * DV + col0, S[i]);
             }
-            fwd_step<RI, CW>(S, sk + t * DK, sa + t * DK, sv + t * DV, sb[t], lane, col0);
+            fwd_step<RI, CW>(S, sk + t * DK, sa + t * DK, sv + t * DV, sb[t], lane, col0,
+                             pbuf + (size_t)(t0 + t) * DV);
         }
     }
     if (tid == 0) stamp_end(prm.stamp);
@@ -168,7 +198,8 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_kernel(const BwdParams prm
     float *sa = sq + CK * DK;        // [CK][DK] alpha
     float *sv = sa + CK * DK;        // [CK][DV]
     float *sd = sv + CK * DV;        // [CK][DV] dout
-    float *sb = sd + CK * DV;        // [CK] beta
+    float *sp = sd + CK * DV;        // [CK][DV] p (from pass 1)
+    float *sb = sp + CK * DV;        // [CK] beta
     float *acq = sb + CK;            // [CK][DK] sums over columns: dq
     float *ack = acq + CK * DK;      //                             dk
     float *aca = ack + CK * DK;      //                             d alpha
@@ -192,11 +223,12 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_kernel(const BwdParams prm
     }
 
     float *scratch = prm.ckpt + ((size_t)prm.B * H * nck1 + (size_t)bh * (BWD_CK1 / CK)) * DK * DV;
+    const float *pbuf = prm.ckpt + (size_t)prm.B * H * (nck1 + BWD_CK1 / CK) * DK * DV + (size_t)bh * T * DV;
     // The reverse walk's inputs for a block of CK tokens: loaded into registers one
     // block ahead (fetch), converted into the shared tiles at the block's start (put).
     constexpr int PK = (CK * DK + BWD_THREADS - 1) / BWD_THREADS, PV = (CK * DV + BWD_THREADS - 1) / BWD_THREADS;
     uint16_t rk[PK], rq[PK], rv[PV], rd[PV];
-    float rg[PK], rb = 0.f;
+    float rg[PK], rp[PV], rb = 0.f;
     int pf_t0 = -1;  // first token of the block held in the registers
     auto fetch = [&](int t0, int nt) {
 #pragma unroll
@@ -215,6 +247,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_kernel(const BwdParams prm
             const size_t row = ((size_t)b * T + (in ? t0 + t : 0)) * H + h;
             rv[x] = in ? prm.v[row * DV + c] : (uint16_t)0;
             rd[x] = (in && prm.dout) ? prm.dout[row * DV + c] : (uint16_t)0;
+            rp[x] = in ? pbuf[(size_t)(t0 + t) * DV + c] : 0.f;
         }
         rb = tid < nt ? prm.beta[((size_t)b * T + t0 + tid) * H + h] : 0.f;
         pf_t0 = t0;
@@ -235,6 +268,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_kernel(const BwdParams prm
             if (e < nt * DV) {
                 sv[e] = bf16_bits_to_f32(rv[x]);
                 sd[e] = bf16_bits_to_f32(rd[x]);
+                sp[e] = rp[x];
             }
         }
         if (tid < nt) sb[tid] = rb;
@@ -273,7 +307,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_kernel(const BwdParams prm
                     fetch(t1, T - t1 < CK ? T - t1 : CK);
                 }
                 for (int t = 0; t < nt; ++t)
-                    fwd_step<RI, CW>(S, sk + t * DK, sa + t * DK, sv + t * DV, sb[t], lane, col0);
+                    fwd_step_p<RI, CW>(S, sk + t * DK, sa + t * DK, sv + t * DV, sp + t * DV, sb[t], lane, col0);
             }
         }
     for (int j = nb - 1; j >= 0; --j) {
@@ -315,7 +349,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_kernel(const BwdParams prm
                 for (int i = 0; i < RI; ++i) load_row<CW>(s0 + (lane + 32 * i) * LD0 + col0, S[i]);
             }
             for (; s < tt; ++s) {
-                fwd_step<RI, CW>(S, sk + s * DK, sa + s * DK, sv + s * DV, sb[s], lane, col0);
+                fwd_step_p<RI, CW>(S, sk + s * DK, sa + s * DK, sv + s * DV, sp + s * DV, sb[s], lane, col0);
                 if (s + 1 == SP && tt > SP) {  // on the way to a later token: keep the state before SP
 #pragma unroll
                     for (int i = 0; i < RI; ++i)
@@ -335,29 +369,25 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_kernel(const BwdParams prm
                 qr[i] = qt[lane + 32 * i];
                 ar[i] = at[lane + 32 * i];
             }
-            // The readout's share of dS first (it needs no forward quantity), then the two
-            // column reductions together: p = (Diag(a) S)^T k and du = dS^T k.
+            // The readout's share of dS first (it needs no forward quantity), then the one
+            // column reduction du = dS^T k; p = (Diag(a) S)^T k is pass 1's.
             float p[CW], du[CW];
 #pragma unroll
             for (int c = 0; c < CW; ++c) {
                 const float d = scale * dot[col0 + c];
-                float pa = 0.f, ua = 0.f;
+                float ua = 0.f;
 #pragma unroll
                 for (int i = 0; i < RI; ++i) {
                     dS[i][c] += qr[i] * d;
-                    pa += kr[i] * ar[i] * S[i][c];
                     ua += dS[i][c] * kr[i];
                 }
-                p[c] = pa;
+                p[c] = sp[tt * DV + col0 + c];
                 du[c] = ua;
             }
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1)
 #pragma unroll
-                for (int c = 0; c < CW; ++c) {
-                    p[c] += __shfl_xor_sync(0xffffffffu, p[c], o);
-                    du[c] += __shfl_xor_sync(0xffffffffu, du[c], o);
-                }
+                for (int c = 0; c < CW; ++c) du[c] += __shfl_xor_sync(0xffffffffu, du[c], o);
             float dqp[RI], dkp[RI], dap[RI];
 #pragma unroll
             for (int i = 0; i < RI; ++i) { dqp[i] = 0.f; dkp[i] = 0.f; dap[i] = 0.f; }
@@ -415,7 +445,7 @@ template <int DK, int DV>
 static cudaError_t launch_bwd_t(const BwdParams &prm, cudaStream_t stream) {
     const int BH = prm.B * prm.H;
     const int s1 = (2 * BWD_FT * DK + BWD_FT * DV + BWD_FT) * 4;
-    const int s2 = (2 * DK * (DV + 4) + 3 * BWD_CK * DK + 2 * BWD_CK * DV + BWD_CK + 3 * BWD_CK * DK + BWD_CK + DK * DV) * 4;
+    const int s2 = (2 * DK * (DV + 4) + 3 * BWD_CK * DK + 3 * BWD_CK * DV + BWD_CK + 3 * BWD_CK * DK + BWD_CK + DK * DV) * 4;
     cudaError_t e = cudaFuncSetAttribute(bwd_ckpt_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, s1);
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(bwd_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, s2);
@@ -426,9 +456,11 @@ static cudaError_t launch_bwd_t(const BwdParams &prm, cudaStream_t stream) {
     return cudaGetLastError();
 }
 
-// Level-1 checkpoints [B H][ceil(T / CK1)] and level-2 scratch [B H][CK1 / CK], each dk x dv fp32.
+// Level-1 checkpoints [B H][ceil(T / CK1)] and level-2 scratch [B H][CK1 / CK], each dk x dv
+// fp32, then every token's p, [B H][T][dv] fp32.
 size_t bwd_ckpt_bytes(int B, int T, int H, int dk, int dv) {
-    return (size_t)B * H * ((T + BWD_CK1 - 1) / BWD_CK1 + BWD_CK1 / BWD_CK) * dk * dv * sizeof(float);
+    return (size_t)B * H * ((T + BWD_CK1 - 1) / BWD_CK1 + BWD_CK1 / BWD_CK) * dk * dv * sizeof(float) +
+           (size_t)B * H * T * dv * sizeof(float);
 }
 
 cudaError_t launch_bwd(const BwdParams &prm, int dk, int dv, cudaStream_t stream) {

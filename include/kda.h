@@ -216,8 +216,9 @@ KDA_API int kda_decode_step_raw(const void *q, const void *k, const void *v,
  *   dbeta : fp32 [B, T, H]
  *   dh0   : fp32 [B, H, dk, dv]  or NULL (not written)
  *
- * Workspace: the checkpoints, B H (ceil(T / 64) + 16) dk dv fp32
- * (kda_chunk_bwd_workspace_bytes: 1.3 GB for B8 H32 T4096 d128, 34 GB for
+ * Workspace: the state checkpoints, B H (ceil(T / 64) + 16) dk dv fp32, and
+ * each token's p = (Diag(alpha) S)^T k from the first pass, B H T dv fp32
+ * (kda_chunk_bwd_workspace_bytes: 1.9 GB for B8 H32 T4096 d128, 51 GB for
  * B1 H32 T1M), held like the prefill's workspace (grown with cudaMalloc,
  * freed by kda_release_workspace).  T == 0 sets dh0 = dhT.
  * Errors as kda_chunk_fwd.

@@ -265,8 +265,8 @@ def test_backward_rejects(lib):
     # T == 0 with no dh0 wanted: nothing to do
     assert bwd(q=None, k=None, v=None, g=None, beta=None, dq=None, dk=None, dv=None, dg=None, db=None, T=0) == \
         kda.KDA_OK
-    # a state every 64 tokens and a scratch of 16 states, per (b, h)
-    assert lib.kda_chunk_bwd_workspace_bytes(2, 100, 3, 128, 64) == 2 * 3 * (2 + 16) * 128 * 64 * 4
+    # a state every 64 tokens and a scratch of 16 states, then every token's p, per (b, h)
+    assert lib.kda_chunk_bwd_workspace_bytes(2, 100, 3, 128, 64) == 2 * 3 * ((2 + 16) * 128 * 64 + 100 * 64) * 4
 
 
 def test_debug_library_exports_the_same_symbols(lib):
