@@ -16,8 +16,9 @@ launching stream, barrier + synchronize on both sides, max over ranks.
 Also measured and reported in the same line:
   decode   64 consecutive kda_decode_step calls on B=256, H=32, d=128 with a
            512 MiB fp32 state (GB/s of algorithmic traffic);
-  e2e      the same prefill metric through the public API with pinned host
-           buffers: H2D of the inputs, the kernel, D2H of out and hT per step;
+  e2e      the same prefill metric through kda_chunk_fwd_host with pinned host
+           buffers: H2D of the inputs, the kernels, D2H of out and hT per step
+           (pieces of the token axis overlapped on three streams);
   roofline achieved algorithmic GB/s of the prefill call (its kernels) vs
            measured HBM peak, with each kernel's busy time from one extra step
            whose launches the kernels stamp themselves (%globaltimer);
