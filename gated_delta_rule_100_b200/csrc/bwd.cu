@@ -410,9 +410,14 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_kernel(const BwdParams prm
                     dS[i][c] = ar[i] * dsd;
                 }
             }
-            if (lane == 0) {
+            if (lane == 0) {  // this warp's CW columns of dv = beta du, one 8- or 16-byte store
+                uint32_t w[CW / 2];
 #pragma unroll
-                for (int c = 0; c < CW; ++c) prm.dv[row * DV + col0 + c] = to_bf16_bits(bt * du[c]);
+                for (int c = 0; c < CW; c += 2) w[c / 2] = pack_bf16x2(bt * du[c], bt * du[c + 1]);
+                if constexpr (CW == 8)
+                    *reinterpret_cast<uint4 *>(prm.dv + row * DV + col0) = make_uint4(w[0], w[1], w[2], w[3]);
+                else
+                    *reinterpret_cast<uint2 *>(prm.dv + row * DV + col0) = make_uint2(w[0], w[1]);
                 atomicAdd(&acb[tt], dbp);
             }
 #pragma unroll
