@@ -201,12 +201,13 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         if (!SG && tid == 32) tma_load_4d(sbase + L::OFF_GIN, &tm_g, bar_in, 0, h, gi.tok0, gi.bcoord);
         tma_pending = true;
         float al[SUB];
-        if constexpr (SG) {  // one gate per (token, head), shared by all channels: plain loads
-            const float *gp = prm.g + (size_t)(gi.row0 + tb) * H + h;
-#pragma unroll
-            for (int u = 0; u < SUB; ++u)
-                al[u] = (tb + u < gi.nvalid && active && KDA_CHECK(prm.st, gi.row0 + tb + u < rows))
-                            ? __ldg(gp + (size_t)u * H) : 0.f;
+        // SG: one gate per (token, head), shared by all channels: threads 64..127 stage
+        // the chunk's 64 gates in shared memory (the prologue's norm slots, unused here)
+        float *s_gsc = reinterpret_cast<float *>(sm + L::OFF_MISC + 256);
+        if (SG && tid >= CH && tid < 2 * CH) {
+            const int t = tid - CH;
+            s_gsc[t] = (t < gi.nvalid && KDA_CHECK(prm.st, gi.row0 + t < rows))
+                           ? __ldg(prm.g + (size_t)(gi.row0 + t) * H + h) : 0.f;
         }
         if (tid < CH) {
             const float braw = (tid < gi.nvalid && KDA_CHECK(prm.st, gi.row0 + tid < rows))
@@ -219,6 +220,9 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             const float *gs = reinterpret_cast<const float *>(sm + L::OFF_GIN) + tb * DK + c;
 #pragma unroll
             for (int u = 0; u < SUB; ++u) al[u] = (tb + u < gi.nvalid && active) ? gs[u * DK] : 0.f;
+        } else {
+#pragma unroll
+            for (int u = 0; u < SUB; ++u) al[u] = (tb + u < gi.nvalid && active) ? s_gsc[tb + u] : 0.f;
         }
         float *s_rn = reinterpret_cast<float *>(sm + L::OFF_MISC + 256);  // PRO: 1 / |q_t|, then 1 / |k_t|
         if constexpr (PRO) {
