@@ -23,6 +23,10 @@ Also measured and reported in the same line:
            measured HBM peak, with each kernel's busy time from one extra step
            whose launches the kernels stamp themselves (%globaltimer);
   training the training-shape prefill (B8 H32 T4096) timed the same way;
+  raw_prologue  kda_chunk_fwd_raw (gate prologue fused) on the step's workload;
+  varlen   kda_chunk_fwd_varlen on a packed batch of 64 sequences of mixed lengths;
+  two_level  a few-heads long sequence (B1 H4 T262144) with and without the
+           two-level pass;
   backward kda_chunk_bwd on the training shape (fp32 CUDA cores, "alu" roofline);
   cpu_baseline  the fp64 oracle on a bounded sample of the workload (rank 0,
            N = 1 only), plus every workload's recipe on 1 thread and all cores.
@@ -110,6 +114,118 @@ def measure_scalar_gate(d, cfg, out, hT, stream, steps, warmup, P):
             "config": {"workload": cfg.name, "gate": "fp32 [B,T,H]: key channel 0 of the workload's gate"},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": P["hbm_gbs"], "unit": "GB/s",
                          "frac": achieved / P["hbm_gbs"], "algorithmic_bytes_per_launch": nbytes}}
+
+
+def _time_calls(step, stream, steps, warmup):
+    """Mean ms of `steps` calls of `step` on `stream` after `warmup` untimed ones,
+    CUDA events on the stream; raises if the library reports a device-side error."""
+    import torch
+
+    from gated_delta_rule_100_b200 import kda
+
+    for _ in range(max(1, warmup)):
+        step()
+    torch.cuda.synchronize()
+    if kda.stream_status(stream) != kda.KDA_OK:
+        raise RuntimeError("device-side error during warm-up")
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if kda.stream_status(stream) != kda.KDA_OK:
+        raise RuntimeError("device-side error in the timed steps")
+    return e0.elapsed_time(e1) / steps
+
+
+def _hbm_roofline(nbytes, ms, P):
+    achieved = nbytes / (ms / 1e3) / 1e9
+    return {"bound": "hbm", "achieved": achieved, "peak": P["hbm_gbs"], "unit": "GB/s",
+            "frac": achieved / P["hbm_gbs"], "algorithmic_bytes_per_launch": nbytes}
+
+
+def measure_raw(d, cfg, out, hT, stream, steps, warmup, P):
+    """The fused gate prologue (kda_chunk_fwd_raw) on the bench workload: its
+    tensors passed as the raw projections (q, k normalised again in the kernels,
+    g = -c softplus(g_raw) with c = the workload's decay scale, beta = sigmoid of
+    the workload's beta), timed like the step."""
+    from gated_delta_rule_100_b200 import kda
+
+    c = cfg.decay
+
+    def step():
+        kda.chunk_fwd_raw(d["q"], d["k"], d["v"], d["g"], d["beta"], c, cfg.scale, d["h0"], out=out, hT=hT,
+                          stream=stream)
+
+    ms = _time_calls(step, stream, steps, warmup)
+    nbytes = prefill_bytes(cfg.B, cfg.T, cfg.H, cfg.dk, cfg.dv, cfg.h0_std > 0, True)
+    return {"metric": "raw-input prefill tokens/s", "value": cfg.B * cfg.T / (ms / 1e3), "unit": "tokens/s",
+            "ms_per_step": ms, "steps": steps, "entry_point": "kda_chunk_fwd_raw",
+            "config": {"workload": cfg.name, "raw": "the workload's q, k, g, beta as raw projections",
+                       "gate_c": c},
+            "roofline": _hbm_roofline(nbytes, ms, P)}
+
+
+def measure_varlen(stream, steps, warmup, P, dev):
+    """A packed batch (kda_chunk_fwd_varlen): 64 sequences of log-uniform lengths in
+    [128, 16384] (269,705 tokens), 32 heads, a state per sequence in and out."""
+    import torch
+
+    from gated_delta_rule_100_b200 import inputs, kda
+
+    vc = inputs.VARLEN_CONFIG
+    d = inputs.make_varlen(vc, device=dev)
+    T = d["q"].shape[0]
+    out = torch.empty((T, vc.H, vc.dv), dtype=torch.bfloat16, device=dev)
+    hT = torch.empty((vc.N, vc.H, vc.dk, vc.dv), dtype=torch.float32, device=dev)
+
+    def step():
+        kda.chunk_fwd_varlen(d["q"], d["k"], d["v"], d["g"], d["beta"], vc.scale, d["cu_seqlens"], d["h0"],
+                             out=out, hT=hT, stream=stream)
+
+    ms = _time_calls(step, stream, steps, warmup)
+    state = 4 * vc.dk * vc.dv * vc.N * vc.H
+    nbytes = prefill_bytes(1, T, vc.H, vc.dk, vc.dv, False, False) + 2 * state
+    lengths = inputs.varlen_lengths(vc)
+    del d, out, hT
+    return {"metric": "packed-batch prefill tokens/s", "value": T / (ms / 1e3), "unit": "tokens/s",
+            "ms_per_step": ms, "steps": steps, "entry_point": "kda_chunk_fwd_varlen",
+            "config": {"workload": vc.name, "N": vc.N, "T_total": T, "H": vc.H, "dk": vc.dk, "dv": vc.dv,
+                       "min_len": min(lengths), "max_len": max(lengths), "seed": vc.seed},
+            "roofline": _hbm_roofline(nbytes, ms, P)}
+
+
+def measure_two_level(stream, steps, warmup, P, dev):
+    """Few heads, long sequence (B1 H4 T262144): kda_chunk_fwd with its automatic
+    two-level pass, and the same call with the two-level pass off (one chain CTA
+    per (b, h, value slice) walking all 4,096 chunks)."""
+    import torch
+
+    from gated_delta_rule_100_b200 import inputs, kda
+
+    tc = inputs.TWO_LEVEL_CONFIG
+    d = inputs.make_config(tc, device=dev)
+    out = torch.empty((tc.B, tc.T, tc.H, tc.dv), dtype=torch.bfloat16, device=dev)
+    hT = torch.empty((tc.B, tc.H, tc.dk, tc.dv), dtype=torch.float32, device=dev)
+
+    def step():
+        kda.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], tc.scale, d["h0"], out=out, hT=hT, stream=stream)
+
+    try:
+        kda.set_parts(0)
+        ms = _time_calls(step, stream, steps, warmup)
+        kda.set_parts(1)
+        ms_plain = _time_calls(step, stream, steps, warmup)
+    finally:
+        kda.set_parts(0)
+    nbytes = prefill_bytes(tc.B, tc.T, tc.H, tc.dk, tc.dv, tc.h0_std > 0, True)
+    del d, out, hT
+    return {"metric": "few-heads long-sequence prefill tokens/s", "value": tc.B * tc.T / (ms / 1e3),
+            "unit": "tokens/s", "ms_per_step": ms, "plain_pass_ms_per_step": ms_plain, "steps": steps,
+            "entry_point": "kda_chunk_fwd (two-level pass chosen automatically)",
+            "config": {"workload": tc.name, "B": tc.B, "H": tc.H, "T": tc.T, "dk": tc.dk, "dv": tc.dv},
+            "roofline": _hbm_roofline(nbytes, ms, P)}
 
 
 def prefill_flops(B, T, H, dk, dv, C=CHUNK):
@@ -672,6 +788,27 @@ def run_ours(args):
         except Exception as exc:  # noqa: BLE001 - an extra item must not cost the measurement above
             training = {"error": f"{type(exc).__name__}: {exc}"[:300]}
 
+    raw = None
+    if not args.no_raw:
+        try:
+            raw = measure_raw(d, cfg, out, hT, stream, args.steps, args.warmup, P)
+        except Exception as exc:  # noqa: BLE001 - an extra item must not cost the measurement above
+            raw = {"error": f"{type(exc).__name__}: {exc}"[:300]}
+
+    varlen = None
+    if not args.no_varlen:
+        try:
+            varlen = measure_varlen(stream, args.steps, args.warmup, P, dev)
+        except Exception as exc:  # noqa: BLE001
+            varlen = {"error": f"{type(exc).__name__}: {exc}"[:300]}
+
+    two_level = None
+    if not args.no_two_level:
+        try:
+            two_level = measure_two_level(stream, args.steps, args.warmup, P, dev)
+        except Exception as exc:  # noqa: BLE001
+            two_level = {"error": f"{type(exc).__name__}: {exc}"[:300]}
+
     backward = None
     if not args.no_backward:
         try:
@@ -762,6 +899,7 @@ def run_ours(args):
                        "parallelism": f"weak: one workload copy per GPU x{world}"},
             "tflops": nflops / (ms_per_step / 1e3) / 1e12 * world,
             "roofline": roof, "decode": dec, "scalar_gate": gdn, "training": training, "backward": backward,
+            "raw_prologue": raw, "varlen": varlen, "two_level": two_level,
             "e2e": e2e,
             "cpu_baseline": cpu,
             "clocks": clk.summary(), "gpu_launches": gpu_launches,
@@ -786,6 +924,9 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-training", action="store_true", help="skip the training-shape prefill line")
     ap.add_argument("--no-backward", action="store_true", help="skip the training-shape backward line")
+    ap.add_argument("--no-raw", action="store_true", help="skip the raw-input (gate prologue) prefill line")
+    ap.add_argument("--no-varlen", action="store_true", help="skip the packed-batch prefill line")
+    ap.add_argument("--no-two-level", action="store_true", help="skip the few-heads long-sequence line")
     ap.add_argument("--record-traffic", metavar="CSV",
                     help="write profiles/traffic.json from an ncu dram-bytes CSV and exit")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -19,7 +19,10 @@ along T so the fp32 temporaries stay small on long sequences):
 Decode draws the fp32 state first (``state_std * randn``), then for every
 step the same five tensors as above with T = 1.
 
-The shapes and decay scales are those of the workloads in ``CONFIGS``.
+The shapes and decay scales are those of the workloads in ``CONFIGS``; two more
+shapes measure paths of their own: a few-heads long sequence
+(``TWO_LEVEL_CONFIG``) and a packed batch of sequences of mixed lengths
+(``VARLEN_CONFIG``, lengths from ``varlen_lengths``).
 """
 from __future__ import annotations
 
@@ -79,6 +82,62 @@ CONFIGS = {
                                                            128, 128, 0.01, 0.0, 3),
 }
 DECODE_CONFIG = DecodeConfig("decode_B256_H32_d128_64steps", 256, 32, 128, 128, 0.05, 0.02, 64, 4)
+
+# Few heads, long sequence: the shape the two-level pass is for (4 heads leave most
+# SMs idle under one chain CTA per head).
+TWO_LEVEL_CONFIG = PrefillConfig("two_level_B1_H4_T262144_d128", 1, 4, 1 << 18, 128, 128, 0.01, 0.02, 5)
+
+
+@dataclass(frozen=True)
+class VarlenConfig:
+    """A packed batch: N sequences whose lengths are drawn log-uniformly in
+    [min_len, max_len] (a serving mix of short and long prompts), back to back
+    along the token axis, each with its own initial state."""
+    name: str
+    N: int
+    H: int
+    dk: int
+    dv: int
+    min_len: int
+    max_len: int
+    decay: float
+    h0_std: float
+    seed: int
+
+    @property
+    def scale(self) -> float:
+        return self.dk ** -0.5
+
+
+VARLEN_CONFIG = VarlenConfig("varlen_N64_H32_d128_len128-16384", 64, 32, 128, 128, 128, 16384, 0.05, 0.02, 6)
+
+
+def varlen_lengths(cfg: VarlenConfig):
+    """The N sequence lengths of a packed-batch workload (a CPU generator seeded with
+    ``seed``: log-uniform draws, rounded down, at least min_len)."""
+    gen = torch.Generator().manual_seed(int(cfg.seed))
+    u = torch.rand(cfg.N, generator=gen, dtype=torch.float64)
+    lo, hi = torch.log(torch.tensor(float(cfg.min_len))), torch.log(torch.tensor(float(cfg.max_len)))
+    return [max(cfg.min_len, int(x)) for x in torch.exp(lo + u * (hi - lo)).tolist()]
+
+
+def make_varlen(cfg: VarlenConfig, device="cpu"):
+    """Packed-batch inputs: dict(q, k, v, g, beta [T_total, ...], h0 [N, H, dk, dv] or
+    None, cu_seqlens int32 [N + 1]) drawn with the prefill recipe on one row of
+    T_total = sum of the lengths tokens (seed + 1 for h0 after the row's draws)."""
+    lengths = varlen_lengths(cfg)
+    T = sum(lengths)
+    d = make_prefill(1, T, cfg.H, cfg.dk, cfg.dv, decay=cfg.decay, h0_std=0.0, seed=cfg.seed, device=device)
+    d = {k: (v[0] if v is not None else None) for k, v in d.items()}
+    if cfg.h0_std > 0:
+        gen = torch.Generator(device=device)
+        gen.manual_seed(int(cfg.seed) + 1)
+        d["h0"] = cfg.h0_std * _randn((cfg.N, cfg.H, cfg.dk, cfg.dv), gen, device)
+    cu = [0]
+    for n in lengths:
+        cu.append(cu[-1] + n)
+    d["cu_seqlens"] = torch.tensor(cu, dtype=torch.int32, device=device)
+    return d
 
 
 def _randn(shape, gen, device):
