@@ -228,19 +228,28 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         if constexpr (PRO) {
 #pragma unroll
             for (int u = 0; u < SUB; ++u) al[u] = (tb + u < gi.nvalid && active) ? gate_logdecay(al[u], prm.gate_c) : 0.f;
-            // warp w: rows 8 w .. 8 w + 7 of [q; k]; each lane sums DK / 32 squares
-            for (int rr = 0; rr < 8; ++rr) {
-                const int row = warp * 8 + rr;
+            // 1 / |row| of the 128 rows of [q; k]: warp w takes rows 8 w .. 8 w + 7, each row
+            // on DK / 8 lanes that load one 16-byte chunk (8 values) apiece; the tile's
+            // swizzle only permutes the chunks of a 128-byte row, which a sum ignores
+            constexpr int CPR = DK / 8, RPI = 32 / CPR;  // chunks per row, rows per pass
+            const int sub = lane / CPR, chunk = lane % CPR;
+#pragma unroll
+            for (int it = 0; it < 8 / RPI; ++it) {
+                const int row = warp * 8 + it * RPI + sub;
                 const uint8_t *tile = sm + (row < CH ? L::OFF_QIN : L::OFF_KIN);
+                const uint4 w = *reinterpret_cast<const uint4 *>(tile + (chunk >> 3) * CH * 128 +
+                                                                 (row & (CH - 1)) * 128 + (chunk & 7) * 16);
+                const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
                 float ss = 0.f;
 #pragma unroll
-                for (int cc = lane; cc < DK; cc += 32) {
-                    const float x = bf16_bits_to_f32(*reinterpret_cast<const uint16_t *>(tile + kmaj<128, 2>(row & (CH - 1), cc, CH)));
-                    ss += x * x;
+                for (int j = 0; j < 4; ++j) {
+                    const float lo = __uint_as_float(wv[j] << 16), hi = __uint_as_float(wv[j] & 0xFFFF0000u);
+                    ss += lo * lo;
+                    ss += hi * hi;
                 }
 #pragma unroll
-                for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-                if (lane == 0) s_rn[row] = rsqrtf(fmaxf(ss, 1e-24f));
+                for (int o = CPR / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+                if (chunk == 0) s_rn[row] = rsqrtf(fmaxf(ss, 1e-24f));
             }
             __syncthreads();
         }
@@ -256,15 +265,16 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 uint32_t k1 = *reinterpret_cast<const uint16_t *>(ks + kmaj<128, 2>(tb + 2 * e + 1, c, CH));
                 uint32_t q0 = *reinterpret_cast<const uint16_t *>(qs + kmaj<128, 2>(tb + 2 * e, c, CH));
                 uint32_t q1 = *reinterpret_cast<const uint16_t *>(qs + kmaj<128, 2>(tb + 2 * e + 1, c, CH));
-                if constexpr (PRO) {
+                if constexpr (PRO) {  // normalised, rounded to bf16 again, two at a time
                     const int t = tb + 2 * e;
-                    k0 = to_bf16_bits(bf16_bits_to_f32((uint16_t)k0) * s_rn[CH + t]);
-                    k1 = to_bf16_bits(bf16_bits_to_f32((uint16_t)k1) * s_rn[CH + t + 1]);
-                    q0 = to_bf16_bits(bf16_bits_to_f32((uint16_t)q0) * s_rn[t]);
-                    q1 = to_bf16_bits(bf16_bits_to_f32((uint16_t)q1) * s_rn[t + 1]);
+                    const float2 nk = *reinterpret_cast<const float2 *>(s_rn + CH + t);
+                    const float2 nq = *reinterpret_cast<const float2 *>(s_rn + t);
+                    kp[e] = pack_bf16x2(bf16_bits_to_f32((uint16_t)k0) * nk.x, bf16_bits_to_f32((uint16_t)k1) * nk.y);
+                    qp[e] = pack_bf16x2(bf16_bits_to_f32((uint16_t)q0) * nq.x, bf16_bits_to_f32((uint16_t)q1) * nq.y);
+                } else {
+                    kp[e] = k0 | (k1 << 16);
+                    qp[e] = q0 | (q1 << 16);
                 }
-                kp[e] = k0 | (k1 << 16);
-                qp[e] = q0 | (q1 << 16);
             }
         }
         auto unpack = [](const uint32_t (&pr)[SUB / 2], int u) {
