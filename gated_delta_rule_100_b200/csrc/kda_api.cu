@@ -99,7 +99,6 @@ size_t record_cap() {
     const unsigned long long c = g_record_cap.load();
     return c ? (size_t)c : kWorkspaceCap;
 }
-constexpr double kPrepCtasPerFreeSm = 2.0;         // prep density beside a chain kernel
 constexpr size_t kTicketBytes = 256;               // per record buffer: item counter, steep-item count
 struct Workspace {
     uint8_t *base = nullptr;  // [counters][steep-item list][records]
@@ -511,13 +510,13 @@ static int chunk_fwd_impl(const void *q, const void *k, const void *v, const flo
     for (int i = 0; i < pl.nbuf; ++i)
         if (make_rec_maps(enc, recs[i], (long long)B * H * seg, dk, rmaps[i]) != KDA_OK) return KDA_ERR_CUDA;
 
-    // Prep CTAs: two per SM when prep runs alone; beside a chain kernel, two
-    // per SM the chain leaves free (lower densities slowed the whole call on
-    // the long-context workload: the chain speeds up less than prep slows).
-    // Its CTAs claim items from a counter, so any that start late only share
-    // the remaining work.
-    const int chain_ctas = B * H * chain_slices(B, H, dv, sms);
-    const int prep_ctas = (multi && chain_ctas < sms) ? (int)(kPrepCtasPerFreeSm * (sms - chain_ctas) + 0.5) : 2 * sms;
+    // Prep CTAs: two per SM, also beside a chain kernel.  The chain's CTAs are
+    // placed first (the next prep waits for them), so the prep CTAs that do not
+    // fit on the SMs the chain leaves free wait in the queue and start on the
+    // chain's SMs as soon as it ends; they claim items from the same counter, so
+    // they take over the segment's tail (long-context call 51.7 -> 49.8 ms
+    // against two CTAs per free SM only; lower densities were slower still).
+    const int prep_ctas = 2 * sms;
     cudaStream_t sp = s, sc = s;  // prep and chain streams
     if (multi) {
         sp = w->lo;
@@ -551,8 +550,7 @@ static int chunk_fwd_impl(const void *q, const void *k, const void *v, const flo
         pp.H = H;
         pp.gm = uniform_geom(B, T, n0, cnt);
         pp.st = dst;
-        // the first segment's prep runs alone: two CTAs on every SM
-        const int ctas = i == 0 ? 2 * sms : (prep_ctas > 0 ? prep_ctas : 1);
+        const int ctas = prep_ctas;
         cudaError_t e = timed_launch(dev, 0, sp, [&](unsigned long long *t) {
             pp.stamp = t;
             return kda::launch_prep(tq, tk, tg, pp, dk, ctas, sp, prologue);
