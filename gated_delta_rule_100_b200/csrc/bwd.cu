@@ -79,35 +79,48 @@ __device__ __forceinline__ void store_row(float *dst, const float (&x)[CW]) {
     for (int c = 0; c < CW; c += 4) *reinterpret_cast<float4 *>(dst + c) = make_float4(x[c], x[c + 1], x[c + 2], x[c + 3]);
 }
 
-// One forward step on this warp's columns: S <- Diag(a) S + k (beta (v - k^T Diag(a) S))^T;
-// lane 0 writes p = k^T Diag(a) S of the columns to p_out (global, 16-byte aligned).
-template <int RI, int CW>
-__device__ __forceinline__ void fwd_step(float (&S)[RI][CW], const float *sk, const float *sa, const float *sv,
-                                         float beta, int lane, int col0, float *p_out) {
-    float kr[RI], p[CW];
+// Pass 1's layout: thread (rg, cg) of an 8 x 64 grid holds rows 4 rg + 32 i + r
+// (i < DK / 32, r < 4) of the state and columns cg CP .. cg CP + CP - 1 (CP = DV / 64),
+// so the column reduction p = (Diag(a) S)^T k is DK / 8 products in the thread and a
+// three-level shuffle over the 8 row groups (lanes rg of one cg).  Rows in blocks of
+// four make each 16-byte read of k or alpha by 8 lanes one conflict-free wavefront.
+// One forward step S <- Diag(a) S + k (beta (v - p))^T; the rg == 0 lanes write p to
+// p_out.  Per element the operations are those of fwd_step_p, in the same order.
+template <int DK, int DV>
+__device__ __forceinline__ void fwd_step_rows(float (&S)[DK / 8][DV / 64], const float *sk, const float *sa,
+                                              const float *sv, float beta, int rg, int c0, float *p_out) {
+    constexpr int RP = DK / 8, CP = DV / 64;
+    float kr[RP], p[CP];
 #pragma unroll
-    for (int i = 0; i < RI; ++i) kr[i] = sk[lane + 32 * i];
+    for (int c = 0; c < CP; ++c) p[c] = 0.f;
 #pragma unroll
-    for (int c = 0; c < CW; ++c) p[c] = 0.f;
+    for (int i = 0; i < RP / 4; ++i) {
+        const float4 k4 = *reinterpret_cast<const float4 *>(sk + 4 * rg + 32 * i);
+        const float4 a4 = *reinterpret_cast<const float4 *>(sa + 4 * rg + 32 * i);
+        const float kk[4] = {k4.x, k4.y, k4.z, k4.w}, aa[4] = {a4.x, a4.y, a4.z, a4.w};
 #pragma unroll
-    for (int i = 0; i < RI; ++i) {
-        const float a = sa[lane + 32 * i];
+        for (int r = 0; r < 4; ++r) {
+            kr[4 * i + r] = kk[r];
 #pragma unroll
-        for (int c = 0; c < CW; ++c) {
-            S[i][c] *= a;
-            p[c] += kr[i] * S[i][c];
+            for (int c = 0; c < CP; ++c) {
+                S[4 * i + r][c] *= aa[r];
+                p[c] += kk[r] * S[4 * i + r][c];
+            }
         }
     }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1)
+    for (int o = 1; o < 8; o <<= 1)
 #pragma unroll
-        for (int c = 0; c < CW; ++c) p[c] += __shfl_xor_sync(0xffffffffu, p[c], o);
-    if (lane == 0) store_row<CW>(p_out + col0, p);
+        for (int c = 0; c < CP; ++c) p[c] += __shfl_xor_sync(0xffffffffu, p[c], o);
+    if (rg == 0) {
+        if constexpr (CP == 2) *reinterpret_cast<float2 *>(p_out + c0) = make_float2(p[0], p[1]);
+        else p_out[c0] = p[0];
+    }
 #pragma unroll
-    for (int c = 0; c < CW; ++c) {
-        const float u = beta * (sv[col0 + c] - p[c]);
+    for (int c = 0; c < CP; ++c) {
+        const float u = beta * (sv[c0 + c] - p[c]);
 #pragma unroll
-        for (int i = 0; i < RI; ++i) S[i][c] += kr[i] * u;
+        for (int i = 0; i < RP; ++i) S[i][c] += kr[i] * u;
     }
 }
 
@@ -135,7 +148,7 @@ __device__ __forceinline__ void fwd_step_p(float (&S)[RI][CW], const float *sk, 
 
 template <int DK, int DV>
 __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_ckpt_kernel(const BwdParams prm) {
-    constexpr int RI = DK / 32, CW = DV / 16;
+    constexpr int RP = DK / 8, CP = DV / 64;  // rows and columns of the state per thread
     extern __shared__ __align__(16) float fsm[];
     float *sk = fsm;                      // [FT][DK]
     float *sa = sk + BWD_FT * DK;         // [FT][DK] alpha
@@ -143,20 +156,18 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_ckpt_kernel(const BwdParam
     float *sb = sv + BWD_FT * DV;         // [FT]
     const int bh = blockIdx.x, b = bh / prm.H, h = bh % prm.H;
     const int T = prm.T, H = prm.H;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, col0 = warp * CW;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int rg = lane & 7, c0 = (warp * 4 + (lane >> 3)) * CP;  // row group, first column
     const int nck = (T + BWD_CK1 - 1) / BWD_CK1;
     float *pbuf = prm.ckpt + (size_t)prm.B * H * (nck + BWD_CK1 / BWD_CK) * DK * DV + (size_t)bh * T * DV;
     if (tid == 0) stamp_start(prm.stamp);
-    float S[RI][CW];
+    auto row_of = [&](int j) { return 4 * rg + 32 * (j >> 2) + (j & 3); };  // this thread's j-th row
+    float S[RP][CP];
 #pragma unroll
-    for (int i = 0; i < RI; ++i) {
-        if (prm.h0) {
-            load_row<CW>(prm.h0 + ((size_t)bh * DK + lane + 32 * i) * DV + col0, S[i]);
-        } else {
+    for (int j = 0; j < RP; ++j)
 #pragma unroll
-            for (int c = 0; c < CW; ++c) S[i][c] = 0.f;
-        }
-    }
+        for (int c = 0; c < CP; ++c)
+            S[j][c] = prm.h0 ? prm.h0[((size_t)bh * DK + row_of(j)) * DV + c0 + c] : 0.f;
     for (int t0 = 0; t0 < T; t0 += BWD_FT) {
         const int nt = T - t0 < BWD_FT ? T - t0 : BWD_FT;
         __syncthreads();  // the previous block's inputs are no longer read
@@ -176,10 +187,14 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_ckpt_kernel(const BwdParam
             if ((t0 + t) % BWD_CK1 == 0) {  // the state before token t0 + t
                 float *dst = prm.ckpt + ((size_t)bh * nck + (t0 + t) / BWD_CK1) * DK * DV;
 #pragma unroll
-                for (int i = 0; i < RI; ++i) store_row<CW>(dst + (size_t)(lane + 32 * i) * DV + col0, S[i]);
+                for (int j = 0; j < RP; ++j) {
+                    float *d = dst + (size_t)row_of(j) * DV + c0;
+                    if constexpr (CP == 2) *reinterpret_cast<float2 *>(d) = make_float2(S[j][0], S[j][1]);
+                    else d[0] = S[j][0];
+                }
             }
-            fwd_step<RI, CW>(S, sk + t * DK, sa + t * DK, sv + t * DV, sb[t], lane, col0,
-                             pbuf + (size_t)(t0 + t) * DV);
+            fwd_step_rows<DK, DV>(S, sk + t * DK, sa + t * DK, sv + t * DV, sb[t], rg, c0,
+                                  pbuf + (size_t)(t0 + t) * DV);
         }
     }
     if (tid == 0) stamp_end(prm.stamp);

@@ -159,10 +159,9 @@ int kda_chunk_fwd_host(const void *q, const void *k, const void *v, const float 
         cudaStreamWaitEvent(st->up, st->fork, 0) != cudaSuccess ||
         cudaStreamWaitEvent(st->down, st->fork, 0) != cudaSuccess)
         return KDA_ERR_CUDA;
-    if (h0 != nullptr && cudaMemcpyAsync(state, h0, state_bytes, cudaMemcpyHostToDevice, st->up) != cudaSuccess)
-        return KDA_ERR_CUDA;
-
     int status = KDA_OK;
+    if (h0 != nullptr && cudaMemcpyAsync(state, h0, state_bytes, cudaMemcpyHostToDevice, st->up) != cudaSuccess)
+        status = KDA_ERR_CUDA;
     int i = 0;
     for (int t0 = 0; t0 < T && status == KDA_OK; t0 += P, ++i) {
         const int n = T - t0 < P ? T - t0 : P;
@@ -202,8 +201,11 @@ int kda_chunk_fwd_host(const void *q, const void *k, const void *v, const float 
     if (status == KDA_OK && hT != nullptr &&
         cudaMemcpyAsync(hT, state, state_bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
         status = KDA_ERR_CUDA;
-    // join: the caller's stream follows the last download (the download stream is serial)
-    if (i > 0 && cudaStreamWaitEvent(s, st->downloaded[(i - 1) & 1], 0) != cudaSuccess) status = KDA_ERR_CUDA;
+    // join: the caller's stream follows everything enqueued on the copy streams (on an
+    // error path too, so that the next call cannot reuse staging under a copy in flight)
+    if (cudaEventRecord(st->uploaded[0], st->up) != cudaSuccess || cudaEventRecord(st->downloaded[0], st->down) != cudaSuccess ||
+        cudaStreamWaitEvent(s, st->uploaded[0], 0) != cudaSuccess || cudaStreamWaitEvent(s, st->downloaded[0], 0) != cudaSuccess)
+        status = KDA_ERR_CUDA;
     if (cudaEventRecord(st->done, s) != cudaSuccess) status = KDA_ERR_CUDA;
     return status;
 }
