@@ -4,6 +4,8 @@ import json
 import os
 import sys
 
+import pytest
+
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 sys.path.insert(0, ROOT)
 
@@ -115,3 +117,90 @@ def test_scalar_gate_line_with_stand_in_device(monkeypatch):
     per_channel = bench.prefill_bytes(cfg.B, cfg.T, cfg.H, cfg.dk, cfg.dv, cfg.h0_std > 0, True)
     assert r["roofline"]["algorithmic_bytes_per_launch"] == per_channel - cfg.B * cfg.T * cfg.H * 4 * (cfg.dk - 1)
     assert r["entry_point"] == "kda_gdn_chunk_fwd"
+
+
+def _stand_in_events(monkeypatch, calls, ms_per_call=2.0):
+    import torch
+
+    class Event:
+        def __init__(self, **kw):
+            self.t = None
+
+        def record(self, stream=None):
+            self.t = len(calls)
+
+        def elapsed_time(self, other):
+            return ms_per_call * (other.t - self.t)
+
+    monkeypatch.setattr(torch.cuda, "Event", Event)
+    monkeypatch.setattr(torch.cuda, "synchronize", lambda: None)
+
+
+def test_raw_prologue_line_with_stand_in_device(monkeypatch):
+    """The raw-input item passes the workload's tensors as the raw projections with
+    the workload's decay scale, and counts the per-channel prefill's bytes."""
+    from gated_delta_rule_100_b200 import inputs, kda
+
+    calls = []
+    monkeypatch.setattr(kda, "chunk_fwd_raw", lambda q, k, v, g, beta, c, scale, h0, **kw: calls.append((g, c)))
+    monkeypatch.setattr(kda, "stream_status", lambda stream=None: kda.KDA_OK)
+    _stand_in_events(monkeypatch, calls)
+    cfg = inputs.CONFIGS["oracle_scale_B1_H1_T256_d64"]
+    d = inputs.make_config(cfg)
+    r = bench.measure_raw(d, cfg, None, None, None, steps=3, warmup=1, P={"hbm_gbs": 1000.0})
+    assert len(calls) == 4 and all(g is d["g"] and c == cfg.decay for g, c in calls)
+    assert r["ms_per_step"] == 2.0 and r["entry_point"] == "kda_chunk_fwd_raw"
+    assert r["roofline"]["algorithmic_bytes_per_launch"] == bench.prefill_bytes(
+        cfg.B, cfg.T, cfg.H, cfg.dk, cfg.dv, cfg.h0_std > 0, True)
+
+
+def test_varlen_line_with_stand_in_device(monkeypatch):
+    """The packed-batch item: the recipe's offsets reach the call, and the bytes are
+    the tokens' plus one initial and one final state per sequence."""
+    from gated_delta_rule_100_b200 import inputs, kda
+
+    vc = inputs.VarlenConfig("tiny_varlen", 5, 2, 64, 64, 16, 300, 0.05, 0.02, 11)
+    monkeypatch.setattr(inputs, "VARLEN_CONFIG", vc)
+    calls = []
+
+    def fake(q, k, v, g, beta, scale, cu, h0, **kw):
+        calls.append(cu.tolist())
+        assert q.shape[0] == cu[-1] and h0.shape == (vc.N, vc.H, vc.dk, vc.dv)
+
+    monkeypatch.setattr(kda, "chunk_fwd_varlen", fake)
+    monkeypatch.setattr(kda, "stream_status", lambda stream=None: kda.KDA_OK)
+    _stand_in_events(monkeypatch, calls)
+    r = bench.measure_varlen(None, steps=2, warmup=1, P={"hbm_gbs": 1000.0}, dev="cpu")
+    lengths = inputs.varlen_lengths(vc)
+    assert calls[0] == [0] + list(__import__("itertools").accumulate(lengths))
+    assert all(vc.min_len <= n <= vc.max_len for n in lengths)
+    T = sum(lengths)
+    state = 4 * vc.dk * vc.dv * vc.N * vc.H
+    assert r["config"]["T_total"] == T and r["value"] == T / 2e-3
+    assert r["roofline"]["algorithmic_bytes_per_launch"] == bench.prefill_bytes(1, T, vc.H, vc.dk, vc.dv,
+                                                                                False, False) + 2 * state
+
+
+def test_two_level_line_restores_the_parts_hook(monkeypatch):
+    """The few-heads item times the automatic choice, then the plain pass, and leaves
+    the parts hook at automatic even when a call fails."""
+    from gated_delta_rule_100_b200 import inputs, kda
+
+    monkeypatch.setattr(inputs, "TWO_LEVEL_CONFIG", inputs.PrefillConfig("tiny", 1, 2, 256, 64, 64, 0.01, 0.02, 5))
+    parts, calls = [], []
+    monkeypatch.setattr(kda, "set_parts", lambda p: parts.append(p))
+    monkeypatch.setattr(kda, "chunk_fwd", lambda *a, **kw: calls.append(parts[-1]))
+    monkeypatch.setattr(kda, "stream_status", lambda stream=None: kda.KDA_OK)
+    _stand_in_events(monkeypatch, calls)
+    r = bench.measure_two_level(None, steps=2, warmup=1, P={"hbm_gbs": 1000.0}, dev="cpu")
+    assert calls == [0, 0, 0, 1, 1, 1] and parts[-1] == 0
+    assert r["ms_per_step"] == 2.0 and r["plain_pass_ms_per_step"] == 2.0
+
+    def boom(*a, **kw):
+        raise RuntimeError("device error")
+
+    parts.clear()
+    monkeypatch.setattr(kda, "chunk_fwd", boom)
+    with pytest.raises(RuntimeError):
+        bench.measure_two_level(None, steps=2, warmup=1, P={"hbm_gbs": 1000.0}, dev="cpu")
+    assert parts[-1] == 0
