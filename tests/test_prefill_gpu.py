@@ -311,3 +311,20 @@ def test_kernel_launch_timeline():
     c = next(x for x in L if x[0] == "chain")
     assert c[1] >= p[2] - 1e-6  # the chain starts after its records are written
     assert kda.kernel_launches() == []
+
+
+@pytest.mark.parametrize("B,H,T", [(64, 32, 100), (256, 16, 1)])
+def test_many_heads_short_sequences(B, H, T):
+    """Thousands of (b, h) with one or two chunks each: one chain CTA per (b, h)
+    (many waves), a partial chunk, h0 read and hT written per (b, h).  Checked
+    against the oracle on every sequence of two heads and on all heads of two
+    batch rows."""
+    d = inputs.make_prefill(B, T, H, 128, 128, decay=0.05, h0_std=0.02, seed=23 + T, device=DEV)
+    out, hT = run(d, 128 ** -0.5)
+    assert kda.stream_status() == kda.KDA_OK
+    o_ref, s_ref = oracle_prefill(d, 128 ** -0.5, heads=[0, H - 1])
+    assert_close(f64(out[:, :, [0, H - 1]]), o_ref, f"B{B} H{H} T{T} out (heads 0, {H - 1})")
+    assert_close(f64(hT[:, [0, H - 1]]), s_ref, f"B{B} H{H} T{T} hT (heads 0, {H - 1})")
+    o_ref, s_ref = oracle_prefill(d, 128 ** -0.5, batches=[0, B - 1])
+    assert_close(f64(out[[0, B - 1]]), o_ref, f"B{B} H{H} T{T} out (batches 0, {B - 1})")
+    assert_close(f64(hT[[0, B - 1]]), s_ref, f"B{B} H{H} T{T} hT (batches 0, {B - 1})")
