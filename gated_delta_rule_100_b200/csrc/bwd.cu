@@ -14,10 +14,11 @@
 // This is the recurrent form: exact, and every step is column-local except
 // for dq, dk, dg and dbeta, which sum over the dv columns.
 //
-// Layout: one CTA of 512 threads per (b, h).  Warp w owns state columns
-// w CW .. w CW + CW - 1, lane l owns rows l + 32 i; so the column reductions
-// (p, du) are warp shuffles, and the sums over columns go through
-// shared-memory atomics per token.
+// Layout: one CTA of 512 threads per (b, h).  In pass 2 warp w owns state
+// columns w CW .. w CW + CW - 1 and lane l rows l + 32 i, so the column
+// reduction du is a warp shuffle and the sums over columns go through
+// shared-memory atomics per token; pass 1, which has no sums over columns,
+// gives each thread 16 rows and 2 columns (see fwd_step_rows).
 //   Pass 1 (bwd_ckpt_kernel): the forward recurrence from h0, storing S every
 //          CK1 = 64 tokens (level-1 checkpoints, fp32, in the workspace) and
 //          every token's p = S'^T k (fp32 [T][dv] per (b, h)).  Every later
@@ -36,7 +37,7 @@
 //          column as it is formed; dh0 at the end.
 // Memory: (ceil(T / 64) + 16) dk dv + T dv fp32 per (b, h); forward steps per token:
 // one in pass 1, one for level 2, one on average for the per-token states
-// (blocks of 8 took 56 ms on B8 H32 T4096, 3.5 recomputed steps per token).
+// (blocks of 8, with 3.5 recomputed steps per token, were slower).
 // Inputs are staged in shared memory per block of tokens, loaded into registers
 // one block ahead.  Level-2 states go through global memory (the scratch); the
 // reverse walk copies each block's state into one of two shared buffers with
