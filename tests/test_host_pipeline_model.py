@@ -20,6 +20,8 @@ import random
 
 import pytest
 
+from stream_model import simulate
+
 
 def enqueue_call(npieces, skip=(), ops=None, call=0, caller="s"):
     """The enqueue sequence of one kda_chunk_fwd_host call made on stream `caller`:
@@ -59,27 +61,6 @@ def enqueue_call(npieces, skip=(), ops=None, call=0, caller="s"):
     add("s", "record", "done")
     add("s", "op", ("after", call, None, None))  # the caller's next work on its stream
     return ops
-
-
-def simulate(ops, rng):
-    """Start and end times of every op under the event semantics."""
-    stream_end = {}  # completion time of the last op enqueued on each stream
-    stream_ready = {}  # earliest start of the next op on each stream (waits included)
-    record_time = {}  # event -> completion time of its most recent record (as enqueued)
-    spans = []
-    for stream, kind, arg in ops:
-        t = stream_end.get(stream, 0.0)
-        if kind == "record":  # captures everything enqueued on the stream so far, waits included
-            record_time[arg] = max(t, stream_ready.get(stream, 0.0))
-        elif kind == "wait":
-            if arg in record_time:
-                stream_ready[stream] = max(stream_ready.get(stream, 0.0), record_time[arg])
-        else:
-            start = max(t, stream_ready.get(stream, 0.0))
-            end = start + rng.uniform(0.1, 3.0)
-            stream_end[stream] = end
-            spans.append((arg, start, end, stream))
-    return spans
 
 
 def violations(spans):
