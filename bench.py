@@ -850,6 +850,29 @@ def run_ours(args):
                             "traffic_note": "ncu dram__bytes_read.sum + dram__bytes_write.sum per launch, "
                                             "captured on this workload",
                             "algorithmic_bytes_per_launch": db}}
+        # the same steps from raw projections (gate prologue and q/k norms in the kernel),
+        # the workload's tensors taken as the raw values; it never fails the line
+        try:
+            def raw_step(s):
+                kda.decode_step_raw(dd["q"][s], dd["k"][s], dd["v"][s], dd["g"][s], dd["beta"][s], dcfg.decay,
+                                    dcfg.scale, state, out=dout, stream=stream)
+
+            for s in range(3):
+                raw_step(s)
+            torch.cuda.synchronize()
+            e0.record(stream)
+            for s in range(dcfg.steps):
+                raw_step(s)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            if kda.stream_status(stream) != kda.KDA_OK:
+                raise RuntimeError("device-side error in the raw decode steps")
+            rms = e0.elapsed_time(e1)
+            rgbs = db * dcfg.steps / (rms / 1e3) / 1e9
+            dec["raw_prologue"] = {"entry_point": "kda_decode_step_raw", "us_per_step": rms * 1e3 / dcfg.steps,
+                                   "achieved_gbs": rgbs, "frac": rgbs / P["hbm_gbs"], "gate_c": dcfg.decay}
+        except Exception as exc:  # noqa: BLE001
+            dec["raw_prologue"] = {"error": f"{type(exc).__name__}: {exc}"[:300]}
         del dd, state
 
     # ---------------- end to end from pinned host buffers ----------------
