@@ -604,8 +604,8 @@ def measure_backward(P, stream, steps, dev):
 
 def cpu_baseline_table(budget_s=3.0):
     """The fp64 oracle on each workload's recipe, on 1 thread and on all host
-    cores: the first two workloads in full, the training shape and the decode
-    workload on samples sized to about `budget_s` each.  Prefill in tokens/s of
+    cores: the first two workloads in full, the training shape (forward and
+    backward) and the decode workload on samples sized to about `budget_s` each.  Prefill in tokens/s of
     the full workload's head count (token-heads/s / H), decode in GB/s of the
     decode step's algorithmic traffic."""
     import numpy as np
@@ -635,6 +635,20 @@ def cpu_baseline_table(budget_s=3.0):
             rows.append({"workload": name, "threads": threads, "seconds": dt,
                          "sample": "full" if full else f"{heads} heads x {T} tokens (batch 1)",
                          "tokens_per_s": th / dt / cfg.H})
+    # the backward on the training shape's recipe: the oracle keeps every state of a
+    # (b, h), so a sample of 512 tokens per head, one head per thread
+    cfg = inputs.CONFIGS["training_B8_H32_T4096_d128"]
+    for threads in (1, cores):
+        heads, T = min(cfg.H, max(1, threads)), 512
+        d = inputs.make_prefill(1, T, heads, cfg.dk, cfg.dv, decay=cfg.decay, h0_std=cfg.h0_std, seed=cfg.seed)
+        gen = __import__("torch").Generator().manual_seed(cfg.seed + 100)
+        dout = __import__("torch").randn((1, T, heads, cfg.dv), generator=gen)
+        t0 = time.perf_counter()
+        oracle.kda_bwd(*(f64(d[k]) for k in ("q", "k", "v", "g", "beta")), cfg.scale,
+                       None if d["h0"] is None else f64(d["h0"]), f64(dout), None, threads=threads)
+        dt = time.perf_counter() - t0
+        rows.append({"workload": cfg.name + " backward", "threads": threads, "seconds": dt,
+                     "sample": f"{heads} heads x {T} tokens (batch 1)", "tokens_per_s": T * heads / dt / cfg.H})
     dcfg = inputs.DECODE_CONFIG
     for threads in (1, cores):
         nbh = min(dcfg.B, 8 * max(1, threads))  # sequences of the sample (all heads of each)
