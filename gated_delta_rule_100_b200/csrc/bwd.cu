@@ -86,7 +86,8 @@ __device__ __forceinline__ void store_row(float *dst, const float (&x)[CW]) {
 // three-level shuffle over the 8 row groups (lanes rg of one cg).  Rows in blocks of
 // four make each 16-byte read of k or alpha by 8 lanes one conflict-free wavefront.
 // One forward step S <- Diag(a) S + k (beta (v - p))^T; the rg == 0 lanes write p to
-// p_out.  Per element the operations are those of fwd_step_p, in the same order.
+// p_out (unless NULL).  Per element the operations are those of fwd_step_p, in the
+// same order.
 template <int DK, int DV>
 __device__ __forceinline__ void fwd_step_rows(float (&S)[DK / 8][DV / 64], const float *sk, const float *sa,
                                               const float *sv, float beta, int rg, int c0, float *p_out) {
@@ -113,7 +114,7 @@ __device__ __forceinline__ void fwd_step_rows(float (&S)[DK / 8][DV / 64], const
     for (int o = 1; o < 8; o <<= 1)
 #pragma unroll
         for (int c = 0; c < CP; ++c) p[c] += __shfl_xor_sync(0xffffffffu, p[c], o);
-    if (rg == 0) {
+    if (rg == 0 && p_out != nullptr) {
         if constexpr (CP == 2) *reinterpret_cast<float2 *>(p_out + c0) = make_float2(p[0], p[1]);
         else p_out[c0] = p[0];
     }
@@ -185,7 +186,9 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_ckpt_kernel(const BwdParam
         if (tid < nt) sb[tid] = prm.beta[((size_t)b * T + t0 + tid) * H + h];
         __syncthreads();
         for (int t = 0; t < nt; ++t) {
-            if ((t0 + t) % BWD_CK1 == 0) {  // the state before token t0 + t
+            if ((t0 + t) % BWD_CK1 == 0 &&  // the state before token t0 + t, into the level-1 region
+                KDA_CHECK(prm.st, ((long long)bh * nck + (t0 + t) / BWD_CK1 + 1) * DK * DV <=
+                                      (long long)prm.B * H * nck * DK * DV)) {
                 float *dst = prm.ckpt + ((size_t)bh * nck + (t0 + t) / BWD_CK1) * DK * DV;
 #pragma unroll
                 for (int j = 0; j < RP; ++j) {
@@ -194,8 +197,9 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_ckpt_kernel(const BwdParam
                     else d[0] = S[j][0];
                 }
             }
+            const bool p_in = KDA_CHECK(prm.st, (pbuf - prm.ckpt) + (long long)(t0 + t + 1) * DV <= prm.ckpt_elems);
             fwd_step_rows<DK, DV>(S, sk + t * DK, sa + t * DK, sv + t * DV, sb[t], rg, c0,
-                                  pbuf + (size_t)(t0 + t) * DV);
+                                  p_in ? pbuf + (size_t)(t0 + t) * DV : nullptr);
         }
     }
     if (tid == 0) stamp_end(prm.stamp);
@@ -263,7 +267,8 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_kernel(const BwdParams prm
             const size_t row = ((size_t)b * T + (in ? t0 + t : 0)) * H + h;
             rv[x] = in ? prm.v[row * DV + c] : (uint16_t)0;
             rd[x] = (in && prm.dout) ? prm.dout[row * DV + c] : (uint16_t)0;
-            rp[x] = in ? pbuf[(size_t)(t0 + t) * DV + c] : 0.f;
+            rp[x] = (in && KDA_CHECK(prm.st, (pbuf - prm.ckpt) + (long long)(t0 + t + 1) * DV <= prm.ckpt_elems))
+                        ? pbuf[(size_t)(t0 + t) * DV + c] : 0.f;
         }
         rb = tid < nt ? prm.beta[((size_t)b * T + t0 + tid) * H + h] : 0.f;
         pf_t0 = t0;
@@ -290,7 +295,12 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_kernel(const BwdParams prm
         if (tid < nt) sb[tid] = rb;
     };
     // a level-2 state from the scratch into a checkpoint tile (this thread's share)
+    [[maybe_unused]] const long long scratch_end = (long long)prm.B * H * (nck1 + BWD_CK1 / CK) * DK * DV;  // floats
     auto copy_state = [&](float *dst, const float *src) {
+        if (!KDA_CHECK(prm.st, (src - prm.ckpt) + (long long)DK * DV <= scratch_end)) {
+            cp_async_commit();  // an empty group keeps the waits' counts
+            return;
+        }
 #pragma unroll
         for (int x = 0; x < DK * DV / 4 / BWD_THREADS; ++x) {
             const int e = (tid + x * BWD_THREADS) * 4;
@@ -305,14 +315,25 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_kernel(const BwdParams prm
         {  // level 2: run the chunk forward from its level-1 checkpoint, leaving a state per block
             float S[RI][CW];
             const float *ck = prm.ckpt + ((size_t)bh * nck1 + n) * DK * DV;
+            const bool ck_in = KDA_CHECK(prm.st, ((long long)bh * nck1 + n + 1) * DK * DV <=
+                                                     (long long)prm.B * H * nck1 * DK * DV);
 #pragma unroll
-            for (int i = 0; i < RI; ++i) load_row<CW>(ck + (size_t)(lane + 32 * i) * DV + col0, S[i]);
+            for (int i = 0; i < RI; ++i) {
+                if (ck_in) {
+                    load_row<CW>(ck + (size_t)(lane + 32 * i) * DV + col0, S[i]);
+                } else {
+#pragma unroll
+                    for (int c = 0; c < CW; ++c) S[i][c] = 0.f;
+                }
+            }
             for (int jb = 0; jb < nb; ++jb) {
                 const int t0 = c0 + jb * CK;
                 const int nt = T - t0 < CK ? T - t0 : CK;
                 float *dst = scratch + (size_t)jb * DK * DV;
+                if (KDA_CHECK(prm.st, (dst - prm.ckpt) + (long long)DK * DV <= scratch_end)) {
 #pragma unroll
-                for (int i = 0; i < RI; ++i) store_row<CW>(dst + (size_t)(lane + 32 * i) * DV + col0, S[i]);
+                    for (int i = 0; i < RI; ++i) store_row<CW>(dst + (size_t)(lane + 32 * i) * DV + col0, S[i]);
+                }
                 if (jb + 1 == nb) break;  // the last block's state is not needed past its start
                 __syncthreads();          // the previous block's inputs are no longer read
                 if (pf_t0 != t0) fetch(t0, nt);

@@ -3,6 +3,8 @@
 #pragma once
 #include <stdint.h>
 
+#include "kda_device.cuh"
+
 namespace kda {
 
 struct BwdParams {
@@ -14,9 +16,12 @@ struct BwdParams {
     uint16_t *dq, *dk, *dv;     // bf16 [B, T, H, dk | dk | dv]
     float *dg, *dbeta;          // [B, T, H, dk], [B, T, H]
     float *dh0;                 // [B, H, dk, dv] or NULL
-    float *ckpt;                // [B H][ceil(T / 64)][dk][dv] level-1 states, then [B H][8][dk][dv] scratch
+    float *ckpt;                // [B H][ceil(T / 64)][dk][dv] level-1 states, [B H][16][dk][dv] level-2
+                                // scratch, then every token's p: [B H][T][dv]
+    long long ckpt_elems;       // floats of the ckpt workspace (the debug build's bound)
     float scale;
     int B, T, H;
+    DeviceStatus st;            // status word (the debug build's index checks report to it)
     unsigned long long *stamp;  // measurement hook: the launch pair's timing slot, or NULL
 };
 

@@ -905,6 +905,8 @@ int kda_chunk_bwd(const void *q, const void *k, const void *v, const float *g, c
     }
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return KDA_ERR_CUDA;
+    uint32_t *word = nullptr;  // before g_mu: current_status_word takes it too
+    if (current_status_word(&word) != KDA_OK) return KDA_ERR_CUDA;
     std::lock_guard<std::mutex> lk(g_mu);
     Workspace *w = nullptr;
     if (int st = reserve_workspace(dev, 0, 0, false, &w); st != KDA_OK) return st;
@@ -933,8 +935,11 @@ int kda_chunk_bwd(const void *q, const void *k, const void *v, const float *g, c
     bp.dbeta = dbeta;
     bp.dh0 = dh0;
     bp.ckpt = w->ckpt;
+    bp.ckpt_elems = (long long)(need / sizeof(float));
     bp.scale = scale;
     bp.B = B; bp.T = T; bp.H = H;
+    bp.st.word = word;
+    bp.st.wait_polls = ~0ull;  // the backward has no bounded waits
     if (timed_launch(dev, 4, s, [&](unsigned long long *t) {
             bp.stamp = t;
             return kda::launch_bwd(bp, dk, dv, s);

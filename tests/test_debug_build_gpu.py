@@ -3,9 +3,10 @@ record index and offset, shared-memory tile and tensor-operand view, token row
 and state slice whose bounds rest on layout constants and launch geometry is
 checked before use; a failed check is reported as KDA_ERR_BOUNDS (the access
 is skipped, nothing traps).  Run through the same binding on the small
-workload, short and ragged lengths, and every path of the prefill (exact,
+workload, short and ragged lengths, every path of the prefill (exact,
 two-level, segmented, packed with windows, no-allocation, raw inputs, scalar
-gate): no check may fail, and the results must still match the oracle."""
+gate) and the backward: no check may fail, and the results must still match
+the oracle."""
 import numpy as np
 import pytest
 import torch
@@ -95,3 +96,24 @@ def test_noalloc_raw_and_scalar_gate():
     kda.gdn_chunk_fwd(d["q"], d["k"], d["v"], gs, d["beta"], 0.1, d["h0"])
     kda.chunk_fwd_raw(d["q"], d["k"], d["v"], d["g"], d["beta"], 0.5, 0.1, d["h0"])
     assert kda.stream_status() == kda.KDA_OK
+
+
+@pytest.mark.parametrize("T", [1, 65, 200])
+@pytest.mark.parametrize("dk,dv", [(64, 128), (128, 64), (128, 128)])
+def test_backward(T, dk, dv):
+    """The backward through the debug library: its checks on the level-1 and level-2
+    checkpoint regions, the per-token p buffer and the asynchronous checkpoint
+    copies never fail, and the gradients match the oracle."""
+    d = inputs.make_prefill(2, T, 2, dk, dv, decay=0.05, h0_std=0.02, seed=3300 + T, device=DEV)
+    gen = torch.Generator(device=DEV).manual_seed(3400 + T)
+    dout = torch.randn((2, T, 2, dv), generator=gen, device=DEV).to(torch.bfloat16)
+    dhT = 0.1 * torch.randn((2, 2, dk, dv), generator=gen, device=DEV)
+    r = kda.chunk_bwd(d["q"], d["k"], d["v"], d["g"], d["beta"], dk ** -0.5, d["h0"], dout, dhT)
+    torch.cuda.synchronize()
+    assert kda.stream_status() == kda.KDA_OK, f"backward T={T} {dk}x{dv}: an index check failed"
+    ref = oracle.kda_bwd(f64(d["q"]), f64(d["k"]), f64(d["v"]), f64(d["g"]), f64(d["beta"]), dk ** -0.5,
+                         f64(d["h0"]), f64(dout), f64(dhT))
+    for n in ("dq", "dk", "dv", "dg", "dbeta", "dh0"):
+        # the bf16 gradients: one bf16 spacing of the largest reference value, as the backward's tests
+        bar = max(2e-2, 2.0 ** -7 * float(np.abs(ref[n]).max())) if n in ("dq", "dk", "dv") else 2e-2
+        assert_close(f64(r[n]), ref[n], f"debug backward T={T} {dk}x{dv} {n}", mabs=bar)
