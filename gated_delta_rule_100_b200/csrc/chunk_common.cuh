@@ -34,6 +34,7 @@ constexpr int NSUB = CH / SUB;  // 4
 constexpr int A_LD = 68;        // fp32 row stride of the A / T scratch
 constexpr float EXP_CLAMP_HI = 5.5406223843935098e34f;  // e^80
 constexpr float EXP_CLAMP_LO = 1.8048513878454153e-35f; // e^-80
+constexpr float MILD_DEC_LO = 4.2483542552915889e-18f;   // e^-40: least e^{Gamma_C} of a mild chunk
 
 constexpr int REC_WQ = 0;         // 32 KB (dk = 64 uses the first 16 KB)
 constexpr int REC_P = 32768;      // 8 KB

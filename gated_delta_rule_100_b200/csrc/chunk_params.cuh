@@ -141,6 +141,7 @@ struct PrepParams {
     int *steep_count;    // zero at launch: items appended to steep_items
     int *steep_items;    // items whose decay needs the exact kernel (room for every item)
     int force_exact;     // test hook: list every item
+    int block_refs;      // test hook: the 16-token block references for every item, mild or not
     float gate_c;        // gate prologue (raw g, beta, q, k): g = -gate_c softplus(g_raw)
     int H;
     SeqGeom gm;

@@ -50,6 +50,7 @@ uint32_t *g_status_ptr[kMaxDevices] = {};
 std::atomic<unsigned long long> g_wait_polls{0};
 std::atomic<unsigned long long> g_inject_polls{0};
 std::atomic<int> g_force_exact{0};
+std::atomic<int> g_block_refs{0};  // test hook: prep's block references for every chunk
 std::atomic<int> g_parts_override{0};  // test hook: parts of the two-level pass (0 = automatic, 1 = off)
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
@@ -395,7 +396,7 @@ kda::ExactParams exact_params(const void *q, const void *k, const float *g, int 
 
 extern "C" {
 
-int kda_abi_version(void) { return 103; }
+int kda_abi_version(void) { return 104; }
 
 const char *kda_status_string(int status) {
     switch (status) {
@@ -416,6 +417,8 @@ void kda_chunk_fwd_debug_wait_limit(unsigned long long polls) { g_wait_polls.sto
 void kda_chunk_fwd_debug_inject_timeout(unsigned long long polls) { g_inject_polls.store(polls); }
 
 void kda_chunk_fwd_debug_force_exact(int enable) { g_force_exact.store(enable != 0); }
+
+void kda_chunk_fwd_debug_block_refs(int enable) { g_block_refs.store(enable != 0); }
 
 void kda_chunk_fwd_debug_record_cap(unsigned long long bytes) { g_record_cap.store(bytes); }
 
@@ -546,6 +549,7 @@ static int chunk_fwd_impl(const void *q, const void *k, const void *v, const flo
         pp.steep_count = counters + 2 * buf + 1;
         pp.steep_items = steep_list;
         pp.force_exact = g_force_exact.load();
+        pp.block_refs = g_block_refs.load();
         pp.gate_c = gate_c;
         pp.H = H;
         pp.gm = uniform_geom(B, T, n0, cnt);
@@ -835,6 +839,7 @@ int kda_chunk_fwd_varlen(const void *q, const void *k, const void *v, const floa
         pp.steep_count = counters + 1;
         pp.steep_items = steep_list;
         pp.force_exact = g_force_exact.load();
+        pp.block_refs = g_block_refs.load();
         pp.gate_c = 0.f;
         pp.H = H;
         pp.gm = gm;
@@ -1094,6 +1099,7 @@ int kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const flo
         pp.steep_count = ticket + 1;
         pp.steep_items = steep_list;
         pp.force_exact = g_force_exact.load();
+        pp.block_refs = g_block_refs.load();
         pp.gate_c = 0.f;
         pp.H = H;
         pp.gm = uniform_geom(B, T, n0, cnt);

@@ -15,7 +15,12 @@
 // each result goes to a per-chunk record (layout in chunk_common.cuh).
 //
 // Decay factors.  e^{Gamma_i - Gamma_j} is split into two factors, one per
-// side of the contraction over key channels.  Rows of 16-token block I use
+// side of the contraction over key channels.  In a mild chunk (every key
+// channel keeps e^{Gamma_C} >= e^-40, which covers ordinary gates) the chunk's
+// start is the reference: row factor e^{Gamma_i}, column factor e^{-Gamma_j},
+// both within [e^-40, e^40], so the formation operands X = [K e^G; Q e^G] and
+// Y = K e^{-G} are products the record needs anyway and one 64-column product
+// forms A and P.  Otherwise rows of 16-token block I use
 // the reference m = 16 I + 8: row factor e^{Gamma_i - Gamma_m}, column factor
 // e^{Gamma_m - Gamma_j}.  For j in an earlier block both factors are <= 1; in
 // the block itself a factor can exceed 1.  It stays below e^80 unless some key
@@ -37,7 +42,8 @@
 // pairs, so the phase fits in 64 registers.  Phases per item:
 //   E  alpha, running products; operand tiles X, Y^(I) (bf16, smem) for the
 //      formation; Q e^G, K-hat (record); (K e^G)^T (tf32, smem)
-//   F  X Y^(I)^T -> A, P                    (UMMA bf16, overlapped with E's tail)
+//   F  X Y^(I)^T -> A, P                    (UMMA bf16, overlapped with E's tail;
+//      a mild chunk: X Y^T after all of E)
 //   AP A -> fp32 scratch, P -> record (fp16)
 //   T  (I + A)^{-1}: 16x16 diagonal blocks by substitution, off-diagonal blocks
 //      from N = D A_off as T = (I - N + N^2 - N^3) D, fp32 on CUDA cores
@@ -307,20 +313,87 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 dec *= btJ;
             }
         }
-        __syncthreads();  // the exchange area becomes X
+        // Mild chunk: no key channel loses more than 40 of log-decay over the chunk.  Then
+        // the chunk's own start is a usable reference for every token (factors e^{Gamma_t}
+        // and e^{-Gamma_t} within [e^-40, e^40]): X = [K e^G; Q e^G], Y = K e^{-G}, one
+        // 64-column formation product.  Otherwise the 16-token block references below.
+        const bool mild = __syncthreads_and(!active || dec >= MILD_DEC_LO) && !prm.block_refs;  // X's area is free
 
-        auto yput = [&](int Iy, int j0, const float (&v8)[8]) {
+        auto yput4 = [&](int Iy, int j0, uint4 w) {
             const uint32_t off = mnmaj<64, 2>(c, yoff(Iy) + j0, DK);
             if (KDA_CHECK(prm.st, off + 16 <= (uint32_t)(DK * 320)))
-                *reinterpret_cast<uint4 *>(sm + L::OFF_Y + off) = pack8_bf16(v8);
+                *reinterpret_cast<uint4 *>(sm + L::OFF_Y + off) = w;
         };
-        auto xput = [&](int col, const float (&v8)[8]) {
+        auto xput4 = [&](int col, uint4 w) {
             const uint32_t off = mnmaj<128, 2>(c, col, DK);
             if (KDA_CHECK(prm.st, off + 16 <= (uint32_t)(DK * 256)))
-                *reinterpret_cast<uint4 *>(sm + L::OFF_X + off) = pack8_bf16(v8);
+                *reinterpret_cast<uint4 *>(sm + L::OFF_X + off) = w;
         };
+        auto yput = [&](int Iy, int j0, const float (&v8)[8]) { yput4(Iy, j0, pack8_bf16(v8)); };
+        auto xput = [&](int col, const float (&v8)[8]) { xput4(col, pack8_bf16(v8)); };
         bool steep = false;  // a split factor of this thread's block would pass e^80
-        if (active) {
+        if (active && mild) {
+            // One pass over this thread's 16 tokens.  From the last token down, r =
+            // e^{Gamma_C - Gamma_t}: K-hat (record) and Y = K-hat / e^{Gamma_C} = K e^{-G}.
+            // From the first token up, p = e^{Gamma_t}: Q e^G (record, and the query rows
+            // of X), K e^G (the key rows of X, and (K e^G)^T).  Values are packed in pairs
+            // as they are formed.
+            if (I == 0 && rec_in && KDA_CHECK(prm.st, REC_DEC + 4 * c + 4 <= REC_BYTES))
+                reinterpret_cast<float *>(rec + REC_DEC)[c] = dec;
+            const float inv_dec = __fdividef(1.0f, dec);
+            {
+                uint16_t *khr = reinterpret_cast<uint16_t *>(rec + REC_KH) + (I * 128 + c) * SUB;
+                const bool kh_in = rec_in && KDA_CHECK(prm.st, ((I * 128 + c) * SUB + 16) * 2 <= REC_T - REC_KH);
+                float r = postB;
+#pragma unroll
+                for (int hh = 1; hh >= 0; --hh) {
+                    uint32_t hk[4], yk[4];
+#pragma unroll
+                    for (int e = 7; e >= 1; e -= 2) {  // tokens e - 1, e of the half
+                        const float hi = kval(hh * 8 + e) * r;
+                        r *= al[hh * 8 + e];
+                        const float lo = kval(hh * 8 + e - 1) * r;
+                        r *= al[hh * 8 + e - 1];
+                        hk[e / 2] = pack_f16x2(lo, hi);
+                        yk[e / 2] = pack_bf16x2(lo * inv_dec, hi * inv_dec);
+                    }
+                    if (kh_in) *reinterpret_cast<uint4 *>(khr + hh * 8) = make_uint4(hk[0], hk[1], hk[2], hk[3]);
+                    yput4(0, tb + hh * 8, make_uint4(yk[0], yk[1], yk[2], yk[3]));
+                }
+            }
+            {
+                uint16_t *qer = reinterpret_cast<uint16_t *>(rec + REC_WQ) + ((NSUB + I) * DK + c) * SUB;
+                const bool qe_in = rec_in && KDA_CHECK(prm.st, (((NSUB + I) * DK + c) * SUB + 16) * 2 <= REC_P - REC_WQ);
+                float p = preB;
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    uint32_t qk[4], xk[4];
+#pragma unroll
+                    for (int e4 = 0; e4 < 2; ++e4) {
+                        float b[4];
+#pragma unroll
+                        for (int ep = 0; ep < 2; ++ep) {
+                            const int u = hh * 8 + e4 * 4 + 2 * ep;
+                            p *= al[u];
+                            const float q0 = qval(u) * p, k0 = kval(u) * p;
+                            p *= al[u + 1];
+                            const float q1 = qval(u + 1) * p, k1 = kval(u + 1) * p;
+                            qk[e4 * 2 + ep] = pack_bf16x2(q0, q1);
+                            xk[e4 * 2 + ep] = pack_bf16x2(k0, k1);
+                            b[2 * ep] = k0;
+                            b[2 * ep + 1] = k1;
+                        }
+                        const uint32_t o = kmaj<128, 4>(c, tb + hh * 8 + e4 * 4, 128);
+                        if (KDA_CHECK(prm.st, o + 16 <= 128 * 64 * 4))
+                            *reinterpret_cast<uint4 *>(sm + L::OFF_BK + o) = pack4_tf32(b[0], b[1], b[2], b[3]);
+                    }
+                    const uint4 qw = make_uint4(qk[0], qk[1], qk[2], qk[3]);
+                    if (qe_in) *reinterpret_cast<uint4 *>(qer + hh * 8) = qw;
+                    xput4(tb + hh * 8, make_uint4(xk[0], xk[1], xk[2], xk[3]));
+                    xput4(CH + tb + hh * 8, qw);
+                }
+            }
+        } else if (active) {
             // Own block, reference m = tb + 8:
             //   u >= 8: f_u = prod_{s=9..u} alpha     X = k f,   Y^(I) = k / f
             //   u <  8: y_u = prod_{s=u+1..8} alpha   X = k / y, Y^(I) = k y
@@ -395,8 +468,10 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         }
 
         // ---------------- F: formation products (bf16), overlapped with the rest of E ----------------
-        if (tid == 0) {  // X [Y^(0) | .. | Y^(3)]^T: 128 x 160, column block I' = D^(I')
-            const uint32_t idesc = make_idesc(1, true, true, 128, yoff(NSUB));
+        // Block references: X [Y^(0) | .. | Y^(3)]^T, 128 x 160, column block I' = D^(I').
+        // Mild chunk: X Y^T, 128 x 64 (E is complete).
+        if (tid == 0) {
+            const uint32_t idesc = make_idesc(1, true, true, 128, mild ? CH : yoff(NSUB));
 #pragma unroll
             for (int kk = 0; kk < DK / 16; ++kk)
                 umma<0>(tmem + L::TM_AP, desc_mnmaj<128>(sbase + L::OFF_X, DK, kk * 16),
@@ -406,38 +481,36 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         mma_pending = true;
 
         // e^{Gamma_C - Gamma_t}: K-hat^T (record);  e^{Gamma_t}: Q e^G (record) and (K e^G)^T (smem)
-        {
-            if (active) {
-                if (I == 0 && rec_in && KDA_CHECK(prm.st, REC_DEC + 4 * c + 4 <= REC_BYTES))
-                    reinterpret_cast<float *>(rec + REC_DEC)[c] = dec;
-                uint16_t *khr = reinterpret_cast<uint16_t *>(rec + REC_KH) + (I * 128 + c) * SUB;
-                const bool kh_in = rec_in && KDA_CHECK(prm.st, ((I * 128 + c) * SUB + 16) * 2 <= REC_T - REC_KH);
-                float r = postB;
+        if (active && !mild) {
+            if (I == 0 && rec_in && KDA_CHECK(prm.st, REC_DEC + 4 * c + 4 <= REC_BYTES))
+                reinterpret_cast<float *>(rec + REC_DEC)[c] = dec;
+            uint16_t *khr = reinterpret_cast<uint16_t *>(rec + REC_KH) + (I * 128 + c) * SUB;
+            const bool kh_in = rec_in && KDA_CHECK(prm.st, ((I * 128 + c) * SUB + 16) * 2 <= REC_T - REC_KH);
+            float r = postB;
 #pragma unroll
-                for (int hh = 1; hh >= 0; --hh) {
-                    float kh[8];
+            for (int hh = 1; hh >= 0; --hh) {
+                float kh[8];
 #pragma unroll
-                    for (int e = 7; e >= 0; --e) { kh[e] = kval(hh * 8 + e) * r; r *= al[hh * 8 + e]; }
-                    if (kh_in) *reinterpret_cast<uint4 *>(khr + hh * 8) = pack8_f16(kh);
+                for (int e = 7; e >= 0; --e) { kh[e] = kval(hh * 8 + e) * r; r *= al[hh * 8 + e]; }
+                if (kh_in) *reinterpret_cast<uint4 *>(khr + hh * 8) = pack8_f16(kh);
+            }
+            uint16_t *qer = reinterpret_cast<uint16_t *>(rec + REC_WQ) + ((NSUB + I) * DK + c) * SUB;
+            const bool qe_in = rec_in && KDA_CHECK(prm.st, (((NSUB + I) * DK + c) * SUB + 16) * 2 <= REC_P - REC_WQ);
+            float p = preB;
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                float qe[8], bk[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    p *= al[hh * 8 + e];
+                    qe[e] = qval(hh * 8 + e) * p;
+                    bk[e] = kval(hh * 8 + e) * p;
                 }
-                uint16_t *qer = reinterpret_cast<uint16_t *>(rec + REC_WQ) + ((NSUB + I) * DK + c) * SUB;
-                const bool qe_in = rec_in && KDA_CHECK(prm.st, (((NSUB + I) * DK + c) * SUB + 16) * 2 <= REC_P - REC_WQ);
-                float p = preB;
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    float qe[8], bk[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        p *= al[hh * 8 + e];
-                        qe[e] = qval(hh * 8 + e) * p;
-                        bk[e] = kval(hh * 8 + e) * p;
-                    }
-                    if (qe_in) *reinterpret_cast<uint4 *>(qer + hh * 8) = pack8_bf16(qe);
-                    const uint32_t o0 = kmaj<128, 4>(c, tb + hh * 8, 128), o1 = kmaj<128, 4>(c, tb + hh * 8 + 4, 128);
-                    if (KDA_CHECK(prm.st, o0 + 16 <= 128 * 64 * 4 && o1 + 16 <= 128 * 64 * 4)) {
-                        *reinterpret_cast<uint4 *>(sm + L::OFF_BK + o0) = pack4_tf32(bk[0], bk[1], bk[2], bk[3]);
-                        *reinterpret_cast<uint4 *>(sm + L::OFF_BK + o1) = pack4_tf32(bk[4], bk[5], bk[6], bk[7]);
-                    }
+                if (qe_in) *reinterpret_cast<uint4 *>(qer + hh * 8) = pack8_bf16(qe);
+                const uint32_t o0 = kmaj<128, 4>(c, tb + hh * 8, 128), o1 = kmaj<128, 4>(c, tb + hh * 8 + 4, 128);
+                if (KDA_CHECK(prm.st, o0 + 16 <= 128 * 64 * 4 && o1 + 16 <= 128 * 64 * 4)) {
+                    *reinterpret_cast<uint4 *>(sm + L::OFF_BK + o0) = pack4_tf32(bk[0], bk[1], bk[2], bk[3]);
+                    *reinterpret_cast<uint4 *>(sm + L::OFF_BK + o1) = pack4_tf32(bk[4], bk[5], bk[6], bk[7]);
                 }
             }
         }
@@ -475,16 +548,23 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             float v16[16];
 #pragma unroll
             for (int e = 0; e < 16; ++e) v16[e] = 0.f;
-#pragma unroll
-            for (int dI = 0; dI < 2; ++dI) {
-                const int Ib = I0 + dI;
-                if (cc <= Ib) {  // warp-uniform
-                    float t[16];
-                    tmem_ld16(tmem + lane_base + L::TM_AP + yoff(Ib) + cc * 16, t);
+            if (mild) {  // column j of the product is token j
+                if (cc <= I0 + 1) {  // warp-uniform: some row of the quarter reaches this chunk
+                    tmem_ld16(tmem + lane_base + L::TM_AP + cc * 16, v16);
                     tmem_wait_ld();
-                    if (myI == Ib) {
+                }
+            } else {
 #pragma unroll
-                        for (int e = 0; e < 16; ++e) v16[e] = t[e];
+                for (int dI = 0; dI < 2; ++dI) {
+                    const int Ib = I0 + dI;
+                    if (cc <= Ib) {  // warp-uniform
+                        float t[16];
+                        tmem_ld16(tmem + lane_base + L::TM_AP + yoff(Ib) + cc * 16, t);
+                        tmem_wait_ld();
+                        if (myI == Ib) {
+#pragma unroll
+                            for (int e = 0; e < 16; ++e) v16[e] = t[e];
+                        }
                     }
                 }
             }

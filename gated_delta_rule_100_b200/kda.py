@@ -37,7 +37,7 @@ EXPORTED = ("kda_chunk_fwd", "kda_chunk_fwd_noalloc", "kda_chunk_fwd_host", "kda
             "kda_chunk_bwd", "kda_chunk_bwd_workspace_bytes",
             "kda_chunk_fwd_workspace_bytes", "kda_chunk_fwd_varlen_workspace_bytes", "kda_release_workspace",
             "kda_status_string", "kda_stream_status", "kda_chunk_fwd_debug_wait_limit",
-            "kda_chunk_fwd_debug_inject_timeout", "kda_chunk_fwd_debug_force_exact", "kda_chunk_fwd_debug_record_cap", "kda_chunk_fwd_debug_parts",
+            "kda_chunk_fwd_debug_inject_timeout", "kda_chunk_fwd_debug_force_exact", "kda_chunk_fwd_debug_block_refs", "kda_chunk_fwd_debug_record_cap", "kda_chunk_fwd_debug_parts",
             "kda_debug_kernel_timing", "kda_debug_kernel_times", "kda_debug_kernel_launches",
             "kda_abi_version")
 
@@ -120,6 +120,8 @@ def _open(path):
     lib.kda_chunk_fwd_debug_record_cap.restype = None
     lib.kda_chunk_fwd_debug_force_exact.argtypes = [i]
     lib.kda_chunk_fwd_debug_force_exact.restype = None
+    lib.kda_chunk_fwd_debug_block_refs.argtypes = [i]
+    lib.kda_chunk_fwd_debug_block_refs.restype = None
     lib.kda_debug_kernel_timing.argtypes = [i]
     lib.kda_debug_kernel_timing.restype = None
     lib.kda_debug_kernel_times.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_longlong), i]
@@ -406,6 +408,12 @@ def inject_timeout(polls: int) -> None:
 def force_exact(enable: bool) -> None:
     """Test hook: every prefill chunk takes the exact path (see ``kda.h``)."""
     load().kda_chunk_fwd_debug_force_exact(1 if enable else 0)
+
+
+def block_refs(enable: bool) -> None:
+    """Test hook: every prefill chunk is formed with its 16-token block
+    references, mild decay or not (see ``kda.h``)."""
+    load().kda_chunk_fwd_debug_block_refs(1 if enable else 0)
 
 
 KERNEL_KINDS = ("prep", "chain", "exact", "fixup", "bwd")

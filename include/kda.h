@@ -411,6 +411,17 @@ KDA_API void kda_chunk_fwd_debug_inject_timeout(unsigned long long polls);
 KDA_API void kda_chunk_fwd_debug_force_exact(int enable);
 
 /*
+ * kda_chunk_fwd_debug_block_refs -- test hook.  A chunk whose decay is mild
+ * (every key channel's log-decay over the chunk >= -40) is normally formed
+ * with one reference at the chunk's start; while enabled (enable != 0), every
+ * chunk of every prefill launched afterwards is formed with the references of
+ * its 16-token blocks instead, the form chunks with stronger decay take, so a
+ * test can compare the two forms on the same inputs.  Process-wide; off by
+ * default.
+ */
+KDA_API void kda_chunk_fwd_debug_block_refs(int enable);
+
+/*
  * kda_chunk_fwd_debug_record_cap -- test hook.  Caps the bytes of chunk
  * records the prefill workspace holds at once (0 restores the default,
  * 2 GiB), so that small problems exercise the paths long ones take: segments
@@ -463,7 +474,8 @@ KDA_API int kda_debug_kernel_launches(int *kind, long long *start_ns, long long 
 /* Version of this ABI (major * 100 + minor): 101 adds the scalar-gate entry
  * points, 102 the packed-batch prefill, the raw-input (fused gate prologue)
  * entry points, the backward pass and the exact-path and two-level test
- * hooks, 103 the host-buffer prefill and the per-launch timing list. */
+ * hooks, 103 the host-buffer prefill and the per-launch timing list, 104 the
+ * block-reference test hook. */
 KDA_API int kda_abi_version(void);
 
 #ifdef __cplusplus

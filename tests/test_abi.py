@@ -33,7 +33,7 @@ def test_header_declares_the_boundary():
 def test_library_exports_every_declared_symbol(lib):
     for name in declared_symbols():
         assert hasattr(lib, name), name
-    assert lib.kda_abi_version() == 103
+    assert lib.kda_abi_version() == 104
 
 
 def test_status_strings(lib):

@@ -3,8 +3,8 @@ record index and offset, shared-memory tile and tensor-operand view, token row
 and state slice whose bounds rest on layout constants and launch geometry is
 checked before use; a failed check is reported as KDA_ERR_BOUNDS (the access
 is skipped, nothing traps).  Run through the same binding on the small
-workload, short and ragged lengths, every path of the prefill (exact,
-two-level, segmented, packed with windows, no-allocation, raw inputs, scalar
+workload, short and ragged lengths, every path of the prefill (exact, block
+references, two-level, segmented, packed with windows, no-allocation, raw inputs, scalar
 gate) and the backward: no check may fail, and the results must still match
 the oracle."""
 import numpy as np
@@ -23,6 +23,7 @@ def _reset():
     kda.set_parts(0)
     kda.set_record_cap(0)
     kda.force_exact(False)
+    kda.block_refs(False)
 
 
 @pytest.fixture(autouse=True)
@@ -60,6 +61,9 @@ def test_exact_two_level_and_segmented_paths():
     kda.force_exact(True)
     run_and_check(d, 0.1, "exact path")
     kda.force_exact(False)
+    kda.block_refs(True)
+    run_and_check(d, 0.1, "block references")
+    kda.block_refs(False)
     kda.set_parts(3)
     run_and_check(d, 0.1, "two-level pass")
     kda.set_record_cap(2 * 2 * 8 * 74240)

@@ -16,10 +16,12 @@ def _reset_hooks():
     kda.inject_timeout(0)
     kda.set_wait_limit(0)
     kda.force_exact(False)
+    kda.block_refs(False)
     yield
     kda.inject_timeout(0)
     kda.set_wait_limit(0)
     kda.force_exact(False)
+    kda.block_refs(False)
     assert kda.stream_status() == kda.KDA_OK
 
 
@@ -233,6 +235,50 @@ def test_exact_path_matches_fast_path(dk, dv):
     kda.force_exact(False)
     assert_close(f64(ex_o), f64(fast_o), "exact vs fast out")
     assert_close(f64(ex_s), f64(fast_s), "exact vs fast hT")
+
+
+@pytest.mark.parametrize("dk,dv", [(64, 128), (128, 64), (128, 128)])
+@pytest.mark.parametrize("T", [77, 1000])
+def test_mild_and_block_forms_agree(T, dk, dv):
+    """A chunk whose decay is mild (every key channel keeps e^{Gamma_C} >= e^-40) is
+    formed with one reference at its start; the 16-token block references (the
+    form of chunks with stronger decay, forced here on every chunk) must give the
+    same results: both match the oracle and each other."""
+    d = inputs.make_prefill(2, T, 2, dk, dv, decay=0.1, h0_std=0.02, seed=650 + T + dk, device=DEV)
+    scale = dk ** -0.5
+    mild_o, mild_s = check(d, scale, f"mild form T={T} {dk}x{dv}")
+    kda.block_refs(True)
+    blk_o, blk_s = check(d, scale, f"block form T={T} {dk}x{dv}")
+    kda.block_refs(False)
+    assert_close(f64(blk_o), f64(mild_o), "block vs mild form out")
+    assert_close(f64(blk_s), f64(mild_s), "block vs mild form hT")
+
+
+@pytest.mark.parametrize("gate", ["per_channel", "scalar"])
+def test_decay_around_the_mild_limit(gate):
+    """Chunks on both sides of the mild limit in one sequence: in each chunk one key
+    channel (channel 0 for the scalar gate) decays at a constant rate whose chunk
+    total ranges from -30 to -70 (mild below 40, block references above, no
+    16-token block steep), the others at the workload's rate; the tail chunk is
+    ragged.  Every chunk must match the oracle whichever form it took."""
+    T = 16 * 64 + 23
+    d = inputs.make_prefill(1, T, 2, 128, 128, decay=0.05, h0_std=0.02, seed=660, device=DEV)
+    g = d["g"]
+    rates = torch.linspace(30.0, 70.0, (T + 63) // 64, device=DEV) / 64.0
+    ch = 0 if gate == "scalar" else 37
+    for n, r in enumerate(rates.tolist()):
+        g[0, 64 * n:64 * (n + 1), :, ch] = -r
+    scale = 128 ** -0.5
+    if gate == "scalar":
+        gs = g[..., 0].contiguous()
+        d["g"] = gs.unsqueeze(-1).expand_as(g).contiguous()
+        out, hT = kda.gdn_chunk_fwd(d["q"], d["k"], d["v"], gs, d["beta"], scale, d["h0"])
+    else:
+        out, hT = kda.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], scale, d["h0"])
+    torch.cuda.synchronize()
+    o_ref, s_ref = oracle_prefill(d, scale)
+    assert_close(f64(out), o_ref, f"mild limit {gate} out")
+    assert_close(f64(hT), s_ref, f"mild limit {gate} hT")
 
 
 def test_large_values_and_state():
