@@ -43,6 +43,7 @@ decode_step_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ 
     __shared__ float s_k[DK], s_q[DK], s_a[DK];
     __shared__ float s_red[2][NRG][DV];
     __shared__ float s_qk;
+    __shared__ float s_nrm[2][DK / 32];  // PRO: per-warp partial sums of q^2, k^2
 
     const int bh = blockIdx.x;
     const int tid = threadIdx.x;
@@ -61,26 +62,37 @@ decode_step_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ 
         const int r = rg * RPT + i;
         s[i] = __ldcs(reinterpret_cast<const float4 *>(S + (size_t)r * DV) + cg);
     }
-    for (int r = tid; r < DK; r += DEC_THREADS) {
-        s_k[r] = bf16_bits_to_f32(kh[r]);
-        s_q[r] = bf16_bits_to_f32(qh[r]);
-        const float gr = gh[g_dk > 1 ? r : 0];
-        s_a[r] = __expf(PRO ? gate_logdecay(gr, gate_c) : gr);
+    static_assert(DK <= DEC_THREADS, "one thread per key channel");
+    float kq = 0.f, qq = 0.f;  // PRO: this thread's raw k and q values
+    if (tid < DK) {
+        kq = bf16_bits_to_f32(kh[tid]);
+        qq = bf16_bits_to_f32(qh[tid]);
+        const float gr = gh[g_dk > 1 ? tid : 0];
+        s_a[tid] = __expf(PRO ? gate_logdecay(gr, gate_c) : gr);
+        if constexpr (PRO) {  // raw q, k: the sums of squares of the L2 norms, per warp
+            float sk = kq * kq, sq = qq * qq;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                sk += __shfl_xor_sync(0xffffffffu, sk, o);
+                sq += __shfl_xor_sync(0xffffffffu, sq, o);
+            }
+            if ((tid & 31) == 0) { s_nrm[0][tid >> 5] = sq; s_nrm[1][tid >> 5] = sk; }
+        } else {
+            s_k[tid] = kq;
+            s_q[tid] = qq;
+        }
+    }
+    if constexpr (PRO) {  // normalised q, k rounded to bf16 again, as the prefill's prologue
+        __syncthreads();
+        if (tid < DK) {
+            float sq = 0.f, sk = 0.f;
+#pragma unroll
+            for (int w = 0; w < DK / 32; ++w) { sq += s_nrm[0][w]; sk += s_nrm[1][w]; }
+            s_q[tid] = bf16_bits_to_f32(to_bf16_bits(qq * rsqrtf(fmaxf(sq, 1e-24f))));
+            s_k[tid] = bf16_bits_to_f32(to_bf16_bits(kq * rsqrtf(fmaxf(sk, 1e-24f))));
+        }
     }
     __syncthreads();
-    if constexpr (PRO) {  // raw q, k: L2-normalise each (warp 0: q, warp 1: k), as the prefill's prologue
-        if (tid < 64) {
-            float *x = tid < 32 ? s_q : s_k;
-            const int ln = tid & 31;
-            float ss = 0.f;
-            for (int r = ln; r < DK; r += 32) ss += x[r] * x[r];
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-            const float rn = rsqrtf(fmaxf(ss, 1e-24f));
-            for (int r = ln; r < DK; r += 32) x[r] = bf16_bits_to_f32(to_bf16_bits(x[r] * rn));
-        }
-        __syncthreads();
-    }
     if (tid < 32) {
         float acc = 0.f;
         for (int r = tid; r < DK; r += 32) acc += s_q[r] * s_k[r];
