@@ -469,7 +469,6 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
             if (more) {  // V^T is free: U(n) completed before product 1(n)
                 build_vt();
                 arrive(B_VT);
-                if (n + 2 < nseg) load_v(n + 2);
             }
             // state update, S = e^{Gamma_C} S0 + K-hat^T Vnew
             if (!(ok = wait_warp(B_M3, (uint32_t)(n & 1)))) break;
@@ -490,6 +489,10 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
             store_state_bf16();  // S0 is free: product 1(n) completed
             tc_fence_before();
             arrive(B_S0);
+            // The values of chunk n + 2, for V^T(n + 2) in the next iteration.  Issued
+            // here, not before the state update: global loads in flight there delayed its
+            // TMEM load (median 870 -> 270 cycles, chunk period 5.2k -> 4.6k cycles).
+            if (n + 2 < nseg) load_v(n + 2);
         }
         if (ok && lq >= 2) {  // the last chunk's output
             if ((ok = wait_warp(B_MB, (uint32_t)((nseg - 1) & 1)))) {
