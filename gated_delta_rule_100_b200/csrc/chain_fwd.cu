@@ -39,7 +39,8 @@
 // The state lives in fp32 registers (compute thread (c, g) holds row c and
 // VS / 4 columns); a bf16 copy in shared memory feeds the tensor core.  The
 // values V are read with plain coalesced loads one chunk before their V^T tile
-// is built.
+// is built, issued after the state update: global loads in flight delay the
+// compute warps' TMEM loads.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <stdint.h>
